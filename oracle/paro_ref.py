@@ -1,0 +1,403 @@
+"""Float64 CPU oracle of per-head block-sparse attention over a token grid.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the bench's
+CPU-baseline / reference legs may import this module.  It shares no code with
+the CUDA library and never imports it; both sides only share the seeded
+input generator.
+
+Every function is the plain definition of one step, written with NumPy in
+float64 (except where the INT8 path fixes float32 rounding), with no
+blocking, fusion or reordering beyond what the step itself states.  Sources:
+
+* PAROAttention (arXiv 2506.16054), Pith verdict page, "key_machinery" and
+  "core_discovery": a per-head permutation of the flattened sequence among
+  the six orders of [F, H, W]; a static block mask; block-wise INT8
+  quantisation of Q/K and of the post-softmax map P, with groups aligned to
+  the FlashAttention block.
+* SPADE (arXiv 2608.03335), Pith verdict page, "key_machinery" (iii) and the
+  referee's minor comments on section 3.1 (MEAN summariser) and section 2.2,
+  Eq. (2) (the mask is additive: 0 on kept block pairs, -inf on pruned ones),
+  and "core_discovery" (Top-K filter); flash block-sparse attention with an
+  online softmax.
+* PASA (arXiv 2604.12219), Pith page, Figure 2 caption: each query block
+  attends to at most k key blocks, cost O(S k) instead of O(S^2).
+
+Readings where the pages are silent (each one also listed in the design doc):
+
+1. An order's letters list the axes outermost -> innermost; FHW is the
+   natural flattening n = f*H*W + h*W + w.  Ids: 0 FHW, 1 FWH, 2 HFW,
+   3 HWF, 4 WFH, 5 WHF.
+2. Blocks are runs of ``block`` consecutive tokens of the permuted order;
+   the permuted sequence is zero-padded at its tail to N_p = NB*block.
+3. Block summary = mean of the block's valid (non-pad) rows; block score
+   = q_bar . k_bar / sqrt(d) (no softmax: it would not change a row's top-k).
+4. k = ceil(density * NB) clamped to [1, NB] (product rounded to 9 decimals
+   first); the diagonal block always kept and counts toward k; the other
+   k-1 are the largest scores, ties to the lower block index, NaN read as
+   -inf.  Selected indices are returned in ascending order.
+5. Pad keys are masked with -inf; pad query rows are never output.
+6. Softmax scale 1/sqrt(d).
+7. INT8: see :func:`quantize_int8` and :func:`attention_int8`.
+
+Parity status: every function here is pinned by the tests under
+``tests/test_oracle_*.py`` (brute force, library routines, closed forms);
+none is "parity unpinned".
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+# Axis letters of each order id, outermost first.
+ORDER_NAMES = ("FHW", "FWH", "HFW", "HWF", "WFH", "WHF")
+
+
+# ---------------------------------------------------------------- reorder --
+
+def order_axes(perm_id: int) -> tuple:
+    """(outer, middle, inner) axis indices of order ``perm_id`` (0=F,1=H,2=W)."""
+    return tuple("FHW".index(c) for c in ORDER_NAMES[int(perm_id)])
+
+
+def reorder_head(x: np.ndarray, grid: tuple, perm_id: int, block: int) -> np.ndarray:
+    """One head's [N, d] rows in natural FHW order -> [N_p, d] in the head's
+    order, zero rows appended at the tail (PAROAttention review,
+    key_machinery: the six axis orders of [F, H, W])."""
+    F, H, W = grid
+    N, d = x.shape
+    assert N == F * H * W
+    ax = order_axes(perm_id)
+    y = x.reshape(F, H, W, d).transpose(ax + (3,)).reshape(N, d)
+    nb = -(-N // block)
+    out = np.zeros((nb * block, d), dtype=x.dtype)
+    out[:N] = y
+    return out
+
+
+def inverse_reorder_head(xp: np.ndarray, grid: tuple, perm_id: int) -> np.ndarray:
+    """Inverse of :func:`reorder_head`: drop the pad rows, undo the order."""
+    F, H, W = grid
+    N = F * H * W
+    d = xp.shape[1]
+    ax = order_axes(perm_id)
+    sizes = tuple((F, H, W)[a] for a in ax)
+    y = xp[:N].reshape(sizes + (d,))
+    inv = tuple(int(i) for i in np.argsort(ax)) + (3,)
+    return y.transpose(inv).reshape(N, d)
+
+
+def reorder(x: np.ndarray, grid: tuple, perms, block: int) -> np.ndarray:
+    """[B, h, N, d] -> [B, h, N_p, d], per-head order ``perms[h]``."""
+    B, nh, N, d = x.shape
+    nb = -(-N // block)
+    out = np.zeros((B, nh, nb * block, d), dtype=x.dtype)
+    for b in range(B):
+        for h in range(nh):
+            out[b, h] = reorder_head(x[b, h], grid, perms[h], block)
+    return out
+
+
+def inverse_reorder(xp: np.ndarray, grid: tuple, perms) -> np.ndarray:
+    """[B, h, N_p, d] -> [B, h, N, d]."""
+    B, nh, _, d = xp.shape
+    N = grid[0] * grid[1] * grid[2]
+    out = np.zeros((B, nh, N, d), dtype=xp.dtype)
+    for b in range(B):
+        for h in range(nh):
+            out[b, h] = inverse_reorder_head(xp[b, h], grid, perms[h])
+    return out
+
+
+# ------------------------------------------------------- pooled scores --
+
+def block_pool(xp: np.ndarray, N: int, block: int) -> np.ndarray:
+    """Mean of each block's valid rows (SPADE review, MEAN summariser).
+    xp: [B, h, N_p, d] permuted; returns [B, h, NB, d] float64."""
+    B, nh, Np, d = xp.shape
+    nb = Np // block
+    out = np.zeros((B, nh, nb, d), dtype=np.float64)
+    for i in range(nb):
+        lo, hi = i * block, min((i + 1) * block, N)
+        out[:, :, i] = xp[:, :, lo:hi].astype(np.float64).mean(axis=2)
+    return out
+
+
+def block_scores(q_pool: np.ndarray, k_pool: np.ndarray) -> np.ndarray:
+    """S_bar[i, j] = q_bar_i . k_bar_j / sqrt(d)  (SPADE review, key_machinery
+    (iii), intra-estimation from the summaries).  [B, h, NB, NB] float64."""
+    d = q_pool.shape[-1]
+    return np.einsum("bhid,bhjd->bhij", q_pool, k_pool) / math.sqrt(d)
+
+
+def pooled_scores(q, k, grid, perms, block):
+    """Reorder -> mean-pool -> block score, from natural-order Q and K."""
+    N = grid[0] * grid[1] * grid[2]
+    qp = reorder(np.asarray(q, dtype=np.float64), grid, perms, block)
+    kp = reorder(np.asarray(k, dtype=np.float64), grid, perms, block)
+    qb = block_pool(qp, N, block)
+    kb = block_pool(kp, N, block)
+    return qb, kb, block_scores(qb, kb)
+
+
+# ---------------------------------------------------------------- top-k --
+
+def k_for_density(nb: int, density: float) -> int:
+    """ceil(density * NB) clamped to [1, NB]; the product is rounded to 9
+    decimals first so that binary round-off cannot add a block."""
+    if nb <= 0:
+        return 0
+    return int(min(nb, max(1, math.ceil(round(density * nb, 9)))))
+
+
+def select_topk_row(s: np.ndarray, i: int, k: int) -> np.ndarray:
+    """One query-block row: the diagonal block, then the k-1 largest other
+    scores, ties to the lower index, NaN as -inf; ascending indices
+    (PASA review, Figure 2: at most k key blocks per query block; SPADE
+    review, core_discovery: Top-K filter)."""
+    nb = s.shape[0]
+    k = min(k, nb)
+    v = np.where(np.isnan(s), -np.inf, s.astype(np.float64))
+    j = np.arange(nb)
+    others = j[j != i]
+    # lexsort: the last key is the primary one -> score descending, then index
+    order = np.lexsort((others, -v[others]))
+    chosen = np.concatenate(([i], others[order[:k - 1]]))
+    return np.sort(chosen).astype(np.int32)
+
+
+def select_topk(scores: np.ndarray, k: int) -> np.ndarray:
+    """[B, h, NB, NB] scores -> [B, h, NB, k] int32 kept block indices."""
+    B, nh, nb, _ = scores.shape
+    k = min(k, nb)
+    out = np.zeros((B, nh, nb, k), dtype=np.int32)
+    for b in range(B):
+        for h in range(nh):
+            for i in range(nb):
+                out[b, h, i] = select_topk_row(scores[b, h, i], i, k)
+    return out
+
+
+# ---------------------------------------------------------- static masks --
+
+def bitmask_from_idx(idx: np.ndarray, nb: int, counts=None) -> np.ndarray:
+    """Kept-index lists -> bitmask [B, h, NB, ceil(NB/32)] uint32, bit j%32 of
+    word j//32 set when key block j is kept (PAROAttention review,
+    key_machinery: static masks stored as bitmasks)."""
+    B, nh, rows, kk = idx.shape
+    words = -(-nb // 32)
+    out = np.zeros((B, nh, rows, words), dtype=np.uint32)
+    for b in range(B):
+        for h in range(nh):
+            for i in range(rows):
+                c = kk if counts is None else int(counts[b, h, i])
+                for j in idx[b, h, i, :c]:
+                    out[b, h, i, j // 32] |= np.uint32(1 << (int(j) % 32))
+    return out
+
+
+def compact_mask(bitmask: np.ndarray, nb: int):
+    """Bitmask -> (idx [B, h, NB, NB] int32 ascending, padded with -1;
+    counts [B, h, NB] int32)."""
+    B, nh, rows, _ = bitmask.shape
+    idx = np.full((B, nh, rows, nb), -1, dtype=np.int32)
+    counts = np.zeros((B, nh, rows), dtype=np.int32)
+    for b in range(B):
+        for h in range(nh):
+            for i in range(rows):
+                js = [j for j in range(nb)
+                      if (int(bitmask[b, h, i, j // 32]) >> (j % 32)) & 1]
+                counts[b, h, i] = len(js)
+                idx[b, h, i, :len(js)] = js
+    return idx, counts
+
+
+# ------------------------------------------------------------- attention --
+
+def attention_permuted(qp, kp, vp, N: int, block: int, idx, counts=None):
+    """Block-sparse softmax(Q K^T / sqrt(d) + M) V in the permuted domain.
+
+    M is the additive block mask (SPADE review, section 2.2, Eq. (2)): 0 where
+    key block j is in query block i's kept list and the key is a real token,
+    -inf elsewhere.  Rows are processed one query block at a time with a
+    max-subtracted softmax; only kept key blocks are gathered.
+    qp/kp/vp: [Np, d] float64; idx [NB, k] (counts [NB] or None).
+    Returns [Np, d] (pad rows zero).
+    """
+    Np, d = qp.shape
+    nb = Np // block
+    out = np.zeros((Np, vp.shape[1]), dtype=np.float64)
+    scale = 1.0 / math.sqrt(d)
+    for i in range(nb):
+        lo, hi = i * block, min((i + 1) * block, N)
+        if hi <= lo:
+            continue
+        c = idx.shape[1] if counts is None else int(counts[i])
+        kept = [int(j) for j in idx[i, :c]]
+        cols = np.concatenate([np.arange(j * block, min((j + 1) * block, N))
+                               for j in kept]) if kept else np.zeros(0, dtype=np.int64)
+        if cols.size == 0:
+            continue  # a row with no valid key: output stays 0
+        s = qp[lo:hi] @ kp[cols].T * scale
+        m = s.max(axis=1, keepdims=True)
+        p = np.exp(s - m)
+        out[lo:hi] = (p @ vp[cols]) / p.sum(axis=1, keepdims=True)
+    return out
+
+
+def attention(q, k, v, grid, perms, block, idx, counts=None):
+    """Reorder -> block-sparse attention over the kept tiles -> inverse
+    reorder.  q/k/v [B, h, N, d] natural order (any float dtype, upcast to
+    float64); idx [B, h, NB, k]; returns [B, h, N, d] float64."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, nh, N, d = q.shape
+    out = np.zeros((B, nh, N, v.shape[-1]), dtype=np.float64)
+    for b in range(B):
+        for h in range(nh):
+            qp = reorder_head(q[b, h], grid, perms[h], block)
+            kp = reorder_head(k[b, h], grid, perms[h], block)
+            vp = reorder_head(v[b, h], grid, perms[h], block)
+            cnt = None if counts is None else counts[b, h]
+            op = attention_permuted(qp, kp, vp, N, block, idx[b, h], cnt)
+            out[b, h] = inverse_reorder_head(op, grid, perms[h])
+    return out
+
+
+def attention_rows(q, k, v, grid, perms, block, idx, rows, counts=None):
+    """Outputs of selected natural-order query rows only: ``rows`` is a list
+    of (b, h, n).  Same definition as :func:`attention`, one row at a time,
+    for full-size checks where the whole output is too costly."""
+    q = np.asarray(q)
+    F, H, W = grid
+    N = F * H * W
+    d = q.shape[-1]
+    res = np.zeros((len(rows), d), dtype=np.float64)
+    pos_cache = {}
+    for r, (b, h, n) in enumerate(rows):
+        pid = int(perms[h])
+        if pid not in pos_cache:
+            perm_rows = reorder_head(np.arange(N, dtype=np.float64)[:, None], grid,
+                                     pid, block)[:N, 0].astype(np.int64)
+            pos = np.empty(N, dtype=np.int64)
+            pos[perm_rows] = np.arange(N)
+            pos_cache[pid] = (perm_rows, pos)
+        perm_rows, pos = pos_cache[pid]
+        i = pos[n] // block
+        c = idx.shape[-1] if counts is None else int(counts[b, h, i])
+        kept = [int(j) for j in idx[b, h, i, :c]]
+        cols_p = np.concatenate([np.arange(j * block, min((j + 1) * block, N))
+                                 for j in kept])
+        cols = perm_rows[cols_p]
+        qr = np.asarray(q[b, h, n], dtype=np.float64)
+        kk = np.asarray(k[b, h][cols], dtype=np.float64)
+        vv = np.asarray(v[b, h][cols], dtype=np.float64)
+        s = kk @ qr / math.sqrt(d)
+        p = np.exp(s - s.max())
+        res[r] = (p @ vv) / p.sum()
+    return res
+
+
+# ------------------------------------------------------------------ INT8 --
+
+def quantize_int8(xp: np.ndarray, N: int, block: int):
+    """Per-block symmetric INT8 quantisation (PAROAttention review,
+    key_machinery: block-wise INT8 with groups aligned to the FlashAttention
+    block; QK^T in INT8 as in its SageAttention baseline).
+
+    Defined in float32 with IEEE round-to-nearest on every operation:
+      absmax = max |x| over the block's valid rows,
+      inv    = fl32(127 / absmax),
+      q      = clamp(round_half_even(fl32(x * inv)), -127, 127),
+      scale  = fl32(absmax / 127);
+    a block with absmax 0 gets q = 0 and scale 0.  Pad rows quantise to 0.
+    xp: [B, h, N_p, d] permuted (values exactly representable in float32).
+    Returns q [B, h, N_p, d] int8 and scales [B, h, NB] float32.
+    """
+    x32 = np.asarray(xp, dtype=np.float32)
+    B, nh, Np, d = x32.shape
+    nb = Np // block
+    q = np.zeros((B, nh, Np, d), dtype=np.int8)
+    sc = np.zeros((B, nh, nb), dtype=np.float32)
+    for b in range(B):
+        for h in range(nh):
+            for i in range(nb):
+                lo, hi = i * block, min((i + 1) * block, N)
+                blk = x32[b, h, lo:hi]
+                amax = np.float32(np.abs(blk).max()) if hi > lo else np.float32(0)
+                if amax == 0:
+                    continue
+                inv = np.float32(np.float32(127.0) / amax)
+                y = np.rint(blk * inv)  # float32 multiply, then half-even
+                q[b, h, lo:hi] = np.clip(y, -127, 127).astype(np.int8)
+                sc[b, h, i] = np.float32(amax / np.float32(127.0))
+    return q, sc
+
+
+def attention_int8(q8, k8, v8, sq, sk, sv, N: int, block: int, idx, counts=None,
+                   mode: str = "online", quantize_p: bool = True):
+    """INT8 block-sparse attention in the permuted domain, one head.
+
+    S = (Q8 K8^T exact in integers) * s_q[i] * s_k[j] / sqrt(d) per tile.
+    P is quantised per (query block, key block) tile with a symmetric scale
+    (PAROAttention review, core_discovery: block-wise INT8 quantisation of
+    the post-softmax map).  The softmax numerator of a tile is bounded by 1
+    after max subtraction, so the tile's symmetric scale is 1/127:
+    p8 = round_half_even(127 * P_tilde), and the tile contributes
+    (p8 V8) * s_v[j] / 127.  The normaliser sums the unquantised P_tilde.
+
+    mode "online": kept tiles in ascending order with a running row max,
+    P_tilde = exp(s - m_run), earlier sums rescaled by exp(m_old - m_new)
+    (SPADE review, key_machinery (iii): flash block-sparse attention with
+    an online softmax) -- the order the pages describe.
+    mode "rowmax": P_tilde = exp(s - m_row) with the row's final max.
+    ``quantize_p=False`` skips the P rounding (P used exactly).
+
+    q8/k8/v8 [Np, d] int8, sq/sk/sv [NB] float32, idx [NB, k]; returns
+    [Np, d] float64 (pad rows zero).
+    """
+    Np, d = q8.shape
+    nb = Np // block
+    out = np.zeros((Np, d), dtype=np.float64)
+    inv_sqrt_d = 1.0 / math.sqrt(d)
+    qi = q8.astype(np.int64)
+    ki = k8.astype(np.int64)
+    vi = v8.astype(np.int64)
+    for i in range(nb):
+        lo, hi = i * block, min((i + 1) * block, N)
+        if hi <= lo:
+            continue
+        c = idx.shape[1] if counts is None else int(counts[i])
+        kept = [int(j) for j in idx[i, :c]]
+        tiles = []
+        for j in kept:
+            klo, khi = j * block, min((j + 1) * block, N)
+            if khi <= klo:
+                continue
+            s_int = qi[lo:hi] @ ki[klo:khi].T
+            s = s_int.astype(np.float64) * (float(sq[i]) * float(sk[j]) * inv_sqrt_d)
+            tiles.append((j, klo, khi, s))
+        rows = hi - lo
+        if not tiles:
+            continue
+        if mode == "rowmax":
+            m_row = np.max([t[3].max(axis=1) for t in tiles], axis=0)[:, None]
+        m = np.full((rows, 1), -np.inf)
+        l = np.zeros((rows, 1))
+        acc = np.zeros((rows, d))
+        for (j, klo, khi, s) in tiles:
+            if mode == "online":
+                m_new = np.maximum(m, s.max(axis=1, keepdims=True))
+                alpha = np.exp(m - m_new)
+            else:
+                m_new = m_row
+                alpha = np.ones((rows, 1))
+            pt = np.exp(s - m_new)
+            pq = np.rint(127.0 * pt) / 127.0 if quantize_p else pt
+            l = l * alpha + pt.sum(axis=1, keepdims=True)
+            acc = acc * alpha + (pq @ vi[klo:khi].astype(np.float64)) * float(sv[j])
+            m = m_new
+        out[lo:hi] = acc / l
+    return out

@@ -1,0 +1,127 @@
+"""Pins of the oracle's INT8 path (PAROAttention, arXiv 2506.16054, review
+key_machinery and core_discovery: block-wise INT8 quantisation with groups
+aligned to the attention block, for QK^T and for the post-softmax map P).
+
+* exact codes on hand-built blocks (round-half-to-even, clamp at +-127,
+  zero blocks, float32 scale arithmetic);
+* special case: integer inputs with absmax 127 quantise to themselves with
+  scale 1, so with P unrounded the INT8 attention equals the float64
+  attention of the same values;
+* analytic bound on the effect of rounding P;
+* online and row-max modes coincide when a row keeps a single block.
+"""
+
+import math
+
+import numpy as np
+
+from oracle import paro_ref as ref
+
+
+def test_codes_half_even_and_clamp():
+    # absmax 127 -> inv = 1, scale = 1: codes are the rounded values
+    blk = np.array([[127.0, 2.5, 3.5, -2.5], [-0.5, 0.5, 1.5, -127.0]], dtype=np.float32)
+    xp = blk.reshape(1, 1, 2, 4)
+    q, s = ref.quantize_int8(xp, 2, 2)
+    assert q[0, 0].tolist() == [[127, 2, 4, -2], [0, 0, 2, -127]]
+    assert s[0, 0, 0] == np.float32(1.0)
+
+
+def test_scale_arithmetic_is_float32():
+    x = np.array([[0.3, -0.1], [0.2, 0.05]], dtype=np.float32).reshape(1, 1, 2, 2)
+    q, s = ref.quantize_int8(x, 2, 2)
+    amax = np.float32(0.3)
+    inv = np.float32(127.0) / amax
+    assert s[0, 0, 0] == np.float32(amax / np.float32(127.0))
+    want = np.clip(np.rint(x[0, 0] * inv), -127, 127)
+    assert (q[0, 0] == want).all()
+    # 0.3 * fl32(127/0.3) rounds to 127 exactly
+    assert q[0, 0, 0, 0] == 127
+
+
+def test_zero_block_and_pad_rows():
+    x = np.zeros((1, 1, 8, 3), dtype=np.float32)
+    x[0, 0, 4:6] = 1.0
+    q, s = ref.quantize_int8(x, 6, 4)  # N = 6: block 1 has 2 real rows, 2 pad rows
+    assert s[0, 0, 0] == 0 and (q[0, 0, :4] == 0).all()
+    assert (q[0, 0, 4:6] == 127).all() and (q[0, 0, 6:] == 0).all()
+
+
+def integer_inputs(rng, Np, d):
+    x = rng.integers(-126, 127, size=(Np, d)).astype(np.float32)
+    x[0, 0] = 127.0  # every block of 4 rows gets absmax 127 below
+    return x
+
+
+def test_integer_inputs_reduce_to_float_attention():
+    rng = np.random.default_rng(3)
+    block, nb, d = 4, 5, 8
+    Np = N = block * nb
+    xs = []
+    for _ in range(3):
+        x = rng.integers(-126, 127, size=(Np, d)).astype(np.float32)
+        for i in range(nb):
+            x[i * block, 0] = 127.0
+        xs.append(x)
+    # shrink the scores so that the softmax is not one-hot
+    q8, sq = ref.quantize_int8(xs[0].reshape(1, 1, Np, d), N, block)
+    k8, sk = ref.quantize_int8(xs[1].reshape(1, 1, Np, d), N, block)
+    v8, sv = ref.quantize_int8(xs[2].reshape(1, 1, Np, d), N, block)
+    assert (sq == 1).all() and (q8[0, 0] == xs[0]).all()
+    idx = np.array([[0, 2, 3], [1, 2, 4], [0, 1, 2], [3, 4, 0], [4, 1, 2]], dtype=np.int32)
+    idx = np.sort(idx, axis=1)
+    # scale inputs by 2^-6 so that S / sqrt(d) stays moderate: use the
+    # float path with the same integer values and scales 2^-6
+    sq = sq * np.float32(2.0 ** -6)
+    sk = sk * np.float32(2.0 ** -6)
+    got = ref.attention_int8(q8[0, 0], k8[0, 0], v8[0, 0], sq[0, 0], sk[0, 0], sv[0, 0],
+                             N, block, idx, quantize_p=False)
+    want = ref.attention_permuted(xs[0].astype(np.float64) * 2.0 ** -6,
+                                  xs[1].astype(np.float64) * 2.0 ** -6,
+                                  xs[2].astype(np.float64), N, block, idx)
+    assert np.abs(got - want).max() < 1e-10
+    got_r = ref.attention_int8(q8[0, 0], k8[0, 0], v8[0, 0], sq[0, 0], sk[0, 0], sv[0, 0],
+                               N, block, idx, mode="rowmax", quantize_p=False)
+    assert np.abs(got_r - want).max() < 1e-10
+
+
+def test_p_rounding_bound():
+    rng = np.random.default_rng(8)
+    block, nb, d = 8, 4, 16
+    N = Np = block * nb
+    x = rng.standard_normal((3, 1, 1, Np, d)).astype(np.float32)
+    q8, sq = ref.quantize_int8(x[0] * 0.5, N, block)
+    k8, sk = ref.quantize_int8(x[1] * 0.5, N, block)
+    v8, sv = ref.quantize_int8(x[2], N, block)
+    idx = np.tile(np.arange(nb, dtype=np.int32), (nb, 1))
+    for mode in ("online", "rowmax"):
+        exact = ref.attention_int8(q8[0, 0], k8[0, 0], v8[0, 0], sq[0, 0], sk[0, 0], sv[0, 0],
+                                   N, block, idx, mode=mode, quantize_p=False)
+        quant = ref.attention_int8(q8[0, 0], k8[0, 0], v8[0, 0], sq[0, 0], sk[0, 0], sv[0, 0],
+                                   N, block, idx, mode=mode)
+        # |dO_r| <= sum_c |dP_rc| |v_c| / l_r with |dP| <= 1/254 and l_r >= 1
+        vabs = np.abs(v8[0, 0].astype(np.float64)) * np.repeat(sv[0, 0], block)[:, None]
+        bound = vabs.sum(axis=0)[None, :] / 254.0
+        assert (np.abs(quant - exact) <= bound + 1e-12).all()
+        assert np.abs(quant - exact).max() > 0  # rounding did something
+
+
+def test_single_block_modes_agree():
+    rng = np.random.default_rng(2)
+    block, nb, d = 8, 3, 8
+    N = Np = block * nb
+    x = rng.standard_normal((3, 1, 1, Np, d)).astype(np.float32)
+    qs = [ref.quantize_int8(x[t], N, block) for t in range(3)]
+    idx = np.arange(nb, dtype=np.int32)[:, None]
+    a = ref.attention_int8(qs[0][0][0, 0], qs[1][0][0, 0], qs[2][0][0, 0], qs[0][1][0, 0],
+                           qs[1][1][0, 0], qs[2][1][0, 0], N, block, idx, mode="online")
+    b = ref.attention_int8(qs[0][0][0, 0], qs[1][0][0, 0], qs[2][0][0, 0], qs[0][1][0, 0],
+                           qs[1][1][0, 0], qs[2][1][0, 0], N, block, idx, mode="rowmax")
+    assert np.abs(a - b).max() < 1e-12
+
+
+def test_int32_dot_is_exact_range():
+    # the largest |Q8 . K8| over d = 128 fits float32's exact-integer range,
+    # so converting the int32 accumulator to float32 loses nothing
+    assert 127 * 127 * 128 < 2 ** 24
+    assert math.isclose(127 * 127 * 128, 2064512)
