@@ -1,0 +1,418 @@
+"""Benchmark of the block-sparse attention path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = the whole path for one 720p-shaped video DiT layer (B=1, 40 heads,
+d=128, 21x45x80 grid = 75,600 tokens, block 128, density 0.15):
+pooled block scores (reorder folded into the loads) -> top-k kept blocks ->
+block-sparse attention over the kept tiles (inverse reorder folded into the
+stores).  Inputs are resident in HBM when the timed region starts and are
+larger than L2 (3 x 774 MB), so no flush is needed between steps.
+
+Prints one JSON line (rank 0).  ``value`` is the effective TFLOPS over kept
+tiles (4*b^2*d FLOPs per kept tile) of the whole step, summed over ranks
+(each rank runs its own independent layer: weak scaling, no collective on
+the data path; the only collectives are the barrier and the max of the
+per-rank times).  The reference arm (``--impl reference``) times the
+float64 CPU oracle on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_attention_34_b200 import paro  # noqa: E402
+from block_sparse_attention_34_b200.configs import WORKLOADS  # noqa: E402
+from block_sparse_attention_34_b200.synth import make_inputs  # noqa: E402
+
+METRIC = "block-sparse attention latency (ms) & effective TFLOPS, % of TC peak, at given density"
+DEFAULT_WORKLOAD = "720p_21x45x80"
+
+
+# ---------------------------------------------------------------- helpers --
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(ws, backend):
+    if ws > 1 and not torch.distributed.is_initialized():
+        from datetime import timedelta
+        torch.distributed.init_process_group(backend=backend, timeout=timedelta(seconds=120))
+
+
+def max_over_ranks(x: float, ws: int, device) -> float:
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("attn_sm100.cu", "tmem.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "block_sparse_attention_34_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str):
+    """DRAM bytes per launch of the attention kernel from the committed ncu
+    summary, or None when the summary is missing or the kernel changed."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("kernel_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ steps --
+
+class Pipeline:
+    """Device buffers and the launches of one step (through the C ABI)."""
+
+    def __init__(self, w, q, k, v, perms, density, baseline=False):
+        self.w = w
+        self.pr = paro.Problem(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, perms)
+        self.k = paro.k_for_density(self.pr.NB, density)
+        self.q, self.k_, self.v = q, k, v
+        dev = q.device
+        pr = self.pr
+        self.q_pool = torch.empty((pr.B, pr.heads, pr.NB, pr.d), dtype=torch.float32, device=dev)
+        self.k_pool = torch.empty_like(self.q_pool)
+        self.scores = torch.empty((pr.B, pr.heads, pr.NB, pr.NB), dtype=torch.float32, device=dev)
+        self.idx = torch.empty((pr.B, pr.heads, pr.NB, self.k), dtype=torch.int32, device=dev)
+        self.out = torch.empty((pr.B, pr.heads, pr.N, pr.d), dtype=q.dtype, device=dev)
+        self.baseline = baseline
+        self.launches_per_step = 5  # pool q, pool k, score, top-k, attention
+
+    def select(self):
+        paro.block_score(self.q, self.k_, self.pr, self.q_pool, self.k_pool, self.scores)
+        paro.select_topk(self.scores, self.pr, self.k, self.idx)
+
+    def attend(self):
+        paro.block_sparse_attn(self.q, self.k_, self.v, self.pr, self.idx, out=self.out,
+                               baseline=self.baseline)
+
+    def step(self, ev=None):
+        self.select()
+        if ev is not None:
+            ev[0].record()
+        self.attend()
+        if ev is not None:
+            ev[1].record()
+
+    def flops(self):
+        return self.w.flops(self.k)
+
+
+def time_steps(pipe, steps, warmup, ws, device):
+    for _ in range(warmup):
+        pipe.step()
+    torch.cuda.synchronize()
+    ev_attn = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    start.record()
+    for s in range(steps):
+        pipe.step(ev_attn[s])
+    end.record()
+    torch.cuda.synchronize()
+    barrier(ws)
+    total_ms = start.elapsed_time(end)
+    attn_ms = [a.elapsed_time(b) for a, b in ev_attn]
+    return total_ms, attn_ms
+
+
+def e2e_steps(pipe, host_q, host_k, host_v, host_out, steps):
+    """The same step through the public API with host buffers: pinned host
+    -> device copies of Q, K, V, the path, and the device -> host copy of O,
+    all inside the timed region."""
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record()
+    for _ in range(steps):
+        pipe.q.copy_(host_q, non_blocking=True)
+        pipe.k_.copy_(host_k, non_blocking=True)
+        pipe.v.copy_(host_v, non_blocking=True)
+        pipe.step()
+        host_out.copy_(pipe.out, non_blocking=True)
+    end.record()
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / steps
+
+
+def cpu_baseline(w, q, k, v, perms, idx_host, budget_s=12.0, max_blocks=None):
+    """The float64 oracle, as it stands, on a bounded sample: head 0, query
+    blocks 0, 1, 2, ... until the time budget is spent.  Returns TFLOPS of
+    kept-tile work and the sample description."""
+    from oracle import paro_ref as ref
+    grid = (w.F, w.H, w.W)
+    qh = q[0, 0].double().numpy()
+    kh = k[0, 0].double().numpy()
+    vh = v[0, 0].double().numpy()
+    qp = ref.reorder_head(qh, grid, perms[0], w.block)
+    kp = ref.reorder_head(kh, grid, perms[0], w.block)
+    vp = ref.reorder_head(vh, grid, perms[0], w.block)
+    kk = idx_host.shape[-1]
+    t0 = time.perf_counter()
+    done = 0
+    nb = w.NB if max_blocks is None else min(w.NB, max_blocks)
+    while done < nb:
+        chunk = min(4, nb - done)
+        lo = done * w.block
+        ref.attention_permuted(qp[lo:lo + chunk * w.block], kp, vp, w.N, w.block,
+                               idx_host[0, 0, done:done + chunk])
+        done += chunk
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    flops = 4.0 * w.block * w.block * w.d * kk * done
+    return flops / dt / 1e12, dt, f"head 0, query blocks 0..{done - 1} of {w.NB} ({done * kk} kept tiles)"
+
+
+def cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+# ------------------------------------------------------------------- main --
+
+def run_ours(a):
+    ws, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU path)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(ws, "nccl")
+    w = WORKLOADS[a.workload]
+    q, k, v, perms = make_inputs(w)
+    qd, kd, vd = (t.to(device) for t in (q, k, v))
+    pipe = Pipeline(w, qd, kd, vd, perms, a.density if a.density is not None else w.density,
+                    baseline=a.kernel == "mma")
+    sampler = ClockSampler(local)
+    sampler.start()
+    total_ms, attn_ms = time_steps(pipe, a.steps, a.warmup, ws, device)
+    clocks = sampler.stop()
+    ms_step = max_over_ranks(total_ms / a.steps, ws, device)
+    attn_avg = max_over_ranks(sum(attn_ms) / len(attn_ms), ws, device)
+    flops = pipe.flops()
+    value = flops * ws / (ms_step / 1e3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", 1400.0))
+    achieved = flops / (attn_avg / 1e3) / 1e12
+
+    # speedup over the same kernel on the dense (density 1.0) layer
+    dense = None
+    if not a.no_dense:
+        dpipe = Pipeline(w, qd, kd, vd, perms, 1.0, baseline=a.kernel == "mma")
+        dsteps = max(2, min(a.steps, 3))
+        _, d_attn = time_steps(dpipe, dsteps, 1, ws, device)
+        dense_ms = max_over_ranks(sum(d_attn) / len(d_attn), ws, device)
+        dense = {"attn_ms": dense_ms, "tflops": dpipe.flops() / (dense_ms / 1e3) / 1e12,
+                 "speedup_attn": dense_ms / attn_avg, "target": 0.8 / (pipe.k / pipe.pr.NB)}
+        del dpipe
+
+    e2e = None
+    if not a.no_e2e:
+        host = [t.pin_memory() for t in (q, k, v)]
+        host_out = torch.empty(pipe.out.shape, dtype=pipe.out.dtype).pin_memory()
+        e_ms = max_over_ranks(e2e_steps(pipe, *host, host_out, max(1, min(a.steps, 5))), ws, device)
+        e2e = {"value": flops * ws / (e_ms / 1e3) / 1e12, "unit": "TFLOPS",
+               "ms_per_step": e_ms,
+               "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in host)),
+               "d2h_bytes_per_step": int(host_out.numel() * host_out.element_size())}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not a.no_cpu_baseline:
+        tf, dt, sample = cpu_baseline(w, q, k, v, perms, pipe.idx.cpu().numpy(), budget_s=a.cpu_budget)
+        cpu = {"value": tf, "unit": "TFLOPS", "cores": cores(), "kind": "oracle",
+               "sample": sample, "seconds": round(dt, 2)}
+
+    if rank == 0:
+        res = {
+            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": ws, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded structured q/k, normal v; no weights)",
+            "config": {
+                "workload": w.name, "B": w.B, "heads": w.heads, "grid": [w.F, w.H, w.W],
+                "N": w.N, "d": w.d, "block": w.block, "density": pipe.k / pipe.pr.NB,
+                "density_requested": a.density if a.density is not None else w.density,
+                "k": pipe.k, "NB": pipe.pr.NB, "kept_tiles": w.kept_tiles(pipe.k),
+                "flops_per_step": flops, "kernel": "tcgen05" if a.kernel == "tcgen05" else "mma.sync",
+                "l2": "inputs larger than L2 (q, k, v 774 MB each); no flush",
+                "parallelism": f"replicas x{ws} (independent layers, no data-path collective)",
+                "attn_ms": attn_avg, "select_ms": ms_step - attn_avg,
+            },
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": ncu_traffic(w.name),
+                         "kernel": "attn_sm100_kernel" if a.kernel == "tcgen05" else "attn_mma_kernel",
+                         "peak_source": f"{peak_src} bf16_tflops_sustained"},
+            "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": pipe.launches_per_step * a.steps,
+            "clocks": clocks, "dense": dense,
+        }
+        print(json.dumps(res), flush=True)
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
+def run_reference(a):
+    """The reference arm: the float64 oracle on the host cores (rank 0 only),
+    each step a bounded sample of the same workload."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    from oracle import paro_ref as ref
+    w = WORKLOADS[a.workload]
+    dens = a.density if a.density is not None else w.density
+    q, k, v, perms = make_inputs(w, heads=1)
+    grid = (w.F, w.H, w.W)
+    # the oracle's own selection for head 0 (pooled scores -> top-k)
+    _, _, s = ref.pooled_scores(q.double().numpy(), k.double().numpy(), grid, perms[:1], w.block)
+    kk = ref.k_for_density(w.NB, dens)
+    idx = ref.select_topk(s, kk)
+    blocks = max(1, a.ref_blocks)
+    times = []
+    for it in range(a.warmup + a.steps):
+        tf, dt, sample = cpu_baseline(w, q, k, v, perms, idx, budget_s=1e9, max_blocks=blocks)
+        if it >= a.warmup:
+            times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    flops = 4.0 * w.block * w.block * w.d * kk * blocks
+    value = flops / (ms / 1e3) / 1e12
+    res = {"metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": ws, "steps": a.steps,
+           "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+           "config": {"workload": w.name, "density": kk / w.NB, "k": kk,
+                      "sample_query_blocks": blocks, "note": "float64 CPU oracle"},
+           "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores(), "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--density", type=float, default=None)
+    ap.add_argument("--kernel", choices=["tcgen05", "mma"], default="tcgen05")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--ref-blocks", type=int, default=8)
+    a = ap.parse_args(argv)
+    if a.warmup < 3 and a.impl == "ours":
+        print("note: warmup raised to 3", file=sys.stderr)
+        a.warmup = 3
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,272 @@
+// The C ABI of libparo (declared in include/paro.h): argument validation,
+// the per-call Grid description, and dispatch to the kernels.  Nothing here
+// allocates device memory or synchronises.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "common.cuh"
+
+namespace paro {
+cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, pa_dtype dt,
+                              const Grid& g, const int32_t* idx, const int32_t* counts,
+                              int k_max, const float* qs, const float* ks, const float* vs,
+                              void* out, int32_t* status, cudaStream_t s);
+bool attn_sm100_supports(pa_dtype dt, const Grid& g);
+}  // namespace paro
+
+namespace {
+
+thread_local std::string g_error;
+
+pa_status fail(pa_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_error = buf;
+  return st;
+}
+
+pa_status ok() {
+  g_error.clear();
+  return PA_OK;
+}
+
+pa_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return ok();
+  return fail(PA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Validates the sizes and fills the grid description (order tables included).
+pa_status make_grid(const pa_shape& s, const int8_t* perms, bool need_perms, paro::Grid* g) {
+  if (s.B < 1 || s.heads < 1 || s.F < 1 || s.H < 1 || s.W < 1 || s.d < 1 || s.block < 1)
+    return fail(PA_ERR_INVALID_ARG, "shape fields must be >= 1 (B=%d heads=%d F=%d H=%d W=%d d=%d block=%d)",
+                s.B, s.heads, s.F, s.H, s.W, s.d, s.block);
+  if (s.heads > paro::kMaxHeads)
+    return fail(PA_ERR_UNSUPPORTED, "heads=%d exceeds the supported maximum %d", s.heads, paro::kMaxHeads);
+  if (s.d != 64 && s.d != 128)
+    return fail(PA_ERR_UNSUPPORTED, "head dim d=%d unsupported (64 or 128)", s.d);
+  if (s.block != 64 && s.block != 128)
+    return fail(PA_ERR_UNSUPPORTED, "block=%d unsupported (64 or 128)", s.block);
+  const int64_t N = (int64_t)s.F * s.H * s.W;
+  const int64_t NB = (N + s.block - 1) / s.block;
+  const int64_t Np = NB * s.block;
+  if (Np > (int64_t)1 << 30)
+    return fail(PA_ERR_UNSUPPORTED, "N=%lld tokens per head exceeds 2^30", (long long)N);
+  if ((int64_t)s.B * s.heads * Np * s.d >= ((int64_t)1 << 40))
+    return fail(PA_ERR_UNSUPPORTED, "tensor of B*heads*N_p*d elements too large");
+  std::memset(g, 0, sizeof(*g));
+  g->B = s.B;
+  g->heads = s.heads;
+  g->F = s.F;
+  g->H = s.H;
+  g->W = s.W;
+  g->d = s.d;
+  g->block = s.block;
+  g->N = (int32_t)N;
+  g->NB = (int32_t)NB;
+  g->Np = (int32_t)Np;
+  const int size[3] = {s.F, s.H, s.W};
+  const int stride[3] = {s.H * s.W, s.W, 1};
+  // axes of each order id, outermost first: FHW FWH HFW HWF WFH WHF
+  static const int axes[6][3] = {{0, 1, 2}, {0, 2, 1}, {1, 0, 2}, {1, 2, 0}, {2, 0, 1}, {2, 1, 0}};
+  for (int o = 0; o < 6; ++o) {
+    g->mid[o] = size[axes[o][1]];
+    g->inn[o] = size[axes[o][2]];
+    g->so[o] = stride[axes[o][0]];
+    g->sm[o] = stride[axes[o][1]];
+    g->si[o] = stride[axes[o][2]];
+  }
+  if (need_perms) {
+    if (perms == nullptr) return fail(PA_ERR_INVALID_ARG, "perms is NULL");
+    for (int h = 0; h < s.heads; ++h) {
+      if (perms[h] < 0 || perms[h] > 5)
+        return fail(PA_ERR_INVALID_ARG, "perms[%d]=%d is not an order id 0..5", h, (int)perms[h]);
+      g->perm[h] = perms[h];
+    }
+  }
+  return PA_OK;
+}
+
+#define PA_REQUIRE(cond, ...)                                   \
+  do {                                                          \
+    if (!(cond)) return fail(PA_ERR_INVALID_ARG, __VA_ARGS__); \
+  } while (0)
+
+pa_status check_float_dtype(pa_dtype dt) {
+  if (dt != PA_F32 && dt != PA_BF16)
+    return fail(PA_ERR_INVALID_ARG, "dtype %d: expected PA_F32 or PA_BF16", (int)dt);
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t pa_abi_version(void) { return 1; }
+
+const char* pa_last_error(void) { return g_error.c_str(); }
+
+int32_t pa_num_blocks(pa_shape s) {
+  if (s.F < 1 || s.H < 1 || s.W < 1 || s.block < 1) return -1;
+  const int64_t N = (int64_t)s.F * s.H * s.W;
+  const int64_t nb = (N + s.block - 1) / s.block;
+  return nb > INT32_MAX ? -1 : (int32_t)nb;
+}
+
+int32_t pa_k_for_density(int32_t nb, double density) {
+  if (nb <= 0) return 0;
+  double x = density * (double)nb;
+  if (!(x == x)) return 1;  // NaN density keeps the diagonal only
+  x = std::nearbyint(x * 1e9) / 1e9;  // round to 9 decimals
+  double c = std::ceil(x);
+  if (c < 1.0) c = 1.0;
+  if (c > (double)nb) c = (double)nb;
+  return (int32_t)c;
+}
+
+pa_status pa_reorder(const void* x, void* x_perm, pa_dtype dtype, pa_shape shape,
+                     const int8_t* perms, void* stream) {
+  paro::Grid g;
+  pa_status st = check_float_dtype(dtype);
+  if (st != PA_OK) return st;
+  if ((st = make_grid(shape, perms, true, &g)) != PA_OK) return st;
+  PA_REQUIRE(x && x_perm, "x and x_perm must be non-NULL");
+  PA_REQUIRE(aligned16(x) && aligned16(x_perm), "x and x_perm must be 16-byte aligned");
+  return cuda_status(paro::launch_reorder(x, x_perm, dtype, g, false, (cudaStream_t)stream),
+                     "pa_reorder launch");
+}
+
+pa_status pa_inverse_reorder(const void* x_perm, void* x, pa_dtype dtype, pa_shape shape,
+                             const int8_t* perms, void* stream) {
+  paro::Grid g;
+  pa_status st = check_float_dtype(dtype);
+  if (st != PA_OK) return st;
+  if ((st = make_grid(shape, perms, true, &g)) != PA_OK) return st;
+  PA_REQUIRE(x && x_perm, "x and x_perm must be non-NULL");
+  PA_REQUIRE(aligned16(x) && aligned16(x_perm), "x and x_perm must be 16-byte aligned");
+  return cuda_status(paro::launch_reorder(x_perm, x, dtype, g, true, (cudaStream_t)stream),
+                     "pa_inverse_reorder launch");
+}
+
+pa_status pa_block_score(const void* q, const void* k, pa_dtype dtype, pa_shape shape,
+                         const int8_t* perms, float* q_pool, float* k_pool, float* scores,
+                         void* stream) {
+  paro::Grid g;
+  pa_status st = check_float_dtype(dtype);
+  if (st != PA_OK) return st;
+  if ((st = make_grid(shape, perms, true, &g)) != PA_OK) return st;
+  PA_REQUIRE(q && k && q_pool && k_pool && scores,
+             "q, k, q_pool, k_pool and scores must be non-NULL");
+  PA_REQUIRE(aligned16(q) && aligned16(k), "q and k must be 16-byte aligned");
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = paro::launch_pool(q, dtype, g, q_pool, s);
+  if (e == cudaSuccess) e = paro::launch_pool(k, dtype, g, k_pool, s);
+  if (e == cudaSuccess) e = paro::launch_score(q_pool, k_pool, g, scores, s);
+  return cuda_status(e, "pa_block_score launch");
+}
+
+pa_status pa_score_pooled(const float* q_pool, const float* k_pool, pa_shape shape,
+                          float* scores, void* stream) {
+  paro::Grid g;
+  pa_status st = make_grid(shape, nullptr, false, &g);
+  if (st != PA_OK) return st;
+  PA_REQUIRE(q_pool && k_pool && scores, "q_pool, k_pool and scores must be non-NULL");
+  return cuda_status(paro::launch_score(q_pool, k_pool, g, scores, (cudaStream_t)stream),
+                     "pa_score_pooled launch");
+}
+
+pa_status pa_select_topk(const float* scores, pa_shape shape, int32_t k, int32_t* idx,
+                         void* stream) {
+  paro::Grid g;
+  pa_status st = make_grid(shape, nullptr, false, &g);
+  if (st != PA_OK) return st;
+  PA_REQUIRE(scores && idx, "scores and idx must be non-NULL");
+  PA_REQUIRE(k >= 1 && k <= g.NB, "k=%d must be in [1, NB=%d]", k, g.NB);
+  PA_REQUIRE(g.NB <= 16384, "NB=%d exceeds 16384 (row keys must fit in shared memory)", g.NB);
+  return cuda_status(paro::launch_topk(scores, g, k, idx, (cudaStream_t)stream),
+                     "pa_select_topk launch");
+}
+
+pa_status pa_compact_mask(const uint32_t* bitmask, pa_shape shape, int32_t* idx, int32_t* counts,
+                          void* stream) {
+  paro::Grid g;
+  pa_status st = make_grid(shape, nullptr, false, &g);
+  if (st != PA_OK) return st;
+  PA_REQUIRE(bitmask && idx && counts, "bitmask, idx and counts must be non-NULL");
+  return cuda_status(paro::launch_compact(bitmask, g, idx, counts, (cudaStream_t)stream),
+                     "pa_compact_mask launch");
+}
+
+pa_status pa_quantize_int8(const void* x, pa_dtype dtype, pa_shape shape, const int8_t* perms,
+                           int8_t* x_q, float* scales, float* pool, void* stream) {
+  paro::Grid g;
+  pa_status st = check_float_dtype(dtype);
+  if (st != PA_OK) return st;
+  if ((st = make_grid(shape, perms, true, &g)) != PA_OK) return st;
+  PA_REQUIRE(x && x_q && scales, "x, x_q and scales must be non-NULL");
+  PA_REQUIRE(aligned16(x) && aligned16(x_q), "x and x_q must be 16-byte aligned");
+  return cuda_status(paro::launch_quantize(x, dtype, g, x_q, scales, pool, (cudaStream_t)stream),
+                     "pa_quantize_int8 launch");
+}
+
+static pa_status attn_common(const void* q, const void* k, const void* v, pa_dtype dtype,
+                             pa_shape shape, const int8_t* perms, const int32_t* idx,
+                             const int32_t* counts, int32_t k_max, const float* q_scale,
+                             const float* k_scale, const float* v_scale, void* out,
+                             int32_t* dev_status, void* stream, bool force_mma) {
+  paro::Grid g;
+  pa_status st = make_grid(shape, perms, true, &g);
+  if (st != PA_OK) return st;
+  PA_REQUIRE(dtype == PA_F32 || dtype == PA_BF16 || dtype == PA_I8, "dtype %d unknown", (int)dtype);
+  PA_REQUIRE(q && k && v && out && idx, "q, k, v, idx and out must be non-NULL");
+  PA_REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out),
+             "q, k, v and out must be 16-byte aligned");
+  PA_REQUIRE(k_max >= 0 && k_max <= g.NB, "k_max=%d must be in [0, NB=%d]", k_max, g.NB);
+  if (dtype == PA_I8) {
+    PA_REQUIRE(q_scale && k_scale && v_scale, "INT8 attention needs q_scale, k_scale, v_scale");
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  const bool sm100 = !force_mma && paro::attn_sm100_supports(dtype, g);
+  if (dtype == PA_I8 && !sm100)
+    return fail(PA_ERR_UNSUPPORTED, "INT8 attention needs d=128, block=128 (tcgen05 kernel)");
+  if (k_max == 0) {
+    // every row has no kept block: the output is all zeros
+    const size_t es = dtype == PA_F32 ? 4 : 2;
+    return cuda_status(cudaMemsetAsync(out, 0, (size_t)g.B * g.heads * g.N * g.d * es, s),
+                       "pa_block_sparse_attn memset");
+  }
+  cudaError_t e;
+  if (sm100)
+    e = paro::launch_attn_sm100(q, k, v, dtype, g, idx, counts, k_max, q_scale, k_scale, v_scale,
+                                out, dev_status, s);
+  else
+    e = paro::launch_attn_mma(q, k, v, dtype, g, idx, counts, k_max, out, dev_status, s);
+  return cuda_status(e, "pa_block_sparse_attn launch");
+}
+
+pa_status pa_block_sparse_attn(const void* q, const void* k, const void* v, pa_dtype dtype,
+                               pa_shape shape, const int8_t* perms, const int32_t* idx,
+                               const int32_t* counts, int32_t k_max, const float* q_scale,
+                               const float* k_scale, const float* v_scale, void* out,
+                               int32_t* dev_status, void* stream) {
+  return attn_common(q, k, v, dtype, shape, perms, idx, counts, k_max, q_scale, k_scale, v_scale,
+                     out, dev_status, stream, false);
+}
+
+pa_status pa_block_sparse_attn_mma(const void* q, const void* k, const void* v, pa_dtype dtype,
+                                   pa_shape shape, const int8_t* perms, const int32_t* idx,
+                                   const int32_t* counts, int32_t k_max, void* out,
+                                   int32_t* dev_status, void* stream) {
+  PA_REQUIRE(dtype != PA_I8, "the mma.sync baseline takes PA_F32 or PA_BF16");
+  return attn_common(q, k, v, dtype, shape, perms, idx, counts, k_max, nullptr, nullptr, nullptr,
+                     out, dev_status, stream, true);
+}
+
+}  // extern "C"

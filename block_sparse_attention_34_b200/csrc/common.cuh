@@ -1,0 +1,99 @@
+// Shared device-side definitions of libparo: the grid/order description every
+// kernel receives by value, the position -> natural-token map of a head's
+// axis order, and the device status word.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "paro.h"
+
+namespace paro {
+
+constexpr int kMaxHeads = 1024;
+
+// Sizes of one call plus the per-order index tables.  For order o (letters
+// outer -> inner, PAROAttention review: the six orders of [F, H, W]) a
+// permuted position p decomposes as p = (c_out * mid[o] + c_mid) * inn[o] +
+// c_in, and the token's natural index is c_out*so[o] + c_mid*sm[o] +
+// c_in*si[o] (natural strides: F -> H*W, H -> W, W -> 1).
+struct Grid {
+  int32_t B, heads, F, H, W, d, block;
+  int32_t N, NB, Np;
+  int32_t mid[6], inn[6], so[6], sm[6], si[6];
+  int8_t perm[kMaxHeads];
+};
+
+__device__ __forceinline__ int natural_index(const Grid& g, int order, int p) {
+  const int inn = g.inn[order], mid = g.mid[order];
+  const int ci = p % inn;
+  const int t = p / inn;
+  const int cm = t % mid;
+  const int co = t / mid;
+  return co * g.so[order] + cm * g.sm[order] + ci * g.si[order];
+}
+
+// First error wins; never traps.
+__device__ __forceinline__ void report(int32_t* status, int code) {
+  if (status != nullptr) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ float to_float(float x) { return x; }
+__device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_float(float x);
+template <>
+__device__ __forceinline__ float from_float<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_float<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Unpack a 16-byte chunk of T into floats (8 bf16 or 4 f32).
+template <typename T>
+struct Chunk;
+template <>
+struct Chunk<__nv_bfloat16> {
+  static constexpr int n = 8;
+  __device__ static void unpack(const uint4& u, float* f) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 t = __bfloat1622float2(h[i]);
+      f[2 * i] = t.x;
+      f[2 * i + 1] = t.y;
+    }
+  }
+};
+template <>
+struct Chunk<float> {
+  static constexpr int n = 4;
+  __device__ static void unpack(const uint4& u, float* f) {
+    f[0] = __uint_as_float(u.x);
+    f[1] = __uint_as_float(u.y);
+    f[2] = __uint_as_float(u.z);
+    f[3] = __uint_as_float(u.w);
+  }
+};
+
+}  // namespace paro
+
+// Launchers implemented in the kernel files, called by the C ABI layer.
+// Each returns cudaGetLastError() of its launch.
+namespace paro {
+cudaError_t launch_reorder(const void* x, void* xp, pa_dtype dt, const Grid& g, bool inverse,
+                           cudaStream_t s);
+cudaError_t launch_pool(const void* x, pa_dtype dt, const Grid& g, float* pool, cudaStream_t s);
+cudaError_t launch_score(const float* qp, const float* kp, const Grid& g, float* scores,
+                         cudaStream_t s);
+cudaError_t launch_topk(const float* scores, const Grid& g, int k, int32_t* idx, cudaStream_t s);
+cudaError_t launch_compact(const uint32_t* bm, const Grid& g, int32_t* idx, int32_t* counts,
+                           cudaStream_t s);
+cudaError_t launch_quantize(const void* x, pa_dtype dt, const Grid& g, int8_t* xq, float* scales,
+                            float* pool, cudaStream_t s);
+cudaError_t launch_attn_mma(const void* q, const void* k, const void* v, pa_dtype dt,
+                            const Grid& g, const int32_t* idx, const int32_t* counts, int k_max,
+                            void* out, int32_t* status, cudaStream_t s);
+}  // namespace paro

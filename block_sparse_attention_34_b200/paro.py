@@ -1,0 +1,239 @@
+"""Thin Python binding of libparo (include/paro.h).
+
+Argument marshalling only: every step runs in the library's CUDA kernels on
+the caller's current torch stream.  Torch supplies device memory and
+streams.  There is no CPU fallback: if the library is missing or a call
+fails, an exception is raised.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libparo.so")
+
+PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_TIMEOUT, PA_ERR_DEVICE_CHECK = range(6)
+PA_F32, PA_BF16, PA_I8 = 0, 1, 2
+STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_CUDA",
+                4: "PA_ERR_TIMEOUT", 5: "PA_ERR_DEVICE_CHECK"}
+ORDER_IDS = {"FHW": 0, "FWH": 1, "HFW": 2, "HWF": 3, "WFH": 4, "WHF": 5}
+
+
+class PaShape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "heads", "F", "H", "W", "d", "block")]
+
+
+class ParoError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+
+
+def load():
+    """Load libparo.so (built by ``python -m block_sparse_attention_34_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m block_sparse_attention_34_b200.build` (needs nvcc)")
+    lib = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "pa_abi_version": ([], _I),
+        "pa_last_error": ([], ctypes.c_char_p),
+        "pa_num_blocks": ([PaShape], _I),
+        "pa_k_for_density": ([_I, ctypes.c_double], _I),
+        "pa_reorder": ([_P, _P, _I, PaShape, _P, _P], _I),
+        "pa_inverse_reorder": ([_P, _P, _I, PaShape, _P, _P], _I),
+        "pa_block_score": ([_P, _P, _I, PaShape, _P, _P, _P, _P, _P], _I),
+        "pa_score_pooled": ([_P, _P, PaShape, _P, _P], _I),
+        "pa_select_topk": ([_P, PaShape, _I, _P, _P], _I),
+        "pa_compact_mask": ([_P, PaShape, _P, _P, _P], _I),
+        "pa_quantize_int8": ([_P, _I, PaShape, _P, _P, _P, _P, _P], _I),
+        "pa_block_sparse_attn": ([_P, _P, _P, _I, PaShape, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P], _I),
+        "pa_block_sparse_attn_mma": ([_P, _P, _P, _I, PaShape, _P, _P, _P, _I, _P, _P, _P], _I),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = lib
+    return lib
+
+
+def _check(status: int):
+    if status != PA_OK:
+        raise ParoError(status, load().pa_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return PA_F32
+    if t.dtype == torch.bfloat16:
+        return PA_BF16
+    if t.dtype == torch.int8:
+        return PA_I8
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("tensors must be on a CUDA device (no CPU path)")
+            if not t.is_contiguous():
+                raise ValueError("tensors must be contiguous")
+
+
+class Problem:
+    """Sizes of one attention call plus the per-head order ids."""
+
+    def __init__(self, B, heads, grid, d, block, perms):
+        self.B, self.heads, self.d, self.block = int(B), int(heads), int(d), int(block)
+        self.F, self.H, self.W = (int(x) for x in grid)
+        self.N = self.F * self.H * self.W
+        self.NB = -(-self.N // self.block)
+        self.N_p = self.NB * self.block
+        p = np.asarray(perms, dtype=np.int8)
+        if p.shape != (self.heads,):
+            raise ValueError(f"perms must have one order id per head ({self.heads})")
+        self._perms = np.ascontiguousarray(p)
+        self.shape = PaShape(self.B, self.heads, self.F, self.H, self.W, self.d, self.block)
+
+    @property
+    def perms_ptr(self):
+        return self._perms.ctypes.data_as(ctypes.c_void_p)
+
+    @classmethod
+    def from_qkv(cls, q, grid, perms, block):
+        B, h, N, d = q.shape
+        return cls(B, h, grid, d, block, perms)
+
+
+def k_for_density(nb: int, density: float) -> int:
+    return int(load().pa_k_for_density(int(nb), float(density)))
+
+
+def reorder(x, pr: Problem, out=None):
+    _need_cuda(x)
+    out = out if out is not None else torch.empty((pr.B, pr.heads, pr.N_p, pr.d), dtype=x.dtype,
+                                                  device=x.device)
+    _check(load().pa_reorder(_ptr(x), _ptr(out), _dtype_code(x), pr.shape, pr.perms_ptr, _stream()))
+    return out
+
+
+def inverse_reorder(xp, pr: Problem, out=None):
+    _need_cuda(xp)
+    out = out if out is not None else torch.empty((pr.B, pr.heads, pr.N, pr.d), dtype=xp.dtype,
+                                                  device=xp.device)
+    _check(load().pa_inverse_reorder(_ptr(xp), _ptr(out), _dtype_code(xp), pr.shape, pr.perms_ptr,
+                                     _stream()))
+    return out
+
+
+def block_score(q, k, pr: Problem, q_pool=None, k_pool=None, scores=None):
+    _need_cuda(q, k)
+    dev = q.device
+    q_pool = q_pool if q_pool is not None else torch.empty((pr.B, pr.heads, pr.NB, pr.d), dtype=torch.float32, device=dev)
+    k_pool = k_pool if k_pool is not None else torch.empty_like(q_pool)
+    scores = scores if scores is not None else torch.empty((pr.B, pr.heads, pr.NB, pr.NB), dtype=torch.float32, device=dev)
+    _check(load().pa_block_score(_ptr(q), _ptr(k), _dtype_code(q), pr.shape, pr.perms_ptr,
+                                 _ptr(q_pool), _ptr(k_pool), _ptr(scores), _stream()))
+    return q_pool, k_pool, scores
+
+
+def score_pooled(q_pool, k_pool, pr: Problem, scores=None):
+    _need_cuda(q_pool, k_pool)
+    scores = scores if scores is not None else torch.empty((pr.B, pr.heads, pr.NB, pr.NB), dtype=torch.float32, device=q_pool.device)
+    _check(load().pa_score_pooled(_ptr(q_pool), _ptr(k_pool), pr.shape, _ptr(scores), _stream()))
+    return scores
+
+
+def select_topk(scores, pr: Problem, k: int, idx=None):
+    _need_cuda(scores)
+    idx = idx if idx is not None else torch.empty((pr.B, pr.heads, pr.NB, k), dtype=torch.int32, device=scores.device)
+    _check(load().pa_select_topk(_ptr(scores), pr.shape, int(k), _ptr(idx), _stream()))
+    return idx
+
+
+def compact_mask(bitmask, pr: Problem, idx=None, counts=None):
+    _need_cuda(bitmask)
+    dev = bitmask.device
+    idx = idx if idx is not None else torch.empty((pr.B, pr.heads, pr.NB, pr.NB), dtype=torch.int32, device=dev)
+    counts = counts if counts is not None else torch.empty((pr.B, pr.heads, pr.NB), dtype=torch.int32, device=dev)
+    _check(load().pa_compact_mask(_ptr(bitmask), pr.shape, _ptr(idx), _ptr(counts), _stream()))
+    return idx, counts
+
+
+def quantize_int8(x, pr: Problem, with_pool=False, x_q=None, scales=None, pool=None):
+    _need_cuda(x)
+    dev = x.device
+    x_q = x_q if x_q is not None else torch.empty((pr.B, pr.heads, pr.N_p, pr.d), dtype=torch.int8, device=dev)
+    scales = scales if scales is not None else torch.empty((pr.B, pr.heads, pr.NB), dtype=torch.float32, device=dev)
+    if with_pool and pool is None:
+        pool = torch.empty((pr.B, pr.heads, pr.NB, pr.d), dtype=torch.float32, device=dev)
+    _check(load().pa_quantize_int8(_ptr(x), _dtype_code(x), pr.shape, pr.perms_ptr, _ptr(x_q),
+                                   _ptr(scales), _ptr(pool), _stream()))
+    return (x_q, scales, pool) if with_pool else (x_q, scales)
+
+
+def block_sparse_attn(q, k, v, pr: Problem, idx, counts=None, scales=None, out=None,
+                      status=None, baseline=False):
+    """O = block-sparse attention over the kept tiles, natural token order.
+
+    ``scales`` = (q_scale, k_scale, v_scale) for int8 q/k/v from
+    :func:`quantize_int8` (output bf16).  ``baseline=True`` runs the
+    mma.sync comparison kernel instead of the tcgen05 one."""
+    _need_cuda(q, k, v, idx, counts)
+    code = _dtype_code(q)
+    out_dtype = torch.bfloat16 if code == PA_I8 else q.dtype
+    out = out if out is not None else torch.empty((pr.B, pr.heads, pr.N, pr.d), dtype=out_dtype, device=q.device)
+    k_max = int(idx.shape[-1])
+    lib = load()
+    if baseline:
+        st = lib.pa_block_sparse_attn_mma(_ptr(q), _ptr(k), _ptr(v), code, pr.shape, pr.perms_ptr,
+                                          _ptr(idx), _ptr(counts), k_max, _ptr(out), _ptr(status),
+                                          _stream())
+    else:
+        qs, ks, vs = scales if scales is not None else (None, None, None)
+        st = lib.pa_block_sparse_attn(_ptr(q), _ptr(k), _ptr(v), code, pr.shape, pr.perms_ptr,
+                                      _ptr(idx), _ptr(counts), k_max, _ptr(qs), _ptr(ks), _ptr(vs),
+                                      _ptr(out), _ptr(status), _stream())
+    _check(st)
+    return out
+
+
+def attention(q, k, v, grid, perms, block, density, int8=False, baseline=False):
+    """The whole path for one call: pooled block scores -> top-k kept
+    blocks -> block-sparse attention (orders applied inside the kernels).
+    Returns (out, idx)."""
+    pr = Problem.from_qkv(q, grid, perms, block)
+    kk = k_for_density(pr.NB, density)
+    if int8:
+        q8, qs, qp = quantize_int8(q, pr, with_pool=True)
+        k8, ks, kp = quantize_int8(k, pr, with_pool=True)
+        v8, vs = quantize_int8(v, pr)
+        scores = score_pooled(qp, kp, pr)
+        idx = select_topk(scores, pr, kk)
+        return block_sparse_attn(q8, k8, v8, pr, idx, scales=(qs, ks, vs)), idx
+    _, _, scores = block_score(q, k, pr)
+    idx = select_topk(scores, pr, kk)
+    return block_sparse_attn(q, k, v, pr, idx, baseline=baseline), idx

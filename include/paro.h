@@ -1,0 +1,202 @@
+/*
+ * paro.h -- C ABI of libparo: per-head block-sparse attention over the
+ * F x H x W token grid of a video diffusion transformer, on NVIDIA B200
+ * (sm_100a).
+ *
+ * The path, one attention call:
+ *   1. per-head reorder of the flattened tokens to one of the six axis orders
+ *      of [F, H, W]                  (PAROAttention, arXiv 2506.16054, Pith
+ *                                     verdict page, key_machinery);
+ *   2. mean-pooled Q/K block summaries and block scores
+ *                                    (SPADE, arXiv 2608.03335, Pith verdict
+ *                                     page, key_machinery (iii) and the
+ *                                     referee's note on the MEAN summariser);
+ *   3. top-k key blocks per query block, or a static bitmask
+ *                                    (PASA, arXiv 2604.12219, Figure 2;
+ *                                     PAROAttention review: bitmask masks);
+ *   4. online-softmax attention over the kept (query block, key block) tiles
+ *      only, optionally with INT8 Q/K/V and INT8 P
+ *                                    (SPADE review, key_machinery (iii);
+ *                                     PAROAttention review, key_machinery);
+ *   5. inverse reorder of the output (fused into step 4's store).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - N = F*H*W tokens per head; NB = ceil(N / block) blocks; N_p = NB*block.
+ * - Order ids (one int8 per head, HOST memory, length shape.heads, the same
+ *   for every batch index): 0 FHW, 1 FWH, 2 HFW, 3 HWF, 4 WFH, 5 WHF, the
+ *   letters listing the axes outermost -> innermost.  FHW is the natural
+ *   flattening n = f*H*W + h*W + w.  Token n of a head sits at position
+ *   pos(n) of that head's order; block i holds positions [i*block,
+ *   (i+1)*block); positions >= N are zero padding.
+ * - Q, K, V and the attention output are [B, heads, N, d] row-major in the
+ *   natural order, contiguous, device memory, base 16-byte aligned.
+ *   INT8 tensors and pooled summaries are in the permuted order.
+ * - Every pointer argument except `perms` is DEVICE memory owned by the
+ *   caller; the library allocates no device memory and keeps no pointer
+ *   after a call returns.
+ * - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *   only enqueues work on it and returns; nothing synchronises.
+ * - Supported: d in {64, 128}; block in {64, 128}; 1 <= heads <= 1024;
+ *   B >= 1; F, H, W >= 1; B*heads*N_p*d < 2^40.
+ * - Errors: argument errors return PA_ERR_INVALID_ARG (or
+ *   PA_ERR_UNSUPPORTED for valid but unsupported sizes) before any launch;
+ *   a failed launch returns PA_ERR_CUDA.  pa_last_error() then gives a
+ *   message (thread-local, valid until the next call on the thread).
+ *   Device-side checks (malformed index lists, a bounded wait that ran
+ *   out) write a nonzero pa_status code into *dev_status when dev_status is
+ *   not NULL (first error wins) and skip the offending work; they never
+ *   trap.  Read it after synchronising the stream.
+ */
+#ifndef PARO_H
+#define PARO_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,
+  PA_ERR_UNSUPPORTED = 2,
+  PA_ERR_CUDA = 3,
+  PA_ERR_TIMEOUT = 4,
+  PA_ERR_DEVICE_CHECK = 5
+} pa_status;
+
+typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_I8 = 2 } pa_dtype;
+
+typedef struct {
+  int32_t B, heads, F, H, W, d, block;
+} pa_shape;
+
+/* Version of this ABI (bumped on any signature change). */
+PA_API int32_t pa_abi_version(void);
+
+/* Message of the last failed call on this thread ("" if none). */
+PA_API const char* pa_last_error(void);
+
+/* NB = ceil(F*H*W / block), or -1 for a malformed shape. */
+PA_API int32_t pa_num_blocks(pa_shape shape);
+
+/* Kept key blocks per query block for a density:
+ * ceil(density * nb) clamped to [1, nb], with density*nb rounded to 9
+ * decimals first (so 0.3 * 10 keeps 3, not 4).  Returns 0 for nb <= 0.
+ * (The pages give the density; the rounding rule is this library's.) */
+PA_API int32_t pa_k_for_density(int32_t nb, double density);
+
+/* Step 1 standalone (PAROAttention review, key_machinery: per-head
+ * permutation among the six axis orders).  x [B,heads,N,d] natural ->
+ * x_perm [B,heads,N_p,d] permuted, pad rows written as zeros.
+ * dtype PA_F32 or PA_BF16 (same for both buffers). */
+PA_API pa_status pa_reorder(const void* x, void* x_perm, pa_dtype dtype, pa_shape shape,
+                     const int8_t* perms, void* stream);
+
+/* Step 5 standalone: x_perm [B,heads,N_p,d] permuted -> x [B,heads,N,d]
+ * natural; pad rows are dropped. */
+PA_API pa_status pa_inverse_reorder(const void* x_perm, void* x, pa_dtype dtype, pa_shape shape,
+                             const int8_t* perms, void* stream);
+
+/* Step 2 (SPADE review: MEAN summariser; intra-estimation).  From
+ * natural-order q, k (PA_F32 or PA_BF16):
+ *   q_pool[b,h,i,:] = mean of the valid rows of permuted block i of q (fp32),
+ *   k_pool likewise,
+ *   scores[b,h,i,j] = dot(q_pool[b,h,i,:], k_pool[b,h,j,:]) / sqrt(d) (fp32).
+ * q_pool, k_pool [B,heads,NB,d] float and scores [B,heads,NB,NB] float are
+ * all outputs and required. */
+PA_API pa_status pa_block_score(const void* q, const void* k, pa_dtype dtype, pa_shape shape,
+                         const int8_t* perms, float* q_pool, float* k_pool, float* scores,
+                         void* stream);
+
+/* The score half of pa_block_score alone, from pooled summaries already in
+ * memory (e.g. the `pool` outputs of pa_quantize_int8):
+ *   scores[b,h,i,j] = dot(q_pool[b,h,i,:], k_pool[b,h,j,:]) / sqrt(d). */
+PA_API pa_status pa_score_pooled(const float* q_pool, const float* k_pool, pa_shape shape,
+                          float* scores, void* stream);
+
+/* Step 3, online (PASA review, Figure 2: at most k key blocks per query
+ * block; SPADE review: Top-K filter).  Row (b,h,i) of scores
+ * [B,heads,NB,NB] -> idx[b,h,i,0..k-1] (int32, ascending): block i itself,
+ * then the k-1 largest other scores, ties to the lower block index, NaN
+ * read as -inf, -0.0 equal to +0.0.  1 <= k <= NB. */
+PA_API pa_status pa_select_topk(const float* scores, pa_shape shape, int32_t k, int32_t* idx,
+                         void* stream);
+
+/* Step 3, static (PAROAttention review, key_machinery: static masks stored
+ * as bitmasks).  bitmask [B,heads,NB,ceil(NB/32)] uint32, bit (j % 32) of
+ * word (j / 32) set when key block j is kept for query block i ->
+ * idx [B,heads,NB,NB] int32 (kept indices ascending, the rest -1) and
+ * counts [B,heads,NB] int32.  Bits at j >= NB are ignored. */
+PA_API pa_status pa_compact_mask(const uint32_t* bitmask, pa_shape shape, int32_t* idx,
+                          int32_t* counts, void* stream);
+
+/* Per-block symmetric INT8 quantisation in the permuted order
+ * (PAROAttention review, key_machinery: block-wise INT8 aligned to the
+ * attention block).  For permuted block i of x (PA_F32 or PA_BF16,
+ * natural order in):
+ *   absmax = max |x| over the block's valid rows,
+ *   x_q    = clamp(round_half_even(x * fl32(127/absmax)), -127, 127),
+ *   scale  = fl32(absmax / 127)   (0 and all-zero codes when absmax = 0),
+ * all in float32 round-to-nearest.  x_q [B,heads,N_p,d] int8 (pad rows 0),
+ * scales [B,heads,NB] float.  pool, if not NULL, [B,heads,NB,d] float,
+ * receives the block mean of x (as pa_block_score's q_pool) from the same
+ * read. */
+PA_API pa_status pa_quantize_int8(const void* x, pa_dtype dtype, pa_shape shape, const int8_t* perms,
+                           int8_t* x_q, float* scales, float* pool, void* stream);
+
+/* Step 4 + fused step 5 (SPADE review, key_machinery (iii): flash
+ * block-sparse attention with an online softmax; the inverse reorder is
+ * the output store).  For every valid query token n of head (b,h), with
+ * i = pos(n) / block:
+ *   out[b,h,n,:] = sum_c softmax_c(q_n . k_c / sqrt(d)) v_c
+ * over the tokens c whose block is listed in idx row (b,h,i) (the first
+ * counts[b,h,i] entries, or all k when counts is NULL).
+ *
+ * idx [B,heads,NB,k] int32; each used entry in [0, NB), ascending, no
+ * repeats (a malformed row is skipped with PA_ERR_DEVICE_CHECK on
+ * dev_status; its rows of out are left unwritten).  A row whose count is
+ * 0 produces zeros.
+ *
+ * dtype PA_BF16: q, k, v, out bf16, natural order; P rounded to bf16 for
+ *   the P V product, fp32 accumulation.
+ * dtype PA_F32: q, k, v, out float, natural order; the products run in
+ *   bf16 (inputs rounded to bf16 on load), fp32 accumulation.
+ * dtype PA_I8: q, k, v are int8 [B,heads,N_p,d] from pa_quantize_int8
+ *   (permuted) with scales q_scale, k_scale, v_scale [B,heads,NB]; out is
+ *   bf16 natural order.  S = (Q8 K8^T in int32) * q_scale * k_scale /
+ *   sqrt(d); per tile P~ = exp(s - running row max) is quantised to
+ *   round_half_even(127 P~) and P V runs in int8 with int32
+ *   accumulation, scaled by v_scale / 127; the normaliser sums the
+ *   unrounded P~.
+ * q_scale/k_scale/v_scale are ignored (may be NULL) unless dtype is PA_I8. */
+PA_API pa_status pa_block_sparse_attn(const void* q, const void* k, const void* v, pa_dtype dtype,
+                               pa_shape shape, const int8_t* perms, const int32_t* idx,
+                               const int32_t* counts, int32_t k_max, const float* q_scale,
+                               const float* k_scale, const float* v_scale, void* out,
+                               int32_t* dev_status, void* stream);
+
+/* The same computation as pa_block_sparse_attn for dtype PA_F32 or PA_BF16,
+ * on the legacy warp-level tensor-core path (mma.sync m16n8k16, one CTA per
+ * query block, K/V tiles gathered into padded shared memory).  It is the
+ * comparison baseline for the tcgen05 kernel, and it is also what
+ * pa_block_sparse_attn itself runs for the shapes the tcgen05 kernel does
+ * not take (d = 64, block = 64, or PA_F32).  Same arguments, layouts,
+ * ownership and errors as pa_block_sparse_attn, without the INT8 scales. */
+PA_API pa_status pa_block_sparse_attn_mma(const void* q, const void* k, const void* v, pa_dtype dtype,
+                                   pa_shape shape, const int8_t* perms, const int32_t* idx,
+                                   const int32_t* counts, int32_t k_max, void* out,
+                                   int32_t* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PARO_H */

@@ -1,0 +1,107 @@
+"""The C ABI library on the CPU: it loads, exports every function that
+include/paro.h declares, and rejects malformed arguments on the host before
+any CUDA call (so these run without a GPU)."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from block_sparse_attention_34_b200 import paro
+from oracle import paro_ref as ref
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(paro.LIB_PATH):
+        from block_sparse_attention_34_b200 import build
+        build.build()
+    return paro.load()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "paro.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    assert lib.pa_abi_version() == 1
+
+
+def test_k_for_density_matches_oracle(lib):
+    rng = np.random.default_rng(0)
+    for nb in [1, 2, 4, 10, 32, 256, 591, 929, 1000]:
+        for dens in [0.0, 1e-9, 0.1, 0.15, 0.2, 0.25, 0.3, 0.5, 0.7, 1.0, 2.0,
+                     *rng.random(20).tolist()]:
+            assert lib.pa_k_for_density(nb, dens) == ref.k_for_density(nb, dens), (nb, dens)
+    assert lib.pa_k_for_density(0, 0.5) == 0
+
+
+def test_num_blocks(lib):
+    assert lib.pa_num_blocks(paro.PaShape(1, 40, 21, 45, 80, 128, 128)) == 591
+    assert lib.pa_num_blocks(paro.PaShape(1, 24, 33, 45, 80, 128, 128)) == 929
+    assert lib.pa_num_blocks(paro.PaShape(1, 1, 0, 4, 4, 64, 64)) == -1
+
+
+FAKE = ctypes.c_void_p(4096)  # never dereferenced: every case fails validation first
+
+
+def perms_of(*ids):
+    a = np.array(ids, dtype=np.int8)
+    return a, a.ctypes.data_as(ctypes.c_void_p)
+
+
+def test_host_validation(lib):
+    good = paro.PaShape(1, 2, 4, 8, 8, 64, 64)
+    keep, pp = perms_of(0, 5)
+    # unsupported head dim and block
+    assert lib.pa_reorder(FAKE, FAKE, paro.PA_BF16, paro.PaShape(1, 2, 4, 8, 8, 96, 64), pp, None) == paro.PA_ERR_UNSUPPORTED
+    assert lib.pa_reorder(FAKE, FAKE, paro.PA_BF16, paro.PaShape(1, 2, 4, 8, 8, 64, 32), pp, None) == paro.PA_ERR_UNSUPPORTED
+    assert b"block=32" in lib.pa_last_error()
+    # malformed shape
+    assert lib.pa_reorder(FAKE, FAKE, paro.PA_BF16, paro.PaShape(1, 0, 4, 8, 8, 64, 64), pp, None) == paro.PA_ERR_INVALID_ARG
+    # wrong dtype for reorder
+    assert lib.pa_reorder(FAKE, FAKE, paro.PA_I8, good, pp, None) == paro.PA_ERR_INVALID_ARG
+    # bad order id
+    keep2, bad = perms_of(0, 6)
+    assert lib.pa_reorder(FAKE, FAKE, paro.PA_BF16, good, bad, None) == paro.PA_ERR_INVALID_ARG
+    assert b"perms[1]=6" in lib.pa_last_error()
+    # NULL perms / pointers / misaligned pointers
+    assert lib.pa_reorder(FAKE, FAKE, paro.PA_BF16, good, None, None) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_reorder(None, FAKE, paro.PA_BF16, good, pp, None) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_reorder(ctypes.c_void_p(4100), FAKE, paro.PA_BF16, good, pp, None) == paro.PA_ERR_INVALID_ARG
+    # top-k: k out of range
+    assert lib.pa_select_topk(FAKE, good, 0, FAKE, None) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_select_topk(FAKE, good, 5, FAKE, None) == paro.PA_ERR_INVALID_ARG  # NB = 4
+    # attention: INT8 without scales; k_max above NB
+    assert lib.pa_block_sparse_attn(FAKE, FAKE, FAKE, paro.PA_I8, paro.PaShape(1, 2, 4, 8, 8, 128, 128),
+                                    pp, FAKE, None, 1, None, None, None, FAKE, None, None) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_block_sparse_attn(FAKE, FAKE, FAKE, paro.PA_BF16, good, pp, FAKE, None, 9,
+                                    None, None, None, FAKE, None, None) == paro.PA_ERR_INVALID_ARG
+    # INT8 needs the tcgen05 shape
+    assert lib.pa_block_sparse_attn(FAKE, FAKE, FAKE, paro.PA_I8, good, pp, FAKE, None, 2,
+                                    FAKE, FAKE, FAKE, FAKE, None, None) == paro.PA_ERR_UNSUPPORTED
+    # baseline refuses INT8
+    assert lib.pa_block_sparse_attn_mma(FAKE, FAKE, FAKE, paro.PA_I8, good, pp, FAKE, None, 2,
+                                        FAKE, None, None) == paro.PA_ERR_INVALID_ARG
+    # too many heads
+    many = np.zeros(2000, dtype=np.int8)
+    assert lib.pa_reorder(FAKE, FAKE, paro.PA_BF16, paro.PaShape(1, 2000, 4, 8, 8, 64, 64),
+                          many.ctypes.data_as(ctypes.c_void_p), None) == paro.PA_ERR_UNSUPPORTED
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    pr = paro.Problem(1, 2, (4, 8, 8), 64, 64, [0, 5])
+    x = torch.zeros(1, 2, 256, 64)
+    with pytest.raises(ValueError):
+        paro.reorder(x, pr)
