@@ -16,11 +16,14 @@
 //              rescales O in TMEM when its row max grows by more than 2^8,
 //              and runs the epilogue;
 //   warp 4     allocates TMEM; one lane issues every tcgen05.mma and commit;
-//   warps 5-8  gather loaders: each token row of K or V is 256 contiguous
-//              bytes at its natural position, copied with 16-byte cp.async
+//   warps 5-8  gather loaders (Q by all four; then warps 5-6 stream K and
+//              warps 7-8 stream V): each token row is 256 contiguous bytes
+//              at its natural position, copied with 16-byte cp.async
 //              straight into the 128-byte-swizzled operand layout -- the
 //              axis order is applied in the address, so no reordered copy
-//              of any tensor exists in HBM.
+//              of any tensor exists in HBM.  A K stage is refilled as soon
+//              as the QK^T that read it completes, a V stage once its P V
+//              completes, so neither stream waits on the other.
 // Tensor memory (512 columns): S double buffer at columns 0 and 128, O at
 // 256.  Shared memory: Q (32 KB), a two-stage K and V ring (4 x 32 KB), a
 // double-buffered P (2 x 32 KB), all in the canonical K-major / MN-major
@@ -60,7 +63,8 @@ constexpr uint32_t kColS = 0, kColO = 256;
 
 // barrier slots (8 bytes each) after kOffBar
 enum : uint32_t {
-  BQ = 0, BK0 = 1, BV0 = 3, BS0 = 5, BSF0 = 7, BP0 = 9, BPV0 = 11, BDRAIN = 13, NBAR = 14
+  BQ = 0, BK0 = 1, BV0 = 3, BS0 = 5, BSF0 = 7, BP0 = 9, BPV0 = 11, BKF0 = 13, BDRAIN = 15,
+  NBAR = 16
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -196,16 +200,17 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c) {
   return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
 }
 
-// One loader warp copies its 32 rows (rows 32*lw .. 32*lw+31 of the tile)
-// of a [128 x 128] bf16 tile.  nat = natural token index of this lane's row
-// (lane l <-> row 32*lw + l), or -1 for a pad row (zero-filled).
+// One loader warp copies 32 rows (row0 .. row0+31) of a [128 x 128] bf16
+// tile.  nat = natural token index of this lane's row (lane l <-> row
+// row0 + l), or -1 for a pad row (zero-filled).  Each 16-lane half of the
+// warp reads one whole 256-byte row per instruction.
 __device__ __forceinline__ void load_rows(uint32_t tile, const __nv_bfloat16* __restrict__ head,
-                                          int lw, int lane, int nat) {
+                                          int row0, int lane, int nat) {
 #pragma unroll 4
   for (int m = 0; m < 16; ++m) {
     const int src_lane = 2 * m + (lane >> 4);
     const int n = __shfl_sync(0xffffffffu, nat, src_lane);
-    const int r = 32 * lw + src_lane;
+    const int r = row0 + src_lane;
     const int cc = lane & 15;
     const int half = cc >> 3, c = cc & 7;
     const char* src = reinterpret_cast<const char*>(head) +
@@ -241,12 +246,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int32_t* ids = idx + row * k_max;
   const int cnt = counts != nullptr ? __ldg(counts + row) : k_max;
   Ctl ctl{abort_flag, status};
+  // a wait of an earlier CTA of this launch already expired: end quickly
+  const bool expired =
+      status != nullptr && *reinterpret_cast<volatile int32_t*>(status) == PA_ERR_TIMEOUT;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(BQ), kLoadWarps * 32);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(BK0 + s), kLoadWarps * 32);
-      mbar_init(bar(BV0 + s), kLoadWarps * 32);
+      mbar_init(bar(BK0 + s), kLoadWarps * 16);
+      mbar_init(bar(BV0 + s), kLoadWarps * 16);
+      mbar_init(bar(BKF0 + s), 1);
       mbar_init(bar(BS0 + s), 1);
       mbar_init(bar(BSF0 + s), kSoftmaxWarps * 32);
       mbar_init(bar(BP0 + s), kSoftmaxWarps * 32);
@@ -283,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const bool run = *bad_flag == 0;
+  const bool run = *bad_flag == 0 && !expired;
   const int n_tiles = run ? cnt : 0;
 
   const __nv_bfloat16* qh = q + bh * (int64_t)g.N * kD;
@@ -297,34 +306,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         const int p = i * kBlock + 32 * lw + lane;
         const int nat = p < g.N ? natural_index(g, order, p) : -1;
-        load_rows(base + kOffQ, qh, lw, lane, nat);
+        load_rows(base + kOffQ, qh, 32 * lw, lane, nat);
         cp_async_commit();
         cp_async_wait<0>();
         fence_async_smem();
         mbar_arrive(bar(BQ));
       }
+      // warps 5-6 stream K (stage free once QK^T of tile j-2 completed),
+      // warps 7-8 stream V (stage free once P V of tile j-2 completed)
+      const bool is_k = lw < 2;
+      const int half_rows = 64 * (lw & 1);
+      const __nv_bfloat16* src = is_k ? kh : vh;
+      const uint32_t ring = base + (is_k ? kOffK : kOffV);
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j & 1;
-        if (j >= 2 && !warp_wait(bar(BPV0 + s), ((j - 2) >> 1) & 1, ctl)) break;
+        if (j >= 2 && !warp_wait(bar((is_k ? BKF0 : BPV0) + s), ((j - 2) >> 1) & 1, ctl)) break;
         const int kb = __ldg(ids + j);
-        const int p = kb * kBlock + 32 * lw + lane;
-        const int nat = p < g.N ? natural_index(g, order, p) : -1;
-        load_rows(base + kOffK + s * kTile, kh, lw, lane, nat);
-        cp_async_commit();
-        load_rows(base + kOffV + s * kTile, vh, lw, lane, nat);
-        cp_async_commit();
-        if (j >= 1) {
-          cp_async_wait<2>();  // the two groups of tile j-1 are complete
-          fence_async_smem();
-          mbar_arrive(bar(BK0 + ((j - 1) & 1)));
-          mbar_arrive(bar(BV0 + ((j - 1) & 1)));
+#pragma unroll
+        for (int g2 = 0; g2 < 2; ++g2) {
+          const int row0 = half_rows + 32 * g2;
+          const int p = kb * kBlock + row0 + lane;
+          const int nat = p < g.N ? natural_index(g, order, p) : -1;
+          load_rows(ring + s * kTile, src, row0, lane, nat);
         }
-        if (j == n_tiles - 1) {
-          cp_async_wait<0>();
-          fence_async_smem();
-          mbar_arrive(bar(BK0 + s));
-          mbar_arrive(bar(BV0 + s));
-        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        fence_async_smem();
+        mbar_arrive(bar((is_k ? BK0 : BV0) + s));
       }
       cp_async_wait<0>();
     }
@@ -363,6 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      sw128_desc(ka + off, 16, 1024), id_qk, kk > 0 ? 1u : 0u);
         }
         mma_commit(bar(BS0 + b));
+        mma_commit(bar(BKF0 + b));
         if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
       }
       if (ok) issue_pv(n_tiles - 1);

@@ -221,7 +221,7 @@ def block_sparse_attn(q, k, v, pr: Problem, idx, counts=None, scales=None, out=N
     return out
 
 
-def attention(q, k, v, grid, perms, block, density, int8=False, baseline=False):
+def attention(q, k, v, grid, perms, block, density, int8=False, baseline=False, status=None):
     """The whole path for one call: pooled block scores -> top-k kept
     blocks -> block-sparse attention (orders applied inside the kernels).
     Returns (out, idx)."""
@@ -233,7 +233,7 @@ def attention(q, k, v, grid, perms, block, density, int8=False, baseline=False):
         v8, vs = quantize_int8(v, pr)
         scores = score_pooled(qp, kp, pr)
         idx = select_topk(scores, pr, kk)
-        return block_sparse_attn(q8, k8, v8, pr, idx, scales=(qs, ks, vs)), idx
+        return block_sparse_attn(q8, k8, v8, pr, idx, scales=(qs, ks, vs), status=status), idx
     _, _, scores = block_score(q, k, pr)
     idx = select_topk(scores, pr, kk)
-    return block_sparse_attn(q, k, v, pr, idx, baseline=baseline), idx
+    return block_sparse_attn(q, k, v, pr, idx, baseline=baseline, status=status), idx

@@ -46,7 +46,9 @@
  *   Device-side checks (malformed index lists, a bounded wait that ran
  *   out) write a nonzero pa_status code into *dev_status when dev_status is
  *   not NULL (first error wins) and skip the offending work; they never
- *   trap.  Read it after synchronising the stream.
+ *   trap.  Read it after synchronising the stream.  A kernel that finds
+ *   PA_ERR_TIMEOUT already recorded there skips its work, so one expired
+ *   wait ends the launch quickly: reset the word to 0 before reusing it.
  */
 #ifndef PARO_H
 #define PARO_H

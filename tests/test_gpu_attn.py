@@ -53,8 +53,11 @@ def test_topk_pipeline_small(w, baseline):
     q, k, v, perms = inputs(w)
     pr = problem(w, perms)
     qd, kd, vd = to_dev(q, k, v)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
     out, idx = paro.attention(qd, kd, vd, (w.F, w.H, w.W), perms, w.block, w.density,
-                              baseline=baseline)
+                              baseline=baseline, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
     idx_h = idx.cpu().numpy()
     want = ref.attention(as_f64(q), as_f64(k), as_f64(v), (w.F, w.H, w.W), perms, w.block, idx_h)
     compare(out, want)
@@ -127,7 +130,11 @@ def test_480p_two_heads_full():
     q, k, v, perms = inputs(w, heads=2)
     pr = problem(w, perms, heads=2)
     qd, kd, vd = to_dev(q, k, v)
-    out, idx = paro.attention(qd, kd, vd, (w.F, w.H, w.W), perms, w.block, w.density)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, idx = paro.attention(qd, kd, vd, (w.F, w.H, w.W), perms, w.block, w.density,
+                              status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
     want = ref.attention(as_f64(q), as_f64(k), as_f64(v), (w.F, w.H, w.W), perms, w.block,
                          idx.cpu().numpy())
     compare(out, want)
