@@ -20,6 +20,7 @@ float64 CPU oracle on a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -282,7 +283,9 @@ def run_ours(a):
     device = torch.device("cuda", local)
     init_dist(ws, "nccl")
     w = WORKLOADS[a.workload]
-    q, k, v, perms = make_inputs(w)
+    q, k, v, perms = make_inputs(w, heads=a.heads)
+    if a.heads is not None:  # leading heads only (same values as the full draw)
+        w = dataclasses.replace(w, heads=a.heads)
     qd, kd, vd = (t.to(device) for t in (q, k, v))
     pipe = Pipeline(w, qd, kd, vd, perms, a.density if a.density is not None else w.density,
                     baseline=a.kernel == "mma")
@@ -333,7 +336,8 @@ def run_ours(a):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded structured q/k, normal v; no weights)",
             "config": {
-                "workload": w.name, "B": w.B, "heads": w.heads, "grid": [w.F, w.H, w.W],
+                "workload": w.name if a.heads is None else f"{w.name} (first {w.heads} heads)",
+                "B": w.B, "heads": w.heads, "grid": [w.F, w.H, w.W],
                 "N": w.N, "d": w.d, "block": w.block, "density": pipe.k / pipe.pr.NB,
                 "density_requested": a.density if a.density is not None else w.density,
                 "k": pipe.k, "NB": pipe.pr.NB, "kept_tiles": w.kept_tiles(pipe.k),
@@ -398,6 +402,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--density", type=float, default=None)
+    ap.add_argument("--heads", type=int, default=None,
+                    help="run only the leading heads (profiling captures)")
     ap.add_argument("--kernel", choices=["tcgen05", "mma"], default="tcgen05")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
