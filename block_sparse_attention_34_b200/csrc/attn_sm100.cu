@@ -10,14 +10,18 @@
 // row max / row sum softmax, and O += P V_j, then O / l written to the
 // natural positions of the block's tokens.
 //
-// One CTA per (query block, head); 9 warps with fixed roles:
-//   warps 0-3  softmax: thread t owns row t of the 128-row tile, i.e. TMEM
-//              lane t; reads S from TMEM, writes P (bf16) to shared memory,
-//              rescales O in TMEM when its row max grows by more than 2^8,
-//              and runs the epilogue;
-//   warp 4     allocates TMEM; one lane issues every tcgen05.mma and commit;
-//   warps 5-8  gather loaders (Q by all four; then warps 5-6 stream K and
-//              warps 7-8 stream V): each token row is 256 contiguous bytes
+// One CTA per (query block, head); 13 warps with fixed roles:
+//   warps 0-7  softmax, two warpgroups splitting every tile by columns:
+//              warp w owns rows 32*(w%4) .. +31 (TMEM lanes; a warp may only
+//              touch its lane quarter) and key columns 64*(w/4) .. +63.  Each
+//              thread reads its 64 scores from TMEM, the two halves of a row
+//              exchange their maxima through shared memory, then each thread
+//              writes its 64 bf16 probabilities into its half of the P tile
+//              and, when the row max grew by more than 2^8, rescales its 64
+//              columns of O in TMEM; the epilogue is split the same way;
+//   warp 8     allocates TMEM; one lane issues every tcgen05.mma and commit;
+//   warps 9-12 gather loaders (Q by all four; then warps 9-10 stream K and
+//              warps 11-12 stream V): each token row is 256 contiguous bytes
 //              at its natural position, copied with 16-byte cp.async
 //              straight into the 128-byte-swizzled operand layout -- the
 //              axis order is applied in the address, so no reordered copy
@@ -27,7 +31,8 @@
 // Tensor memory (512 columns): S double buffer at columns 0 and 128, O at
 // 256.  Shared memory: Q (32 KB), a two-stage K and V ring (4 x 32 KB), a
 // double-buffered P (2 x 32 KB), all in the canonical K-major / MN-major
-// SWIZZLE_128B layouts the MMA descriptors name.
+// SWIZZLE_128B layouts the MMA descriptors name, after a small region of
+// mbarriers and the row-max exchange buffer.
 //
 // The MMA warp runs one step ahead: QK^T of tile j is issued before P V of
 // tile j-1, so the tensor core works on S_j while the softmax warps turn
@@ -43,29 +48,36 @@ namespace {
 
 constexpr int kBlock = 128;
 constexpr int kD = 128;
-constexpr int kSoftmaxWarps = 4;
-constexpr int kMmaWarp = 4;
-constexpr int kLoadWarp0 = 5;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp0 = 9;
 constexpr int kLoadWarps = 4;
-constexpr int kThreads = (kSoftmaxWarps + 1 + kLoadWarps) * 32;  // 288
+constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;                // 256
+constexpr int kThreads = (kSoftmaxWarps + 1 + kLoadWarps) * 32;  // 416
 constexpr uint32_t kTile = kBlock * kD * 2;                       // 32 KB
 constexpr uint32_t kHalf = kBlock * 128;                          // 16 KB: 64 columns
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kTile;          // 2 stages
-constexpr uint32_t kOffV = 3 * kTile;      // 2 stages
-constexpr uint32_t kOffP = 5 * kTile;      // 2 buffers
-constexpr uint32_t kOffBar = 7 * kTile;    // mbarriers and flags
-constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
+// small region first: mbarriers (19 x 8 B), TMEM slot and flags (16 B),
+// row-max exchange [2 tiles][2 halves][128 rows] float (2 KB)
+constexpr uint32_t kOffBar = 0;
+constexpr uint32_t kOffSlot = 192;
+constexpr uint32_t kOffXmax = 256;
+constexpr uint32_t kSmall = 3072;  // operand tiles start 1024-aligned after it
+constexpr uint32_t kOffQ = kSmall;
+constexpr uint32_t kOffK = kOffQ + kTile;      // 2 stages
+constexpr uint32_t kOffV = kOffK + 2 * kTile;  // 2 stages
+constexpr uint32_t kOffP = kOffV + 2 * kTile;  // 2 buffers
+constexpr uint32_t kSmemBytes = kOffP + 2 * kTile;  // 232,448 B = 227 KB
 constexpr uint64_t kTimeoutNs = 1000000000ull;
 constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold (factor 256)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;
 
-// barrier slots (8 bytes each) after kOffBar
+// barrier slots
 enum : uint32_t {
-  BQ = 0, BK0 = 1, BV0 = 3, BS0 = 5, BSF0 = 7, BP0 = 9, BPV0 = 11, BKF0 = 13, BDRAIN = 15,
-  NBAR = 16
+  BQ = 0, BK0 = 1, BV0 = 3, BS0 = 5, BSF0 = 7, BP0 = 9, BPV0 = 11, BKF0 = 13, BX0 = 15,
+  BDRAIN = 17, BL = 18, NBAR = 19
 };
+static_assert(NBAR * 8 <= kOffSlot, "barrier region");
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -102,7 +114,7 @@ struct Ctl {
 };
 
 // Bounded wait on one phase of an mbarrier (one thread).
-__device__ __noinline__ bool wait_phase(uint32_t bar, uint32_t parity, Ctl c) {
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, Ctl c) {
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
@@ -123,6 +135,13 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, Ctl c) 
   int ok = 0;
   if ((threadIdx.x & 31) == 0) ok = wait_phase(bar, parity, c) ? 1 : 0;
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Bounded wait by every lane (each acquires the data published before the
+// phase completed); the outcome is made warp-uniform.
+__device__ __forceinline__ bool all_wait(uint32_t bar, uint32_t parity, Ctl c) {
+  const bool ok = wait_phase(bar, parity, c);
+  return __all_sync(0xffffffffu, ok);
 }
 
 // --- tcgen05 -------------------------------------------------------------
@@ -226,15 +245,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                       int k_max, float scale_log2, __nv_bfloat16* __restrict__ out,
                       int32_t* __restrict__ status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  // 1024-byte alignment of the operand tiles (the swizzle pattern repeats
-  // every 8 rows of 128 bytes)
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  unsigned char* gbase = smem_raw + (base - raw);
+  // the operand tiles need 1024-byte alignment (the swizzle pattern repeats
+  // every 8 rows of 128 bytes); dynamic shared memory starts at the window
+  // base when, as here, there is no static shared memory
+  const uint32_t base = smem_u32(smem_raw);
+  if ((base & 1023u) != 0) {
+    if (threadIdx.x == 0) report(status, PA_ERR_UNSUPPORTED);
+    return;
+  }
+  unsigned char* gbase = smem_raw;
   const uint32_t bars = base + kOffBar;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOffBar + NBAR * 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOffSlot);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile uint32_t* bad_flag = tmem_slot + 2;
+  float* xmax = reinterpret_cast<float*>(gbase + kOffXmax);
   auto bar = [&](uint32_t slot) { return bars + slot * 8u; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -257,11 +281,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(BV0 + s), kLoadWarps * 16);
       mbar_init(bar(BKF0 + s), 1);
       mbar_init(bar(BS0 + s), 1);
-      mbar_init(bar(BSF0 + s), kSoftmaxWarps * 32);
-      mbar_init(bar(BP0 + s), kSoftmaxWarps * 32);
+      mbar_init(bar(BSF0 + s), kSoftmaxThreads);
+      mbar_init(bar(BP0 + s), kSoftmaxThreads);
       mbar_init(bar(BPV0 + s), 1);
+      mbar_init(bar(BX0 + s), kSoftmaxThreads);
     }
     mbar_init(bar(BDRAIN), 1);
+    mbar_init(bar(BL), kSoftmaxThreads);
     *abort_flag = 0;
     *bad_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -381,28 +407,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------ softmax ----
-    const int r = threadIdx.x;  // tile row == TMEM lane
-    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const int quarter = warp & 3, hc = warp >> 2;
+    const int r = quarter * 32 + lane;  // tile row == TMEM lane
+    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       const int b = j & 1;
       if (!warp_wait(bar(BS0 + b), (j >> 1) & 1, ctl)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[128];
-      tmem_ld128(lane_addr + kColS + b * 128, sr);
+      uint32_t sr[64];
+      tmem_ld64(lane_addr + kColS + b * 128 + hc * 64, sr);
       tc_fence_before();
       mbar_arrive(bar(BSF0 + b));
       const int kb = __ldg(ids + j);
-      const int valid = g.N - kb * kBlock;  // keys of this block that exist
-      float mx = -INFINITY;
+      const int valid = g.N - kb * kBlock - hc * 64;  // existing keys in my half
+      if (valid < 64) {  // only the ragged last block (warp-uniform)
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        float s = __uint_as_float(sr[c]) * scale_log2;
-        s = c < valid ? s : -INFINITY;
-        sr[c] = __float_as_uint(s);
-        mx = fmaxf(mx, s);
+        for (int c = 0; c < 64; ++c)
+          if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
       }
+      // raw row max of my half (8 independent chains), exchanged with the
+      // other half of the row
+      float mp[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mp[u] = __uint_as_float(sr[u]);
+#pragma unroll
+      for (int c = 8; c < 64; ++c) mp[c & 7] = fmaxf(mp[c & 7], __uint_as_float(sr[c]));
+      const float mh = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+      float* xm = xmax + b * 256;
+      xm[hc * 128 + r] = mh;
+      mbar_arrive(bar(BX0 + b));
+      if (!all_wait(bar(BX0 + b), (j >> 1) & 1, ctl)) { ok = false; break; }
+      const float mx = fmaxf(mh, xm[(hc ^ 1) * 128 + r]) * scale_log2;
       // lazy rescale: keep the reference max unless the row max grew by
       // more than 2^8 (exact either way: O and l share the reference)
       const bool need = j == 0 ? false : (mx > m_used + kRescaleLog2);
@@ -412,59 +450,69 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const float alpha = need ? ex2(m_used - mx) : 1.f;
 #pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 32) {
+        for (int c0 = 0; c0 < 64; c0 += 32) {
           uint32_t orr[32];
-          tmem_ld32(lane_addr + kColO + c0, orr);
+          tmem_ld32(lane_addr + kColO + hc * 64 + c0, orr);
 #pragma unroll
           for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
-          tmem_st32(lane_addr + kColO + c0, orr);
+          tmem_st32(lane_addr + kColO + hc * 64 + c0, orr);
         }
         l *= alpha;
         if (need) m_used = mx;
       }
       if (j >= 2 && !warp_wait(bar(BPV0 + b), ((j - 2) >> 1) & 1, ctl)) { ok = false; break; }
-      // P = 2^(s - m), row sum, bf16 into the swizzled K-major P tile
-      unsigned char* pt = gbase + kOffP + b * kTile;
-      float rs = 0.f;
+      // P = 2^(s*scale - m) in bf16 into my half of the swizzled K-major P
+      // tile; row sum in 8 independent chains
+      unsigned char* pt = gbase + kOffP + b * kTile + hc * kHalf;
+      const float neg_m = -m_used;
+      float rs[8];
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
+      for (int u = 0; u < 8; ++u) rs[u] = 0.f;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          float e[8];
+      for (int c = 0; c < 8; ++c) {
+        float e[8];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            e[u] = ex2(__uint_as_float(sr[hf * 64 + c * 8 + u]) - m_used);
-            rs += e[u];
-          }
-          uint4 w;
-          w.x = pack_bf16(e[0], e[1]);
-          w.y = pack_bf16(e[2], e[3]);
-          w.z = pack_bf16(e[4], e[5]);
-          w.w = pack_bf16(e[6], e[7]);
-          *reinterpret_cast<uint4*>(pt + hf * kHalf + sw128_off(r, c)) = w;
+        for (int u = 0; u < 8; ++u) {
+          e[u] = ex2(fmaf(__uint_as_float(sr[c * 8 + u]), scale_log2, neg_m));
+          rs[u] += e[u];
         }
+        uint4 w;
+        w.x = pack_bf16(e[0], e[1]);
+        w.y = pack_bf16(e[2], e[3]);
+        w.z = pack_bf16(e[4], e[5]);
+        w.w = pack_bf16(e[6], e[7]);
+        *reinterpret_cast<uint4*>(pt + sw128_off(r, c)) = w;
       }
-      l += rs;
+      l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(bar(BP0 + b));
     }
-    // epilogue: O / l at the natural positions of the block's tokens
+    // epilogue: the two halves add their row sums, then each writes O / l
+    // for its 64 columns at the natural position of the row's token
     const int p = i * kBlock + r;
     __nv_bfloat16* orow = p < g.N ? out + (bh * (int64_t)g.N + natural_index(g, order, p)) * kD
                                   : nullptr;
     if (run && cnt == 0) {
       if (orow != nullptr)
-        for (int c = 0; c < 16; ++c) reinterpret_cast<uint4*>(orow)[c] = make_uint4(0, 0, 0, 0);
+        for (int c = 0; c < 8; ++c)
+          reinterpret_cast<uint4*>(orow + hc * 64)[c] = make_uint4(0, 0, 0, 0);
     } else if (ok && n_tiles > 0) {
       const int jl = n_tiles - 1;
-      if (warp_wait(bar(BPV0 + (jl & 1)), (jl >> 1) & 1, ctl)) {
+      // the exchange buffer the last tile did not use: its previous reads
+      // (tile jl-1) finished before every thread arrived for tile jl
+      float* xl = xmax + ((jl & 1) ^ 1) * 256;
+      xl[hc * 128 + r] = l;
+      mbar_arrive(bar(BL));
+      const bool okl = all_wait(bar(BL), 0, ctl);
+      const float lt = okl ? l + xl[(hc ^ 1) * 128 + r] : 0.f;
+      if (okl && warp_wait(bar(BPV0 + (jl & 1)), (jl >> 1) & 1, ctl)) {
         tc_fence_after();
-        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
 #pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 32) {
+        for (int c0 = 0; c0 < 64; c0 += 32) {
           uint32_t orr[32];
-          tmem_ld32(lane_addr + kColO + c0, orr);
+          tmem_ld32(lane_addr + kColO + hc * 64 + c0, orr);
           if (orow != nullptr) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -474,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               w.y = pack_bf16(f[2] * inv, f[3] * inv);
               w.z = pack_bf16(f[4] * inv, f[5] * inv);
               w.w = pack_bf16(f[6] * inv, f[7] * inv);
-              reinterpret_cast<uint4*>(orow + c0)[c] = w;
+              reinterpret_cast<uint4*>(orow + hc * 64 + c0)[c] = w;
             }
           }
         }
