@@ -6,241 +6,123 @@
 // softmax over the kept block pairs; PAROAttention, arXiv 2506.16054, review
 // key_machinery: the per-head axis order of the tokens, fused into the
 // kernel's loads and stores): for query block i of head (b, h) and every key
-// block j of its ascending kept list, S = Q_i K_j^T / sqrt(d), a running
-// row max / row sum softmax, and O += P V_j, then O / l written to the
-// natural positions of the block's tokens.
+// block j of its ascending kept list, S = Q_i K_j^T / sqrt(d), softmax, and
+// O = sum_j P_j V_j / l, written to the natural positions of the block's
+// tokens.
 //
-// One CTA per (query block, head); 13 warps with fixed roles:
-//   warps 0-7  softmax, two warpgroups splitting every tile by columns:
-//              warp w owns rows 32*(w%4) .. +31 (TMEM lanes; a warp may only
-//              touch its lane quarter) and key columns 64*(w/4) .. +63.  Each
-//              thread reads its 64 scores from TMEM, the two halves of a row
-//              exchange their maxima through shared memory, then each thread
-//              writes its 64 bf16 probabilities into its half of the P tile
-//              and, when the row max grew by more than 2^8, rescales its 64
-//              columns of O in TMEM; the epilogue is split the same way;
+// One CTA per (query block, head); 12 warps with fixed roles:
+//   warps 0-3  softmax A: the even-numbered kept tiles (0, 2, 4, ...);
+//   warps 4-7  softmax B: the odd-numbered kept tiles.  A thread owns one
+//              row of the 128-row tile (TMEM lane); each group keeps its own
+//              running max, row sum and O accumulator in TMEM -- an exact
+//              split of the row's kept keys into two disjoint sets -- and
+//              the two partial results are merged once at the end
+//              (O = (O_A 2^(m_A-m) + O_B 2^(m_B-m)) / (l_A 2^(m_A-m) +
+//              l_B 2^(m_B-m))).  The two groups share the SM's sub-cores,
+//              so the exponentials of one overlap the TMEM reads and max of
+//              the other;
 //   warp 8     allocates TMEM; one lane issues every tcgen05.mma and commit;
-//   warps 9-12 gather loaders (Q by all four; then warps 9-10 stream K and
-//              warps 11-12 stream V): each token row is 256 contiguous bytes
-//              at its natural position, copied with 16-byte cp.async
-//              straight into the 128-byte-swizzled operand layout -- the
-//              axis order is applied in the address, so no reordered copy
-//              of any tensor exists in HBM.  A K stage is refilled as soon
-//              as the QK^T that read it completes, a V stage once its P V
-//              completes, so neither stream waits on the other.
-// Tensor memory (512 columns): S double buffer at columns 0 and 128, O at
-// 256.  Shared memory: Q (32 KB), a two-stage K and V ring (4 x 32 KB), a
-// double-buffered P (2 x 32 KB), all in the canonical K-major / MN-major
-// SWIZZLE_128B layouts the MMA descriptors name, after a small region of
-// mbarriers and the row-max exchange buffer.
+//   warp 9     gathers Q and then K tiles, warp 10 gathers V tiles, both with
+//              TMA tile::gather4: lane l computes the natural positions of
+//              rows 4l..4l+3 of the tile from the head's axis order and
+//              issues two 4-row gathers (one per 64-column half) straight
+//              into the 128-byte-swizzled operand layout, so the reorder
+//              costs no pass over HBM;
+//   warp 11    validates the kept list, then idles.
+// Tensor memory (512 columns): S_A, S_B at columns 0 and 128, O_A, O_B at
+// 256 and 384.  Shared memory: Q (32 KB), two-stage K and V rings
+// (4 x 32 KB), P_A and P_B (2 x 32 KB) in the canonical K-major / MN-major
+// SWIZZLE_128B layouts the MMA descriptors name.
 //
-// The MMA warp runs one step ahead: QK^T of tile j is issued before P V of
-// tile j-1, so the tensor core works on S_j while the softmax warps turn
-// S_{j-1} into P_{j-1}.  Every wait on an mbarrier is bounded (about one
-// second of %globaltimer); on expiry the kernel records PA_ERR_TIMEOUT in the
-// device status word, every role leaves its loop, in-flight copies and MMAs
-// are drained and TMEM is released before the CTA exits.
-#include "common.cuh"
-#include "tmem.cuh"
+// MMA issue order: QK(0), QK(1), PV(0), QK(2), PV(1), ... -- a K stage is
+// refilled once the QK^T that read it completes, a V stage once its P V
+// completes.  Every mbarrier wait is bounded (about one second of
+// %globaltimer); on expiry the kernel records PA_ERR_TIMEOUT in the device
+// status word, each role leaves its loop, in-flight TMA loads and MMAs are
+// drained and TMEM is released before the CTA exits.
+#include "sm100.cuh"
 
 namespace paro {
+
+#ifdef PARO_TRACE
+// Phase trace (debug builds only): clock64() of each role's key events for
+// one CTA, event e of tile j at g_paro_trace[e * 128 + j].
+__device__ long long* g_paro_trace = nullptr;
+__device__ int g_paro_trace_cta = 7;
+#define PARO_T(ev, j)                                                                    \
+  do {                                                                                   \
+    if (g_paro_trace != nullptr && blockIdx.x == g_paro_trace_cta && blockIdx.y == 0 &&  \
+        (j) < 128)                                                                       \
+      g_paro_trace[(ev) * 128 + (j)] = clock64();                                        \
+  } while (0)
+#else
+#define PARO_T(ev, j) \
+  do {                \
+  } while (0)
+#endif
+
 namespace {
+
+using namespace sm100;
 
 constexpr int kBlock = 128;
 constexpr int kD = 128;
-constexpr int kSoftmaxWarps = 8;
 constexpr int kMmaWarp = 8;
-constexpr int kLoadWarp0 = 9;
-constexpr int kLoadWarps = 4;
-constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;                // 256
-constexpr int kThreads = (kSoftmaxWarps + 1 + kLoadWarps) * 32;  // 416
-constexpr uint32_t kTile = kBlock * kD * 2;                       // 32 KB
-constexpr uint32_t kHalf = kBlock * 128;                          // 16 KB: 64 columns
-// small region first: mbarriers (19 x 8 B), TMEM slot and flags (16 B),
-// row-max exchange [2 tiles][2 halves][128 rows] float (2 KB)
+constexpr int kKWarp = 9;
+constexpr int kVWarp = 10;
+constexpr int kCheckWarp = 11;
+constexpr int kThreads = 12 * 32;  // 384
+constexpr int kGroupThreads = 128;
+constexpr uint32_t kTile = kBlock * kD * 2;  // 32 KB
+constexpr uint32_t kHalf = kBlock * 128;     // 16 KB: 64 columns
+// small region first: mbarriers, TMEM slot and flags, merge buffers
+// [m, l][group][128 rows] float; the operand tiles start 1024-aligned
 constexpr uint32_t kOffBar = 0;
 constexpr uint32_t kOffSlot = 192;
-constexpr uint32_t kOffXmax = 256;
-constexpr uint32_t kSmall = 3072;  // operand tiles start 1024-aligned after it
+constexpr uint32_t kOffMerge = 256;
+constexpr uint32_t kSmall = 3072;
 constexpr uint32_t kOffQ = kSmall;
 constexpr uint32_t kOffK = kOffQ + kTile;      // 2 stages
 constexpr uint32_t kOffV = kOffK + 2 * kTile;  // 2 stages
-constexpr uint32_t kOffP = kOffV + 2 * kTile;  // 2 buffers
+constexpr uint32_t kOffP = kOffV + 2 * kTile;  // P_A, P_B
 constexpr uint32_t kSmemBytes = kOffP + 2 * kTile;  // 232,448 B = 227 KB
-constexpr uint64_t kTimeoutNs = 1000000000ull;
 constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold (factor 256)
+constexpr int kRegsLaunch = 168;  // 65,536 / 384 rounded down to a multiple of 8
+constexpr int kRegsSoftmax = 200, kRegsAux = 56;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsAux <= kThreads * kRegsLaunch, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;
 
-// barrier slots
 enum : uint32_t {
-  BQ = 0, BK0 = 1, BV0 = 3, BS0 = 5, BSF0 = 7, BP0 = 9, BPV0 = 11, BKF0 = 13, BX0 = 15,
-  BDRAIN = 17, BL = 18, NBAR = 19
+  BQ = 0, BK0 = 1, BV0 = 3, BS0 = 5, BSF0 = 7, BP0 = 9, BPV0 = 11, BKF0 = 13, BDRAIN = 15,
+  BM = 16, NBAR = 17
 };
 static_assert(NBAR * 8 <= kOffSlot, "barrier region");
+static_assert(kOffMerge + 2 * 2 * 128 * 4 <= kSmall, "merge region");
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.shared::cta.b64 st, [%0];\n}\n" ::"r"(bar)
-               : "memory");
+// Natural row (in the [B*heads*N, d] matrix) of tile row p of head bh;
+// pad rows (p >= N) point at the head's first row: their keys are masked
+// to -inf and their query rows are never stored.
+__device__ __forceinline__ int gather_row(const Grid& g, int order, int64_t bh, int p) {
+  return (int)(bh * g.N) + (p < g.N ? natural_index(g, order, p) : 0);
 }
 
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-struct Ctl {
-  volatile uint32_t* abort;
-  int32_t* status;
-};
-
-// Bounded wait on one phase of an mbarrier (one thread).
-__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, Ctl c) {
-  if (mbar_try(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*c.abort) return false;
-      if (global_ns() - t0 > kTimeoutNs) {
-        *c.abort = 1;
-        report(c.status, PA_ERR_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
-
-// Warp-uniform bounded wait: lane 0 waits, the outcome is broadcast.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, Ctl c) {
-  int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = wait_phase(bar, parity, c) ? 1 : 0;
-  return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
-
-// Bounded wait by every lane (each acquires the data published before the
-// phase completed); the outcome is made warp-uniform.
-__device__ __forceinline__ bool all_wait(uint32_t bar, uint32_t parity, Ctl c) {
-  const bool ok = wait_phase(bar, parity, c);
-  return __all_sync(0xffffffffu, ok);
-}
-
-// --- tcgen05 -------------------------------------------------------------
-
-// Shared-memory matrix descriptor, SWIZZLE_128B, sm_100 version field.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
-  return d;
-}
-
-// Instruction descriptor, kind::f16: D f32, A and B bf16, A K-major.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
-         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                           uint32_t accumulate) {
-  asm volatile(
-      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
-                   bar)
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-}
-__device__ __forceinline__ void fence_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;\n" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
-}
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&t);
-}
-
-// Byte offset of the 16-byte chunk c (0..7) of row r inside one 64-column
-// half of a SWIZZLE_128B tile: rows are 128 bytes, chunks XOR-permuted by
-// the row's position within its 8-row group.
-__device__ __forceinline__ uint32_t sw128_off(int r, int c) {
-  return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
-}
-
-// One loader warp copies 32 rows (row0 .. row0+31) of a [128 x 128] bf16
-// tile.  nat = natural token index of this lane's row (lane l <-> row
-// row0 + l), or -1 for a pad row (zero-filled).  Each 16-lane half of the
-// warp reads one whole 256-byte row per instruction.
-__device__ __forceinline__ void load_rows(uint32_t tile, const __nv_bfloat16* __restrict__ head,
-                                          int row0, int lane, int nat) {
-#pragma unroll 4
-  for (int m = 0; m < 16; ++m) {
-    const int src_lane = 2 * m + (lane >> 4);
-    const int n = __shfl_sync(0xffffffffu, nat, src_lane);
-    const int r = row0 + src_lane;
-    const int cc = lane & 15;
-    const int half = cc >> 3, c = cc & 7;
-    const char* src = reinterpret_cast<const char*>(head) +
-                      (n >= 0 ? (int64_t)n * (kD * 2) : 0) + half * 128 + c * 16;
-    cp_async16(tile + half * kHalf + sw128_off(r, c), src, n >= 0 ? 16u : 0u);
-  }
+// Lane l gathers rows 4l..4l+3 of a 128 x 128 bf16 tile (both halves).
+__device__ __forceinline__ void gather_tile(uint32_t tile, const CUtensorMap* map, const Grid& g,
+                                            int order, int64_t bh, int p0, int lane, uint32_t bar) {
+  const int r = 4 * lane;
+  const int r0 = gather_row(g, order, bh, p0 + r);
+  const int r1 = gather_row(g, order, bh, p0 + r + 1);
+  const int r2 = gather_row(g, order, bh, p0 + r + 2);
+  const int r3 = gather_row(g, order, bh, p0 + r + 3);
+  tma_gather4(tile + r * 128, map, 0, r0, r1, r2, r3, bar);
+  tma_gather4(tile + kHalf + r * 128, map, 64, r0, r1, r2, r3, bar);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_sm100_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                      const __nv_bfloat16* __restrict__ v, const __grid_constant__ Grid g,
+    attn_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
+                      const __grid_constant__ CUtensorMap map_k,
+                      const __grid_constant__ CUtensorMap map_v, const __grid_constant__ Grid g,
                       const int32_t* __restrict__ idx, const int32_t* __restrict__ counts,
                       int k_max, float scale_log2, __nv_bfloat16* __restrict__ out,
                       int32_t* __restrict__ status) {
@@ -254,12 +136,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
   unsigned char* gbase = smem_raw;
-  const uint32_t bars = base + kOffBar;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOffSlot);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile uint32_t* bad_flag = tmem_slot + 2;
-  float* xmax = reinterpret_cast<float*>(gbase + kOffXmax);
-  auto bar = [&](uint32_t slot) { return bars + slot * 8u; };
+  float* merge = reinterpret_cast<float*>(gbase + kOffMerge);  // [m|l][group][row]
+  auto bar = [&](uint32_t slot) { return base + kOffBar + slot * 8u; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x;
@@ -275,32 +156,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       status != nullptr && *reinterpret_cast<volatile int32_t*>(status) == PA_ERR_TIMEOUT;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(BQ), kLoadWarps * 32);
+    mbar_init(bar(BQ), 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(BK0 + s), kLoadWarps * 16);
-      mbar_init(bar(BV0 + s), kLoadWarps * 16);
-      mbar_init(bar(BKF0 + s), 1);
+      mbar_init(bar(BK0 + s), 1);
+      mbar_init(bar(BV0 + s), 1);
       mbar_init(bar(BS0 + s), 1);
-      mbar_init(bar(BSF0 + s), kSoftmaxThreads);
-      mbar_init(bar(BP0 + s), kSoftmaxThreads);
+      mbar_init(bar(BSF0 + s), kGroupThreads);
+      mbar_init(bar(BP0 + s), kGroupThreads);
       mbar_init(bar(BPV0 + s), 1);
-      mbar_init(bar(BX0 + s), kSoftmaxThreads);
+      mbar_init(bar(BKF0 + s), 1);
     }
     mbar_init(bar(BDRAIN), 1);
-    mbar_init(bar(BL), kSoftmaxThreads);
+    mbar_init(bar(BM), 2 * kGroupThreads);
     *abort_flag = 0;
     *bad_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
-  if (warp == kMmaWarp) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"(kTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
-  }
-  if (warp == kLoadWarp0) {
-    // validate the kept list once: count in range, indices ascending in [0, NB)
+  if (warp == kMmaWarp) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+  if (warp == kCheckWarp) {
+    // the kept list: count in range, indices ascending in [0, NB)
     bool bad = cnt < 0 || cnt > k_max;
     if (!bad) {
       for (int e = lane; e < cnt; e += 32) {
@@ -320,47 +194,42 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const bool run = *bad_flag == 0 && !expired;
   const int n_tiles = run ? cnt : 0;
-
-  const __nv_bfloat16* qh = q + bh * (int64_t)g.N * kD;
-  const __nv_bfloat16* kh = k + bh * (int64_t)g.N * kD;
-  const __nv_bfloat16* vh = v + bh * (int64_t)g.N * kD;
-
-  if (warp >= kLoadWarp0) {
-    // ------------------------------------------------------ loaders ----
-    const int lw = warp - kLoadWarp0;
+  // registers: launched at 168 per thread (384 x 168 = 64,512); the two
+  // softmax warpgroups take 200, the MMA / gather / check warpgroup 56
+  // (2 x 128 x 200 + 128 x 56 = 58,368 <= 64,512), and every warpgroup
+  // returns to 168 before the common exit
+  if (warp >= 8) {
+  regs_dec<kRegsAux>();
+  if (warp == kKWarp || warp == kVWarp) {
+    // ------------------------------------------------------ gathers ----
+    const bool is_k = warp == kKWarp;
+    const CUtensorMap* map = is_k ? &map_k : &map_v;
+    const uint32_t ring = base + (is_k ? kOffK : kOffV);
+    int issued = 0;
     if (n_tiles > 0) {
-      {
-        const int p = i * kBlock + 32 * lw + lane;
-        const int nat = p < g.N ? natural_index(g, order, p) : -1;
-        load_rows(base + kOffQ, qh, 32 * lw, lane, nat);
-        cp_async_commit();
-        cp_async_wait<0>();
-        fence_async_smem();
-        mbar_arrive(bar(BQ));
+      if (is_k) {
+        if (lane == 0) mbar_arrive_tx(bar(BQ), kTile);
+        __syncwarp();
+        gather_tile(base + kOffQ, &map_q, g, order, bh, i * kBlock, lane, bar(BQ));
       }
-      // warps 5-6 stream K (stage free once QK^T of tile j-2 completed),
-      // warps 7-8 stream V (stage free once P V of tile j-2 completed)
-      const bool is_k = lw < 2;
-      const int half_rows = 64 * (lw & 1);
-      const __nv_bfloat16* src = is_k ? kh : vh;
-      const uint32_t ring = base + (is_k ? kOffK : kOffV);
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j & 1;
+        // the stage is free once QK^T (K) or P V (V) of tile j-2 completed
         if (j >= 2 && !warp_wait(bar((is_k ? BKF0 : BPV0) + s), ((j - 2) >> 1) & 1, ctl)) break;
+        PARO_T(is_k ? 0 : 2, j);
         const int kb = __ldg(ids + j);
-#pragma unroll
-        for (int g2 = 0; g2 < 2; ++g2) {
-          const int row0 = half_rows + 32 * g2;
-          const int p = kb * kBlock + row0 + lane;
-          const int nat = p < g.N ? natural_index(g, order, p) : -1;
-          load_rows(ring + s * kTile, src, row0, lane, nat);
-        }
-        cp_async_commit();
-        cp_async_wait<0>();
-        fence_async_smem();
-        mbar_arrive(bar((is_k ? BK0 : BV0) + s));
+        if (lane == 0) mbar_arrive_tx(bar((is_k ? BK0 : BV0) + s), kTile);
+        __syncwarp();
+        gather_tile(ring + s * kTile, map, g, order, bh, kb * kBlock, lane,
+                    bar((is_k ? BK0 : BV0) + s));
+        issued = j + 1;
       }
-      cp_async_wait<0>();
+      // on the way out make sure this warp's last loads have landed
+      if (lane == 0) {
+        if (is_k) drain_phase(bar(BQ), 0);
+        for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j)
+          drain_phase(bar((is_k ? BK0 : BV0) + (j & 1)), (j >> 1) & 1);
+      }
     }
   } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------- MMA ----
@@ -379,9 +248,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < kBlock / 16; ++kk) {
           const uint64_t ad = sw128_desc(pa + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = sw128_desc(va + kk * 16 * 128, kHalf, 1024);
-          mma_f16_ss(tmem + kColO, ad, bd, id_pv, (jp > 0 || kk > 0) ? 1u : 0u);
+          mma_f16_ss(tmem + kColO + b * 128, ad, bd, id_pv, (jp >= 2 || kk > 0) ? 1u : 0u);
         }
         mma_commit(bar(BPV0 + b));
+        PARO_T(5, jp);
         return true;
       };
       for (int j = 0; ok && j < n_tiles; ++j) {
@@ -398,78 +268,85 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(bar(BS0 + b));
         mma_commit(bar(BKF0 + b));
+        PARO_T(4, j);
         if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
       }
       if (ok) issue_pv(n_tiles - 1);
       // drain: every MMA issued above has completed once this commit fires
       mma_commit(bar(BDRAIN));
-      wait_phase(bar(BDRAIN), 0, ctl);
+      drain_phase(bar(BDRAIN), 0);
     }
+  }
+  __syncwarp();  // setmaxnreg is warp-aligned: reconverge after the lane-0 roles
+  regs_inc<kRegsLaunch>();
   } else {
+    regs_inc<kRegsSoftmax>();
     // ------------------------------------------------------ softmax ----
-    const int quarter = warp & 3, hc = warp >> 2;
+    const int grp = warp >> 2;  // 0: even tiles, 1: odd tiles
+    const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // tile row == TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t s_col = kColS + grp * 128, o_col = kColO + grp * 128;
+    unsigned char* pt = gbase + kOffP + grp * kTile;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      const int b = j & 1;
-      if (!warp_wait(bar(BS0 + b), (j >> 1) & 1, ctl)) { ok = false; break; }
+    int t = 0;  // this group's tile counter
+    for (int j = grp; j < n_tiles; j += 2, ++t) {
+      if (!warp_wait(bar(BS0 + grp), t & 1, ctl)) { ok = false; break; }
+      if (lane == 0 && quarter == 0) PARO_T(6 + 4 * grp, j);
       tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld64(lane_addr + kColS + b * 128 + hc * 64, sr);
+      uint32_t sr[128];
+      tmem_ld128(lane_addr + s_col, sr);
       tc_fence_before();
-      mbar_arrive(bar(BSF0 + b));
+      mbar_arrive(bar(BSF0 + grp));
+      if (lane == 0 && quarter == 0) PARO_T(7 + 4 * grp, j);
       const int kb = __ldg(ids + j);
-      const int valid = g.N - kb * kBlock - hc * 64;  // existing keys in my half
-      if (valid < 64) {  // only the ragged last block (warp-uniform)
+      const int valid = g.N - kb * kBlock;  // keys of this block that exist
+      if (valid < kBlock) {  // only the ragged last block (warp-uniform)
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
+        for (int c = 0; c < 128; ++c)
           if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
       }
-      // raw row max of my half (8 independent chains), exchanged with the
-      // other half of the row
       float mp[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) mp[u] = __uint_as_float(sr[u]);
 #pragma unroll
-      for (int c = 8; c < 64; ++c) mp[c & 7] = fmaxf(mp[c & 7], __uint_as_float(sr[c]));
-      const float mh = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-      float* xm = xmax + b * 256;
-      xm[hc * 128 + r] = mh;
-      mbar_arrive(bar(BX0 + b));
-      if (!all_wait(bar(BX0 + b), (j >> 1) & 1, ctl)) { ok = false; break; }
-      const float mx = fmaxf(mh, xm[(hc ^ 1) * 128 + r]) * scale_log2;
+      for (int c = 8; c < 128; ++c) mp[c & 7] = fmaxf(mp[c & 7], __uint_as_float(sr[c]));
+      const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) *
+                       scale_log2;
+      if (lane == 0 && quarter == 0) PARO_T(8 + 4 * grp, j);
       // lazy rescale: keep the reference max unless the row max grew by
       // more than 2^8 (exact either way: O and l share the reference)
-      const bool need = j == 0 ? false : (mx > m_used + kRescaleLog2);
-      if (j == 0) m_used = mx == -INFINITY ? 0.f : mx;
-      if (__any_sync(0xffffffffu, need)) {
-        if (!warp_wait(bar(BPV0 + ((j - 1) & 1)), ((j - 1) >> 1) & 1, ctl)) { ok = false; break; }
-        tc_fence_after();
-        const float alpha = need ? ex2(m_used - mx) : 1.f;
+      const bool need = t == 0 ? false : (mx > m_used + kRescaleLog2);
+      if (t == 0) m_used = mx == -INFINITY ? 0.f : mx;
+      if (t >= 1) {
+        // O_grp and P_grp are free once P V of this group's previous tile
+        // (tile j-2) completed
+        if (!warp_wait(bar(BPV0 + grp), (t - 1) & 1, ctl)) { ok = false; break; }
+        if (__any_sync(0xffffffffu, need)) {
+          tc_fence_after();
+          const float alpha = need ? ex2(m_used - mx) : 1.f;
 #pragma unroll 1
-        for (int c0 = 0; c0 < 64; c0 += 32) {
-          uint32_t orr[32];
-          tmem_ld32(lane_addr + kColO + hc * 64 + c0, orr);
+          for (int c0 = 0; c0 < 128; c0 += 32) {
+            uint32_t orr[32];
+            tmem_ld32(lane_addr + o_col + c0, orr);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
-          tmem_st32(lane_addr + kColO + hc * 64 + c0, orr);
+            for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
+            tmem_st32(lane_addr + o_col + c0, orr);
+          }
+          l *= alpha;
+          if (need) m_used = mx;
         }
-        l *= alpha;
-        if (need) m_used = mx;
       }
-      if (j >= 2 && !warp_wait(bar(BPV0 + b), ((j - 2) >> 1) & 1, ctl)) { ok = false; break; }
-      // P = 2^(s*scale - m) in bf16 into my half of the swizzled K-major P
-      // tile; row sum in 8 independent chains
-      unsigned char* pt = gbase + kOffP + b * kTile + hc * kHalf;
+      // P = 2^(s*scale - m) in bf16 into the swizzled K-major P tile; row
+      // sum in 8 independent chains
       const float neg_m = -m_used;
       float rs[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) rs[u] = 0.f;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < 16; ++c) {
         float e[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -481,53 +358,78 @@ __global__ void __launch_bounds__(kThreads, 1)
         w.y = pack_bf16(e[2], e[3]);
         w.z = pack_bf16(e[4], e[5]);
         w.w = pack_bf16(e[6], e[7]);
-        *reinterpret_cast<uint4*>(pt + sw128_off(r, c)) = w;
+        *reinterpret_cast<uint4*>(pt + (c >> 3) * kHalf + sw128_off(r, c & 7)) = w;
       }
       l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
+      if (lane == 0 && quarter == 0) PARO_T(9 + 4 * grp, j);
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(bar(BP0 + b));
+      mbar_arrive(bar(BP0 + grp));
     }
-    // epilogue: the two halves add their row sums, then each writes O / l
-    // for its 64 columns at the natural position of the row's token
+    // ---- merge the two groups and store (group g writes columns 64g..)
     const int p = i * kBlock + r;
     __nv_bfloat16* orow = p < g.N ? out + (bh * (int64_t)g.N + natural_index(g, order, p)) * kD
                                   : nullptr;
     if (run && cnt == 0) {
       if (orow != nullptr)
         for (int c = 0; c < 8; ++c)
-          reinterpret_cast<uint4*>(orow + hc * 64)[c] = make_uint4(0, 0, 0, 0);
+          reinterpret_cast<uint4*>(orow + grp * 64)[c] = make_uint4(0, 0, 0, 0);
     } else if (ok && n_tiles > 0) {
-      const int jl = n_tiles - 1;
-      // the exchange buffer the last tile did not use: its previous reads
-      // (tile jl-1) finished before every thread arrived for tile jl
-      float* xl = xmax + ((jl & 1) ^ 1) * 256;
-      xl[hc * 128 + r] = l;
-      mbar_arrive(bar(BL));
-      const bool okl = all_wait(bar(BL), 0, ctl);
-      const float lt = okl ? l + xl[(hc ^ 1) * 128 + r] : 0.f;
-      if (okl && warp_wait(bar(BPV0 + (jl & 1)), (jl >> 1) & 1, ctl)) {
+      const bool has_b = n_tiles >= 2;
+      merge[(0 * 2 + grp) * 128 + r] = m_used;
+      merge[(1 * 2 + grp) * 128 + r] = l;
+      mbar_arrive(bar(BM));
+      bool okm = all_wait(bar(BM), 0, ctl);
+      float fa = 0.f, fb = 0.f, lt = 0.f;
+      if (okm) {
+        const float ma = merge[r], mb = has_b ? merge[128 + r] : -INFINITY;
+        const float m = fmaxf(ma, mb);
+        fa = ex2(ma - m);
+        fb = has_b ? ex2(mb - m) : 0.f;
+        lt = merge[256 + r] * fa + (has_b ? merge[384 + r] * fb : 0.f);
+      }
+      // both groups' last P V must be complete
+      for (int gg = 0; okm && gg < 2; ++gg) {
+        if (gg == 1 && !has_b) continue;
+        const int jl = ((n_tiles - 1) & 1) == gg ? n_tiles - 1 : n_tiles - 2;
+        okm = warp_wait(bar(BPV0 + gg), (jl >> 1) & 1, ctl);
+      }
+      if (okm) {
         tc_fence_after();
         const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        fa *= inv;
+        fb *= inv;
 #pragma unroll 1
         for (int c0 = 0; c0 < 64; c0 += 32) {
-          uint32_t orr[32];
-          tmem_ld32(lane_addr + kColO + hc * 64 + c0, orr);
+          const int col = grp * 64 + c0;
+          uint32_t oa[32], ob[32];
+          tmem_ld32(lane_addr + kColO + col, oa);
+          if (has_b) {
+            tmem_ld32(lane_addr + kColO + 128 + col, ob);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) ob[c] = 0u;
+          }
           if (orow != nullptr) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-              const float* f = reinterpret_cast<const float*>(orr) + c * 8;
+              float v[8];
+#pragma unroll
+              for (int u = 0; u < 8; ++u)
+                v[u] = __uint_as_float(oa[c * 8 + u]) * fa + __uint_as_float(ob[c * 8 + u]) * fb;
               uint4 w;
-              w.x = pack_bf16(f[0] * inv, f[1] * inv);
-              w.y = pack_bf16(f[2] * inv, f[3] * inv);
-              w.z = pack_bf16(f[4] * inv, f[5] * inv);
-              w.w = pack_bf16(f[6] * inv, f[7] * inv);
-              reinterpret_cast<uint4*>(orow + hc * 64 + c0)[c] = w;
+              w.x = pack_bf16(v[0], v[1]);
+              w.y = pack_bf16(v[2], v[3]);
+              w.z = pack_bf16(v[4], v[5]);
+              w.w = pack_bf16(v[6], v[7]);
+              reinterpret_cast<uint4*>(orow + col)[c] = w;
             }
           }
         }
       }
     }
+    __syncwarp();
+    regs_dec<kRegsLaunch>();
   }
 
   tc_fence_before();
@@ -535,16 +437,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) {
     __syncwarp();
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem),
-                 "r"(kTmemCols)
-                 : "memory");
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
 }  // namespace
 
 bool attn_sm100_supports(pa_dtype dt, const Grid& g) {
-  return dt == PA_BF16 && g.d == kD && g.block == kBlock;
+  return dt == PA_BF16 && g.d == kD && g.block == kBlock &&
+         (int64_t)g.B * g.heads * g.N < ((int64_t)1 << 31);
 }
 
 cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, pa_dtype dt,
@@ -555,15 +456,19 @@ cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, pa_dt
   (void)ks;
   (void)vs;
   if (!attn_sm100_supports(dt, g)) return cudaErrorInvalidValue;
+  const uint64_t rows = (uint64_t)g.B * g.heads * g.N;
+  CUtensorMap mq, mk, mv;
+  if (!encode_gather_map(&mq, q, rows, kD, 2, 64) || !encode_gather_map(&mk, k, rows, kD, 2, 64) ||
+      !encode_gather_map(&mv, v, rows, kD, 2, 64))
+    return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)kD));
   dim3 grid(g.NB, g.B * g.heads);
-  attn_sm100_kernel<<<grid, kThreads, kSmemBytes, s>>>(
-      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-      static_cast<const __nv_bfloat16*>(v), g, idx, counts, k_max, scale_log2,
-      static_cast<__nv_bfloat16*>(out), status);
+  attn_sm100_kernel<<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, g, idx, counts, k_max,
+                                                       scale_log2,
+                                                       static_cast<__nv_bfloat16*>(out), status);
   return cudaGetLastError();
 }
 

@@ -1,0 +1,233 @@
+// sm_100a building blocks shared by the tcgen05 attention kernels: mbarrier
+// waits bounded by %globaltimer, shared-memory matrix and instruction
+// descriptors for tcgen05.mma, TMEM allocation, commits and fences, and TMA
+// row gathers (cp.async.bulk.tensor ... tile::gather4).
+#pragma once
+
+#include <cuda.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "tmem.cuh"
+
+namespace paro {
+namespace sm100 {
+
+constexpr uint64_t kTimeoutNs = 1000000000ull;  // a legitimate wait lasts microseconds
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.shared::cta.b64 st, [%0];\n}\n" ::"r"(bar)
+               : "memory");
+}
+
+// One arrival that also raises the transaction count by `bytes` (TMA loads
+// then complete the phase as their bytes land).
+__device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}\n" ::"r"(
+                   bar),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, "
+      "p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Abort flag shared by the CTA's roles plus the device status word.
+struct Ctl {
+  volatile uint32_t* abort;
+  int32_t* status;
+};
+
+// Bounded wait on one phase of an mbarrier (one thread).  Gives up when the
+// CTA's abort flag is raised, or after kTimeoutNs, raising it and recording
+// PA_ERR_TIMEOUT.
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, Ctl c) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*c.abort) return false;
+      if (global_ns() - t0 > kTimeoutNs) {
+        *c.abort = 1;
+        report(c.status, PA_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait that ignores the abort flag: used on the way out to let this
+// thread's own copies land before the CTA releases its shared memory.
+__device__ __forceinline__ bool drain_phase(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = global_ns();
+  while (!mbar_try(bar, parity))
+    if (global_ns() - t0 > kTimeoutNs) return false;
+  return true;
+}
+
+// Warp-uniform bounded wait: lane 0 waits, the outcome is broadcast.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, Ctl c) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = wait_phase(bar, parity, c) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Bounded wait by every lane (each acquires what was published before the
+// phase completed); the outcome is made warp-uniform.
+__device__ __forceinline__ bool all_wait(uint32_t bar, uint32_t parity, Ctl c) {
+  const bool ok = wait_phase(bar, parity, c);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// --- tcgen05 ----------------------------------------------------------------
+
+// Shared-memory matrix descriptor, SWIZZLE_128B, sm_100 version field.
+// K-major operands: lbo = 16 (unused), sbo = 1024 (8-row groups of 128 B).
+// MN-major operands: lbo = byte distance of 64-element MN chunks, sbo = 1024.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16: D f32, A and B bf16, A K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Instruction descriptor, kind::i8: D s32, A and B signed int8, A K-major.
+__host__ __device__ constexpr uint32_t idesc_s8(int M, int N, bool b_mn_major) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+                   bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t slot_smem, uint32_t cols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(slot_smem),
+               "r"(cols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t tmem, uint32_t cols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(cols)
+               : "memory");
+}
+
+// Per-warpgroup register budget (every warp of the warpgroup executes it).
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+// Generic-proxy shared-memory writes (st.shared) become visible to the
+// async proxy (tcgen05.mma operand reads).
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+
+// --- TMA ----------------------------------------------------------------
+
+// Four rows (r0..r3) x 64 columns starting at column `col` of a 2D tensor
+// map whose box is {64, 1}, into 4 consecutive 128-byte rows at `dst`; the
+// map's SWIZZLE_128B is applied on the destination address bits.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int col, int r0,
+                                            int r1, int r2, int r3, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cta.global.tile::gather4.mbarrier::complete_tx::bytes [%0], "
+      "[%1, {%2, %3, %4, %5, %6}], [%7];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
+      : "memory");
+}
+
+// --- math ---------------------------------------------------------------
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&t);
+}
+
+// Byte offset of the 16-byte chunk c (0..7) of row r inside one 128-byte
+// wide SWIZZLE_128B panel: rows are 128 bytes, chunks XOR-permuted by the
+// row's position within its 8-row group.
+__device__ __forceinline__ uint32_t sw128_off(int r, int c) {
+  return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
+}
+
+}  // namespace sm100
+
+// Host: encode a 2D row-gather tensor map over a row-major [rows, cols]
+// matrix of `elem_bytes`-byte elements with a {box_cols, 1} box and
+// SWIZZLE_128B (box_cols * elem_bytes must be 128).  Returns false when the
+// driver entry point is unavailable or the encode fails.
+bool encode_gather_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                       int elem_bytes, uint32_t box_cols);
+
+}  // namespace paro
