@@ -3,10 +3,10 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 One step = the whole path for one 720p-shaped video DiT layer (B=1, 40 heads,
-d=128, 21x45x80 grid = 75,600 tokens, block 128, density 0.15):
-pooled block scores (reorder folded into the loads) -> top-k kept blocks ->
-block-sparse attention over the kept tiles (inverse reorder folded into the
-stores).  Inputs are resident in HBM when the timed region starts and are
+d=128, 21x45x80 grid = 75,600 tokens, block 128, density 0.15): reorder of
+q, k, v with the block means taken from the same read -> pooled block scores
+-> top-k kept blocks -> block-sparse attention over the kept tiles (inverse
+reorder folded into its stores).  Inputs are resident in HBM when the timed region starts and are
 larger than L2 (3 x 774 MB), so no flush is needed between steps.
 
 Prints one JSON line (rank 0).  ``value`` is the effective TFLOPS over kept
@@ -39,6 +39,7 @@ sys.path.insert(0, ROOT)
 
 from block_sparse_attention_34_b200 import paro  # noqa: E402
 from block_sparse_attention_34_b200.configs import WORKLOADS  # noqa: E402
+from block_sparse_attention_34_b200.pipeline import Pipeline  # noqa: E402
 from block_sparse_attention_34_b200.synth import make_inputs  # noqa: E402
 
 METRIC = "block-sparse attention latency (ms) & effective TFLOPS, % of TC peak, at given density"
@@ -161,47 +162,23 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ steps --
 
-class Pipeline:
-    """Device buffers and the launches of one step (through the C ABI)."""
-
-    def __init__(self, w, q, k, v, perms, density, baseline=False):
-        self.w = w
-        self.pr = paro.Problem(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, perms)
-        self.k = paro.k_for_density(self.pr.NB, density)
-        self.q, self.k_, self.v = q, k, v
-        dev = q.device
-        pr = self.pr
-        self.q_pool = torch.empty((pr.B, pr.heads, pr.NB, pr.d), dtype=torch.float32, device=dev)
-        self.k_pool = torch.empty_like(self.q_pool)
-        self.scores = torch.empty((pr.B, pr.heads, pr.NB, pr.NB), dtype=torch.float32, device=dev)
-        self.idx = torch.empty((pr.B, pr.heads, pr.NB, self.k), dtype=torch.int32, device=dev)
-        self.out = torch.empty((pr.B, pr.heads, pr.N, pr.d), dtype=q.dtype, device=dev)
-        self.baseline = baseline
-        self.launches_per_step = 5  # pool q, pool k, score, top-k, attention
-
-    def select(self):
-        paro.block_score(self.q, self.k_, self.pr, self.q_pool, self.k_pool, self.scores)
-        paro.select_topk(self.scores, self.pr, self.k, self.idx)
-
-    def attend(self):
-        paro.block_sparse_attn(self.q, self.k_, self.v, self.pr, self.idx, out=self.out,
-                               baseline=self.baseline)
-
-    def step(self, ev=None):
-        self.select()
-        if ev is not None:
-            ev[0].record()
-        self.attend()
-        if ev is not None:
-            ev[1].record()
-
-    def flops(self):
-        return self.w.flops(self.k)
+def make_pipeline(w, perms, density, kernel, device):
+    return Pipeline(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, perms, density,
+                    device=device, int8=w.int8, baseline=kernel == "mma")
 
 
-def time_steps(pipe, steps, warmup, ws, device):
+def step(pipe, qkv, ev=None):
+    pipe.select(*qkv)
+    if ev is not None:
+        ev[0].record()
+    pipe.attend(*qkv)
+    if ev is not None:
+        ev[1].record()
+
+
+def time_steps(pipe, qkv, steps, warmup, ws, device):
     for _ in range(warmup):
-        pipe.step()
+        step(pipe, qkv)
     torch.cuda.synchronize()
     ev_attn = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(steps)]
@@ -210,16 +187,18 @@ def time_steps(pipe, steps, warmup, ws, device):
     torch.cuda.synchronize()
     start.record()
     for s in range(steps):
-        pipe.step(ev_attn[s])
+        step(pipe, qkv, ev_attn[s])
     end.record()
     torch.cuda.synchronize()
     barrier(ws)
+    if int(pipe.status.item()) != 0:
+        raise RuntimeError(f"device status {int(pipe.status.item())} after the timed steps")
     total_ms = start.elapsed_time(end)
     attn_ms = [a.elapsed_time(b) for a, b in ev_attn]
     return total_ms, attn_ms
 
 
-def e2e_steps(pipe, host_q, host_k, host_v, host_out, steps):
+def e2e_steps(pipe, qkv, host_q, host_k, host_v, host_out, steps):
     """The same step through the public API with host buffers: pinned host
     -> device copies of Q, K, V, the path, and the device -> host copy of O,
     all inside the timed region."""
@@ -227,10 +206,10 @@ def e2e_steps(pipe, host_q, host_k, host_v, host_out, steps):
     torch.cuda.synchronize()
     start.record()
     for _ in range(steps):
-        pipe.q.copy_(host_q, non_blocking=True)
-        pipe.k_.copy_(host_k, non_blocking=True)
-        pipe.v.copy_(host_v, non_blocking=True)
-        pipe.step()
+        qkv[0].copy_(host_q, non_blocking=True)
+        qkv[1].copy_(host_k, non_blocking=True)
+        qkv[2].copy_(host_v, non_blocking=True)
+        pipe.run(*qkv)
         host_out.copy_(pipe.out, non_blocking=True)
     end.record()
     torch.cuda.synchronize()
@@ -286,16 +265,16 @@ def run_ours(a):
     q, k, v, perms = make_inputs(w, heads=a.heads)
     if a.heads is not None:  # leading heads only (same values as the full draw)
         w = dataclasses.replace(w, heads=a.heads)
-    qd, kd, vd = (t.to(device) for t in (q, k, v))
-    pipe = Pipeline(w, qd, kd, vd, perms, a.density if a.density is not None else w.density,
-                    baseline=a.kernel == "mma")
+    qkv = [t.to(device) for t in (q, k, v)]
+    dens = a.density if a.density is not None else w.density
+    pipe = make_pipeline(w, perms, dens, a.kernel, device)
     sampler = ClockSampler(local)
     sampler.start()
-    total_ms, attn_ms = time_steps(pipe, a.steps, a.warmup, ws, device)
+    total_ms, attn_ms = time_steps(pipe, qkv, a.steps, a.warmup, ws, device)
     clocks = sampler.stop()
     ms_step = max_over_ranks(total_ms / a.steps, ws, device)
     attn_avg = max_over_ranks(sum(attn_ms) / len(attn_ms), ws, device)
-    flops = pipe.flops()
+    flops = w.flops(pipe.k)
     value = flops * ws / (ms_step / 1e3) / 1e12
 
     peaks, peak_src = load_peaks()
@@ -305,11 +284,11 @@ def run_ours(a):
     # speedup over the same kernel on the dense (density 1.0) layer
     dense = None
     if not a.no_dense:
-        dpipe = Pipeline(w, qd, kd, vd, perms, 1.0, baseline=a.kernel == "mma")
+        dpipe = make_pipeline(w, perms, 1.0, a.kernel, device)
         dsteps = max(2, min(a.steps, 3))
-        _, d_attn = time_steps(dpipe, dsteps, 1, ws, device)
+        _, d_attn = time_steps(dpipe, qkv, dsteps, 1, ws, device)
         dense_ms = max_over_ranks(sum(d_attn) / len(d_attn), ws, device)
-        dense = {"attn_ms": dense_ms, "tflops": dpipe.flops() / (dense_ms / 1e3) / 1e12,
+        dense = {"attn_ms": dense_ms, "tflops": w.flops(dpipe.k) / (dense_ms / 1e3) / 1e12,
                  "speedup_attn": dense_ms / attn_avg, "target": 0.8 / (pipe.k / pipe.pr.NB)}
         del dpipe
 
@@ -317,7 +296,8 @@ def run_ours(a):
     if not a.no_e2e:
         host = [t.pin_memory() for t in (q, k, v)]
         host_out = torch.empty(pipe.out.shape, dtype=pipe.out.dtype).pin_memory()
-        e_ms = max_over_ranks(e2e_steps(pipe, *host, host_out, max(1, min(a.steps, 5))), ws, device)
+        e_ms = max_over_ranks(e2e_steps(pipe, qkv, *host, host_out, max(1, min(a.steps, 5))), ws,
+                              device)
         e2e = {"value": flops * ws / (e_ms / 1e3) / 1e12, "unit": "TFLOPS",
                "ms_per_step": e_ms,
                "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in host)),
@@ -341,17 +321,19 @@ def run_ours(a):
                 "N": w.N, "d": w.d, "block": w.block, "density": pipe.k / pipe.pr.NB,
                 "density_requested": a.density if a.density is not None else w.density,
                 "k": pipe.k, "NB": pipe.pr.NB, "kept_tiles": w.kept_tiles(pipe.k),
-                "flops_per_step": flops, "kernel": "tcgen05" if a.kernel == "tcgen05" else "mma.sync",
+                "flops_per_step": flops,
+                "kernel": ("tcgen05, permuted tiles" if a.kernel == "tcgen05" else "mma.sync, gathered rows"),
                 "l2": "inputs larger than L2 (q, k, v 774 MB each); no flush",
                 "parallelism": f"replicas x{ws} (independent layers, no data-path collective)",
-                "attn_ms": attn_avg, "select_ms": ms_step - attn_avg,
+                "attn_ms": attn_avg, "prep_ms": ms_step - attn_avg,
+                "prep": "reorder+pool q,k; reorder v; pooled scores; top-k",
             },
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": ncu_traffic(w.name),
                          "kernel": "attn_sm100_kernel" if a.kernel == "tcgen05" else "attn_mma_kernel",
                          "peak_source": f"{peak_src} bf16_tflops_sustained"},
             "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": pipe.launches_per_step * a.steps,
+            "gpu_launches": pipe.launches * a.steps,
             "clocks": clocks, "dense": dense,
         }
         print(json.dumps(res), flush=True)

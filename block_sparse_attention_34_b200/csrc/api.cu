@@ -13,7 +13,7 @@ namespace paro {
 cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, pa_dtype dt,
                               const Grid& g, const int32_t* idx, const int32_t* counts,
                               int k_max, const float* qs, const float* ks, const float* vs,
-                              void* out, int32_t* status, cudaStream_t s);
+                              void* out, int32_t* status, bool permuted, cudaStream_t s);
 bool attn_sm100_supports(pa_dtype dt, const Grid& g);
 }  // namespace paro
 
@@ -109,7 +109,7 @@ pa_status check_float_dtype(pa_dtype dt) {
 
 extern "C" {
 
-int32_t pa_abi_version(void) { return 1; }
+int32_t pa_abi_version(void) { return 2; }
 
 const char* pa_last_error(void) { return g_error.c_str(); }
 
@@ -132,14 +132,14 @@ int32_t pa_k_for_density(int32_t nb, double density) {
 }
 
 pa_status pa_reorder(const void* x, void* x_perm, pa_dtype dtype, pa_shape shape,
-                     const int8_t* perms, void* stream) {
+                     const int8_t* perms, float* pool, void* stream) {
   paro::Grid g;
   pa_status st = check_float_dtype(dtype);
   if (st != PA_OK) return st;
   if ((st = make_grid(shape, perms, true, &g)) != PA_OK) return st;
   PA_REQUIRE(x && x_perm, "x and x_perm must be non-NULL");
   PA_REQUIRE(aligned16(x) && aligned16(x_perm), "x and x_perm must be 16-byte aligned");
-  return cuda_status(paro::launch_reorder(x, x_perm, dtype, g, false, (cudaStream_t)stream),
+  return cuda_status(paro::launch_reorder_pool(x, x_perm, dtype, g, pool, (cudaStream_t)stream),
                      "pa_reorder launch");
 }
 
@@ -217,7 +217,7 @@ pa_status pa_quantize_int8(const void* x, pa_dtype dtype, pa_shape shape, const 
 }
 
 static pa_status attn_common(const void* q, const void* k, const void* v, pa_dtype dtype,
-                             pa_shape shape, const int8_t* perms, const int32_t* idx,
+                             uint32_t flags, pa_shape shape, const int8_t* perms, const int32_t* idx,
                              const int32_t* counts, int32_t k_max, const float* q_scale,
                              const float* k_scale, const float* v_scale, void* out,
                              int32_t* dev_status, void* stream, bool force_mma) {
@@ -232,6 +232,8 @@ static pa_status attn_common(const void* q, const void* k, const void* v, pa_dty
   if (dtype == PA_I8) {
     PA_REQUIRE(q_scale && k_scale && v_scale, "INT8 attention needs q_scale, k_scale, v_scale");
   }
+  PA_REQUIRE((flags & ~PA_ATTN_PERMUTED) == 0, "unknown flags 0x%x", flags);
+  const bool permuted = dtype == PA_I8 || (flags & PA_ATTN_PERMUTED) != 0;
   cudaStream_t s = (cudaStream_t)stream;
   const bool sm100 = !force_mma && paro::attn_sm100_supports(dtype, g);
   if (dtype == PA_I8 && !sm100)
@@ -245,28 +247,28 @@ static pa_status attn_common(const void* q, const void* k, const void* v, pa_dty
   cudaError_t e;
   if (sm100)
     e = paro::launch_attn_sm100(q, k, v, dtype, g, idx, counts, k_max, q_scale, k_scale, v_scale,
-                                out, dev_status, s);
+                                out, dev_status, permuted, s);
   else
-    e = paro::launch_attn_mma(q, k, v, dtype, g, idx, counts, k_max, out, dev_status, s);
+    e = paro::launch_attn_mma(q, k, v, dtype, g, idx, counts, k_max, out, dev_status, permuted, s);
   return cuda_status(e, "pa_block_sparse_attn launch");
 }
 
 pa_status pa_block_sparse_attn(const void* q, const void* k, const void* v, pa_dtype dtype,
-                               pa_shape shape, const int8_t* perms, const int32_t* idx,
-                               const int32_t* counts, int32_t k_max, const float* q_scale,
-                               const float* k_scale, const float* v_scale, void* out,
-                               int32_t* dev_status, void* stream) {
-  return attn_common(q, k, v, dtype, shape, perms, idx, counts, k_max, q_scale, k_scale, v_scale,
-                     out, dev_status, stream, false);
+                               uint32_t flags, pa_shape shape, const int8_t* perms,
+                               const int32_t* idx, const int32_t* counts, int32_t k_max,
+                               const float* q_scale, const float* k_scale, const float* v_scale,
+                               void* out, int32_t* dev_status, void* stream) {
+  return attn_common(q, k, v, dtype, flags, shape, perms, idx, counts, k_max, q_scale, k_scale,
+                     v_scale, out, dev_status, stream, false);
 }
 
 pa_status pa_block_sparse_attn_mma(const void* q, const void* k, const void* v, pa_dtype dtype,
-                                   pa_shape shape, const int8_t* perms, const int32_t* idx,
-                                   const int32_t* counts, int32_t k_max, void* out,
-                                   int32_t* dev_status, void* stream) {
+                                   uint32_t flags, pa_shape shape, const int8_t* perms,
+                                   const int32_t* idx, const int32_t* counts, int32_t k_max,
+                                   void* out, int32_t* dev_status, void* stream) {
   PA_REQUIRE(dtype != PA_I8, "the mma.sync baseline takes PA_F32 or PA_BF16");
-  return attn_common(q, k, v, dtype, shape, perms, idx, counts, k_max, nullptr, nullptr, nullptr,
-                     out, dev_status, stream, true);
+  return attn_common(q, k, v, dtype, flags, shape, perms, idx, counts, k_max, nullptr, nullptr,
+                     nullptr, out, dev_status, stream, true);
 }
 
 }  // extern "C"

@@ -55,7 +55,8 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // a bf16 smem tile with row stride LD elements; rows past N become zeros.
 template <typename TIn, int D, int LD>
 __device__ __forceinline__ void gather_tile(__nv_bfloat16* dst, const TIn* __restrict__ head,
-                                            const Grid& g, int order, int p0, int rows) {
+                                            const Grid& g, int order, int p0, int rows,
+                                            bool permuted) {
   constexpr int E = 16 / sizeof(TIn);
   constexpr int VPR = D / E;
   for (int e = threadIdx.x; e < rows * VPR; e += blockDim.x) {
@@ -63,7 +64,7 @@ __device__ __forceinline__ void gather_tile(__nv_bfloat16* dst, const TIn* __res
     const int p = p0 + r;
     __nv_bfloat16* d = dst + r * LD + c * E;
     if (p < g.N) {
-      const int n = natural_index(g, order, p);
+      const int n = permuted ? p : natural_index(g, order, p);
       const uint4 u = __ldg(reinterpret_cast<const uint4*>(head + (int64_t)n * D) + c);
       if constexpr (E == 8) {
         *reinterpret_cast<uint4*>(d) = u;
@@ -89,7 +90,7 @@ __global__ void __launch_bounds__(BLOCK * 2)
                     const TIn* __restrict__ v, const __grid_constant__ Grid g,
                     const int32_t* __restrict__ idx, const int32_t* __restrict__ counts,
                     int k_max, float scale_log2, TIn* __restrict__ out,
-                    int32_t* __restrict__ status) {
+                    int32_t* __restrict__ status, int permuted) {
   constexpr int LD = D + 8;  // padded row: conflict-free ldmatrix
   constexpr int NT = BLOCK / 8;  // n-tiles of S
   constexpr int DT = D / 8;  // n-tiles of O
@@ -104,9 +105,10 @@ __global__ void __launch_bounds__(BLOCK * 2)
   const int order = g.perm[h];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t row = bh * g.NB + i;
-  const TIn* qh = q + bh * (int64_t)g.N * D;
-  const TIn* kh = k + bh * (int64_t)g.N * D;
-  const TIn* vh = v + bh * (int64_t)g.N * D;
+  const int64_t rows_per_head = permuted ? g.Np : g.N;
+  const TIn* qh = q + bh * rows_per_head * D;
+  const TIn* kh = k + bh * rows_per_head * D;
+  const TIn* vh = v + bh * rows_per_head * D;
 
   int cnt = counts != nullptr ? __ldg(counts + row) : k_max;
   if (cnt < 0 || cnt > k_max) {
@@ -115,7 +117,7 @@ __global__ void __launch_bounds__(BLOCK * 2)
   }
   const int32_t* ids = idx + row * k_max;
 
-  gather_tile<TIn, D, LD>(Qs, qh, g, order, i * BLOCK, BLOCK);
+  gather_tile<TIn, D, LD>(Qs, qh, g, order, i * BLOCK, BLOCK, permuted != 0);
   __syncthreads();
   uint32_t qf[D / 16][4];
 #pragma unroll
@@ -139,8 +141,8 @@ __global__ void __launch_bounds__(BLOCK * 2)
     }
     prev = j;
     __syncthreads();  // previous tiles fully consumed
-    gather_tile<TIn, D, LD>(Ks, kh, g, order, j * BLOCK, BLOCK);
-    gather_tile<TIn, D, LD>(Vs, vh, g, order, j * BLOCK, BLOCK);
+    gather_tile<TIn, D, LD>(Ks, kh, g, order, j * BLOCK, BLOCK, permuted != 0);
+    gather_tile<TIn, D, LD>(Vs, vh, g, order, j * BLOCK, BLOCK, permuted != 0);
     __syncthreads();
 
     float s[NT][4];
@@ -256,7 +258,7 @@ __global__ void __launch_bounds__(BLOCK * 2)
 template <typename TIn, int D, int BLOCK>
 cudaError_t launch_typed(const void* q, const void* k, const void* v, const Grid& g,
                          const int32_t* idx, const int32_t* counts, int k_max, void* out,
-                         int32_t* status, cudaStream_t s) {
+                         int32_t* status, bool permuted, cudaStream_t s) {
   constexpr int LD = D + 8;
   const size_t smem = (size_t)3 * BLOCK * LD * sizeof(__nv_bfloat16);
   static_assert((size_t)BLOCK * D * sizeof(TIn) <= (size_t)2 * BLOCK * LD * 2,
@@ -268,7 +270,8 @@ cudaError_t launch_typed(const void* q, const void* k, const void* v, const Grid
   dim3 grid(g.NB, g.B * g.heads);
   kern<<<grid, BLOCK * 2, smem, s>>>(static_cast<const TIn*>(q), static_cast<const TIn*>(k),
                                      static_cast<const TIn*>(v), g, idx, counts, k_max,
-                                     scale_log2, static_cast<TIn*>(out), status);
+                                     scale_log2, static_cast<TIn*>(out), status,
+                                     permuted ? 1 : 0);
   return cudaGetLastError();
 }
 
@@ -276,10 +279,10 @@ cudaError_t launch_typed(const void* q, const void* k, const void* v, const Grid
 
 cudaError_t launch_attn_mma(const void* q, const void* k, const void* v, pa_dtype dt,
                             const Grid& g, const int32_t* idx, const int32_t* counts, int k_max,
-                            void* out, int32_t* status, cudaStream_t s) {
-#define PARO_A(T, D, BL)                                                              \
-  if (g.d == D && g.block == BL)                                                      \
-    return launch_typed<T, D, BL>(q, k, v, g, idx, counts, k_max, out, status, s);
+                            void* out, int32_t* status, bool permuted, cudaStream_t s) {
+#define PARO_A(T, D, BL)                                                                    \
+  if (g.d == D && g.block == BL)                                                            \
+    return launch_typed<T, D, BL>(q, k, v, g, idx, counts, k_max, out, status, permuted, s);
   if (dt == PA_BF16) {
     PARO_A(__nv_bfloat16, 64, 64)
     PARO_A(__nv_bfloat16, 64, 128)

@@ -139,8 +139,16 @@ __device__ __forceinline__ void copy_tile(uint32_t tile, const __nv_bfloat16* __
   }
 }
 
+// kTma: q, k, v are in the permuted order ([B*heads*N_p, d], as written by
+// pa_reorder): every tile is 128 contiguous rows, loaded with two TMA tiled
+// boxes (one per 64-column half) by one lane.  Otherwise q, k, v are in the
+// natural order and the copy warps gather the rows with cp.async.
+template <bool kTma>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_sm100_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+    attn_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
+                      const __grid_constant__ CUtensorMap map_k,
+                      const __grid_constant__ CUtensorMap map_v,
+                      const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                       const __nv_bfloat16* __restrict__ v, const __grid_constant__ Grid g,
                       const int32_t* __restrict__ idx, const int32_t* __restrict__ counts,
                       int k_max, float scale_log2, __nv_bfloat16* __restrict__ out,
@@ -175,10 +183,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       status != nullptr && *reinterpret_cast<volatile int32_t*>(status) == PA_ERR_TIMEOUT;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(BQ), 32);
+    constexpr uint32_t kLoadArrivals = kTma ? 1 : 32;  // one expect-tx, or one per lane
+    mbar_init(bar(BQ), kLoadArrivals);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar(BK0 + s), 32);
-      mbar_init(bar(BV0 + s), 32);
+      mbar_init(bar(BK0 + s), kLoadArrivals);
+      mbar_init(bar(BV0 + s), kLoadArrivals);
       mbar_init(bar(BKF0 + s), 1);
       mbar_init(bar(BVF0 + s), 1);
     }
@@ -228,11 +237,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------- copies ----
       const bool is_k = warp == kKWarp;
       const __nv_bfloat16* src = is_k ? kh : vh;
+      const CUtensorMap* map = is_k ? &map_k : &map_v;
       const uint32_t ring = base + (is_k ? kOffK : kOffV);
+      const int row0 = (int)(bh * g.Np);  // first row of this head (permuted order)
+      int issued = 0;
       if (n_tiles > 0) {
         if (is_k) {
-          copy_tile(base + kOffQ, qh, g, order, i * kBlock, lane);
-          cp_async_arrive(bar(BQ));
+          if constexpr (kTma) {
+            if (lane == 0) {
+              mbar_arrive_tx(bar(BQ), kTile);
+              tma_load_2d(base + kOffQ, &map_q, 0, row0 + i * kBlock, bar(BQ));
+              tma_load_2d(base + kOffQ + kHalf, &map_q, 64, row0 + i * kBlock, bar(BQ));
+            }
+          } else {
+            copy_tile(base + kOffQ, qh, g, order, i * kBlock, lane);
+            cp_async_arrive(bar(BQ));
+          }
         }
         for (int j = 0; j < n_tiles; ++j) {
           const int s = j % kStages;
@@ -241,10 +261,30 @@ __global__ void __launch_bounds__(kThreads, 1)
               !warp_wait(bar((is_k ? BKF0 : BVF0) + s), ((j / kStages) - 1) & 1, ctl))
             break;
           PARO_T(is_k ? 0 : 2, j);
-          copy_tile(ring + s * kTile, src, g, order, __ldg(ids + j) * kBlock, lane);
-          cp_async_arrive(bar((is_k ? BK0 : BV0) + s));
+          const int kb = __ldg(ids + j);
+          const uint32_t full = bar((is_k ? BK0 : BV0) + s);
+          if constexpr (kTma) {
+            if (lane == 0) {
+              mbar_arrive_tx(full, kTile);
+              tma_load_2d(ring + s * kTile, map, 0, row0 + kb * kBlock, full);
+              tma_load_2d(ring + s * kTile + kHalf, map, 64, row0 + kb * kBlock, full);
+            }
+          } else {
+            copy_tile(ring + s * kTile, src, g, order, kb * kBlock, lane);
+            cp_async_arrive(full);
+          }
+          issued = j + 1;
         }
-        cp_async_wait_all();  // on every path: this warp's copies have landed
+        // on every path this warp's copies have landed before it leaves
+        if constexpr (kTma) {
+          if (lane == 0) {
+            if (is_k) drain_phase(bar(BQ), 0);
+            for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
+              drain_phase(bar((is_k ? BK0 : BV0) + j % kStages), (j / kStages) & 1);
+          }
+        } else {
+          cp_async_wait_all();
+        }
       }
     } else if (warp == kMmaWarp) {
       // -------------------------------------------------------- MMA ----
@@ -443,30 +483,48 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+template <bool kTma>
+cudaError_t launch_typed(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         const void* q, const void* k, const void* v, const Grid& g,
+                         const int32_t* idx, const int32_t* counts, int k_max, void* out,
+                         int32_t* status, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel<kTma>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)kD));
+  dim3 grid(g.NB, g.B * g.heads);
+  attn_sm100_kernel<kTma><<<grid, kThreads, kSmemBytes, s>>>(
+      mq, mk, mv, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+      static_cast<const __nv_bfloat16*>(v), g, idx, counts, k_max, scale_log2,
+      static_cast<__nv_bfloat16*>(out), status);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 bool attn_sm100_supports(pa_dtype dt, const Grid& g) {
-  return dt == PA_BF16 && g.d == kD && g.block == kBlock;
+  return dt == PA_BF16 && g.d == kD && g.block == kBlock &&
+         (int64_t)g.B * g.heads * g.Np < ((int64_t)1 << 31);
 }
 
 cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, pa_dtype dt,
                               const Grid& g, const int32_t* idx, const int32_t* counts,
                               int k_max, const float* qs, const float* ks, const float* vs,
-                              void* out, int32_t* status, cudaStream_t s) {
+                              void* out, int32_t* status, bool permuted, cudaStream_t s) {
   (void)qs;
   (void)ks;
   (void)vs;
   if (!attn_sm100_supports(dt, g)) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-  if (e != cudaSuccess) return e;
-  const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)kD));
-  dim3 grid(g.NB, g.B * g.heads);
-  attn_sm100_kernel<<<grid, kThreads, kSmemBytes, s>>>(
-      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-      static_cast<const __nv_bfloat16*>(v), g, idx, counts, k_max, scale_log2,
-      static_cast<__nv_bfloat16*>(out), status);
-  return cudaGetLastError();
+  CUtensorMap mq{}, mk{}, mv{};
+  if (permuted) {
+    const uint64_t rows = (uint64_t)g.B * g.heads * g.Np;
+    if (!encode_tile_map(&mq, q, rows, kD, 2, 64, kBlock) ||
+        !encode_tile_map(&mk, k, rows, kD, 2, 64, kBlock) ||
+        !encode_tile_map(&mv, v, rows, kD, 2, 64, kBlock))
+      return cudaErrorInvalidValue;
+    return launch_typed<true>(mq, mk, mv, q, k, v, g, idx, counts, k_max, out, status, s);
+  }
+  return launch_typed<false>(mq, mk, mv, q, k, v, g, idx, counts, k_max, out, status, s);
 }
 
 }  // namespace paro

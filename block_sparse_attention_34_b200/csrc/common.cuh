@@ -85,6 +85,8 @@ struct Chunk<float> {
 namespace paro {
 cudaError_t launch_reorder(const void* x, void* xp, pa_dtype dt, const Grid& g, bool inverse,
                            cudaStream_t s);
+cudaError_t launch_reorder_pool(const void* x, void* xp, pa_dtype dt, const Grid& g, float* pool,
+                                cudaStream_t s);
 cudaError_t launch_pool(const void* x, pa_dtype dt, const Grid& g, float* pool, cudaStream_t s);
 cudaError_t launch_score(const float* qp, const float* kp, const Grid& g, float* scores,
                          cudaStream_t s);
@@ -95,5 +97,5 @@ cudaError_t launch_quantize(const void* x, pa_dtype dt, const Grid& g, int8_t* x
                             float* pool, cudaStream_t s);
 cudaError_t launch_attn_mma(const void* q, const void* k, const void* v, pa_dtype dt,
                             const Grid& g, const int32_t* idx, const int32_t* counts, int k_max,
-                            void* out, int32_t* status, cudaStream_t s);
+                            void* out, int32_t* status, bool permuted, cudaStream_t s);
 }  // namespace paro

@@ -47,12 +47,16 @@ __global__ void __launch_bounds__(kThreads) reorder_kernel(const uint4* __restri
   }
 }
 
-// -------------------------------------------------------------- pooling ---
-// One CTA per (permuted block i, head bh): mean of the block's valid rows in
-// fp32.  Thread t owns chunk (t % vpr) of rows t / vpr, + kThreads/vpr, ...
+// ------------------------------------------------- pooling and reorder ---
+// One CTA per (permuted block i, head bh).  Reads the block's token rows
+// once (natural positions from the head's order); optionally writes them
+// contiguously to the permuted tensor xp (pad rows as zeros) and/or the
+// fp32 mean of the block's valid rows to pool.  Thread t owns chunk
+// (t % vpr) of rows t / vpr, + kThreads/vpr, ...
 template <typename T>
 __global__ void __launch_bounds__(kThreads) pool_kernel(const T* __restrict__ x, const __grid_constant__ Grid g,
-                                                        float* __restrict__ pool) {
+                                                        float* __restrict__ pool,
+                                                        T* __restrict__ xp) {
   constexpr int E = Chunk<T>::n;
   extern __shared__ float red[];  // [groups][d]
   const int vpr = g.d / E;
@@ -69,13 +73,22 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(const T* __restrict__ x,
   const int p0 = i * g.block;
   const int valid = min(g.block, g.N - p0);
   const uint4* base = reinterpret_cast<const uint4*>(x + bh * (int64_t)g.N * g.d);
-  for (int r = rg; r < valid; r += groups) {
-    const int n = natural_index(g, order, p0 + r);
-    float f[E];
-    Chunk<T>::unpack(__ldg(base + (int64_t)n * vpr + c), f);
+  uint4* dst = xp != nullptr
+                   ? reinterpret_cast<uint4*>(xp + (bh * (int64_t)g.Np + p0) * g.d)
+                   : nullptr;
+  const int rows = dst != nullptr ? g.block : valid;
+  for (int r = rg; r < rows; r += groups) {
+    uint4 u = make_uint4(0, 0, 0, 0);
+    if (r < valid) u = __ldg(base + (int64_t)natural_index(g, order, p0 + r) * vpr + c);
+    if (dst != nullptr) dst[(int64_t)r * vpr + c] = u;
+    if (pool != nullptr) {
+      float f[E];
+      Chunk<T>::unpack(u, f);
 #pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] += f[e];
+      for (int e = 0; e < E; ++e) acc[e] += f[e];
+    }
   }
+  if (pool == nullptr) return;  // uniform across the CTA
 #pragma unroll
   for (int e = 0; e < E; ++e) red[rg * g.d + c * E + e] = acc[e];
   __syncthreads();
@@ -332,17 +345,23 @@ cudaError_t launch_reorder(const void* x, void* xp, pa_dtype dt, const Grid& g, 
   return cudaGetLastError();
 }
 
-cudaError_t launch_pool(const void* x, pa_dtype dt, const Grid& g, float* pool, cudaStream_t s) {
+cudaError_t launch_reorder_pool(const void* x, void* xp, pa_dtype dt, const Grid& g, float* pool,
+                                cudaStream_t s) {
   const int E = dt == PA_F32 ? 4 : 8;
   const int groups = kThreads / (g.d / E);
   const size_t smem = (size_t)groups * g.d * sizeof(float);
   dim3 grid(g.NB, g.B * g.heads);
   if (dt == PA_F32)
-    pool_kernel<float><<<grid, kThreads, smem, s>>>(static_cast<const float*>(x), g, pool);
+    pool_kernel<float><<<grid, kThreads, smem, s>>>(static_cast<const float*>(x), g, pool,
+                                                    static_cast<float*>(xp));
   else
-    pool_kernel<__nv_bfloat16>
-        <<<grid, kThreads, smem, s>>>(static_cast<const __nv_bfloat16*>(x), g, pool);
+    pool_kernel<__nv_bfloat16><<<grid, kThreads, smem, s>>>(
+        static_cast<const __nv_bfloat16*>(x), g, pool, static_cast<__nv_bfloat16*>(xp));
   return cudaGetLastError();
+}
+
+cudaError_t launch_pool(const void* x, pa_dtype dt, const Grid& g, float* pool, cudaStream_t s) {
+  return launch_reorder_pool(x, nullptr, dt, g, pool, s);
 }
 
 cudaError_t launch_score(const float* qp, const float* kp, const Grid& g, float* scores,

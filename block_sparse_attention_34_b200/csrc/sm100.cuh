@@ -229,6 +229,17 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// A box of a 2D tensor map (columns x, rows y) into shared memory at dst,
+// completing `bar`'s transaction count as the bytes land.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, "
+      "{%2, %3}], [%4];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
 // --- math ---------------------------------------------------------------
 
 __device__ __forceinline__ float ex2(float x) {
@@ -257,5 +268,10 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c) {
 // driver entry point is unavailable or the encode fails.
 bool encode_gather_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                        int elem_bytes, uint32_t box_cols);
+
+// Host: the same matrix with a {box_cols, box_rows} box (tiled loads of
+// contiguous rows).
+bool encode_tile_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                     int elem_bytes, uint32_t box_cols, uint32_t box_rows);
 
 }  // namespace paro

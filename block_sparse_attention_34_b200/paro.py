@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libparo.so")
 
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_TIMEOUT, PA_ERR_DEVICE_CHECK = range(6)
 PA_F32, PA_BF16, PA_I8 = 0, 1, 2
+PA_ATTN_PERMUTED = 1
 STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_CUDA",
                 4: "PA_ERR_TIMEOUT", 5: "PA_ERR_DEVICE_CHECK"}
 ORDER_IDS = {"FHW": 0, "FWH": 1, "HFW": 2, "HWF": 3, "WFH": 4, "WHF": 5}
@@ -53,15 +54,17 @@ def load():
         "pa_last_error": ([], ctypes.c_char_p),
         "pa_num_blocks": ([PaShape], _I),
         "pa_k_for_density": ([_I, ctypes.c_double], _I),
-        "pa_reorder": ([_P, _P, _I, PaShape, _P, _P], _I),
+        "pa_reorder": ([_P, _P, _I, PaShape, _P, _P, _P], _I),
         "pa_inverse_reorder": ([_P, _P, _I, PaShape, _P, _P], _I),
         "pa_block_score": ([_P, _P, _I, PaShape, _P, _P, _P, _P, _P], _I),
         "pa_score_pooled": ([_P, _P, PaShape, _P, _P], _I),
         "pa_select_topk": ([_P, PaShape, _I, _P, _P], _I),
         "pa_compact_mask": ([_P, PaShape, _P, _P, _P], _I),
         "pa_quantize_int8": ([_P, _I, PaShape, _P, _P, _P, _P, _P], _I),
-        "pa_block_sparse_attn": ([_P, _P, _P, _I, PaShape, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P], _I),
-        "pa_block_sparse_attn_mma": ([_P, _P, _P, _I, PaShape, _P, _P, _P, _I, _P, _P, _P], _I),
+        "pa_block_sparse_attn": ([_P, _P, _P, _I, ctypes.c_uint32, PaShape, _P, _P, _P, _I, _P, _P, _P,
+                                  _P, _P, _P], _I),
+        "pa_block_sparse_attn_mma": ([_P, _P, _P, _I, ctypes.c_uint32, PaShape, _P, _P, _P, _I, _P, _P,
+                                      _P], _I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -132,12 +135,18 @@ def k_for_density(nb: int, density: float) -> int:
     return int(load().pa_k_for_density(int(nb), float(density)))
 
 
-def reorder(x, pr: Problem, out=None):
+def reorder(x, pr: Problem, out=None, pool=None, with_pool=False):
+    """Permuted copy [B, heads, N_p, d] of natural-order x; with
+    ``with_pool`` (or a given ``pool`` buffer) also the block means, from
+    the same read: returns (x_perm, pool)."""
     _need_cuda(x)
     out = out if out is not None else torch.empty((pr.B, pr.heads, pr.N_p, pr.d), dtype=x.dtype,
                                                   device=x.device)
-    _check(load().pa_reorder(_ptr(x), _ptr(out), _dtype_code(x), pr.shape, pr.perms_ptr, _stream()))
-    return out
+    if with_pool and pool is None:
+        pool = torch.empty((pr.B, pr.heads, pr.NB, pr.d), dtype=torch.float32, device=x.device)
+    _check(load().pa_reorder(_ptr(x), _ptr(out), _dtype_code(x), pr.shape, pr.perms_ptr,
+                             _ptr(pool), _stream()))
+    return (out, pool) if (with_pool or pool is not None) else out
 
 
 def inverse_reorder(xp, pr: Problem, out=None):
@@ -196,9 +205,10 @@ def quantize_int8(x, pr: Problem, with_pool=False, x_q=None, scales=None, pool=N
 
 
 def block_sparse_attn(q, k, v, pr: Problem, idx, counts=None, scales=None, out=None,
-                      status=None, baseline=False):
+                      status=None, baseline=False, permuted=False):
     """O = block-sparse attention over the kept tiles, natural token order.
 
+    ``permuted``: q, k, v are [B, heads, N_p, d] from :func:`reorder`.
     ``scales`` = (q_scale, k_scale, v_scale) for int8 q/k/v from
     :func:`quantize_int8` (output bf16).  ``baseline=True`` runs the
     mma.sync comparison kernel instead of the tcgen05 one."""
@@ -207,23 +217,28 @@ def block_sparse_attn(q, k, v, pr: Problem, idx, counts=None, scales=None, out=N
     out_dtype = torch.bfloat16 if code == PA_I8 else q.dtype
     out = out if out is not None else torch.empty((pr.B, pr.heads, pr.N, pr.d), dtype=out_dtype, device=q.device)
     k_max = int(idx.shape[-1])
+    flags = PA_ATTN_PERMUTED if permuted else 0
     lib = load()
     if baseline:
-        st = lib.pa_block_sparse_attn_mma(_ptr(q), _ptr(k), _ptr(v), code, pr.shape, pr.perms_ptr,
-                                          _ptr(idx), _ptr(counts), k_max, _ptr(out), _ptr(status),
-                                          _stream())
+        st = lib.pa_block_sparse_attn_mma(_ptr(q), _ptr(k), _ptr(v), code, flags, pr.shape,
+                                          pr.perms_ptr, _ptr(idx), _ptr(counts), k_max, _ptr(out),
+                                          _ptr(status), _stream())
     else:
         qs, ks, vs = scales if scales is not None else (None, None, None)
-        st = lib.pa_block_sparse_attn(_ptr(q), _ptr(k), _ptr(v), code, pr.shape, pr.perms_ptr,
-                                      _ptr(idx), _ptr(counts), k_max, _ptr(qs), _ptr(ks), _ptr(vs),
-                                      _ptr(out), _ptr(status), _stream())
+        st = lib.pa_block_sparse_attn(_ptr(q), _ptr(k), _ptr(v), code, flags, pr.shape,
+                                      pr.perms_ptr, _ptr(idx), _ptr(counts), k_max, _ptr(qs),
+                                      _ptr(ks), _ptr(vs), _ptr(out), _ptr(status), _stream())
     _check(st)
     return out
 
 
-def attention(q, k, v, grid, perms, block, density, int8=False, baseline=False, status=None):
-    """The whole path for one call: pooled block scores -> top-k kept
-    blocks -> block-sparse attention (orders applied inside the kernels).
+def attention(q, k, v, grid, perms, block, density, int8=False, baseline=False, status=None,
+              permuted=True):
+    """The whole path for one call: reorder with block means (one read of
+    q, k, v) -> pooled block scores -> top-k kept blocks -> block-sparse
+    attention over the permuted tiles, stored back in natural order.
+    ``permuted=False`` skips the reorder pass: the block means are taken
+    from the natural layout and the attention kernel gathers token rows.
     Returns (out, idx)."""
     pr = Problem.from_qkv(q, grid, perms, block)
     kk = k_for_density(pr.NB, density)
@@ -234,6 +249,13 @@ def attention(q, k, v, grid, perms, block, density, int8=False, baseline=False, 
         scores = score_pooled(qp, kp, pr)
         idx = select_topk(scores, pr, kk)
         return block_sparse_attn(q8, k8, v8, pr, idx, scales=(qs, ks, vs), status=status), idx
+    if permuted and not baseline:
+        qp, q_pool = reorder(q, pr, with_pool=True)
+        kp, k_pool = reorder(k, pr, with_pool=True)
+        vp = reorder(v, pr)
+        scores = score_pooled(q_pool, k_pool, pr)
+        idx = select_topk(scores, pr, kk)
+        return block_sparse_attn(qp, kp, vp, pr, idx, status=status, permuted=True), idx
     _, _, scores = block_score(q, k, pr)
     idx = select_topk(scores, pr, kk)
     return block_sparse_attn(q, k, v, pr, idx, baseline=baseline, status=status), idx

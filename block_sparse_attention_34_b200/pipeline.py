@@ -1,0 +1,81 @@
+"""One attention call of the path with its device buffers preallocated, so
+that repeated calls (a DiT's layers and denoising steps) launch kernels only.
+
+Launch sequence of :meth:`Pipeline.run` (every step through the C ABI, on the
+current torch stream):
+
+  bf16:  reorder+pool(q), reorder+pool(k), reorder(v)  -- one HBM pass each
+         score_pooled -> select_topk -> block_sparse_attn(permuted tiles)
+  int8:  quantize+pool(q), quantize+pool(k), quantize(v)
+         score_pooled -> select_topk -> block_sparse_attn(int8)
+
+The output is written in natural token order; the inverse reorder is the
+attention kernel's store.
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import paro
+
+
+class Pipeline:
+    def __init__(self, B, heads, grid, d, block, perms, density, dtype=torch.bfloat16,
+                 device="cuda", int8=False, baseline=False):
+        self.pr = paro.Problem(B, heads, grid, d, block, perms)
+        pr = self.pr
+        self.k = paro.k_for_density(pr.NB, density)
+        self.int8 = int8
+        self.baseline = baseline
+        dev = torch.device(device)
+        if int8:
+            self.xq = [torch.empty((B, heads, pr.N_p, d), dtype=torch.int8, device=dev) for _ in range(3)]
+            self.sc = [torch.empty((B, heads, pr.NB), dtype=torch.float32, device=dev) for _ in range(3)]
+        elif not baseline:
+            self.xp = [torch.empty((B, heads, pr.N_p, d), dtype=dtype, device=dev) for _ in range(3)]
+        self.q_pool = torch.empty((B, heads, pr.NB, d), dtype=torch.float32, device=dev)
+        self.k_pool = torch.empty_like(self.q_pool)
+        self.scores = torch.empty((B, heads, pr.NB, pr.NB), dtype=torch.float32, device=dev)
+        self.idx = torch.empty((B, heads, pr.NB, self.k), dtype=torch.int32, device=dev)
+        out_dtype = torch.bfloat16 if int8 else dtype
+        self.out = torch.empty((B, heads, pr.N, d), dtype=out_dtype, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    @property
+    def launches(self) -> int:
+        """Kernel launches of one :meth:`run` (all of them this library's)."""
+        return 5 if self.baseline else 6
+
+    def select(self, q, k, v):
+        pr = self.pr
+        if self.int8:
+            paro.quantize_int8(q, pr, x_q=self.xq[0], scales=self.sc[0], pool=self.q_pool)
+            paro.quantize_int8(k, pr, x_q=self.xq[1], scales=self.sc[1], pool=self.k_pool)
+            paro.quantize_int8(v, pr, x_q=self.xq[2], scales=self.sc[2])
+            paro.score_pooled(self.q_pool, self.k_pool, pr, scores=self.scores)
+        elif self.baseline:
+            paro.block_score(q, k, pr, self.q_pool, self.k_pool, self.scores)
+        else:
+            paro.reorder(q, pr, out=self.xp[0], pool=self.q_pool)
+            paro.reorder(k, pr, out=self.xp[1], pool=self.k_pool)
+            paro.reorder(v, pr, out=self.xp[2])
+            paro.score_pooled(self.q_pool, self.k_pool, pr, scores=self.scores)
+        paro.select_topk(self.scores, pr, self.k, self.idx)
+
+    def attend(self, q, k, v):
+        pr = self.pr
+        if self.int8:
+            paro.block_sparse_attn(*self.xq, pr, self.idx, scales=tuple(self.sc), out=self.out,
+                                   status=self.status)
+        elif self.baseline:
+            paro.block_sparse_attn(q, k, v, pr, self.idx, out=self.out, status=self.status,
+                                   baseline=True)
+        else:
+            paro.block_sparse_attn(*self.xp, pr, self.idx, out=self.out, status=self.status,
+                                   permuted=True)
+
+    def run(self, q, k, v):
+        self.select(q, k, v)
+        self.attend(q, k, v)
+        return self.out

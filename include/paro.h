@@ -80,7 +80,7 @@ typedef struct {
   int32_t B, heads, F, H, W, d, block;
 } pa_shape;
 
-/* Version of this ABI (bumped on any signature change). */
+/* Version of this ABI (bumped on any signature change): 2. */
 PA_API int32_t pa_abi_version(void);
 
 /* Message of the last failed call on this thread ("" if none). */
@@ -95,12 +95,14 @@ PA_API int32_t pa_num_blocks(pa_shape shape);
  * (The pages give the density; the rounding rule is this library's.) */
 PA_API int32_t pa_k_for_density(int32_t nb, double density);
 
-/* Step 1 standalone (PAROAttention review, key_machinery: per-head
- * permutation among the six axis orders).  x [B,heads,N,d] natural ->
- * x_perm [B,heads,N_p,d] permuted, pad rows written as zeros.
- * dtype PA_F32 or PA_BF16 (same for both buffers). */
+/* Step 1 (PAROAttention review, key_machinery: per-head permutation among
+ * the six axis orders).  x [B,heads,N,d] natural -> x_perm [B,heads,N_p,d]
+ * permuted, pad rows written as zeros.  dtype PA_F32 or PA_BF16 (same for
+ * both buffers).  pool, if not NULL, [B,heads,NB,d] float, receives the
+ * mean of each permuted block's valid rows (step 2's summary, as
+ * pa_block_score's q_pool) from the same read of x. */
 PA_API pa_status pa_reorder(const void* x, void* x_perm, pa_dtype dtype, pa_shape shape,
-                     const int8_t* perms, void* stream);
+                            const int8_t* perms, float* pool, void* stream);
 
 /* Step 5 standalone: x_perm [B,heads,N_p,d] permuted -> x [B,heads,N,d]
  * natural; pad rows are dropped. */
@@ -178,9 +180,19 @@ PA_API pa_status pa_quantize_int8(const void* x, pa_dtype dtype, pa_shape shape,
  *   round_half_even(127 P~) and P V runs in int8 with int32
  *   accumulation, scaled by v_scale / 127; the normaliser sums the
  *   unrounded P~.
- * q_scale/k_scale/v_scale are ignored (may be NULL) unless dtype is PA_I8. */
+ * q_scale/k_scale/v_scale are ignored (may be NULL) unless dtype is PA_I8.
+ *
+ * flags: PA_ATTN_PERMUTED when q, k, v are [B,heads,N_p,d] in the permuted
+ * order (pa_reorder's output) instead of [B,heads,N,d] natural.  Then every
+ * tile of a head is 128 contiguous rows and the sm_100a kernel loads it with
+ * TMA tiled boxes; with natural-order inputs the kernel gathers token rows
+ * itself (no extra pass, but gathers feed the tensor cores more slowly).
+ * PA_I8 inputs are always permuted (the flag is implied).  The output is
+ * always natural order. */
+#define PA_ATTN_PERMUTED 1u
+
 PA_API pa_status pa_block_sparse_attn(const void* q, const void* k, const void* v, pa_dtype dtype,
-                               pa_shape shape, const int8_t* perms, const int32_t* idx,
+                               uint32_t flags, pa_shape shape, const int8_t* perms, const int32_t* idx,
                                const int32_t* counts, int32_t k_max, const float* q_scale,
                                const float* k_scale, const float* v_scale, void* out,
                                int32_t* dev_status, void* stream);
@@ -193,7 +205,7 @@ PA_API pa_status pa_block_sparse_attn(const void* q, const void* k, const void* 
  * not take (d = 64, block = 64, or PA_F32).  Same arguments, layouts,
  * ownership and errors as pa_block_sparse_attn, without the INT8 scales. */
 PA_API pa_status pa_block_sparse_attn_mma(const void* q, const void* k, const void* v, pa_dtype dtype,
-                                   pa_shape shape, const int8_t* perms, const int32_t* idx,
+                                   uint32_t flags, pa_shape shape, const int8_t* perms, const int32_t* idx,
                                    const int32_t* counts, int32_t k_max, void* out,
                                    int32_t* dev_status, void* stream);
 

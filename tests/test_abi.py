@@ -34,7 +34,7 @@ def test_exports_every_declared_symbol(lib):
     assert len(names) >= 12
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.pa_abi_version() == 1
+    assert lib.pa_abi_version() == 2
 
 
 def test_k_for_density_matches_oracle(lib):
@@ -64,39 +64,42 @@ def test_host_validation(lib):
     good = paro.PaShape(1, 2, 4, 8, 8, 64, 64)
     keep, pp = perms_of(0, 5)
     # unsupported head dim and block
-    assert lib.pa_reorder(FAKE, FAKE, paro.PA_BF16, paro.PaShape(1, 2, 4, 8, 8, 96, 64), pp, None) == paro.PA_ERR_UNSUPPORTED
-    assert lib.pa_reorder(FAKE, FAKE, paro.PA_BF16, paro.PaShape(1, 2, 4, 8, 8, 64, 32), pp, None) == paro.PA_ERR_UNSUPPORTED
+    assert lib.pa_reorder(FAKE, FAKE, paro.PA_BF16, paro.PaShape(1, 2, 4, 8, 8, 96, 64), pp, None, None) == paro.PA_ERR_UNSUPPORTED
+    assert lib.pa_reorder(FAKE, FAKE, paro.PA_BF16, paro.PaShape(1, 2, 4, 8, 8, 64, 32), pp, None, None) == paro.PA_ERR_UNSUPPORTED
     assert b"block=32" in lib.pa_last_error()
     # malformed shape
-    assert lib.pa_reorder(FAKE, FAKE, paro.PA_BF16, paro.PaShape(1, 0, 4, 8, 8, 64, 64), pp, None) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_reorder(FAKE, FAKE, paro.PA_BF16, paro.PaShape(1, 0, 4, 8, 8, 64, 64), pp, None, None) == paro.PA_ERR_INVALID_ARG
     # wrong dtype for reorder
-    assert lib.pa_reorder(FAKE, FAKE, paro.PA_I8, good, pp, None) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_reorder(FAKE, FAKE, paro.PA_I8, good, pp, None, None) == paro.PA_ERR_INVALID_ARG
     # bad order id
     keep2, bad = perms_of(0, 6)
-    assert lib.pa_reorder(FAKE, FAKE, paro.PA_BF16, good, bad, None) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_reorder(FAKE, FAKE, paro.PA_BF16, good, bad, None, None) == paro.PA_ERR_INVALID_ARG
     assert b"perms[1]=6" in lib.pa_last_error()
     # NULL perms / pointers / misaligned pointers
-    assert lib.pa_reorder(FAKE, FAKE, paro.PA_BF16, good, None, None) == paro.PA_ERR_INVALID_ARG
-    assert lib.pa_reorder(None, FAKE, paro.PA_BF16, good, pp, None) == paro.PA_ERR_INVALID_ARG
-    assert lib.pa_reorder(ctypes.c_void_p(4100), FAKE, paro.PA_BF16, good, pp, None) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_reorder(FAKE, FAKE, paro.PA_BF16, good, None, None, None) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_reorder(None, FAKE, paro.PA_BF16, good, pp, None, None) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_reorder(ctypes.c_void_p(4100), FAKE, paro.PA_BF16, good, pp, None, None) == paro.PA_ERR_INVALID_ARG
     # top-k: k out of range
     assert lib.pa_select_topk(FAKE, good, 0, FAKE, None) == paro.PA_ERR_INVALID_ARG
     assert lib.pa_select_topk(FAKE, good, 5, FAKE, None) == paro.PA_ERR_INVALID_ARG  # NB = 4
     # attention: INT8 without scales; k_max above NB
-    assert lib.pa_block_sparse_attn(FAKE, FAKE, FAKE, paro.PA_I8, paro.PaShape(1, 2, 4, 8, 8, 128, 128),
+    assert lib.pa_block_sparse_attn(FAKE, FAKE, FAKE, paro.PA_I8, 0, paro.PaShape(1, 2, 4, 8, 8, 128, 128),
                                     pp, FAKE, None, 1, None, None, None, FAKE, None, None) == paro.PA_ERR_INVALID_ARG
-    assert lib.pa_block_sparse_attn(FAKE, FAKE, FAKE, paro.PA_BF16, good, pp, FAKE, None, 9,
+    assert lib.pa_block_sparse_attn(FAKE, FAKE, FAKE, paro.PA_BF16, 0, good, pp, FAKE, None, 9,
                                     None, None, None, FAKE, None, None) == paro.PA_ERR_INVALID_ARG
     # INT8 needs the tcgen05 shape
-    assert lib.pa_block_sparse_attn(FAKE, FAKE, FAKE, paro.PA_I8, good, pp, FAKE, None, 2,
+    assert lib.pa_block_sparse_attn(FAKE, FAKE, FAKE, paro.PA_I8, 0, good, pp, FAKE, None, 2,
                                     FAKE, FAKE, FAKE, FAKE, None, None) == paro.PA_ERR_UNSUPPORTED
     # baseline refuses INT8
-    assert lib.pa_block_sparse_attn_mma(FAKE, FAKE, FAKE, paro.PA_I8, good, pp, FAKE, None, 2,
+    assert lib.pa_block_sparse_attn_mma(FAKE, FAKE, FAKE, paro.PA_I8, 0, good, pp, FAKE, None, 2,
                                         FAKE, None, None) == paro.PA_ERR_INVALID_ARG
+    # unknown flag bits
+    assert lib.pa_block_sparse_attn(FAKE, FAKE, FAKE, paro.PA_BF16, 6, good, pp, FAKE, None, 2,
+                                    None, None, None, FAKE, None, None) == paro.PA_ERR_INVALID_ARG
     # too many heads
     many = np.zeros(2000, dtype=np.int8)
     assert lib.pa_reorder(FAKE, FAKE, paro.PA_BF16, paro.PaShape(1, 2000, 4, 8, 8, 64, 64),
-                          many.ctypes.data_as(ctypes.c_void_p), None) == paro.PA_ERR_UNSUPPORTED
+                          many.ctypes.data_as(ctypes.c_void_p), None, None) == paro.PA_ERR_UNSUPPORTED
 
 
 def test_binding_refuses_cpu_tensors(lib):

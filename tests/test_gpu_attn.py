@@ -10,6 +10,7 @@ import torch
 
 from block_sparse_attention_34_b200 import paro
 from block_sparse_attention_34_b200.configs import WORKLOADS
+from block_sparse_attention_34_b200.pipeline import Pipeline
 from block_sparse_attention_34_b200.synth import as_f64
 from oracle import paro_ref as ref
 
@@ -47,15 +48,19 @@ TC_CASES = [
 ]
 
 
-@pytest.mark.parametrize("baseline", [False, True], ids=["tcgen05", "mma_sync"])
+PATHS = {"tcgen05_permuted": dict(permuted=True), "tcgen05_gather": dict(permuted=False),
+         "mma_sync": dict(baseline=True)}
+
+
+@pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("w", TC_CASES, ids=lambda w: w.name)
-def test_topk_pipeline_small(w, baseline):
+def test_topk_pipeline_small(w, path):
     q, k, v, perms = inputs(w)
     pr = problem(w, perms)
     qd, kd, vd = to_dev(q, k, v)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     out, idx = paro.attention(qd, kd, vd, (w.F, w.H, w.W), perms, w.block, w.density,
-                              baseline=baseline, status=status)
+                              status=status, **PATHS[path])
     torch.cuda.synchronize()
     assert status.item() == 0
     idx_h = idx.cpu().numpy()
@@ -63,8 +68,8 @@ def test_topk_pipeline_small(w, baseline):
     compare(out, want)
 
 
-@pytest.mark.parametrize("baseline", [False, True], ids=["tcgen05", "mma_sync"])
-def test_variable_counts_and_edge_rows(baseline):
+@pytest.mark.parametrize("path", list(PATHS))
+def test_variable_counts_and_edge_rows(path):
     """Ragged kept lists (counts), rows that skip their diagonal, an empty
     row (zeros), and the last (partial) block kept by every row."""
     w = custom("edge_1300", 1, 4, 128, (5, 10, 26), 128, "bf16", 1.0, perms=(0, 3, 5, 1))
@@ -86,9 +91,11 @@ def test_variable_counts_and_edge_rows(baseline):
     counts[0, 1, 2] = 0  # empty row -> zeros
     pr = problem(w, perms)
     qd, kd, vd = to_dev(q, k, v)
+    if PATHS[path].get("permuted"):
+        qd, kd, vd = (paro.reorder(x, pr) for x in (qd, kd, vd))
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = paro.block_sparse_attn(qd, kd, vd, pr, torch.from_numpy(idx).cuda(),
-                                 torch.from_numpy(counts).cuda(), status=status, baseline=baseline)
+                                 torch.from_numpy(counts).cuda(), status=status, **PATHS[path])
     torch.cuda.synchronize()
     assert status.item() == 0
     want = ref.attention(as_f64(q), as_f64(k), as_f64(v), (w.F, w.H, w.W), perms, w.block, idx,
@@ -96,17 +103,19 @@ def test_variable_counts_and_edge_rows(baseline):
     compare(out, want)
 
 
-@pytest.mark.parametrize("baseline", [False, True], ids=["tcgen05", "mma_sync"])
-def test_malformed_list_is_reported_not_fatal(baseline):
+@pytest.mark.parametrize("path", list(PATHS))
+def test_malformed_list_is_reported_not_fatal(path):
     w = custom("bad_list", 1, 2, 128, (4, 8, 16), 128, "bf16", 1.0, perms=(0, 5))
     q, k, v, perms = inputs(w)
     pr = problem(w, perms)
     qd, kd, vd = to_dev(q, k, v)
+    if PATHS[path].get("permuted"):
+        qd, kd, vd = (paro.reorder(x, pr) for x in (qd, kd, vd))
     idx = torch.tensor([[[[0, 1], [1, 1], [2, 3], [0, 9]], [[0, 1], [1, 0], [2, 3], [3, 2]]]],
                        dtype=torch.int32, device="cuda")  # repeats, out of range, descending
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = torch.full((1, 2, w.N, w.d), 7.0, dtype=torch.bfloat16, device="cuda")
-    paro.block_sparse_attn(qd, kd, vd, pr, idx, out=out, status=status, baseline=baseline)
+    paro.block_sparse_attn(qd, kd, vd, pr, idx, out=out, status=status, **PATHS[path])
     torch.cuda.synchronize()
     assert status.item() == paro.PA_ERR_DEVICE_CHECK
     # the well-formed rows are still right
@@ -157,21 +166,24 @@ def sampled_rows(w, n, seed):
 
 @pytest.mark.parametrize("density", [0.15, 1.0])
 def test_720p_full_size_sampled(c720, density):
+    """The bench's launch sequence (Pipeline) on the full 720p-shaped layer."""
     w, q, k, v, perms = c720
-    pr = problem(w, perms)
-    qd, kd, vd = to_dev(q, k, v)
-    _, _, s = paro.block_score(qd, kd, pr)
-    kk = paro.k_for_density(pr.NB, density)
-    assert kk == ref.k_for_density(pr.NB, density)
-    idx = paro.select_topk(s, pr, kk)
-    status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    out = paro.block_sparse_attn(qd, kd, vd, pr, idx, status=status)
+    pipe = Pipeline(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, perms, density)
+    assert pipe.k == ref.k_for_density(w.NB, density)
+    qkv = to_dev(q, k, v)
+    out = pipe.run(*qkv)
     torch.cuda.synchronize()
-    assert status.item() == 0
-    idx_h = idx.cpu().numpy()
+    assert pipe.status.item() == 0
+    idx_h = pipe.idx.cpu().numpy()
     if density < 1.0:
         # the kept lists are the oracle's top-k of the same fp32 scores
-        assert (idx_h == ref.select_topk(s.cpu().double().numpy(), kk)).all()
+        assert (idx_h == ref.select_topk(pipe.scores.cpu().double().numpy(), pipe.k)).all()
+        # and the scores are the oracle's pooled scores (sampled heads)
+        for hh in (0, w.heads - 1):
+            _, _, s_ref = ref.pooled_scores(as_f64(q[:, hh:hh + 1]), as_f64(k[:, hh:hh + 1]),
+                                            (w.F, w.H, w.W), perms[hh:hh + 1], w.block)
+            got = pipe.scores[:, hh:hh + 1].cpu().double().numpy()
+            assert np.abs(got - s_ref).max() < 1e-4 * max(1.0, np.abs(s_ref).max())
     rows = sampled_rows(w, 192 if density < 1.0 else 48, seed=11)
     want = ref.attention_rows(as_f64(q), as_f64(k), as_f64(v), (w.F, w.H, w.W), perms, w.block,
                               idx_h, rows)

@@ -41,6 +41,12 @@ def test_reorder_bit_exact(w):
     got = xp.cpu()
     got = got.numpy() if got.dtype == torch.float32 else got.view(torch.int16).numpy()
     assert (got == want).all()
+    # the fused block means from the same read
+    xp2, pool = paro.reorder(qd, pr, with_pool=True)
+    assert torch.equal(xp2, xp)
+    oq = ref.block_pool(ref.reorder(q.double().numpy(), (w.F, w.H, w.W), perms, w.block),
+                        w.N, w.block)
+    assert np.abs(pool.cpu().double().numpy() - oq).max() < 1e-5
     back = paro.inverse_reorder(xp, pr).cpu()
     assert torch.equal(back.view(torch.int16) if back.dtype == torch.bfloat16 else back,
                        q.view(torch.int16) if q.dtype == torch.bfloat16 else q)
