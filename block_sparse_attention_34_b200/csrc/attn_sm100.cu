@@ -17,11 +17,11 @@
 //              running max, row sum and O accumulator -- an exact split of
 //              the row's kept keys into two disjoint sets -- merged once at
 //              the end: O = (O_A 2^(m_A-m) + O_B 2^(m_B-m)) /
-//              (l_A 2^(m_A-m) + l_B 2^(m_B-m)).  The two groups share the
-//              SM's sub-cores, so the exponentials of one overlap the TMEM
-//              reads and max of the other.  P (bf16) goes back into the
-//              group's S columns of tensor memory and feeds the P V MMA from
-//              there;
+//              (l_A 2^(m_A-m) + l_B 2^(m_B-m)).  The groups take turns on
+//              the exponential units (tile j's exponentials start when tile
+//              j-1's are done), so each group's exponentials overlap the
+//              other group's MMAs.  P (bf16) goes back into the group's S
+//              columns of tensor memory and feeds the P V MMA from there;
 //   warp 8     allocates TMEM; one lane issues every tcgen05.mma and commit;
 //   warp 9     gathers Q, then K tiles; warp 10 gathers V tiles.  Each token
 //              row is 256 contiguous bytes at its natural position (the
@@ -92,7 +92,7 @@ constexpr uint32_t kOffV = kOffK + kStages * kTile;  // kStages stages
 constexpr uint32_t kSmemBytes = kOffV + kStages * kTile;  // 232,448 B = 227 KB
 constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold (factor 256)
 constexpr int kRegsLaunch = 168;     // 65,536 / 384 rounded down to a multiple of 8
-constexpr int kRegsSoftmax = 200, kRegsAux = 72;
+constexpr int kRegsSoftmax = 200, kRegsAux = 56;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsAux <= kThreads * kRegsLaunch, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;
@@ -107,7 +107,8 @@ enum : uint32_t {
   BP0 = 15,   // P of group written (2)
   BDRAIN = 17,
   BM = 18,
-  NBAR = 19
+  BE0 = 19,   // exponential phase of group done (2)
+  NBAR = 21
 };
 static_assert(NBAR * 8 <= kOffSlot, "barrier region");
 static_assert(kOffMerge + 2 * 2 * 128 * 4 <= kSmall, "merge region");
@@ -197,6 +198,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar(BDRAIN), 1);
     mbar_init(bar(BM), 2 * kGroupThreads);
+    mbar_init(bar(BE0), kGroupThreads);
+    mbar_init(bar(BE0 + 1), kGroupThreads);
     *abort_flag = 0;
     *bad_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -387,6 +390,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         l *= alpha;
         if (need) m_used = mx;
       }
+      // ping-pong: the exponentials of tile j start once those of tile j-1
+      // (the other group) are done, so the two groups take turns on the
+      // SM's exponential units and each group's exponentials overlap the
+      // other group's MMAs instead of competing with them
+      if (j >= 1 && !warp_wait(bar(BE0 + (grp ^ 1)), ((j - 1) >> 1) & 1, ctl)) { ok = false; break; }
       // P = 2^(s*scale - m) packed as bf16 pairs into the first 64 columns
       // of the group's S region; row sum in 8 independent chains
       const float neg_m = -m_used;
@@ -407,6 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st32(lane_addr + s_col + h2 * 32, pk);
       }
+      mbar_arrive(bar(BE0 + grp));
       l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
       if (lane == 0 && quarter == 0) PARO_T(9 + 4 * grp, j);
       tc_fence_before();
