@@ -91,9 +91,6 @@ constexpr uint32_t kOffK = kOffQ + kTile;            // kStages stages
 constexpr uint32_t kOffV = kOffK + kStages * kTile;  // kStages stages
 constexpr uint32_t kSmemBytes = kOffV + kStages * kTile;  // 232,448 B = 227 KB
 constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold (factor 256)
-constexpr int kRegsLaunch = 168;     // 65,536 / 384 rounded down to a multiple of 8
-constexpr int kRegsSoftmax = 200, kRegsAux = 56;
-static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsAux <= kThreads * kRegsLaunch, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;
 
@@ -230,12 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const __nv_bfloat16* kh = k + bh * (int64_t)g.N * kD;
   const __nv_bfloat16* vh = v + bh * (int64_t)g.N * kD;
 
-  // registers: launched at 168 per thread (384 x 168 = 64,512); the two
-  // softmax warpgroups take 200, the MMA / copy / check warpgroup 56
-  // (2 x 128 x 200 + 128 x 56 = 58,368 <= 64,512), and every warpgroup
-  // returns to 168 before the common exit
   if (warp >= 8) {
-    regs_dec<kRegsAux>();
     if (warp == kKWarp || warp == kVWarp) {
       // ---------------------------------------------------- copies ----
       const bool is_k = warp == kKWarp;
@@ -335,10 +327,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_phase(bar(BDRAIN), 0);
       }
     }
-    __syncwarp();  // setmaxnreg is warp-aligned: reconverge after the lane-0 roles
-    regs_inc<kRegsLaunch>();
+    __syncwarp();  // reconverge after the lane-0 roles
   } else {
-    regs_inc<kRegsSoftmax>();
     // ------------------------------------------------------ softmax ----
     const int grp = warp >> 2;  // 0: even tiles, 1: odd tiles
     const int quarter = warp & 3;
@@ -354,21 +344,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!warp_wait(bar(BS0 + grp), t & 1, ctl)) { ok = false; break; }
       if (lane == 0 && quarter == 0) PARO_T(6 + 4 * grp, j);
       tc_fence_after();
-      uint32_t sr[128];
-      tmem_ld128(lane_addr + s_col, sr);
-      if (lane == 0 && quarter == 0) PARO_T(7 + 4 * grp, j);
       const int kb = __ldg(ids + j);
       const int valid = g.N - kb * kBlock;  // keys of this block that exist
-      if (valid < kBlock) {  // only the ragged last block (warp-uniform)
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
-      }
+      // pass 1: row max, 64 columns at a time (8 independent chains)
       float mp[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) mp[u] = __uint_as_float(sr[u]);
+      for (int u = 0; u < 8; ++u) mp[u] = -INFINITY;
 #pragma unroll
-      for (int c = 8; c < 128; ++c) mp[c & 7] = fmaxf(mp[c & 7], __uint_as_float(sr[c]));
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t sr[64];
+        tmem_ld64(lane_addr + s_col + h2 * 64, sr);
+        if (valid < kBlock) {  // only the ragged last block (warp-uniform)
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (h2 * 64 + c >= valid) sr[c] = __float_as_uint(-INFINITY);
+        }
+#pragma unroll
+        for (int c = 0; c < 64; ++c) mp[c & 7] = fmaxf(mp[c & 7], __uint_as_float(sr[c]));
+      }
+      if (lane == 0 && quarter == 0) PARO_T(7 + 4 * grp, j);
       const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
                              fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) *
                        scale_log2;
@@ -401,14 +395,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       float rs[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) rs[u] = 0.f;
+      // pass 2: S re-read 64 columns at a time (P of columns 0..63 lands in
+      // S columns 0..31, already consumed; columns 64..127 stay intact)
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t sr[64];
+        tmem_ld64(lane_addr + s_col + h2 * 64, sr);
+        if (valid < kBlock) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (h2 * 64 + c >= valid) sr[c] = __float_as_uint(-INFINITY);
+        }
         uint32_t pk[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const int e = h2 * 64 + 2 * c;
-          const float e0 = ex2(fmaf(__uint_as_float(sr[e]), scale_log2, neg_m));
-          const float e1 = ex2(fmaf(__uint_as_float(sr[e + 1]), scale_log2, neg_m));
+          const float e0 = ex2(fmaf(__uint_as_float(sr[2 * c]), scale_log2, neg_m));
+          const float e1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), scale_log2, neg_m));
           rs[(2 * c) & 7] += e0;
           rs[(2 * c + 1) & 7] += e1;
           pk[c] = pack_bf16(e0, e1);
@@ -480,7 +482,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-    regs_dec<kRegsLaunch>();
   }
 
   tc_fence_before();
