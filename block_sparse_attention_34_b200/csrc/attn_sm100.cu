@@ -11,36 +11,36 @@
 // tokens.
 //
 // One CTA per (query block, head); 12 warps with fixed roles:
-//   warps 0-3  softmax A: the even-numbered kept tiles (0, 2, 4, ...);
-//   warps 4-7  softmax B: the odd-numbered kept tiles.  A thread owns one
-//              row of the 128-row tile (TMEM lane).  Each group keeps its own
-//              running max, row sum and O accumulator -- an exact split of
-//              the row's kept keys into two disjoint sets -- merged once at
-//              the end: O = (O_A 2^(m_A-m) + O_B 2^(m_B-m)) /
-//              (l_A 2^(m_A-m) + l_B 2^(m_B-m)).  The groups take turns on
-//              the exponential units (tile j's exponentials start when tile
-//              j-1's are done), so each group's exponentials overlap the
-//              other group's MMAs.  P (bf16) goes back into the group's S
-//              columns of tensor memory and feeds the P V MMA from there;
+//   warps 0-7  softmax, two warpgroups splitting every tile by columns: warp
+//              w owns rows 32*(w%4) .. +31 (its TMEM lane quarter; a warp
+//              may only touch its own quarter) and key columns
+//              64*(w/4) .. +63.  A thread reads its 64 scores from TMEM, the
+//              two halves of a row exchange their maxima through shared
+//              memory, and each thread writes its 64 probabilities (bf16
+//              pairs) into its half of the tile's P region of tensor memory,
+//              from which the P V MMA reads them; when a row's max grows by
+//              more than 2^8 the thread rescales its 64 columns of O;
 //   warp 8     allocates TMEM; one lane issues every tcgen05.mma and commit;
-//   warp 9     gathers Q, then K tiles; warp 10 gathers V tiles.  Each token
-//              row is 256 contiguous bytes at its natural position (the
-//              head's axis order is applied in the address: no reordered
-//              copy of any tensor exists in HBM); 16 lanes copy a row with
-//              16-byte cp.async straight into the 128-byte-swizzled operand
-//              layout, and each lane's arrival on the stage's mbarrier fires
-//              when its copies land, so several tiles are in flight;
+//   warp 9     loads Q, then K tiles; warp 10 loads V tiles.  With inputs in
+//              the permuted order (pa_reorder) every tile is 128 contiguous
+//              rows: one lane issues two TMA tiled boxes (one per 64-column
+//              half) into the 128-byte-swizzled operand layout.  With
+//              natural-order inputs the warp gathers the token rows itself
+//              (16-byte cp.async, 16 lanes per 256-byte row, natural
+//              positions from the head's axis order) and each lane's arrival
+//              on the stage's mbarrier fires when its copies land;
 //   warp 11    validates the kept list, then idles.
-// Tensor memory (512 columns): S_A/P_A, S_B/P_B at columns 0 and 128, O_A,
-// O_B at 256 and 384.  Shared memory: Q (32 KB) and three-stage K and V
-// rings (6 x 32 KB) in the canonical K-major / MN-major SWIZZLE_128B
-// layouts the MMA descriptors name.
+// Tensor memory (512 columns): S double buffer at 0 and 128, P double
+// buffer (64 columns each) at 256 and 320, O at 384.  Shared memory: Q
+// (32 KB) and three-stage K and V rings (6 x 32 KB) in the canonical
+// K-major / MN-major SWIZZLE_128B layouts the MMA descriptors name.
 //
-// MMA issue order QK(0), QK(1), PV(0), QK(2), PV(1), ...: tcgen05 operations
-// of one thread complete in order, so S(j) being ready implies P V(j-2) --
-// the last reader of that group's P columns and writer of its O -- has
-// completed; a K stage is refilled once its QK^T completes, a V stage once
-// its P V completes.  Every mbarrier wait is bounded (about one second of
+// MMA issue order QK(0), QK(1), PV(0), QK(2), PV(1), ...: QK^T of tile j+1
+// runs on the tensor core while the softmax warps turn S(j) into P(j).
+// tcgen05 operations of one thread complete in order, so S(j) being ready
+// implies P V(j-2), the previous reader of P(j)'s buffer, has completed.  A
+// K stage is refilled once its QK^T completes, a V stage once its P V
+// completes.  Every mbarrier wait is bounded (about one second of
 // %globaltimer); on expiry the kernel records PA_ERR_TIMEOUT in the device
 // status word, each role leaves its loop, in-flight copies and MMAs are
 // drained and TMEM is released before the CTA exits.
@@ -77,14 +77,14 @@ constexpr int kKWarp = 9;
 constexpr int kVWarp = 10;
 constexpr int kCheckWarp = 11;
 constexpr int kThreads = 12 * 32;  // 384
-constexpr int kGroupThreads = 128;
+constexpr int kSoftThreads = 256;
 constexpr uint32_t kTile = kBlock * kD * 2;  // 32 KB
 constexpr uint32_t kHalf = kBlock * 128;     // 16 KB: 64 columns
-// small region first: mbarriers, TMEM slot and flags, merge buffers
-// [m, l][group][128 rows] float; the operand tiles start 1024-aligned
+// small region first: mbarriers, TMEM slot and flags, the row-max exchange
+// [2 tiles][2 halves][128 rows] float; the operand tiles start 1024-aligned
 constexpr uint32_t kOffBar = 0;
-constexpr uint32_t kOffSlot = 192;
-constexpr uint32_t kOffMerge = 256;
+constexpr uint32_t kOffSlot = 256;
+constexpr uint32_t kOffXmax = 512;
 constexpr uint32_t kSmall = 3072;
 constexpr uint32_t kOffQ = kSmall;
 constexpr uint32_t kOffK = kOffQ + kTile;            // kStages stages
@@ -92,7 +92,7 @@ constexpr uint32_t kOffV = kOffK + kStages * kTile;  // kStages stages
 constexpr uint32_t kSmemBytes = kOffV + kStages * kTile;  // 232,448 B = 227 KB
 constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold (factor 256)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColO = 256;
+constexpr uint32_t kColS = 0, kColP = 256, kColO = 384;
 
 enum : uint32_t {
   BQ = 0,
@@ -100,15 +100,17 @@ enum : uint32_t {
   BV0 = 4,    // V stage full (3)
   BKF0 = 7,   // K stage free (3)
   BVF0 = 10,  // V stage free (3)
-  BS0 = 13,   // S of group ready (2)
-  BP0 = 15,   // P of group written (2)
-  BDRAIN = 17,
-  BM = 18,
-  BE0 = 19,   // exponential phase of group done (2)
-  NBAR = 21
+  BS0 = 13,   // S(j) ready (2, by j & 1)
+  BSF0 = 15,  // S(j) read by both halves (2)
+  BP0 = 17,   // P(j) written by both halves (2)
+  BPV0 = 19,  // P V(j) complete (2)
+  BX0 = 21,   // row maxima of tile j exchanged (2)
+  BDRAIN = 23,
+  BL = 24,    // row sums exchanged at the end
+  NBAR = 25
 };
 static_assert(NBAR * 8 <= kOffSlot, "barrier region");
-static_assert(kOffMerge + 2 * 2 * 128 * 4 <= kSmall, "merge region");
+static_assert(kOffXmax + 2 * 2 * 128 * 4 <= kSmall, "exchange region");
 
 // One warp copies a 128 x 128 bf16 tile whose row r is the token at
 // permuted position p0 + r of head `head` (rows past N zero-filled).  Lane l
@@ -164,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOffSlot);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile uint32_t* bad_flag = tmem_slot + 2;
-  float* merge = reinterpret_cast<float*>(gbase + kOffMerge);  // [m|l][group][row]
+  float* xmax = reinterpret_cast<float*>(gbase + kOffXmax);  // [tile & 1][half][row]
   auto bar = [&](uint32_t slot) { return base + kOffBar + slot * 8u; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -191,12 +193,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(BS0 + b), 1);
-      mbar_init(bar(BP0 + b), kGroupThreads);
+      mbar_init(bar(BSF0 + b), kSoftThreads);
+      mbar_init(bar(BP0 + b), kSoftThreads);
+      mbar_init(bar(BPV0 + b), 1);
+      mbar_init(bar(BX0 + b), kSoftThreads);
     }
     mbar_init(bar(BDRAIN), 1);
-    mbar_init(bar(BM), 2 * kGroupThreads);
-    mbar_init(bar(BE0), kGroupThreads);
-    mbar_init(bar(BE0 + 1), kGroupThreads);
+    mbar_init(bar(BL), kSoftThreads);
     *abort_flag = 0;
     *bad_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -288,25 +291,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t id_pv = idesc_bf16(kBlock, kD, true);
         bool ok = wait_phase(bar(BQ), 0, ctl);
         fence_async_smem();  // cp.async (generic proxy) writes -> MMA operand reads
-        auto issue_pv = [&](int jp) -> bool {
-          const int b = jp & 1, s = jp % kStages;
-          if (!wait_phase(bar(BP0 + b), (jp >> 1) & 1, ctl)) return false;
-          if (!wait_phase(bar(BV0 + s), (jp / kStages) & 1, ctl)) return false;
-          fence_async_smem();
-          tc_fence_after();
-          const uint32_t va = base + kOffV + s * kTile;
-#pragma unroll
-          for (int kk = 0; kk < kBlock / 16; ++kk)
-            mma_f16_ts(tmem + kColO + b * 128, tmem + kColS + b * 128 + kk * 8,
-                       sw128_desc(va + kk * 16 * 128, kHalf, 1024), id_pv,
-                       (jp >= 2 || kk > 0) ? 1u : 0u);
-          mma_commit(bar(BVF0 + s));
-          PARO_T(5, jp);
-          return true;
-        };
-        for (int j = 0; ok && j < n_tiles; ++j) {
+        // QK^T of tile j into S buffer j & 1: needs K(j) and, for j >= 2,
+        // both halves to have read S(j-2) out of that buffer
+        auto issue_qk = [&](int j) -> bool {
           const int b = j & 1, s = j % kStages;
-          if (!wait_phase(bar(BK0 + s), (j / kStages) & 1, ctl)) { ok = false; break; }
+          if (!wait_phase(bar(BK0 + s), (j / kStages) & 1, ctl)) return false;
+          if (j >= 2 && !wait_phase(bar(BSF0 + b), ((j - 2) >> 1) & 1, ctl)) return false;
           fence_async_smem();
           tc_fence_after();
           const uint32_t ka = base + kOffK + s * kTile;
@@ -319,9 +309,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(bar(BS0 + b));
           mma_commit(bar(BKF0 + s));
           PARO_T(4, j);
-          if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+          return true;
+        };
+        // O += P(j) V(j): P from tensor memory (bf16 pairs), V from the ring
+        auto issue_pv = [&](int j) -> bool {
+          const int b = j & 1, s = j % kStages;
+          if (!wait_phase(bar(BP0 + b), (j >> 1) & 1, ctl)) return false;
+          if (!wait_phase(bar(BV0 + s), (j / kStages) & 1, ctl)) return false;
+          fence_async_smem();
+          tc_fence_after();
+          const uint32_t va = base + kOffV + s * kTile;
+#pragma unroll
+          for (int kk = 0; kk < kBlock / 16; ++kk)
+            mma_f16_ts(tmem + kColO, tmem + kColP + b * 64 + kk * 8,
+                       sw128_desc(va + kk * 16 * 128, kHalf, 1024), id_pv,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(BPV0 + b));
+          mma_commit(bar(BVF0 + s));
+          PARO_T(5, j);
+          return true;
+        };
+        ok = ok && issue_qk(0);
+        for (int j = 0; ok && j < n_tiles; ++j) {
+          if (j + 1 < n_tiles && !issue_qk(j + 1)) { ok = false; break; }
+          if (!issue_pv(j)) { ok = false; break; }
         }
-        if (ok) issue_pv(n_tiles - 1);
         // drain: every MMA issued above has completed once this commit fires
         mma_commit(bar(BDRAIN));
         drain_phase(bar(BDRAIN), 0);
@@ -330,151 +342,118 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();  // reconverge after the lane-0 roles
   } else {
     // ------------------------------------------------------ softmax ----
-    const int grp = warp >> 2;  // 0: even tiles, 1: odd tiles
+    const int hc = warp >> 2;     // column half: keys 64*hc .. 64*hc+63
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // tile row == TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t s_col = kColS + grp * 128, o_col = kColO + grp * 128;
-    float m_used = -INFINITY, l = 0.f;
+    float m_used = -INFINITY, l = 0.f;  // m_used is the same in both halves
     bool ok = true;
-    int t = 0;  // this group's tile counter
-    for (int j = grp; j < n_tiles; j += 2, ++t) {
-      // S(j) ready also means P V(j-2) -- the previous reader of these P
-      // columns and writer of this group's O -- has completed
-      if (!warp_wait(bar(BS0 + grp), t & 1, ctl)) { ok = false; break; }
-      if (lane == 0 && quarter == 0) PARO_T(6 + 4 * grp, j);
+    for (int j = 0; j < n_tiles; ++j) {
+      const int b = j & 1;
+      if (!warp_wait(bar(BS0 + b), (j >> 1) & 1, ctl)) { ok = false; break; }
+      if (lane == 0 && quarter == 0) PARO_T(6 + 4 * hc, j);
       tc_fence_after();
-      const int kb = __ldg(ids + j);
-      const int valid = g.N - kb * kBlock;  // keys of this block that exist
-      // pass 1: row max, 64 columns at a time (8 independent chains)
+      uint32_t sr[64];
+      tmem_ld64(lane_addr + kColS + b * 128 + hc * 64, sr);
+      tc_fence_before();
+      mbar_arrive(bar(BSF0 + b));  // S buffer b may take QK^T(j+2)
+      if (lane == 0 && quarter == 0) PARO_T(7 + 4 * hc, j);
+      const int valid = g.N - __ldg(ids + j) * kBlock - hc * 64;  // existing keys of my half
+      if (valid < 64) {  // only the ragged last block (warp-uniform)
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
+      }
       float mp[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) mp[u] = -INFINITY;
+      for (int u = 0; u < 8; ++u) mp[u] = __uint_as_float(sr[u]);
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        uint32_t sr[64];
-        tmem_ld64(lane_addr + s_col + h2 * 64, sr);
-        if (valid < kBlock) {  // only the ragged last block (warp-uniform)
-#pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (h2 * 64 + c >= valid) sr[c] = __float_as_uint(-INFINITY);
-        }
-#pragma unroll
-        for (int c = 0; c < 64; ++c) mp[c & 7] = fmaxf(mp[c & 7], __uint_as_float(sr[c]));
-      }
-      if (lane == 0 && quarter == 0) PARO_T(7 + 4 * grp, j);
-      const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) *
-                       scale_log2;
-      if (lane == 0 && quarter == 0) PARO_T(8 + 4 * grp, j);
+      for (int c = 8; c < 64; ++c) mp[c & 7] = fmaxf(mp[c & 7], __uint_as_float(sr[c]));
+      const float mh = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+      float* xm = xmax + b * 256;
+      xm[hc * 128 + r] = mh;
+      mbar_arrive(bar(BX0 + b));
+      if (!all_wait(bar(BX0 + b), (j >> 1) & 1, ctl)) { ok = false; break; }
+      const float mx = fmaxf(mh, xm[(hc ^ 1) * 128 + r]) * scale_log2;
+      if (lane == 0 && quarter == 0) PARO_T(8 + 4 * hc, j);
       // lazy rescale: keep the reference max unless the row max grew by
       // more than 2^8 (exact either way: O and l share the reference)
-      const bool need = t == 0 ? false : (mx > m_used + kRescaleLog2);
-      if (t == 0) m_used = mx == -INFINITY ? 0.f : mx;
+      const bool need = j == 0 ? false : (mx > m_used + kRescaleLog2);
+      if (j == 0) m_used = mx == -INFINITY ? 0.f : mx;
       if (__any_sync(0xffffffffu, need)) {
+        // O holds P V up to tile j-1 once that MMA completed
+        if (!warp_wait(bar(BPV0 + ((j - 1) & 1)), ((j - 1) >> 1) & 1, ctl)) { ok = false; break; }
+        tc_fence_after();
         const float alpha = need ? ex2(m_used - mx) : 1.f;
 #pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 32) {
+        for (int c0 = 0; c0 < 64; c0 += 32) {
           uint32_t orr[32];
-          tmem_ld32(lane_addr + o_col + c0, orr);
+          tmem_ld32(lane_addr + kColO + hc * 64 + c0, orr);
 #pragma unroll
           for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
-          tmem_st32(lane_addr + o_col + c0, orr);
+          tmem_st32(lane_addr + kColO + hc * 64 + c0, orr);
         }
         l *= alpha;
         if (need) m_used = mx;
       }
-      // ping-pong: the exponentials of tile j start once those of tile j-1
-      // (the other group) are done, so the two groups take turns on the
-      // SM's exponential units and each group's exponentials overlap the
-      // other group's MMAs instead of competing with them
-      if (j >= 1 && !warp_wait(bar(BE0 + (grp ^ 1)), ((j - 1) >> 1) & 1, ctl)) { ok = false; break; }
-      // P = 2^(s*scale - m) packed as bf16 pairs into the first 64 columns
-      // of the group's S region; row sum in 8 independent chains
+      // P = 2^(s*scale - m) as bf16 pairs into my half of P buffer b (free:
+      // S(j) ready means P V(j-2) completed); row sum in 8 chains
       const float neg_m = -m_used;
       float rs[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) rs[u] = 0.f;
-      // pass 2: S re-read 64 columns at a time (P of columns 0..63 lands in
-      // S columns 0..31, already consumed; columns 64..127 stay intact)
+      uint32_t pk[32];
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        uint32_t sr[64];
-        tmem_ld64(lane_addr + s_col + h2 * 64, sr);
-        if (valid < kBlock) {
-#pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (h2 * 64 + c >= valid) sr[c] = __float_as_uint(-INFINITY);
-        }
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float e0 = ex2(fmaf(__uint_as_float(sr[2 * c]), scale_log2, neg_m));
-          const float e1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), scale_log2, neg_m));
-          rs[(2 * c) & 7] += e0;
-          rs[(2 * c + 1) & 7] += e1;
-          pk[c] = pack_bf16(e0, e1);
-        }
-        tmem_st32(lane_addr + s_col + h2 * 32, pk);
+      for (int c = 0; c < 32; ++c) {
+        const float e0 = ex2(fmaf(__uint_as_float(sr[2 * c]), scale_log2, neg_m));
+        const float e1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), scale_log2, neg_m));
+        rs[(2 * c) & 7] += e0;
+        rs[(2 * c + 1) & 7] += e1;
+        pk[c] = pack_bf16(e0, e1);
       }
-      mbar_arrive(bar(BE0 + grp));
+      tmem_st32(lane_addr + kColP + b * 64 + hc * 32, pk);
       l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
-      if (lane == 0 && quarter == 0) PARO_T(9 + 4 * grp, j);
+      if (lane == 0 && quarter == 0) PARO_T(9 + 4 * hc, j);
       tc_fence_before();
-      mbar_arrive(bar(BP0 + grp));
+      mbar_arrive(bar(BP0 + b));
     }
-    // ---- merge the two groups and store (group g writes columns 64g..)
+    // ---- epilogue: add the two halves' row sums, then each half writes
+    // O / l for its 64 columns at the natural position of the row's token
     const int p = i * kBlock + r;
     __nv_bfloat16* orow = p < g.N ? out + (bh * (int64_t)g.N + natural_index(g, order, p)) * kD
                                   : nullptr;
     if (run && cnt == 0) {
       if (orow != nullptr)
         for (int c = 0; c < 8; ++c)
-          reinterpret_cast<uint4*>(orow + grp * 64)[c] = make_uint4(0, 0, 0, 0);
+          reinterpret_cast<uint4*>(orow + hc * 64)[c] = make_uint4(0, 0, 0, 0);
     } else if (ok && n_tiles > 0) {
-      const bool has_b = n_tiles >= 2;
-      merge[(0 * 2 + grp) * 128 + r] = m_used;
-      merge[(1 * 2 + grp) * 128 + r] = l;
-      mbar_arrive(bar(BM));
-      bool okm = all_wait(bar(BM), 0, ctl);
-      float fa = 0.f, fb = 0.f, lt = 0.f;
-      if (okm) {
-        const float ma = merge[r], mb = has_b ? merge[128 + r] : -INFINITY;
-        const float m = fmaxf(ma, mb);
-        fa = ex2(ma - m);
-        fb = has_b ? ex2(mb - m) : 0.f;
-        lt = merge[256 + r] * fa + (has_b ? merge[384 + r] * fb : 0.f);
-      }
+      // the exchange buffer the last tile did not use: its last reads
+      // (tile n-2) finished before every thread arrived for tile n-1
+      float* xl = xmax + (((n_tiles - 1) & 1) ^ 1) * 256;
+      xl[hc * 128 + r] = l;
+      mbar_arrive(bar(BL));
+      bool okl = all_wait(bar(BL), 0, ctl);
+      const float lt = okl ? l + xl[(hc ^ 1) * 128 + r] : 0.f;
       // every P V has completed once the MMA lane's drain commit fired
-      if (okm) okm = warp_wait(bar(BDRAIN), 0, ctl);
-      if (okm) {
+      if (okl) okl = warp_wait(bar(BDRAIN), 0, ctl);
+      if (okl) {
         tc_fence_after();
         const float inv = lt > 0.f ? 1.f / lt : 0.f;
-        fa *= inv;
-        fb *= inv;
 #pragma unroll 1
         for (int c0 = 0; c0 < 64; c0 += 32) {
-          const int col = grp * 64 + c0;
-          uint32_t oa[32], ob[32];
+          const int col = hc * 64 + c0;
+          uint32_t oa[32];
           tmem_ld32(lane_addr + kColO + col, oa);
-          if (has_b) {
-            tmem_ld32(lane_addr + kColO + 128 + col, ob);
-          } else {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) ob[c] = 0u;
-          }
           if (orow != nullptr) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-              float vv[8];
-#pragma unroll
-              for (int u = 0; u < 8; ++u)
-                vv[u] = __uint_as_float(oa[c * 8 + u]) * fa + __uint_as_float(ob[c * 8 + u]) * fb;
+              const float* f = reinterpret_cast<const float*>(oa) + c * 8;
               uint4 w;
-              w.x = pack_bf16(vv[0], vv[1]);
-              w.y = pack_bf16(vv[2], vv[3]);
-              w.z = pack_bf16(vv[4], vv[5]);
-              w.w = pack_bf16(vv[6], vv[7]);
+              w.x = pack_bf16(f[0] * inv, f[1] * inv);
+              w.y = pack_bf16(f[2] * inv, f[3] * inv);
+              w.z = pack_bf16(f[4] * inv, f[5] * inv);
+              w.w = pack_bf16(f[6] * inv, f[7] * inv);
               reinterpret_cast<uint4*>(orow + col)[c] = w;
             }
           }
