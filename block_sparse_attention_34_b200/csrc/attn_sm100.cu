@@ -14,12 +14,15 @@
 //   warps 0-7  softmax, two warpgroups splitting every tile by columns: warp
 //              w owns rows 32*(w%4) .. +31 (its TMEM lane quarter; a warp
 //              may only touch its own quarter) and key columns
-//              64*(w/4) .. +63.  A thread reads its 64 scores from TMEM, the
-//              two halves of a row exchange their maxima through shared
-//              memory, and each thread writes its 64 probabilities (bf16
-//              pairs) into its half of the tile's P region of tensor memory,
-//              from which the P V MMA reads them; when a row's max grows by
-//              more than 2^8 the thread rescales its 64 columns of O;
+//              64*(w/4) .. +63 of every tile.  Each column half is an exact
+//              split of the row's keys and keeps its own running max, row
+//              sum and O accumulator, so no cross-warp exchange happens per
+//              tile; the halves are merged once at the end:
+//              O = (O_0 2^(m_0-m) + O_1 2^(m_1-m)) / (l_0 2^(m_0-m) +
+//              l_1 2^(m_1-m)).  A thread reads its 64 scores from TMEM,
+//              writes its 64 probabilities (bf16 pairs) into its half of the
+//              tile's P region of tensor memory (the P V MMA's A operand),
+//              and when its max grows by more than 2^8 rescales its O;
 //   warp 8     allocates TMEM; one lane issues every tcgen05.mma and commit;
 //   warp 9     loads Q, then K tiles; warp 10 loads V tiles.  With inputs in
 //              the permuted order (pa_reorder) every tile is 128 contiguous
@@ -30,15 +33,16 @@
 //              positions from the head's axis order) and each lane's arrival
 //              on the stage's mbarrier fires when its copies land;
 //   warp 11    validates the kept list, then idles.
-// Tensor memory (512 columns): S double buffer at 0 and 128, P double
-// buffer (64 columns each) at 256 and 320, O at 384.  Shared memory: Q
+// Tensor memory (512 columns): S at 0, P double buffer (64 columns each)
+// at 128 and 192, O_0 and O_1 at 256 and 384.  Shared memory: Q
 // (32 KB) and three-stage K and V rings (6 x 32 KB) in the canonical
 // K-major / MN-major SWIZZLE_128B layouts the MMA descriptors name.
 //
 // MMA issue order QK(0), QK(1), PV(0), QK(2), PV(1), ...: QK^T of tile j+1
-// runs on the tensor core while the softmax warps turn S(j) into P(j).
-// tcgen05 operations of one thread complete in order, so S(j) being ready
-// implies P V(j-2), the previous reader of P(j)'s buffer, has completed.  A
+// is issued as soon as both halves have read S(j) out of tensor memory, so
+// it runs while the softmax warps turn S(j) into P(j).  tcgen05 operations
+// of one thread complete in order, so S(j) being ready implies P V(j-2),
+// the previous reader of P(j)'s buffer, has completed.  A
 // K stage is refilled once its QK^T completes, a V stage once its P V
 // completes.  Every mbarrier wait is bounded (about one second of
 // %globaltimer); on expiry the kernel records PA_ERR_TIMEOUT in the device
@@ -80,11 +84,12 @@ constexpr int kThreads = 12 * 32;  // 384
 constexpr int kSoftThreads = 256;
 constexpr uint32_t kTile = kBlock * kD * 2;  // 32 KB
 constexpr uint32_t kHalf = kBlock * 128;     // 16 KB: 64 columns
-// small region first: mbarriers, TMEM slot and flags, the row-max exchange
-// [2 tiles][2 halves][128 rows] float; the operand tiles start 1024-aligned
+// small region first: mbarriers, TMEM slot and flags, the final merge
+// buffer [m, l][2 halves][128 rows] float; the operand tiles start
+// 1024-aligned
 constexpr uint32_t kOffBar = 0;
 constexpr uint32_t kOffSlot = 256;
-constexpr uint32_t kOffXmax = 512;
+constexpr uint32_t kOffMerge = 512;
 constexpr uint32_t kSmall = 3072;
 constexpr uint32_t kOffQ = kSmall;
 constexpr uint32_t kOffK = kOffQ + kTile;            // kStages stages
@@ -92,7 +97,7 @@ constexpr uint32_t kOffV = kOffK + kStages * kTile;  // kStages stages
 constexpr uint32_t kSmemBytes = kOffV + kStages * kTile;  // 232,448 B = 227 KB
 constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold (factor 256)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColP = 256, kColO = 384;
+constexpr uint32_t kColS = 0, kColP = 128, kColO = 256;
 
 enum : uint32_t {
   BQ = 0,
@@ -100,17 +105,16 @@ enum : uint32_t {
   BV0 = 4,    // V stage full (3)
   BKF0 = 7,   // K stage free (3)
   BVF0 = 10,  // V stage free (3)
-  BS0 = 13,   // S(j) ready (2, by j & 1)
-  BSF0 = 15,  // S(j) read by both halves (2)
-  BP0 = 17,   // P(j) written by both halves (2)
-  BPV0 = 19,  // P V(j) complete (2)
-  BX0 = 21,   // row maxima of tile j exchanged (2)
-  BDRAIN = 23,
-  BL = 24,    // row sums exchanged at the end
-  NBAR = 25
+  BS = 13,    // S(j) ready
+  BSF = 14,   // S(j) read by every softmax thread
+  BP0 = 15,   // P(j) written by every softmax thread (2, by j & 1)
+  BPV0 = 17,  // P V(j) complete (2)
+  BDRAIN = 19,
+  BM = 20,    // final merge exchange
+  NBAR = 21
 };
 static_assert(NBAR * 8 <= kOffSlot, "barrier region");
-static_assert(kOffXmax + 2 * 2 * 128 * 4 <= kSmall, "exchange region");
+static_assert(kOffMerge + 2 * 2 * 128 * 4 <= kSmall, "merge region");
 
 // One warp copies a 128 x 128 bf16 tile whose row r is the token at
 // permuted position p0 + r of head `head` (rows past N zero-filled).  Lane l
@@ -166,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOffSlot);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile uint32_t* bad_flag = tmem_slot + 2;
-  float* xmax = reinterpret_cast<float*>(gbase + kOffXmax);  // [tile & 1][half][row]
+  float* merge = reinterpret_cast<float*>(gbase + kOffMerge);  // [m|l][half][row]
   auto bar = [&](uint32_t slot) { return base + kOffBar + slot * 8u; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -191,15 +195,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(BKF0 + s), 1);
       mbar_init(bar(BVF0 + s), 1);
     }
+    mbar_init(bar(BS), 1);
+    mbar_init(bar(BSF), kSoftThreads);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(BS0 + b), 1);
-      mbar_init(bar(BSF0 + b), kSoftThreads);
       mbar_init(bar(BP0 + b), kSoftThreads);
       mbar_init(bar(BPV0 + b), 1);
-      mbar_init(bar(BX0 + b), kSoftThreads);
     }
     mbar_init(bar(BDRAIN), 1);
-    mbar_init(bar(BL), kSoftThreads);
+    mbar_init(bar(BM), kSoftThreads);
     *abort_flag = 0;
     *bad_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -291,27 +294,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t id_pv = idesc_bf16(kBlock, kD, true);
         bool ok = wait_phase(bar(BQ), 0, ctl);
         fence_async_smem();  // cp.async (generic proxy) writes -> MMA operand reads
-        // QK^T of tile j into S buffer j & 1: needs K(j) and, for j >= 2,
-        // both halves to have read S(j-2) out of that buffer
+        // QK^T of tile j into S: needs K(j) and, for j >= 1, every softmax
+        // thread to have read S(j-1)
         auto issue_qk = [&](int j) -> bool {
-          const int b = j & 1, s = j % kStages;
+          const int s = j % kStages;
           if (!wait_phase(bar(BK0 + s), (j / kStages) & 1, ctl)) return false;
-          if (j >= 2 && !wait_phase(bar(BSF0 + b), ((j - 2) >> 1) & 1, ctl)) return false;
+          if (j >= 1 && !wait_phase(bar(BSF), (j - 1) & 1, ctl)) return false;
           fence_async_smem();
           tc_fence_after();
           const uint32_t ka = base + kOffK + s * kTile;
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk) {
             const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-            mma_f16_ss(tmem + kColS + b * 128, sw128_desc(base + kOffQ + off, 16, 1024),
+            mma_f16_ss(tmem + kColS, sw128_desc(base + kOffQ + off, 16, 1024),
                        sw128_desc(ka + off, 16, 1024), id_qk, kk > 0 ? 1u : 0u);
           }
-          mma_commit(bar(BS0 + b));
+          mma_commit(bar(BS));
           mma_commit(bar(BKF0 + s));
           PARO_T(4, j);
           return true;
         };
-        // O += P(j) V(j): P from tensor memory (bf16 pairs), V from the ring
+        // O_h += P(j)[:, keys of half h] V(j)[rows of half h], h = 0, 1:
+        // P from tensor memory (bf16 pairs), V from the ring
         auto issue_pv = [&](int j) -> bool {
           const int b = j & 1, s = j % kStages;
           if (!wait_phase(bar(BP0 + b), (j >> 1) & 1, ctl)) return false;
@@ -321,9 +325,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t va = base + kOffV + s * kTile;
 #pragma unroll
           for (int kk = 0; kk < kBlock / 16; ++kk)
-            mma_f16_ts(tmem + kColO, tmem + kColP + b * 64 + kk * 8,
+            mma_f16_ts(tmem + kColO + (kk >> 2) * 128, tmem + kColP + b * 64 + kk * 8,
                        sw128_desc(va + kk * 16 * 128, kHalf, 1024), id_pv,
-                       (j > 0 || kk > 0) ? 1u : 0u);
+                       (j > 0 || (kk & 3) > 0) ? 1u : 0u);
           mma_commit(bar(BPV0 + b));
           mma_commit(bar(BVF0 + s));
           PARO_T(5, j);
@@ -346,17 +350,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // tile row == TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
-    float m_used = -INFINITY, l = 0.f;  // m_used is the same in both halves
+    const uint32_t o_col = kColO + hc * 128;
+    float m_used = -INFINITY, l = 0.f;  // this half's reference max and row sum
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       const int b = j & 1;
-      if (!warp_wait(bar(BS0 + b), (j >> 1) & 1, ctl)) { ok = false; break; }
+      if (!warp_wait(bar(BS), j & 1, ctl)) { ok = false; break; }
       if (lane == 0 && quarter == 0) PARO_T(6 + 4 * hc, j);
       tc_fence_after();
       uint32_t sr[64];
-      tmem_ld64(lane_addr + kColS + b * 128 + hc * 64, sr);
+      tmem_ld64(lane_addr + kColS + hc * 64, sr);
       tc_fence_before();
-      mbar_arrive(bar(BSF0 + b));  // S buffer b may take QK^T(j+2)
+      mbar_arrive(bar(BSF));  // S may take QK^T(j+1)
       if (lane == 0 && quarter == 0) PARO_T(7 + 4 * hc, j);
       const int valid = g.N - __ldg(ids + j) * kBlock - hc * 64;  // existing keys of my half
       if (valid < 64) {  // only the ragged last block (warp-uniform)
@@ -369,37 +374,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int u = 0; u < 8; ++u) mp[u] = __uint_as_float(sr[u]);
 #pragma unroll
       for (int c = 8; c < 64; ++c) mp[c & 7] = fmaxf(mp[c & 7], __uint_as_float(sr[c]));
-      const float mh = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-      float* xm = xmax + b * 256;
-      xm[hc * 128 + r] = mh;
-      mbar_arrive(bar(BX0 + b));
-      if (!all_wait(bar(BX0 + b), (j >> 1) & 1, ctl)) { ok = false; break; }
-      const float mx = fmaxf(mh, xm[(hc ^ 1) * 128 + r]) * scale_log2;
+      const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) *
+                       scale_log2;
       if (lane == 0 && quarter == 0) PARO_T(8 + 4 * hc, j);
-      // lazy rescale: keep the reference max unless the row max grew by
-      // more than 2^8 (exact either way: O and l share the reference)
-      const bool need = j == 0 ? false : (mx > m_used + kRescaleLog2);
-      if (j == 0) m_used = mx == -INFINITY ? 0.f : mx;
+      // lazy rescale: keep the reference max unless this half's max grew
+      // by more than 2^8 (exact either way: O_h and l share the reference).
+      // A half whose keys are all padding (mx = -inf) keeps its reference.
+      const bool first = m_used == -INFINITY;
+      const bool need = !first && mx > m_used + kRescaleLog2;
+      if (first && mx != -INFINITY) m_used = mx;
       if (__any_sync(0xffffffffu, need)) {
-        // O holds P V up to tile j-1 once that MMA completed
+        // O_h holds P V up to tile j-1 once that MMA completed
         if (!warp_wait(bar(BPV0 + ((j - 1) & 1)), ((j - 1) >> 1) & 1, ctl)) { ok = false; break; }
         tc_fence_after();
         const float alpha = need ? ex2(m_used - mx) : 1.f;
 #pragma unroll 1
-        for (int c0 = 0; c0 < 64; c0 += 32) {
+        for (int c0 = 0; c0 < 128; c0 += 32) {
           uint32_t orr[32];
-          tmem_ld32(lane_addr + kColO + hc * 64 + c0, orr);
+          tmem_ld32(lane_addr + o_col + c0, orr);
 #pragma unroll
           for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
-          tmem_st32(lane_addr + kColO + hc * 64 + c0, orr);
+          tmem_st32(lane_addr + o_col + c0, orr);
         }
         l *= alpha;
         if (need) m_used = mx;
       }
       // P = 2^(s*scale - m) as bf16 pairs into my half of P buffer b (free:
       // S(j) ready means P V(j-2) completed); row sum in 8 chains
-      const float neg_m = -m_used;
+      const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
       float rs[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) rs[u] = 0.f;
@@ -418,8 +421,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(BP0 + b));
     }
-    // ---- epilogue: add the two halves' row sums, then each half writes
-    // O / l for its 64 columns at the natural position of the row's token
+    // ---- epilogue: merge the halves, then half h writes output columns
+    // 64h .. 64h+63 of the row at the natural position of its token
     const int p = i * kBlock + r;
     __nv_bfloat16* orow = p < g.N ? out + (bh * (int64_t)g.N + natural_index(g, order, p)) * kD
                                   : nullptr;
@@ -428,32 +431,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 8; ++c)
           reinterpret_cast<uint4*>(orow + hc * 64)[c] = make_uint4(0, 0, 0, 0);
     } else if (ok && n_tiles > 0) {
-      // the exchange buffer the last tile did not use: its last reads
-      // (tile n-2) finished before every thread arrived for tile n-1
-      float* xl = xmax + (((n_tiles - 1) & 1) ^ 1) * 256;
-      xl[hc * 128 + r] = l;
-      mbar_arrive(bar(BL));
-      bool okl = all_wait(bar(BL), 0, ctl);
-      const float lt = okl ? l + xl[(hc ^ 1) * 128 + r] : 0.f;
+      merge[(0 * 2 + hc) * 128 + r] = m_used;
+      merge[(1 * 2 + hc) * 128 + r] = l;
+      mbar_arrive(bar(BM));
+      bool okm = all_wait(bar(BM), 0, ctl);
+      float f0 = 0.f, f1 = 0.f, lt = 0.f;
+      if (okm) {
+        const float m0 = merge[r], m1 = merge[128 + r];
+        const float m = fmaxf(m0, m1);
+        // a half that saw only padding has l = 0 and an untouched O: weight 0
+        f0 = m0 == -INFINITY ? 0.f : ex2(m0 - m);
+        f1 = m1 == -INFINITY ? 0.f : ex2(m1 - m);
+        lt = merge[256 + r] * f0 + merge[384 + r] * f1;
+      }
       // every P V has completed once the MMA lane's drain commit fired
-      if (okl) okl = warp_wait(bar(BDRAIN), 0, ctl);
-      if (okl) {
+      if (okm) okm = warp_wait(bar(BDRAIN), 0, ctl);
+      if (okm) {
         tc_fence_after();
         const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        f0 *= inv;
+        f1 *= inv;
 #pragma unroll 1
         for (int c0 = 0; c0 < 64; c0 += 32) {
           const int col = hc * 64 + c0;
-          uint32_t oa[32];
+          uint32_t oa[32], ob[32];
           tmem_ld32(lane_addr + kColO + col, oa);
+          tmem_ld32(lane_addr + kColO + 128 + col, ob);
           if (orow != nullptr) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-              const float* f = reinterpret_cast<const float*>(oa) + c * 8;
+              float vv[8];
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                const float a0 = f0 != 0.f ? __uint_as_float(oa[c * 8 + u]) * f0 : 0.f;
+                const float a1 = f1 != 0.f ? __uint_as_float(ob[c * 8 + u]) * f1 : 0.f;
+                vv[u] = a0 + a1;
+              }
               uint4 w;
-              w.x = pack_bf16(f[0] * inv, f[1] * inv);
-              w.y = pack_bf16(f[2] * inv, f[3] * inv);
-              w.z = pack_bf16(f[4] * inv, f[5] * inv);
-              w.w = pack_bf16(f[6] * inv, f[7] * inv);
+              w.x = pack_bf16(vv[0], vv[1]);
+              w.y = pack_bf16(vv[2], vv[3]);
+              w.z = pack_bf16(vv[4], vv[5]);
+              w.w = pack_bf16(vv[6], vv[7]);
               reinterpret_cast<uint4*>(orow + col)[c] = w;
             }
           }
