@@ -510,7 +510,7 @@ cudaError_t launch_typed(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
 }  // namespace
 
 bool attn_sm100_supports(pa_dtype dt, const Grid& g) {
-  return dt == PA_BF16 && g.d == kD && g.block == kBlock &&
+  return (dt == PA_BF16 || dt == PA_I8) && g.d == kD && g.block == kBlock &&
          (int64_t)g.B * g.heads * g.Np < ((int64_t)1 << 31);
 }
 
@@ -518,10 +518,9 @@ cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, pa_dt
                               const Grid& g, const int32_t* idx, const int32_t* counts,
                               int k_max, const float* qs, const float* ks, const float* vs,
                               void* out, int32_t* status, bool permuted, cudaStream_t s) {
-  (void)qs;
-  (void)ks;
-  (void)vs;
   if (!attn_sm100_supports(dt, g)) return cudaErrorInvalidValue;
+  if (dt == PA_I8)
+    return launch_attn_i8(q, k, v, g, idx, counts, k_max, qs, ks, vs, out, status, s);
   CUtensorMap mq{}, mk{}, mv{};
   if (permuted) {
     const uint64_t rows = (uint64_t)g.B * g.heads * g.Np;

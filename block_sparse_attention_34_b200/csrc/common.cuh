@@ -98,4 +98,9 @@ cudaError_t launch_quantize(const void* x, pa_dtype dt, const Grid& g, int8_t* x
 cudaError_t launch_attn_mma(const void* q, const void* k, const void* v, pa_dtype dt,
                             const Grid& g, const int32_t* idx, const int32_t* counts, int k_max,
                             void* out, int32_t* status, bool permuted, cudaStream_t s);
+// INT8 tcgen05 attention (d = 128, block = 128, permuted int8 inputs)
+cudaError_t launch_attn_i8(const void* q, const void* k, const void* v, const Grid& g,
+                           const int32_t* idx, const int32_t* counts, int k_max, const float* qs,
+                           const float* ks, const float* vs, void* out, int32_t* status,
+                           cudaStream_t s);
 }  // namespace paro

@@ -336,6 +336,44 @@ def quantize_int8(xp: np.ndarray, N: int, block: int):
     return q, sc
 
 
+def _int8_query_rows(qi, ki, vi, sq_i, sk, sv, N, block, kept, mode, quantize_p):
+    """INT8 attention of some query rows of one query block (int64 codes
+    ``qi`` [r, d], block scale ``sq_i``) over the kept key blocks, in the
+    order listed.  Every step is row-wise, so any subset of a block's rows
+    gets the same values as the whole block.  Returns [r, d] float64."""
+    d = qi.shape[1]
+    inv_sqrt_d = 1.0 / math.sqrt(d)
+    tiles = []
+    for j in kept:
+        klo, khi = j * block, min((j + 1) * block, N)
+        if khi <= klo:
+            continue
+        s_int = qi @ ki[klo:khi].T
+        s = s_int.astype(np.float64) * (float(sq_i) * float(sk[j]) * inv_sqrt_d)
+        tiles.append((j, klo, khi, s))
+    rows = qi.shape[0]
+    if not tiles:
+        return np.zeros((rows, vi.shape[1]), dtype=np.float64)
+    if mode == "rowmax":
+        m_row = np.max([t[3].max(axis=1) for t in tiles], axis=0)[:, None]
+    m = np.full((rows, 1), -np.inf)
+    l = np.zeros((rows, 1))
+    acc = np.zeros((rows, vi.shape[1]))
+    for (j, klo, khi, s) in tiles:
+        if mode == "online":
+            m_new = np.maximum(m, s.max(axis=1, keepdims=True))
+            alpha = np.exp(m - m_new)
+        else:
+            m_new = m_row
+            alpha = np.ones((rows, 1))
+        pt = np.exp(s - m_new)
+        pq = np.rint(127.0 * pt) / 127.0 if quantize_p else pt
+        l = l * alpha + pt.sum(axis=1, keepdims=True)
+        acc = acc * alpha + (pq @ vi[klo:khi].astype(np.float64)) * float(sv[j])
+        m = m_new
+    return acc / l
+
+
 def attention_int8(q8, k8, v8, sq, sk, sv, N: int, block: int, idx, counts=None,
                    mode: str = "online", quantize_p: bool = True):
     """INT8 block-sparse attention in the permuted domain, one head.
@@ -360,8 +398,7 @@ def attention_int8(q8, k8, v8, sq, sk, sv, N: int, block: int, idx, counts=None,
     """
     Np, d = q8.shape
     nb = Np // block
-    out = np.zeros((Np, d), dtype=np.float64)
-    inv_sqrt_d = 1.0 / math.sqrt(d)
+    out = np.zeros((Np, v8.shape[1]), dtype=np.float64)
     qi = q8.astype(np.int64)
     ki = k8.astype(np.int64)
     vi = v8.astype(np.int64)
@@ -371,33 +408,24 @@ def attention_int8(q8, k8, v8, sq, sk, sv, N: int, block: int, idx, counts=None,
             continue
         c = idx.shape[1] if counts is None else int(counts[i])
         kept = [int(j) for j in idx[i, :c]]
-        tiles = []
-        for j in kept:
-            klo, khi = j * block, min((j + 1) * block, N)
-            if khi <= klo:
-                continue
-            s_int = qi[lo:hi] @ ki[klo:khi].T
-            s = s_int.astype(np.float64) * (float(sq[i]) * float(sk[j]) * inv_sqrt_d)
-            tiles.append((j, klo, khi, s))
-        rows = hi - lo
-        if not tiles:
-            continue
-        if mode == "rowmax":
-            m_row = np.max([t[3].max(axis=1) for t in tiles], axis=0)[:, None]
-        m = np.full((rows, 1), -np.inf)
-        l = np.zeros((rows, 1))
-        acc = np.zeros((rows, d))
-        for (j, klo, khi, s) in tiles:
-            if mode == "online":
-                m_new = np.maximum(m, s.max(axis=1, keepdims=True))
-                alpha = np.exp(m - m_new)
-            else:
-                m_new = m_row
-                alpha = np.ones((rows, 1))
-            pt = np.exp(s - m_new)
-            pq = np.rint(127.0 * pt) / 127.0 if quantize_p else pt
-            l = l * alpha + pt.sum(axis=1, keepdims=True)
-            acc = acc * alpha + (pq @ vi[klo:khi].astype(np.float64)) * float(sv[j])
-            m = m_new
-        out[lo:hi] = acc / l
+        out[lo:hi] = _int8_query_rows(qi[lo:hi], ki, vi, sq[i], sk, sv, N, block, kept, mode,
+                                      quantize_p)
     return out
+
+
+def attention_int8_rows(q8, k8, v8, sq, sk, sv, N: int, block: int, idx, positions,
+                        counts=None, mode: str = "online", quantize_p: bool = True):
+    """Rows of :func:`attention_int8` at the given permuted positions only
+    (one head), for full-size checks where the whole head is too costly.
+    Returns [len(positions), d] float64."""
+    qi = q8.astype(np.int64)
+    ki = k8.astype(np.int64)
+    vi = v8.astype(np.int64)
+    res = np.zeros((len(positions), v8.shape[1]), dtype=np.float64)
+    for r, p in enumerate(positions):
+        i = int(p) // block
+        c = idx.shape[1] if counts is None else int(counts[i])
+        kept = [int(j) for j in idx[i, :c]]
+        res[r] = _int8_query_rows(qi[p:p + 1], ki, vi, sq[i], sk, sv, N, block, kept, mode,
+                                  quantize_p)[0]
+    return res

@@ -14,7 +14,8 @@ from block_sparse_attention_34_b200.pipeline import Pipeline
 from block_sparse_attention_34_b200.synth import as_f64
 from oracle import paro_ref as ref
 
-from helpers import BF16_MAX_ABS, BF16_MEAN_ABS, compare, custom, inputs, static_mask, to_dev
+from helpers import (BF16_MAX_ABS, BF16_MEAN_ABS, compare, compare_rows, custom, inputs,
+                     oracle_topk, selection_agreement, static_mask, to_dev, token_mask)
 
 pytestmark = pytest.mark.gpu
 
@@ -63,9 +64,17 @@ def test_topk_pipeline_small(w, path):
                               status=status, **PATHS[path])
     torch.cuda.synchronize()
     assert status.item() == 0
-    idx_h = idx.cpu().numpy()
-    want = ref.attention(as_f64(q), as_f64(k), as_f64(v), (w.F, w.H, w.W), perms, w.block, idx_h)
-    compare(out, want)
+    check_against_oracle_selection(w, q, k, v, perms, out, idx)
+
+
+def check_against_oracle_selection(w, q, k, v, perms, out, idx):
+    """Kept lists equal the oracle's (near ties excepted) and the output
+    equals the oracle's attention over the oracle's lists on those rows."""
+    idx_ref, s_ref, _ = oracle_topk(q, k, w, perms)
+    agree = selection_agreement(idx.cpu().numpy(), idx_ref, s_ref)
+    assert agree.mean() >= 0.95
+    want = ref.attention(as_f64(q), as_f64(k), as_f64(v), (w.F, w.H, w.W), perms, w.block, idx_ref)
+    compare_rows(out, want, token_mask(agree, (w.F, w.H, w.W), perms, w.block))
 
 
 @pytest.mark.parametrize("path", list(PATHS))
@@ -144,9 +153,7 @@ def test_480p_two_heads_full():
                               status=status)
     torch.cuda.synchronize()
     assert status.item() == 0
-    want = ref.attention(as_f64(q), as_f64(k), as_f64(v), (w.F, w.H, w.W), perms, w.block,
-                         idx.cpu().numpy())
-    compare(out, want)
+    check_against_oracle_selection(w, q, k, v, perms, out, idx)
 
 
 @pytest.fixture(scope="module")
@@ -175,18 +182,29 @@ def test_720p_full_size_sampled(c720, density):
     torch.cuda.synchronize()
     assert pipe.status.item() == 0
     idx_h = pipe.idx.cpu().numpy()
+    rows = sampled_rows(w, 192 if density < 1.0 else 48, seed=11)
+    heads = sorted({h for (_, h, _) in rows})
+    idx_ref = np.zeros_like(idx_h)
     if density < 1.0:
-        # the kept lists are the oracle's top-k of the same fp32 scores
-        assert (idx_h == ref.select_topk(pipe.scores.cpu().double().numpy(), pipe.k)).all()
-        # and the scores are the oracle's pooled scores (sampled heads)
-        for hh in (0, w.heads - 1):
+        # the kept lists of the sampled heads are the oracle's top-k of its
+        # float64 pooled scores (near ties excepted), and the scores agree
+        agree = np.ones(idx_h.shape[:3], dtype=bool)
+        for hh in heads:
             _, _, s_ref = ref.pooled_scores(as_f64(q[:, hh:hh + 1]), as_f64(k[:, hh:hh + 1]),
                                             (w.F, w.H, w.W), perms[hh:hh + 1], w.block)
-            got = pipe.scores[:, hh:hh + 1].cpu().double().numpy()
-            assert np.abs(got - s_ref).max() < 1e-4 * max(1.0, np.abs(s_ref).max())
-    rows = sampled_rows(w, 192 if density < 1.0 else 48, seed=11)
+            got_s = pipe.scores[:, hh:hh + 1].cpu().double().numpy()
+            assert np.abs(got_s - s_ref).max() < 1e-4 * max(1.0, np.abs(s_ref).max())
+            idx_ref[:, hh:hh + 1] = ref.select_topk(s_ref, pipe.k)
+            agree[:, hh:hh + 1] = selection_agreement(idx_h[:, hh:hh + 1], idx_ref[:, hh:hh + 1],
+                                                      s_ref)
+        tok_ok = token_mask(agree, (w.F, w.H, w.W), perms, w.block)
+        rows = [r for r in rows if tok_ok[r]]
+        assert len(rows) >= 150
+    else:
+        idx_ref[:] = np.arange(w.NB, dtype=np.int32)
+        assert (idx_h == idx_ref).all()
     want = ref.attention_rows(as_f64(q), as_f64(k), as_f64(v), (w.F, w.H, w.W), perms, w.block,
-                              idx_h, rows)
+                              idx_ref, rows)
     got = out[0].float().cpu().numpy()
     got = np.stack([got[h, n] for (_, h, n) in rows]).astype(np.float64)
     err = np.abs(got - want)

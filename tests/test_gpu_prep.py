@@ -97,15 +97,17 @@ def test_topk_bit_exact(nb, k, kind):
 
 
 @pytest.mark.parametrize("w", CASES[:3] + [WORKLOADS["480p_21x30x52"]], ids=lambda w: w.name)
-def test_topk_on_gpu_scores(w):
+def test_topk_on_pooled_scores(w):
+    """Selection on realistic score structure: the oracle's pooled scores of
+    the synthetic inputs, rounded to float32, given to both sides."""
     q, k, _, perms = inputs(w, heads=2 if w.heads > 2 else None)
+    _, _, s = ref.pooled_scores(as_f64(q), as_f64(k), (w.F, w.H, w.W), perms, w.block)
+    s32 = s.astype(np.float32)
     heads = q.shape[1]
     pr = paro.Problem(w.B, heads, (w.F, w.H, w.W), w.d, w.block, perms)
-    qd, kd = to_dev(q, k)
-    _, _, s = paro.block_score(qd, kd, pr)
     kk = paro.k_for_density(pr.NB, w.density)
-    idx = paro.select_topk(s, pr, kk).cpu().numpy()
-    want = ref.select_topk(s.cpu().double().numpy(), kk)
+    idx = paro.select_topk(torch.from_numpy(s32).cuda(), pr, kk).cpu().numpy()
+    want = ref.select_topk(s32.astype(np.float64), kk)
     assert (idx == want).all()
 
 

@@ -125,3 +125,27 @@ def test_int32_dot_is_exact_range():
     # so converting the int32 accumulator to float32 loses nothing
     assert 127 * 127 * 128 < 2 ** 24
     assert math.isclose(127 * 127 * 128, 2064512)
+
+
+def test_row_subset_matches_whole_head():
+    """attention_int8_rows evaluates single rows with the same row-wise
+    steps: the whole-head function's values (up to float64 summation order,
+    which differs between a one-row and a block matrix product), ragged tail
+    and a row with an empty kept list included."""
+    rng = np.random.default_rng(12)
+    block, nb, d = 8, 5, 16
+    N = block * nb - 3
+    Np = block * nb
+    x = rng.standard_normal((3, 1, 1, Np, d)).astype(np.float32)
+    x[:, :, :, N:] = 0
+    qs = [ref.quantize_int8(x[t], N, block) for t in range(3)]
+    idx = np.array([[0, 2, 4], [1, 3, 4], [0, 2, -1], [0, 1, 3], [2, 3, 4]], dtype=np.int32)
+    counts = np.array([3, 3, 2, 0, 3], dtype=np.int32)
+    args = (qs[0][0][0, 0], qs[1][0][0, 0], qs[2][0][0, 0], qs[0][1][0, 0], qs[1][1][0, 0],
+            qs[2][1][0, 0], N, block, idx)
+    for mode in ("online", "rowmax"):
+        whole = ref.attention_int8(*args, counts=counts, mode=mode)
+        pos = [0, 5, 17, 24, 31, 33, N - 1]
+        rows = ref.attention_int8_rows(*args, pos, counts=counts, mode=mode)
+        assert np.abs(rows - whole[pos]).max() < 1e-12
+        assert (rows[3] == 0).all() and (rows[4] == 0).all()  # block 3: empty list
