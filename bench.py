@@ -83,15 +83,22 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def kernel_source_hash() -> str:
+KERNEL_SOURCES = {
+    "attn_sm100_kernel": ("attn_sm100.cu", "sm100.cuh", "tmem.cuh", "common.cuh"),
+    "attn_i8_kernel": ("attn_sm100_i8.cu", "sm100.cuh", "tmem.cuh", "common.cuh"),
+    "attn_mma_kernel": ("attn_mma.cu", "common.cuh"),
+}
+
+
+def kernel_source_hash(kernel: str = "attn_sm100_kernel") -> str:
     h = hashlib.sha256()
-    for f in ("attn_sm100.cu", "tmem.cuh", "common.cuh"):
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "block_sparse_attention_34_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(workload: str):
+def ncu_traffic(workload: str, kernel: str):
     """DRAM bytes per launch of the attention kernel from the committed ncu
     summary, or None when the summary is missing or the kernel changed."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -99,10 +106,19 @@ def ncu_traffic(workload: str):
         return None
     with open(p) as f:
         d = json.load(f)
-    e = d.get(workload)
-    if not e or e.get("kernel_hash") != kernel_source_hash():
+    e = d.get(f"{workload}/{kernel}")
+    if not e or e.get("kernel_hash") != kernel_source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
+
+
+# tensor-core peak of a dtype from the measured bf16 GEMM peak and the
+# nominal dense ratio (int8 / fp8 4.5 PFLOP/s vs bf16 2.25 PFLOP/s)
+NOMINAL_RATIO = {"bf16": 1.0, "int8": 2.0}
+
+
+def tensor_peak(peaks, dtype: str, which: str = "bf16_tflops_sustained") -> float:
+    return float(peaks.get(which, 1400.0)) * NOMINAL_RATIO[dtype]
 
 
 class ClockSampler:
@@ -162,9 +178,16 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ steps --
 
-def make_pipeline(w, perms, density, kernel, device):
+def make_pipeline(w, perms, density, kernel, device, int8=None):
     return Pipeline(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, perms, density,
-                    device=device, int8=w.int8, baseline=kernel == "mma")
+                    device=device, int8=w.int8 if int8 is None else int8,
+                    baseline=kernel == "mma")
+
+
+def attn_kernel_name(pipe) -> str:
+    if pipe.int8:
+        return "attn_i8_kernel"
+    return "attn_mma_kernel" if pipe.baseline else "attn_sm100_kernel"
 
 
 def step(pipe, qkv, ev=None):
@@ -216,27 +239,35 @@ def e2e_steps(pipe, qkv, host_q, host_k, host_v, host_out, steps):
     return start.elapsed_time(end) / steps
 
 
-def cpu_baseline(w, q, k, v, perms, idx_host, budget_s=12.0, max_blocks=None):
-    """The float64 oracle, as it stands, on a bounded sample: head 0, query
-    blocks 0, 1, 2, ... until the time budget is spent.  Returns TFLOPS of
-    kept-tile work and the sample description."""
+def cpu_baseline(w, q, k, v, perms, idx_host, budget_s=12.0, max_blocks=None, int8=False):
+    """The oracle, as it stands, on a bounded sample: head 0, query blocks
+    0, 1, 2, ... until the time budget is spent (float64 attention, or the
+    oracle's INT8 attention on its own codes when ``int8``).  Returns TFLOPS
+    of kept-tile work and the sample description.  The last query block
+    (ragged rows) is never in the sample."""
     from oracle import paro_ref as ref
     grid = (w.F, w.H, w.W)
-    qh = q[0, 0].double().numpy()
-    kh = k[0, 0].double().numpy()
-    vh = v[0, 0].double().numpy()
-    qp = ref.reorder_head(qh, grid, perms[0], w.block)
-    kp = ref.reorder_head(kh, grid, perms[0], w.block)
-    vp = ref.reorder_head(vh, grid, perms[0], w.block)
+    if int8:
+        xs = [ref.reorder(x[:, :1].float().numpy(), grid, perms[:1], w.block) for x in (q, k, v)]
+        (q8, sq), (k8, sk), (v8, sv) = [ref.quantize_int8(x, w.N, w.block) for x in xs]
+    else:
+        qp = ref.reorder_head(q[0, 0].double().numpy(), grid, perms[0], w.block)
+        kp = ref.reorder_head(k[0, 0].double().numpy(), grid, perms[0], w.block)
+        vp = ref.reorder_head(v[0, 0].double().numpy(), grid, perms[0], w.block)
     kk = idx_host.shape[-1]
     t0 = time.perf_counter()
     done = 0
-    nb = w.NB if max_blocks is None else min(w.NB, max_blocks)
+    nb = w.NB - 1 if max_blocks is None else min(w.NB - 1, max_blocks)
     while done < nb:
         chunk = min(4, nb - done)
         lo = done * w.block
-        ref.attention_permuted(qp[lo:lo + chunk * w.block], kp, vp, w.N, w.block,
+        if int8:
+            ref.attention_int8(q8[0, 0, lo:lo + chunk * w.block], k8[0, 0], v8[0, 0],
+                               sq[0, 0, done:done + chunk], sk[0, 0], sv[0, 0], w.N, w.block,
                                idx_host[0, 0, done:done + chunk])
+        else:
+            ref.attention_permuted(qp[lo:lo + chunk * w.block], kp, vp, w.N, w.block,
+                                   idx_host[0, 0, done:done + chunk])
         done += chunk
         if time.perf_counter() - t0 > budget_s:
             break
@@ -267,7 +298,10 @@ def run_ours(a):
         w = dataclasses.replace(w, heads=a.heads)
     qkv = [t.to(device) for t in (q, k, v)]
     dens = a.density if a.density is not None else w.density
-    pipe = make_pipeline(w, perms, dens, a.kernel, device)
+    int8 = {"auto": w.int8, "bf16": False, "int8": True}[a.precision]
+    pipe = make_pipeline(w, perms, dens, a.kernel, device, int8=int8)
+    kname = attn_kernel_name(pipe)
+    dtype = "int8" if int8 else "bf16"
     sampler = ClockSampler(local)
     sampler.start()
     total_ms, attn_ms = time_steps(pipe, qkv, a.steps, a.warmup, ws, device)
@@ -278,19 +312,36 @@ def run_ours(a):
     value = flops * ws / (ms_step / 1e3) / 1e12
 
     peaks, peak_src = load_peaks()
-    peak = float(peaks.get("bf16_tflops_sustained", 1400.0))
+    peak = tensor_peak(peaks, dtype)
     achieved = flops / (attn_avg / 1e3) / 1e12
 
     # speedup over the same kernel on the dense (density 1.0) layer
     dense = None
     if not a.no_dense:
-        dpipe = make_pipeline(w, perms, 1.0, a.kernel, device)
+        dpipe = make_pipeline(w, perms, 1.0, a.kernel, device, int8=int8)
         dsteps = max(2, min(a.steps, 3))
         _, d_attn = time_steps(dpipe, qkv, dsteps, 1, ws, device)
         dense_ms = max_over_ranks(sum(d_attn) / len(d_attn), ws, device)
         dense = {"attn_ms": dense_ms, "tflops": w.flops(dpipe.k) / (dense_ms / 1e3) / 1e12,
                  "speedup_attn": dense_ms / attn_avg, "target": 0.8 / (pipe.k / pipe.pr.NB)}
         del dpipe
+
+    # the INT8 kernel on the same layer and kept lists' density, beside bf16
+    i8 = None
+    if not int8 and not a.no_int8_compare and a.kernel == "tcgen05" and w.d == 128 \
+            and w.block == 128:
+        ipipe = make_pipeline(w, perms, dens, a.kernel, device, int8=True)
+        isteps = max(2, min(a.steps, 5))
+        i_total, i_attn = time_steps(ipipe, qkv, isteps, 3, ws, device)
+        i_ms = max_over_ranks(sum(i_attn) / len(i_attn), ws, device)
+        i_step = max_over_ranks(i_total / isteps, ws, device)
+        i_tops = flops / (i_ms / 1e3) / 1e12
+        i_peak = tensor_peak(peaks, "int8")
+        i8 = {"attn_ms": i_ms, "ms_per_step": i_step, "tops": i_tops, "peak": i_peak,
+              "frac": i_tops / i_peak, "speedup_attn_vs_bf16": attn_avg / i_ms,
+              "kernel": "attn_i8_kernel",
+              "prep": "quantize+pool q,k; quantize v; pooled scores; top-k"}
+        del ipipe
 
     e2e = None
     if not a.no_e2e:
@@ -305,7 +356,8 @@ def run_ours(a):
 
     cpu = None
     if rank == 0 and ws == 1 and not a.no_cpu_baseline:
-        tf, dt, sample = cpu_baseline(w, q, k, v, perms, pipe.idx.cpu().numpy(), budget_s=a.cpu_budget)
+        tf, dt, sample = cpu_baseline(w, q, k, v, perms, pipe.idx.cpu().numpy(),
+                                      budget_s=a.cpu_budget, int8=int8)
         cpu = {"value": tf, "unit": "TFLOPS", "cores": cores(), "kind": "oracle",
                "sample": sample, "seconds": round(dt, 2)}
 
@@ -313,7 +365,7 @@ def run_ours(a):
         res = {
             "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": ws, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "scaling": "weak", "vs_baseline": None, "dtype": dtype,
             "data": "synthetic (seeded structured q/k, normal v; no weights)",
             "config": {
                 "workload": w.name if a.heads is None else f"{w.name} (first {w.heads} heads)",
@@ -322,19 +374,24 @@ def run_ours(a):
                 "density_requested": a.density if a.density is not None else w.density,
                 "k": pipe.k, "NB": pipe.pr.NB, "kept_tiles": w.kept_tiles(pipe.k),
                 "flops_per_step": flops,
-                "kernel": ("tcgen05, permuted tiles" if a.kernel == "tcgen05" else "mma.sync, gathered rows"),
-                "l2": "inputs larger than L2 (q, k, v 774 MB each); no flush",
+                "kernel": ("mma.sync, gathered rows" if a.kernel == "mma" else
+                           "tcgen05 kind::i8, permuted int8 tiles" if int8 else
+                           "tcgen05 kind::f16, permuted tiles"),
+                "l2": (f"inputs larger than L2 (q, k, v {q.numel() * q.element_size() / 1e6:.0f} MB"
+                       " each); no flush"),
                 "parallelism": f"replicas x{ws} (independent layers, no data-path collective)",
                 "attn_ms": attn_avg, "prep_ms": ms_step - attn_avg,
-                "prep": "reorder+pool q,k; reorder v; pooled scores; top-k",
+                "prep": ("quantize+pool q,k; quantize v; pooled scores; top-k" if int8 else
+                         "reorder+pool q,k; reorder v; pooled scores; top-k"),
             },
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": ncu_traffic(w.name),
-                         "kernel": "attn_sm100_kernel" if a.kernel == "tcgen05" else "attn_mma_kernel",
-                         "peak_source": f"{peak_src} bf16_tflops_sustained"},
+                         "frac": achieved / peak, "traffic": ncu_traffic(w.name, kname),
+                         "kernel": kname,
+                         "peak_source": (f"{peak_src} bf16_tflops_sustained"
+                                         + (" x 2 (nominal int8/bf16 dense ratio)" if int8 else ""))},
             "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": pipe.launches * a.steps,
-            "clocks": clocks, "dense": dense,
+            "clocks": clocks, "dense": dense, "int8": i8,
         }
         print(json.dumps(res), flush=True)
     if ws > 1:
@@ -387,6 +444,9 @@ def main(argv=None):
     ap.add_argument("--heads", type=int, default=None,
                     help="run only the leading heads (profiling captures)")
     ap.add_argument("--kernel", choices=["tcgen05", "mma"], default="tcgen05")
+    ap.add_argument("--precision", choices=["auto", "bf16", "int8"], default="auto",
+                    help="auto: the workload's own (INT8 for the long-clip workload)")
+    ap.add_argument("--no-int8-compare", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -15,76 +15,146 @@
 //   O      = O 2^(m_old - m) + (P8 V8_j, exact int32) * s_v[j] / 127
 // and O / l is stored at the natural positions of the block's tokens.
 //
-// One CTA per (query block, head); 8 warps:
-//   warps 0-3  softmax + correction: thread t owns row t (TMEM lane t); it
-//              turns S(j) into P8(j) (packed 4 per 32-bit TMEM column, the
-//              A operand of the P V MMA), then folds the int32 P V result of
-//              the previous tile into the fp32 O accumulator in TMEM;
-//   warp 4     allocates TMEM; one lane issues every tcgen05.mma and commit;
-//   warp 5     loads Q, then K tiles; warp 6 loads V tiles: one lane issues
-//              one TMA tiled box (128 rows x 128 bytes) per tile;
-//   warp 7     validates the kept list, then idles.
-// Tensor memory (512 columns): S int32 at 0, P8 double buffer (32 columns
-// each) at 128 and 160, the P V int32 result at 192, O fp32 at 320.
-// Shared memory: Q (16 KB) and four-stage K and V rings, each tile one
-// 128-byte-swizzled panel.
+// One CTA per (query block, head); 14 warps in four roles:
+//   warps 0-7   softmax: warp w serves tile rows 32 (w & 3) .. +31 (its
+//               TMEM lane quarter) and S columns 64 (w >> 2) .. +63.  Per
+//               tile: row max of its half, traded with the partner warp of
+//               the other half through shared memory (a bounded mbarrier
+//               exchange: the running max stays exact), P8 of its half into
+//               a 128-byte-swizzled shared-memory tile (the A operand of
+//               P V), the row sum, and the tile's rescale factors;
+//   warps 8-11  correction: warp w folds the int32 P V result of its 32
+//               rows into the fp32 O accumulator in TMEM,
+//               O = O alpha + (s_v / 127) (P8 V8), and stores O / l at the end;
+//   warp 12     allocates TMEM; one lane issues every tcgen05.mma and commit;
+//   warp 13     validates the kept list; one lane then issues the TMA loads
+//               (Q once, then K and V tiles of 128 rows x 128 bytes).
+// Tensor memory (512 columns): S int32 at 0, O fp32 at 128, the P V int32
+// result double buffer at 256 and 384.
+// Shared memory: Q (16 KB), five-stage K and V rings and a P8 double buffer
+// (16 KB per tile, each one 128-byte-swizzled panel).
 //
-// MMA order QK(0), QK(1), PV(0), QK(2), PV(1), ...; S(j) ready implies
-// P V(j-2) completed (in-order tcgen05 completion), so P8 buffer j & 1 is
-// free.  Every mbarrier wait is bounded as in the bf16 kernel; on expiry the
-// kernel records PA_ERR_TIMEOUT and unwinds.
+// int32 -> float conversions avoid the conversion unit: |S|, |P V| <=
+// 128 * 127 * 127 < 2^22, so adding the bits of 1.5 * 2^23 gives a float
+// equal to 1.5 * 2^23 + x exactly, and subtracting 1.5 * 2^23 recovers x.
+//
+// MMA order QK(0), QK(1), PV(0), QK(2), PV(1), ...  S(j) ready implies
+// P V(j-2) completed (tcgen05 operations complete in issue order), so P8
+// buffer j & 1 is free when the softmax writes P8(j); P V(j) waits for the
+// correction of tile j-2 to free result buffer j & 1.  The softmax reads the
+// kept index and block scales of tile j+1 while it works on tile j.  Every mbarrier wait
+// is bounded as in the bf16 kernel; on expiry the kernel records
+// PA_ERR_TIMEOUT and unwinds.
 #include "sm100.cuh"
+#include "tmem.cuh"
 
 namespace paro {
+
+#ifdef PARO_TRACE
+// Phase trace (debug builds only): clock64() of each role's key events for
+// one CTA, event e of tile j at g_paro_trace_i8[e * 128 + j].
+__device__ long long* g_paro_trace_i8 = nullptr;
+__device__ int g_paro_trace_i8_cta = 7;
+#define PARO_T8(ev, j)                                                                      \
+  do {                                                                                      \
+    if (g_paro_trace_i8 != nullptr && blockIdx.x == g_paro_trace_i8_cta && blockIdx.y == 0 && \
+        (j) < 128)                                                                          \
+      g_paro_trace_i8[(ev) * 128 + (j)] = clock64();                                        \
+  } while (0)
+#else
+#define PARO_T8(ev, j) \
+  do {                 \
+  } while (0)
+#endif
+
 namespace {
 
 using namespace sm100;
 
 constexpr int kBlock = 128;
 constexpr int kD = 128;
-constexpr int kStages = 4;
-constexpr int kMmaWarp = 4;
-constexpr int kKWarp = 5;
-constexpr int kVWarp = 6;
-constexpr int kCheckWarp = 7;
-constexpr int kThreads = 8 * 32;
-constexpr int kSoftThreads = 128;
+constexpr int kStages = 5;
+constexpr int kSoftWarps = 8;
+constexpr int kCorrWarp0 = 8;  // warps 8..11
+constexpr int kMmaWarp = 12;
+constexpr int kLoadWarp = 13;
+constexpr int kThreads = 14 * 32;
+constexpr int kSoftThreads = kSoftWarps * 32;
+constexpr int kCorrThreads = 4 * 32;
+constexpr int kScaleSlots = 4;
 constexpr uint32_t kTile = kBlock * kD;  // 16 KB: one 128-byte-swizzled panel
 constexpr uint32_t kOffBar = 0;
-constexpr uint32_t kOffSlot = 256;
-constexpr uint32_t kSmall = 1024;
-constexpr uint32_t kOffQ = kSmall;
+constexpr uint32_t kOffSlot = 512;
+constexpr uint32_t kOffX = 1024;   // row-max exchange [2 parity][2 half][128] f32
+constexpr uint32_t kOffA = 3072;   // rescale factor alpha [4 slots][128] f32
+constexpr uint32_t kOffC = 5120;   // P V scale s_v / 127 [4 slots][128] f32
+constexpr uint32_t kOffL = 7168;   // final row sums [2 half][128] f32
+constexpr uint32_t kOffQ = 8192;
 constexpr uint32_t kOffK = kOffQ + kTile;
 constexpr uint32_t kOffV = kOffK + kStages * kTile;
-constexpr uint32_t kSmemBytes = kOffV + kStages * kTile;  // 148,480 B
+constexpr uint32_t kOffP = kOffV + kStages * kTile;
+constexpr uint32_t kSmemBytes = kOffP + 2 * kTile;  // 221,184 B
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+static_assert(kOffQ % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColP = 128, kColR = 192, kColO = 320;
+constexpr uint32_t kColS = 0, kColO = 128, kColR = 256;
+constexpr int32_t kMagicBits = 0x4B400000;  // bits of 1.5 * 2^23
+constexpr float kMagic = 12582912.0f;       // 1.5 * 2^23
 
 enum : uint32_t {
   BQ = 0,
-  BK0 = 1,    // K stage full (4)
-  BV0 = 5,    // V stage full (4)
-  BKF0 = 9,   // K stage free (4)
-  BVF0 = 13,  // V stage free (4)
-  BS = 17,    // S(j) ready
-  BSF = 18,   // S(j) read
-  BP0 = 19,   // P8(j) written (2)
-  BPV = 21,   // P V(j) result ready
-  BPVF = 22,  // P V(j) result folded into O (result columns free)
-  BDRAIN = 23,
-  NBAR = 24
+  BK0 = 1,                // K stage full (kStages)
+  BV0 = BK0 + kStages,    // V stage full
+  BKF0 = BV0 + kStages,   // K stage free
+  BVF0 = BKF0 + kStages,  // V stage free
+  BS = BVF0 + kStages,    // S(j) ready
+  BSF,                    // S(j) read by the softmax
+  BP0,                    // P8(j) written (2)
+  BSC0 = BP0 + 2,         // rescale factors of tile j written in slot j % 4 (4)
+  BPV0 = BSC0 + kScaleSlots,  // P V(j) ready in result buffer j & 1 (2)
+  BPVF0 = BPV0 + 2,       // result buffer folded into O, free (2)
+  BX0 = BPVF0 + 2,        // row-max exchange of lane quarter q (4)
+  BL = BX0 + 4,           // final row sums written
+  BDRAIN,
+  NBAR
 };
 static_assert(NBAR * 8 <= kOffSlot, "barrier region");
 
-// int32 -> float exactly for |x| < 2^22 without the conversion unit:
-// 1.5 * 2^23 + x lies in [2^23, 2^24), where floats are spaced by 1.
-__device__ __forceinline__ float i2f_small(int32_t x) {
-  return __int_as_float(x + 0x4B400000) - 12582912.0f;
+// float of an int32 |x| < 2^22 held in the bits of a 32-bit register (two
+// such values at once: the subtraction is one paired instruction)
+__device__ __forceinline__ float2 exact_float2(uint32_t a, uint32_t b) {
+  return fadd2(make_float2(__int_as_float((int32_t)a + kMagicBits),
+                           __int_as_float((int32_t)b + kMagicBits)),
+               make_float2(-kMagic, -kMagic));
 }
-// round-half-even of 0 <= y < 2^22 with one float add (the add rounds to
-// the nearest representable value, spacing 1, ties to even)
-__device__ __forceinline__ uint32_t rne_small(float y) {
-  return (uint32_t)(__float_as_int(y + 12582912.0f) - 0x4B400000);
+
+// P~ = 2^(s - m) <= 1 for 64 columns of one row, P8 = rne(127 P~) as the
+// low byte of the float 127 P~ + 1.5 * 2^23 (one rounding to the nearest
+// integer, ties to even), packed 4 per 32-bit word; row sums of P~ in rs.
+template <bool kRagged>
+__device__ __forceinline__ void tile_exp(const uint32_t (&sr)[64], float2 cq2, float2 nm2,
+                                         int valid, float2& rs0, float2& rs1,
+                                         uint32_t (&pk)[16]) {
+  const float2 k127 = make_float2(127.f, 127.f), mg2 = make_float2(kMagic, kMagic);
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    const float2 t0 = ffma2(exact_float2(sr[4 * c], sr[4 * c + 1]), cq2, nm2);
+    const float2 t1 = ffma2(exact_float2(sr[4 * c + 2], sr[4 * c + 3]), cq2, nm2);
+    float2 e0 = make_float2(ex2(t0.x), ex2(t0.y));
+    float2 e1 = make_float2(ex2(t1.x), ex2(t1.y));
+    if (kRagged) {
+      if (4 * c >= valid) e0.x = 0.f;
+      if (4 * c + 1 >= valid) e0.y = 0.f;
+      if (4 * c + 2 >= valid) e1.x = 0.f;
+      if (4 * c + 3 >= valid) e1.y = 0.f;
+    }
+    rs0 = fadd2(rs0, e0);
+    rs1 = fadd2(rs1, e1);
+    const float2 b0 = ffma2(e0, k127, mg2);
+    const float2 b1 = ffma2(e1, k127, mg2);
+    pk[c] = __byte_perm(__byte_perm(__float_as_uint(b0.x), __float_as_uint(b0.y), 0x0040),
+                        __byte_perm(__float_as_uint(b1.x), __float_as_uint(b1.y), 0x0040), 0x5410);
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -104,6 +174,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem_raw + kOffSlot);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile uint32_t* bad_flag = tmem_slot + 2;
+  float* xch = reinterpret_cast<float*>(smem_raw + kOffX);
+  float* s_alpha = reinterpret_cast<float*>(smem_raw + kOffA);
+  float* s_cv = reinterpret_cast<float*>(smem_raw + kOffC);
+  float* s_l = reinterpret_cast<float*>(smem_raw + kOffL);
   auto bar = [&](uint32_t slot) { return base + kOffBar + slot * 8u; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -128,17 +202,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar(BS), 1);
     mbar_init(bar(BSF), kSoftThreads);
-    mbar_init(bar(BP0), kSoftThreads);
-    mbar_init(bar(BP0 + 1), kSoftThreads);
-    mbar_init(bar(BPV), 1);
-    mbar_init(bar(BPVF), kSoftThreads);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(BP0 + b), kSoftThreads);
+      mbar_init(bar(BPV0 + b), 1);
+      mbar_init(bar(BPVF0 + b), kCorrThreads);
+    }
+    for (int b = 0; b < kScaleSlots; ++b) mbar_init(bar(BSC0 + b), kSoftThreads / 2);
+    for (int q = 0; q < 4; ++q) mbar_init(bar(BX0 + q), 64);
+    mbar_init(bar(BL), kSoftThreads);
     mbar_init(bar(BDRAIN), 1);
     *abort_flag = 0;
     *bad_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   if (warp == kMmaWarp) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-  if (warp == kCheckWarp) {
+  if (warp == kLoadWarp) {
     bool bad = cnt < 0 || cnt > k_max;
     if (!bad) {
       for (int e = lane; e < cnt; e += 32) {
@@ -160,30 +238,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_tiles = run ? cnt : 0;
   const int row0 = (int)(bh * g.Np);
 
-  if (warp == kKWarp || warp == kVWarp) {
+  if (warp == kLoadWarp) {
     // ------------------------------------------------------ loads ------
-    const bool is_k = warp == kKWarp;
-    const CUtensorMap* map = is_k ? &map_k : &map_v;
-    const uint32_t ring = base + (is_k ? kOffK : kOffV);
-    int issued = 0;
     if (n_tiles > 0 && lane == 0) {
-      if (is_k) {
-        mbar_arrive_tx(bar(BQ), kTile);
-        tma_load_2d(base + kOffQ, &map_q, 0, row0 + i * kBlock, bar(BQ));
-      }
+      mbar_arrive_tx(bar(BQ), kTile);
+      tma_load_2d(base + kOffQ, &map_q, 0, row0 + i * kBlock, bar(BQ));
+      int nk = 0, nv = 0;  // K and V tiles issued
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j % kStages;
-        if (j >= kStages &&
-            !wait_phase(bar((is_k ? BKF0 : BVF0) + s), ((j / kStages) - 1) & 1, ctl))
-          break;
-        const uint32_t full = bar((is_k ? BK0 : BV0) + s);
-        mbar_arrive_tx(full, kTile);
-        tma_load_2d(ring + s * kTile, map, 0, row0 + __ldg(ids + j) * kBlock, full);
-        issued = j + 1;
+        const int y = row0 + __ldg(ids + j) * kBlock;
+        if (j >= kStages && !wait_phase(bar(BKF0 + s), ((j / kStages) - 1) & 1, ctl)) break;
+        PARO_T8(0, j);
+        mbar_arrive_tx(bar(BK0 + s), kTile);
+        tma_load_2d(base + kOffK + s * kTile, &map_k, 0, y, bar(BK0 + s));
+        nk = j + 1;
+        if (j >= kStages && !wait_phase(bar(BVF0 + s), ((j / kStages) - 1) & 1, ctl)) break;
+        PARO_T8(11, j);
+        mbar_arrive_tx(bar(BV0 + s), kTile);
+        tma_load_2d(base + kOffV + s * kTile, &map_v, 0, y, bar(BV0 + s));
+        nv = j + 1;
       }
-      if (is_k) drain_phase(bar(BQ), 0);
-      for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
-        drain_phase(bar((is_k ? BK0 : BV0) + j % kStages), (j / kStages) & 1);
+      // copies still in flight land before the CTA exits
+      drain_phase(bar(BQ), 0);
+      for (int j = nk > kStages ? nk - kStages : 0; j < nk; ++j)
+        drain_phase(bar(BK0 + j % kStages), (j / kStages) & 1);
+      for (int j = nv > kStages ? nv - kStages : 0; j < nv; ++j)
+        drain_phase(bar(BV0 + j % kStages), (j / kStages) & 1);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
@@ -196,6 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = j % kStages;
         if (!wait_phase(bar(BK0 + s), (j / kStages) & 1, ctl)) return false;
         if (j >= 1 && !wait_phase(bar(BSF), (j - 1) & 1, ctl)) return false;
+        PARO_T8(1, j);
         tc_fence_after();
         const uint32_t ka = base + kOffK + s * kTile;
 #pragma unroll
@@ -210,122 +291,98 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b = j & 1, s = j % kStages;
         if (!wait_phase(bar(BP0 + b), (j >> 1) & 1, ctl)) return false;
         if (!wait_phase(bar(BV0 + s), (j / kStages) & 1, ctl)) return false;
-        if (j >= 1 && !wait_phase(bar(BPVF), (j - 1) & 1, ctl)) return false;
+        if (j >= 2 && !wait_phase(bar(BPVF0 + b), ((j >> 1) - 1) & 1, ctl)) return false;
+        PARO_T8(2, j);
         tc_fence_after();
-        const uint32_t va = base + kOffV + s * kTile;
+        const uint32_t va = base + kOffV + s * kTile, pa = base + kOffP + b * kTile;
 #pragma unroll
-        for (int kk = 0; kk < kBlock / 32; ++kk) {
-          asm volatile(
-              "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
-              "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n}\n" ::"r"(tmem + kColR),
-              "r"(tmem + kColP + b * 32 + kk * 8), "l"(sw128_desc(va + kk * 32 * 128, kTile, 1024)),
-              "r"(id_pv), "r"(kk > 0 ? 1u : 0u)
-              : "memory");
-        }
-        mma_commit(bar(BPV));
+        for (int kk = 0; kk < kBlock / 32; ++kk)
+          mma_i8_ss(tmem + kColR + b * 128, sw128_desc(pa + kk * 32, 16, 1024),
+                    sw128_desc(va + kk * 32 * 128, kTile, 1024), id_pv, kk > 0 ? 1u : 0u);
+        mma_commit(bar(BPV0 + b));
         mma_commit(bar(BVF0 + s));
         return true;
       };
       ok = ok && issue_qk(0);
       for (int j = 0; ok && j < n_tiles; ++j) {
-        if (j + 1 < n_tiles && !issue_qk(j + 1)) { ok = false; break; }
-        if (!issue_pv(j)) { ok = false; break; }
+        if (j + 1 < n_tiles && !issue_qk(j + 1)) break;
+        if (!issue_pv(j)) break;
       }
       mma_commit(bar(BDRAIN));
       drain_phase(bar(BDRAIN), 0);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // -------------------------------------------- softmax + correction --
-    const int r = threadIdx.x;  // tile row == TMEM lane
-    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-    const float sq = __ldg(q_scale + row) * log2e_over_sqrt_d;
-    float m_run = -INFINITY, l = 0.f;
-    float fold_alpha = 0.f, fold_c = 0.f;  // pending fold of the previous tile
+  } else if (warp >= kCorrWarp0) {
+    // -------------------------------------------------- correction ----
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     bool ok = true;
-    // O = O * alpha + c * (P V result): the previous tile's contribution
-    auto fold = [&](int jp, float alpha, float c) -> bool {
-      if (!warp_wait(bar(BPV), jp & 1, ctl)) return false;
-      tc_fence_after();
-#pragma unroll 1
-      for (int c0 = 0; c0 < 128; c0 += 32) {
-        uint32_t pv[32], o[32];
-        tmem_ld32(lane_addr + kColR + c0, pv);
-        if (jp > 0) tmem_ld32(lane_addr + kColO + c0, o);
-#pragma unroll
-        for (int u = 0; u < 32; ++u) {
-          const float add = (float)(int32_t)pv[u] * c;
-          o[u] = __float_as_uint(jp > 0 ? fmaf(__uint_as_float(o[u]), alpha, add) : add);
-        }
-        tmem_st32(lane_addr + kColO + c0, o);
-      }
-      tc_fence_before();
-      mbar_arrive(bar(BPVF));
-      return true;
-    };
     for (int j = 0; j < n_tiles; ++j) {
-      if (!warp_wait(bar(BS), j & 1, ctl)) { ok = false; break; }
+      const int sl = j & (kScaleSlots - 1), b = j & 1;
+      if (!all_wait(bar(BSC0 + sl), (j / kScaleSlots) & 1, ctl)) { ok = false; break; }
+      const float alpha = s_alpha[sl * 128 + r];
+      const float2 cv2 = make_float2(s_cv[sl * 128 + r], s_cv[sl * 128 + r]);
+      const float2 al2 = make_float2(alpha, alpha);
+      if (lane == 0 && quarter == 0) PARO_T8(9, j);
+      if (!warp_wait(bar(BPV0 + b), (j >> 1) & 1, ctl)) { ok = false; break; }
+      if (lane == 0 && quarter == 0) PARO_T8(10, j);
       tc_fence_after();
-      uint32_t sr[128];
-      tmem_ld128(lane_addr + kColS, sr);
-      tc_fence_before();
-      mbar_arrive(bar(BSF));  // S may take QK^T(j+1)
-      const int kb = __ldg(ids + j);
-      const int valid = g.N - kb * kBlock;
-      const float cq = sq * __ldg(k_scale + bh * g.NB + kb);
-      float mp[8];
+      // alpha is 1 while the row max holds
+      const bool keep = __all_sync(0xffffffffu, alpha == 1.f);
+      const uint32_t ra = lane_addr + kColR + b * 128;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kD; c0 += 32) {
+        uint32_t pv[32], o[32];
+        if (j == 0) {
+          tmem_ld32(ra + c0, pv);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) mp[u] = -INFINITY;
+          for (int u = 0; u < 32; u += 2) {
+            const float2 f = fmul2(exact_float2(pv[u], pv[u + 1]), cv2);
+            o[u] = __float_as_uint(f.x);
+            o[u + 1] = __float_as_uint(f.y);
+          }
+        } else {
+          tmem_ld32x2(ra + c0, pv, lane_addr + kColO + c0, o);
+          if (keep) {
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        float s = i2f_small((int32_t)sr[c]) * cq;
-        if (valid < kBlock && c >= valid) s = -INFINITY;
-        sr[c] = __float_as_uint(s);
-        mp[c & 7] = fmaxf(mp[c & 7], s);
-      }
-      const float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-      const float m_new = fmaxf(m_run, mt);
-      const float alpha = m_run == -INFINITY ? 0.f : ex2(m_run - m_new);
-      // P~ = 2^(s - m) <= 1, P8 = rne(127 P~), packed 4 per column
-      float rs[8];
+            for (int u = 0; u < 32; u += 2) {
+              const float2 f = ffma2(exact_float2(pv[u], pv[u + 1]), cv2,
+                                     make_float2(__uint_as_float(o[u]), __uint_as_float(o[u + 1])));
+              o[u] = __float_as_uint(f.x);
+              o[u + 1] = __float_as_uint(f.y);
+            }
+          } else {
 #pragma unroll
-      for (int u = 0; u < 8; ++u) rs[u] = 0.f;
-      uint32_t pk[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        uint32_t w = 0;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const float e = ex2(__uint_as_float(sr[4 * c + b]) - m_new);
-          rs[b] += e;
-          w |= rne_small(127.f * e) << (8 * b);
+            for (int u = 0; u < 32; u += 2) {
+              const float2 oa =
+                  fmul2(make_float2(__uint_as_float(o[u]), __uint_as_float(o[u + 1])), al2);
+              const float2 f = ffma2(exact_float2(pv[u], pv[u + 1]), cv2, oa);
+              o[u] = __float_as_uint(f.x);
+              o[u + 1] = __float_as_uint(f.y);
+            }
+          }
         }
-        pk[c] = w;
+        tmem_st32_async(lane_addr + kColO + c0, o);
       }
-      l = l * alpha + (((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7])));
-      tmem_st32(lane_addr + kColP + (j & 1) * 32, pk);
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(BP0 + (j & 1)));
-      // fold the previous tile's P V (its P used reference m_run)
-      if (j >= 1 && !fold(j - 1, fold_alpha, fold_c)) { ok = false; break; }
-      fold_alpha = alpha;  // O (ref m_run) -> ref m_new when tile j is folded
-      fold_c = __ldg(v_scale + bh * g.NB + kb) * (1.f / 127.f);
-      m_run = m_new;
+      mbar_arrive(bar(BPVF0 + b));
+      if (lane == 0 && quarter == 0) PARO_T8(12, j);
     }
-    if (ok && n_tiles > 0) ok = fold(n_tiles - 1, fold_alpha, fold_c);
     // epilogue: O / l at the natural position of the row's token
     const int p = i * kBlock + r;
-    __nv_bfloat16* orow = p < g.N ? out + (bh * (int64_t)g.N + natural_index(g, order, p)) * kD
-                                  : nullptr;
+    __nv_bfloat16* orow =
+        p < g.N ? out + (bh * (int64_t)g.N + natural_index(g, order, p)) * kD : nullptr;
     if (run && cnt == 0) {
       if (orow != nullptr)
         for (int c = 0; c < 16; ++c) reinterpret_cast<uint4*>(orow)[c] = make_uint4(0, 0, 0, 0);
-    } else if (ok && n_tiles > 0) {
+    } else if (ok && n_tiles > 0 && all_wait(bar(BL), 0, ctl)) {
+      const float lt = s_l[r] + s_l[128 + r];
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
-      for (int c0 = 0; c0 < 128; c0 += 32) {
+      for (int c0 = 0; c0 < kD; c0 += 32) {
         uint32_t o[32];
         tmem_ld32(lane_addr + kColO + c0, o);
         if (orow != nullptr) {
@@ -341,6 +398,102 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+    }
+    __syncwarp();
+  } else {
+    // ----------------------------------------------------- softmax ----
+    const int quarter = warp & 3, hc = warp >> 2;
+    const int r = quarter * 32 + lane;  // tile row == TMEM lane
+    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t xbar = bar(BX0 + quarter);
+    const float sq = __ldg(q_scale + row) * log2e_over_sqrt_d;
+    float m_run = -INFINITY;
+    float2 l2 = make_float2(0.f, 0.f);
+    bool ok = true;
+    // kept index and block scales of the current tile, read a tile ahead
+    int kb_next = 0;
+    float ks_next = 0.f, vs_next = 0.f;
+    if (n_tiles > 0) {
+      kb_next = __ldg(ids);
+      ks_next = __ldg(k_scale + bh * g.NB + kb_next);
+      vs_next = __ldg(v_scale + bh * g.NB + kb_next);
+    }
+    for (int j = 0; j < n_tiles; ++j) {
+      const int kb = kb_next;
+      const float ksc = ks_next, vsc = vs_next;
+      if (j + 1 < n_tiles) {
+        kb_next = __ldg(ids + j + 1);
+        ks_next = __ldg(k_scale + bh * g.NB + kb_next);
+        vs_next = __ldg(v_scale + bh * g.NB + kb_next);
+      }
+      if (!warp_wait(bar(BS), j & 1, ctl)) { ok = false; break; }
+      if (lane == 0 && quarter == 0) PARO_T8(3 + 3 * hc, j);
+      tc_fence_after();
+      uint32_t sr[64];
+      tmem_ld64(lane_addr + kColS + hc * 64, sr);
+      tc_fence_before();
+      mbar_arrive(bar(BSF));  // S may take QK^T(j+1)
+      const int valid = g.N - kb * kBlock - hc * 64;  // valid columns of this half
+      const float cq = sq * ksc;
+      // row max of this half in integers (cq >= 0 keeps the order)
+      int32_t mi = INT32_MIN;
+      if (valid >= 64) {
+        int32_t mp[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mp[u] = INT32_MIN;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) mp[c & 7] = max(mp[c & 7], (int32_t)sr[c]);
+        mi = max(max(max(mp[0], mp[1]), max(mp[2], mp[3])),
+                 max(max(mp[4], mp[5]), max(mp[6], mp[7])));
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (c < valid) mi = max(mi, (int32_t)sr[c]);
+      }
+      const float m_half =
+          mi == INT32_MIN ? -INFINITY : (__int_as_float(mi + kMagicBits) - kMagic) * cq;
+      // trade the half maxima with the partner warp (same rows, other half)
+      float* xs = xch + (j & 1) * 256;
+      xs[hc * 128 + r] = m_half;
+      mbar_arrive(xbar);
+      if (!all_wait(xbar, j & 1, ctl)) { ok = false; break; }
+      if (lane == 0 && quarter == 0) PARO_T8(4 + 3 * hc, j);
+      const float m_new = fmaxf(m_run, fmaxf(m_half, xs[(1 - hc) * 128 + r]));
+      const float alpha = m_run == -INFINITY ? 0.f : ex2(m_run - m_new);
+      if (hc == 0) {
+        // slot j % 4 was last read by the correction of tile j - 4, which
+        // completed before P V(j - 2) was issued, and so before QK(j)
+        const int sl = j & (kScaleSlots - 1);
+        s_alpha[sl * 128 + r] = alpha;
+        s_cv[sl * 128 + r] = vsc * (1.f / 127.f);
+        mbar_arrive(bar(BSC0 + sl));
+      }
+      // P~ = 2^(s - m) <= 1, P8 = rne(127 P~): the low byte of the float
+      // 127 P~ + 1.5 * 2^23 (one rounding, to the nearest integer, ties even)
+      const float2 cq2 = make_float2(cq, cq), nm2 = make_float2(-m_new, -m_new);
+      float2 rs0 = make_float2(0.f, 0.f), rs1 = make_float2(0.f, 0.f);
+      uint32_t pk[16];
+      if (valid >= 64)
+        tile_exp<false>(sr, cq2, nm2, valid, rs0, rs1, pk);
+      else
+        tile_exp<true>(sr, cq2, nm2, valid, rs0, rs1, pk);
+      const float2 rs = fadd2(rs0, rs1);
+      l2 = ffma2(l2, make_float2(alpha, alpha), rs);
+      // this half row of P8 (64 bytes = 4 chunks of 16) into the swizzled
+      // tile; the async proxy (the MMA) reads it after the fence
+      unsigned char* prow = smem_raw + kOffP + (j & 1) * kTile + r * 128;
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        *reinterpret_cast<uint4*>(prow + (((hc * 4 + t) ^ (r & 7)) << 4)) =
+            make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+      fence_async_smem();
+      mbar_arrive(bar(BP0 + (j & 1)));
+      if (lane == 0 && quarter == 0) PARO_T8(5 + 3 * hc, j);
+      m_run = m_new;
+    }
+    if (ok && n_tiles > 0) {
+      s_l[hc * 128 + r] = l2.x + l2.y;
+      mbar_arrive(bar(BL));
     }
     __syncwarp();
   }
