@@ -180,8 +180,15 @@ class ClockSampler:
 
 def make_pipeline(w, perms, density, kernel, device, int8=None):
     return Pipeline(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, perms, density,
+                    dtype=torch.float32 if w.dtype == "f32" else torch.bfloat16,
                     device=device, int8=w.int8 if int8 is None else int8,
                     baseline=kernel == "mma")
+
+
+def percentiles(xs):
+    v = sorted(xs)
+    pick = lambda q: v[min(len(v) - 1, int(round(q * (len(v) - 1))))]
+    return {"p10": pick(0.1), "p50": pick(0.5), "p90": pick(0.9)}
 
 
 def attn_kernel_name(pipe) -> str:
@@ -381,6 +388,7 @@ def run_ours(a):
                        " each); no flush"),
                 "parallelism": f"replicas x{ws} (independent layers, no data-path collective)",
                 "attn_ms": attn_avg, "prep_ms": ms_step - attn_avg,
+                "attn_ms_pct": percentiles(attn_ms),
                 "prep": ("quantize+pool q,k; quantize v; pooled scores; top-k" if int8 else
                          "reorder+pool q,k; reorder v; pooled scores; top-k"),
             },
@@ -396,6 +404,58 @@ def run_ours(a):
         print(json.dumps(res), flush=True)
     if ws > 1:
         torch.distributed.destroy_process_group()
+
+
+def run_sweep(a):
+    """Every workload of the configs table on one GPU: per-step device times
+    of the attention kernel and of the whole step (selection included) after
+    10 warm-up steps, as p10 / p50 / p90 over the timed steps, one JSON line
+    per workload.  Not the default contract line (that is the default run)."""
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU path)")
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    peaks, peak_src = load_peaks()
+    for name, w in WORKLOADS.items():
+        q, k, v, perms = make_inputs(w)
+        qkv = [t.to(device) for t in (q, k, v)]
+        for precision in (["bf16", "int8"] if w.int8 else [w.dtype]):
+            int8 = precision == "int8"
+            pipe = make_pipeline(w, perms, w.density, a.kernel, device, int8=int8)
+            for _ in range(10):
+                step(pipe, qkv)
+            torch.cuda.synchronize()
+            attn, total = [], []
+            for _ in range(max(20, a.steps)):
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                e[0].record()
+                pipe.select(*qkv)
+                e[1].record()
+                pipe.attend(*qkv)
+                e[2].record()
+                torch.cuda.synchronize()
+                attn.append(e[1].elapsed_time(e[2]))
+                total.append(e[0].elapsed_time(e[2]))
+            if int(pipe.status.item()) != 0:
+                raise RuntimeError(f"{name}: device status {int(pipe.status.item())}")
+            flops = w.flops(pipe.k)
+            pa, pt = percentiles(attn), percentiles(total)
+            dt = "int8" if int8 else w.dtype
+            peak = tensor_peak(peaks, "int8" if int8 else "bf16", "bf16_tflops")
+            print(json.dumps({
+                "workload": name, "precision": dt, "B": w.B, "heads": w.heads,
+                "grid": [w.F, w.H, w.W], "d": w.d, "block": w.block, "k": pipe.k,
+                "NB": pipe.pr.NB, "kept_tiles": w.kept_tiles(pipe.k), "flops": flops,
+                "attn_ms": pa, "step_ms": pt,
+                "select_ms_p50": pt["p50"] - pa["p50"],
+                "tflops_p50": flops / (pa["p50"] / 1e3) / 1e12,
+                "frac_of_burst_peak_p50": flops / (pa["p50"] / 1e3) / 1e12 / peak,
+                "peak": peak, "peak_source": f"{peak_src} bf16_tflops"
+                + (" x 2 (nominal int8/bf16 dense ratio)" if int8 else ""),
+                "kernel": attn_kernel_name(pipe), "steps": len(attn), "warmup": 10,
+            }), flush=True)
+            del pipe
+        del qkv
 
 
 def run_reference(a):
@@ -447,6 +507,8 @@ def main(argv=None):
     ap.add_argument("--precision", choices=["auto", "bf16", "int8"], default="auto",
                     help="auto: the workload's own (INT8 for the long-clip workload)")
     ap.add_argument("--no-int8-compare", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="per-workload latency percentiles, one JSON line per workload")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -458,6 +520,8 @@ def main(argv=None):
         a.warmup = 3
     if a.impl == "reference":
         run_reference(a)
+    elif a.sweep:
+        run_sweep(a)
     else:
         run_ours(a)
 

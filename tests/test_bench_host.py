@@ -110,3 +110,13 @@ def test_int8_peak_uses_nominal_ratio():
     assert bench.tensor_peak(peaks, "bf16") == 1000.0
     assert bench.tensor_peak(peaks, "int8") == 2000.0
     assert bench.tensor_peak(peaks, "int8", "bf16_tflops") == 3000.0
+
+
+def test_percentiles_pick_order_statistics():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    xs = [5.0, 1.0, 3.0, 2.0, 4.0, 9.0, 7.0, 8.0, 6.0, 10.0, 0.0]
+    p = bench.percentiles(xs)
+    assert p == {"p10": 1.0, "p50": 5.0, "p90": 9.0}
+    assert bench.percentiles([2.5]) == {"p10": 2.5, "p50": 2.5, "p90": 2.5}
