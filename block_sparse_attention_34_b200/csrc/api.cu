@@ -109,7 +109,7 @@ pa_status check_float_dtype(pa_dtype dt) {
 
 extern "C" {
 
-int32_t pa_abi_version(void) { return 2; }
+int32_t pa_abi_version(void) { return 3; }
 
 const char* pa_last_error(void) { return g_error.c_str(); }
 
@@ -192,6 +192,36 @@ pa_status pa_select_topk(const float* scores, pa_shape shape, int32_t k, int32_t
   PA_REQUIRE(g.NB <= 16384, "NB=%d exceeds 16384 (row keys must fit in shared memory)", g.NB);
   return cuda_status(paro::launch_topk(scores, g, k, idx, (cudaStream_t)stream),
                      "pa_select_topk launch");
+}
+
+pa_status pa_select_hybrid(const float* scores, pa_shape shape, int32_t k, double top_p,
+                           int32_t window, int32_t* idx, int32_t* counts, void* stream) {
+  paro::Grid g;
+  pa_status st = make_grid(shape, nullptr, false, &g);
+  if (st != PA_OK) return st;
+  PA_REQUIRE(scores && idx && counts, "scores, idx and counts must be non-NULL");
+  PA_REQUIRE(k >= 0 && k <= g.NB, "k=%d must be in [0, NB=%d]", k, g.NB);
+  PA_REQUIRE(std::isfinite(top_p), "top_p must be finite");
+  if (g.NB > 4096) return fail(PA_ERR_UNSUPPORTED, "NB=%d exceeds 4096 for pa_select_hybrid", g.NB);
+  return cuda_status(
+      paro::launch_hybrid(scores, g, k, top_p, window, idx, counts, (cudaStream_t)stream),
+      "pa_select_hybrid launch");
+}
+
+pa_status pa_sics_scores(const void* q, const void* k, pa_dtype dtype, pa_shape shape,
+                         float* scores, void* stream) {
+  paro::Grid g;
+  pa_status st = make_grid(shape, nullptr, false, &g);
+  if (st != PA_OK) return st;
+  PA_REQUIRE(dtype == PA_F32 || dtype == PA_BF16, "dtype %d: pa_sics_scores takes F32 or BF16",
+             (int)dtype);
+  PA_REQUIRE(q && k && scores, "q, k and scores must be non-NULL");
+  PA_REQUIRE(g.d % 32 == 0 && g.d <= 256, "d=%d must be a multiple of 32 and <= 256", g.d);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(scores, 0, (size_t)g.B * g.heads * 6 * sizeof(float), s);
+  if (e == cudaSuccess) e = paro::launch_sics(q, dtype, g, scores, s);
+  if (e == cudaSuccess) e = paro::launch_sics(k, dtype, g, scores, s);
+  return cuda_status(e, "pa_sics_scores launch");
 }
 
 pa_status pa_compact_mask(const uint32_t* bitmask, pa_shape shape, int32_t* idx, int32_t* counts,

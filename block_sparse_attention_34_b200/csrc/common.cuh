@@ -98,6 +98,10 @@ cudaError_t launch_quantize(const void* x, pa_dtype dt, const Grid& g, int8_t* x
 cudaError_t launch_attn_mma(const void* q, const void* k, const void* v, pa_dtype dt,
                             const Grid& g, const int32_t* idx, const int32_t* counts, int k_max,
                             void* out, int32_t* status, bool permuted, cudaStream_t s);
+// Selection variants (select_variants.cu)
+cudaError_t launch_sics(const void* x, pa_dtype dt, const Grid& g, float* scores, cudaStream_t s);
+cudaError_t launch_hybrid(const float* scores, const Grid& g, int k, double p, int w,
+                          int32_t* idx, int32_t* counts, cudaStream_t s);
 // INT8 tcgen05 attention (d = 128, block = 128, permuted int8 inputs)
 cudaError_t launch_attn_i8(const void* q, const void* k, const void* v, const Grid& g,
                            const int32_t* idx, const int32_t* counts, int k_max, const float* qs,

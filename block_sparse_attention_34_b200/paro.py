@@ -60,6 +60,8 @@ def load():
         "pa_score_pooled": ([_P, _P, PaShape, _P, _P], _I),
         "pa_select_topk": ([_P, PaShape, _I, _P, _P], _I),
         "pa_compact_mask": ([_P, PaShape, _P, _P, _P], _I),
+        "pa_select_hybrid": ([_P, PaShape, _I, ctypes.c_double, _I, _P, _P, _P], _I),
+        "pa_sics_scores": ([_P, _P, _I, PaShape, _P, _P], _I),
         "pa_quantize_int8": ([_P, _I, PaShape, _P, _P, _P, _P, _P], _I),
         "pa_block_sparse_attn": ([_P, _P, _P, _I, ctypes.c_uint32, PaShape, _P, _P, _P, _I, _P, _P, _P,
                                   _P, _P, _P], _I),
@@ -190,6 +192,27 @@ def compact_mask(bitmask, pr: Problem, idx=None, counts=None):
     counts = counts if counts is not None else torch.empty((pr.B, pr.heads, pr.NB), dtype=torch.int32, device=dev)
     _check(load().pa_compact_mask(_ptr(bitmask), pr.shape, _ptr(idx), _ptr(counts), _stream()))
     return idx, counts
+
+
+def select_hybrid(scores, pr: Problem, k: int, top_p: float, window: int, idx=None, counts=None):
+    """Union of the diagonal, a local window, Top-K and Top-P per query-block
+    row -> (idx [B,h,NB,NB] ascending, -1 padded; counts [B,h,NB])."""
+    _need_cuda(scores)
+    dev = scores.device
+    idx = idx if idx is not None else torch.empty((pr.B, pr.heads, pr.NB, pr.NB), dtype=torch.int32, device=dev)
+    counts = counts if counts is not None else torch.empty((pr.B, pr.heads, pr.NB), dtype=torch.int32, device=dev)
+    _check(load().pa_select_hybrid(_ptr(scores), pr.shape, int(k), float(top_p), int(window), _ptr(idx),
+                                   _ptr(counts), _stream()))
+    return idx, counts
+
+
+def sics_scores(q, k, pr: Problem, scores=None):
+    """[B,h,6] blocking scores of the six axis orders (SICS of q's and k's
+    blocks); the argmax per head is the order SPADE's rule picks."""
+    _need_cuda(q, k)
+    scores = scores if scores is not None else torch.empty((pr.B, pr.heads, 6), dtype=torch.float32, device=q.device)
+    _check(load().pa_sics_scores(_ptr(q), _ptr(k), _dtype_code(q), pr.shape, _ptr(scores), _stream()))
+    return scores
 
 
 def quantize_int8(x, pr: Problem, with_pool=False, x_q=None, scales=None, pool=None):

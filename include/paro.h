@@ -80,7 +80,7 @@ typedef struct {
   int32_t B, heads, F, H, W, d, block;
 } pa_shape;
 
-/* Version of this ABI (bumped on any signature change): 2. */
+/* Version of this ABI (bumped on any signature change): 3. */
 PA_API int32_t pa_abi_version(void);
 
 /* Message of the last failed call on this thread ("" if none). */
@@ -133,6 +133,39 @@ PA_API pa_status pa_score_pooled(const float* q_pool, const float* k_pool, pa_sh
  * read as -inf, -0.0 equal to +0.0.  1 <= k <= NB. */
 PA_API pa_status pa_select_topk(const float* scores, pa_shape shape, int32_t k, int32_t* idx,
                          void* stream);
+
+/* Step 3, hybrid filter (SPADE review, core_discovery: head-wise Top-K /
+ * Top-P and local-window filters).  Row (b,h,i) of scores [B,heads,NB,NB]
+ * keeps the union of
+ *   - block i itself,
+ *   - the local window {j : |i - j| <= window} (window < 0: none),
+ *   - the Top-K set of pa_select_topk (k >= 1; k = 0: none),
+ *   - the Top-P set: blocks in decreasing score order (ties to the lower
+ *     index, NaN read as -inf), the shortest run whose softmax weights
+ *     exp(s_j - max_j s_j) (summed in fp64; NaN weighs 0; a row whose max
+ *     is +inf weighs its +inf entries 1 and the rest 0) reach
+ *     top_p * (their row total); all blocks if none does; none if
+ *     top_p <= 0 or the row is all -inf / NaN.
+ * Output idx [B,heads,NB,NB] int32 (kept indices ascending, the rest -1)
+ * and counts [B,heads,NB] int32, the format pa_block_sparse_attn takes with
+ * k_max = NB.  0 <= k <= NB, top_p finite, NB <= 4096 (PA_ERR_UNSUPPORTED
+ * above: a row is sorted in shared memory). */
+PA_API pa_status pa_select_hybrid(const float* scores, pa_shape shape, int32_t k, double top_p,
+                           int32_t window, int32_t* idx, int32_t* counts, void* stream);
+
+/* Blocking-scheme score (SPADE review, key_machinery (ii): the Sum of
+ * Intra-block Cosine Similarities, one pass per block by the identity
+ * sum_{s != t} cos(x_s, x_t) = |sum_t xh_t|^2 - sum_t |xh_t|^2, xh = x/|x|,
+ * zero rows adding nothing).  For every axis order o (0..5, the ids of the
+ * order table above) and every (b,h):
+ *   scores[b,h,o] = sum over the blocks of order o (runs of `block`
+ *                   permuted tokens) of SICS(q's rows) + SICS(k's rows).
+ * q, k natural order [B,heads,N,d] (PA_F32 or PA_BF16), d a multiple of 32
+ * and <= 256; scores [B,heads,6] float, overwritten (accumulated in fp32
+ * with atomics, so the last bits vary between runs).  The order with the
+ * largest score is SPADE's pick for the head. */
+PA_API pa_status pa_sics_scores(const void* q, const void* k, pa_dtype dtype, pa_shape shape,
+                         float* scores, void* stream);
 
 /* Step 3, static (PAROAttention review, key_machinery: static masks stored
  * as bitmasks).  bitmask [B,heads,NB,ceil(NB/32)] uint32, bit (j % 32) of

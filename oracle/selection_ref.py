@@ -30,9 +30,11 @@ S3. The score of an order is SICS over Q's blocks plus SICS over K's blocks
 S4. Top-P on a query-block row: weights w_j = exp(s_j - max_j s_j) over all
     key blocks (NaN scores weigh 0 and sort as -inf); blocks in order of
     decreasing score, ties to the lower index; keep the shortest prefix
-    whose cumulative weight reaches p * sum(w) (all blocks if none does;
-    none if p <= 0 or every score is -inf / NaN).  A row whose maximum is
-    +inf gives weight 1 to its +inf entries and 0 to the rest.
+    whose running sum reaches p times the full running sum (the total is
+    the last prefix sum, so that p = 1 stops at the last block of nonzero
+    weight whatever the rounding); all blocks if none does; none if
+    p <= 0 or every score is -inf / NaN.  A row whose maximum is +inf gives
+    weight 1 to its +inf entries and 0 to the rest.
 S5. The kept set of row i is the union of the diagonal block, the local
     window {j : |i - j| <= w} (w >= 0; w < 0 adds nothing), the Top-K set of
     paro_ref.select_topk_row (k >= 1; k = 0 adds nothing) and the Top-P set;
@@ -111,7 +113,7 @@ def topp_row(s: np.ndarray, p: float) -> np.ndarray:
     j = np.arange(nb)
     order = np.lexsort((j, -key))  # score descending, then index ascending
     cum = np.cumsum(w[order])
-    target = p * w.sum()
+    target = p * cum[-1]  # the total as the same left-to-right sum
     reach = np.nonzero(cum >= target)[0]
     length = int(reach[0]) + 1 if reach.size else nb
     return np.sort(order[:length]).astype(np.int32)

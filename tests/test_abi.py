@@ -34,7 +34,7 @@ def test_exports_every_declared_symbol(lib):
     assert len(names) >= 12
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.pa_abi_version() == 2
+    assert lib.pa_abi_version() == 3
 
 
 def test_k_for_density_matches_oracle(lib):
@@ -108,3 +108,18 @@ def test_binding_refuses_cpu_tensors(lib):
     x = torch.zeros(1, 2, 256, 64)
     with pytest.raises(ValueError):
         paro.reorder(x, pr)
+
+
+def test_selection_variant_validation(lib):
+    good = paro.PaShape(1, 2, 4, 8, 8, 64, 64)  # NB = 4
+    # hybrid: k range, finite top_p, null outputs, NB limit
+    assert lib.pa_select_hybrid(FAKE, good, -1, 0.5, 1, FAKE, FAKE, None) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_select_hybrid(FAKE, good, 5, 0.5, 1, FAKE, FAKE, None) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_select_hybrid(FAKE, good, 2, float("nan"), 1, FAKE, FAKE, None) == paro.PA_ERR_INVALID_ARG
+    assert b"top_p" in lib.pa_last_error()
+    assert lib.pa_select_hybrid(FAKE, good, 2, 0.5, 1, FAKE, None, None) == paro.PA_ERR_INVALID_ARG
+    big = paro.PaShape(1, 1, 1, 1, 4097 * 64, 64, 64)  # NB = 4097
+    assert lib.pa_select_hybrid(FAKE, big, 2, 0.5, 1, FAKE, FAKE, None) == paro.PA_ERR_UNSUPPORTED
+    # SICS: float inputs only, non-null buffers
+    assert lib.pa_sics_scores(FAKE, FAKE, paro.PA_I8, good, FAKE, None) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_sics_scores(FAKE, None, paro.PA_BF16, good, FAKE, None) == paro.PA_ERR_INVALID_ARG

@@ -1,0 +1,170 @@
+"""GPU parity of the selection variants (SICS blocking score, hybrid Top-K /
+Top-P / local-window filter) against the oracle (oracle/selection_ref.py),
+through the C ABI, and the hybrid kept lists driving the attention kernel.
+
+Scores and the order pick are compared within a float tolerance derived
+from fp32 accumulation (the kernel sums with atomics); the hybrid lists are
+compared bit-exact on identical fp32 scores, except rows whose Top-P
+boundary is a rounding tie (the fp64 prefix sums of the two sides differ in
+association), which must then equal the rule's row for a prefix that stops
+where the oracle's running sum is within 1e-9 of p times its total."""
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_34_b200 import paro
+from block_sparse_attention_34_b200.configs import WORKLOADS
+from block_sparse_attention_34_b200.synth import as_f64
+from oracle import paro_ref as ref
+from oracle import selection_ref as sel
+
+from helpers import compare_rows, custom, inputs, to_dev, token_mask
+
+pytestmark = pytest.mark.gpu
+
+SICS_CASES = [
+    custom("sics_ragged_bf16", 1, 3, 128, (5, 7, 9), 128, "bf16", 0.5, perms=(0, 0, 0)),
+    custom("sics_ragged_f32", 2, 2, 64, (3, 5, 7), 64, "f32", 0.5, perms=(0, 0)),
+    custom("sics_tiny_bf16", 1, 2, 64, (4, 8, 8), 64, "bf16", 0.5, perms=(0, 0)),
+]
+
+
+def dummy_problem(w, heads=None):
+    h = heads or w.heads
+    return paro.Problem(w.B, h, (w.F, w.H, w.W), w.d, w.block, [0] * h)
+
+
+def check_sics(w, q, k):
+    pr = dummy_problem(w, q.shape[1])
+    qd, kd = to_dev(q, k)
+    got = paro.sics_scores(qd, kd, pr).cpu().double().numpy()
+    want = sel.sics_scores(as_f64(q), as_f64(k), (w.F, w.H, w.W), w.block)
+    # |SICS| of one order <= sum over blocks n (n - 1) <= N (block - 1), per tensor;
+    # per-block fp32 sums (relative ~n eps) plus fp32 atomics over NB block
+    # values: 4e-5 of that bound covers both
+    tol = 4e-5 * 2 * w.N * (w.block - 1)
+    assert np.abs(got - want).max() <= tol, (np.abs(got - want).max(), tol)
+    # the pick agrees wherever the oracle's best order leads by more than tol
+    top2 = np.sort(want, axis=-1)[..., -2:]
+    clear = (top2[..., 1] - top2[..., 0]) > 2 * tol
+    assert (sel.select_orders(got)[clear] == sel.select_orders(want)[clear]).all()
+    return got, want
+
+
+@pytest.mark.parametrize("w", SICS_CASES, ids=lambda w: w.name)
+def test_sics_scores(w):
+    q, k, _, _ = inputs(w)
+    check_sics(w, q, k)
+
+
+def test_sics_finds_the_frame_blocking():
+    # every frame's tokens share one direction (per tensor): the frame-major
+    # orders (FHW, FWH) put each frame in its own block and must win
+    F, H, W, d = 6, 4, 16, 64  # H*W = 64 = block
+    rng = np.random.default_rng(4)
+    dirs = rng.standard_normal((2, F, d))
+    scale = rng.uniform(0.5, 2.0, size=(2, F * H * W, 1))
+    q = torch.from_numpy(np.repeat(dirs[0], H * W, axis=0) * scale[0]).float()[None, None]
+    k = torch.from_numpy(np.repeat(dirs[1], H * W, axis=0) * scale[1]).float()[None, None]
+    w = custom("frames", 1, 1, d, (F, H, W), 64, "f32", 0.5, perms=(0,))
+    got, want = check_sics(w, q, k)
+    assert sel.select_orders(want)[0, 0] == 0
+    assert got[0, 0, :2].min() > got[0, 0, 2:].max()
+
+
+def test_sics_480p_two_heads():
+    w = WORKLOADS["480p_21x30x52"]
+    q, k, _, _ = inputs(w, heads=2)
+    check_sics(w, q, k)
+
+
+def random_scores(rng, heads, nb, kind):
+    if kind == "normal":
+        return (rng.standard_normal((1, heads, nb, nb)) * 2.0).astype(np.float32)
+    s = rng.integers(-2, 3, size=(1, heads, nb, nb)).astype(np.float32)
+    m = rng.random(s.shape)
+    s[m < 0.05] = np.nan
+    s[(m >= 0.05) & (m < 0.07)] = -np.inf
+    s[(m >= 0.07) & (m < 0.075)] = np.inf
+    s[(m >= 0.075) & (m < 0.1)] = -0.0
+    return s
+
+
+def near_tie_rows(s_row, i, k, p, w, rel=1e-9):
+    """Every kept set the hybrid rule gives for row i when the Top-P prefix
+    stops anywhere the float64 running sum is within rel of p * total (the
+    two sides sum the same weights in different association)."""
+    v = np.asarray(s_row, dtype=np.float64)
+    key = np.where(np.isnan(v), -np.inf, v)
+    nb = key.size
+    order = np.lexsort((np.arange(nb), -key))
+    lengths = {len(sel.topp_row(s_row, p))}
+    if p > 0 and key.max() > -np.inf:
+        wgt = (key == np.inf).astype(np.float64) if key.max() == np.inf else np.exp(key - key.max())
+        cum = np.cumsum(wgt[order])
+        target = p * cum[-1]
+        for n in range(nb):
+            if cum[n] >= target * (1 - rel) and (n == 0 or cum[n - 1] < target * (1 + rel)):
+                lengths.add(n + 1)
+        if cum[-1] < target * (1 + rel):
+            lengths.add(nb)
+    base = [np.array([i]), sel.window_row(i, w, nb)]
+    if k >= 1:
+        base.append(ref.select_topk_row(s_row, i, k))
+    return [np.unique(np.concatenate(base + [order[:n]])).tolist() for n in sorted(lengths)]
+
+
+def check_hybrid(s, k, p, w):
+    heads, nb = s.shape[1], s.shape[2]
+    pr = paro.Problem(1, heads, (1, 1, nb * 64), 64, 64, [0] * heads)
+    assert pr.NB == nb
+    idx, cnt = paro.select_hybrid(torch.from_numpy(s).cuda(), pr, k, p, w)
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    want_idx, want_cnt = sel.hybrid_select(s, k, p, w)
+    same = (idx == want_idx).all(axis=-1) & (cnt == want_cnt)
+    for b, h, i in zip(*np.nonzero(~same)):
+        row = idx[b, h, i, :cnt[b, h, i]].tolist()
+        assert row in near_tie_rows(s[b, h, i], i, k, p, w), (b, h, i, row)
+        assert (idx[b, h, i, cnt[b, h, i]:] == -1).all()
+    return same.mean()
+
+
+@pytest.mark.parametrize("nb", [1, 5, 33, 100, 591, 929, 3000])
+@pytest.mark.parametrize("kind", ["normal", "special"])
+def test_hybrid_select_matches_oracle(nb, kind):
+    rng = np.random.default_rng(nb + (7 if kind == "special" else 0))
+    heads = 2 if nb <= 600 else 1
+    s = random_scores(rng, heads, nb, kind)
+    params = [(0, 0.5, -1), (3, 0.9, 1), (1, 0.0, 2), (min(4, nb), 0.3, 0), (0, 1.0, -1),
+              (nb, 0.0, -1), (0, 1e-12, -1)]
+    if nb >= 2000:
+        params = [(3, 0.9, 1)]
+    for k, p, w in params:
+        assert check_hybrid(s, min(k, nb), p, w) > 0.99
+
+
+def test_hybrid_attention_end_to_end():
+    """pooled scores -> hybrid lists -> bf16 attention over the permuted
+    tiles with per-row counts, against the oracle's attention over the
+    oracle's hybrid lists (rows whose lists differ at near ties left out)."""
+    w = custom("hybrid_780", 2, 3, 128, (6, 10, 13), 128, "bf16", 0.6, perms=(5, 2, 4))
+    q, k, v, perms = inputs(w)
+    pr = paro.Problem(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, perms)
+    qd, kd, vd = to_dev(q, k, v)
+    qp, q_pool = paro.reorder(qd, pr, with_pool=True)
+    kp, k_pool = paro.reorder(kd, pr, with_pool=True)
+    vp = paro.reorder(vd, pr)
+    scores = paro.score_pooled(q_pool, k_pool, pr)
+    idx, cnt = paro.select_hybrid(scores, pr, 2, 0.5, 1)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = paro.block_sparse_attn(qp, kp, vp, pr, idx, cnt, status=status, permuted=True)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    _, _, s_ref = ref.pooled_scores(as_f64(q), as_f64(k), (w.F, w.H, w.W), perms, w.block)
+    idx_ref, cnt_ref = sel.hybrid_select(s_ref, 2, 0.5, 1)
+    agree = (idx.cpu().numpy() == idx_ref).all(axis=-1) & (cnt.cpu().numpy() == cnt_ref)
+    assert agree.mean() >= 0.9
+    want = ref.attention(as_f64(q), as_f64(k), as_f64(v), (w.F, w.H, w.W), perms, w.block,
+                         idx_ref, cnt_ref)
+    compare_rows(out, want, token_mask(agree, (w.F, w.H, w.W), perms, w.block))

@@ -81,7 +81,9 @@ def brute_topp(s, p):
     else:
         w = [math.exp(v - key.max()) for v in key]
     order = sorted(range(len(key)), key=lambda j: (-key[j], j))
-    total = sum(w)
+    total = 0.0
+    for j in order:
+        total += w[j]
     acc = 0.0
     for n, j in enumerate(order):
         acc += w[j]
@@ -109,6 +111,9 @@ def test_topp_limits_ties_and_non_finite():
     assert sel.topp_row(np.array([-np.inf, np.nan]), 0.5).tolist() == []
     assert sel.topp_row(np.array([np.inf, 0.0, np.inf]), 0.5).tolist() == [0]
     assert sel.topp_row(np.array([np.inf, 0.0, np.inf]), 0.9).tolist() == [0, 2]
+    # p = 1 stops at the last block of nonzero weight (-inf / NaN weigh 0)
+    s3 = np.array([0.3, -np.inf, 1.7, np.nan, -2.0, 0.9], dtype=np.float32)
+    assert sel.topp_row(s3, 1.0).tolist() == [0, 2, 4, 5]
     # the mass of two equal leaders covers p = 2 / (2 + e^-3)
     s2 = np.array([0.0, 0.0, -3.0])
     lead = 2.0 / (2.0 + math.exp(-3.0))
