@@ -416,7 +416,7 @@ def run_sweep(a):
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     peaks, peak_src = load_peaks()
-    for name, w in WORKLOADS.items():
+    for name, w in ([] if a.selection_only else WORKLOADS.items()):
         q, k, v, perms = make_inputs(w)
         qkv = [t.to(device) for t in (q, k, v)]
         for precision in (["bf16", "int8"] if w.int8 else [w.dtype]):
@@ -456,6 +456,75 @@ def run_sweep(a):
             }), flush=True)
             del pipe
         del qkv
+    run_sweep_selection(device, peaks, peak_src, a.heads)
+
+
+def timed_calls(fn, reps=20, warm=5):
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    return ms
+
+
+def run_sweep_selection(device, peaks, peak_src, heads=None):
+    """The selection variants on the 720p layer: the SICS blocking score of
+    the six orders (HBM-bound: q and k read once per order) and a layer
+    whose kept lists come from the hybrid filter (diagonal, window 1,
+    Top-K at density 0.10, Top-P 0.5)."""
+    w = WORKLOADS["720p_21x45x80"]
+    q, k, v, perms = make_inputs(w, heads=heads)
+    if heads is not None:
+        w = dataclasses.replace(w, heads=heads)
+    qkv = [t.to(device) for t in (q, k, v)]
+    pr = paro.Problem(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, [0] * w.heads)
+    sc = torch.empty((w.B, w.heads, 6), dtype=torch.float32, device=device)
+    ms = timed_calls(lambda: paro.sics_scores(qkv[0], qkv[1], pr, sc))
+    nbytes = 2 * 6 * w.B * w.heads * w.N * w.d * qkv[0].element_size()
+    pm = percentiles(ms)
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
+    print(json.dumps({
+        "workload": w.name, "kernel": "sics_kernel", "what": "SICS of the six orders, q and k",
+        "ms": pm, "bytes": nbytes, "gbs_p50": nbytes / (pm["p50"] / 1e3) / 1e9,
+        "frac_of_hbm_p50": nbytes / (pm["p50"] / 1e3) / 1e9 / hbm,
+        "peak_source": f"{peak_src} hbm_gbs", "steps": len(ms),
+    }), flush=True)
+    pipe = Pipeline(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, perms, 0.10, device=device,
+                    selection="hybrid", top_p=0.5, window=1)
+    attn, total = [], []
+    for it in range(30):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record()
+        pipe.select(*qkv)
+        e[1].record()
+        pipe.attend(*qkv)
+        e[2].record()
+        torch.cuda.synchronize()
+        if it >= 10:
+            attn.append(e[1].elapsed_time(e[2]))
+            total.append(e[0].elapsed_time(e[2]))
+    if int(pipe.status.item()) != 0:
+        raise RuntimeError(f"hybrid: device status {int(pipe.status.item())}")
+    kept = pipe.kept_tiles()
+    flops = 4.0 * w.block * w.block * w.d * kept
+    pa, pt = percentiles(attn), percentiles(total)
+    peak = tensor_peak(peaks, "bf16", "bf16_tflops")
+    print(json.dumps({
+        "workload": w.name, "precision": "bf16", "selection": "hybrid k=0.10*NB p=0.5 window=1",
+        "kept_tiles": kept, "density": kept / (w.B * w.heads * pipe.pr.NB ** 2), "flops": flops,
+        "attn_ms": pa, "step_ms": pt, "select_ms_p50": pt["p50"] - pa["p50"],
+        "tflops_p50": flops / (pa["p50"] / 1e3) / 1e12,
+        "frac_of_burst_peak_p50": flops / (pa["p50"] / 1e3) / 1e12 / peak,
+        "peak_source": f"{peak_src} bf16_tflops", "kernel": attn_kernel_name(pipe),
+        "steps": len(attn), "warmup": 10,
+    }), flush=True)
 
 
 def run_reference(a):
@@ -509,6 +578,8 @@ def main(argv=None):
     ap.add_argument("--no-int8-compare", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="per-workload latency percentiles, one JSON line per workload")
+    ap.add_argument("--selection-only", action="store_true",
+                    help="with --sweep: only the selection-variant lines")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -216,7 +216,7 @@ pa_status pa_sics_scores(const void* q, const void* k, pa_dtype dtype, pa_shape 
   PA_REQUIRE(dtype == PA_F32 || dtype == PA_BF16, "dtype %d: pa_sics_scores takes F32 or BF16",
              (int)dtype);
   PA_REQUIRE(q && k && scores, "q, k and scores must be non-NULL");
-  PA_REQUIRE(g.d % 32 == 0 && g.d <= 256, "d=%d must be a multiple of 32 and <= 256", g.d);
+  PA_REQUIRE(aligned16(q) && aligned16(k), "q and k must be 16-byte aligned");
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaMemsetAsync(scores, 0, (size_t)g.B * g.heads * 6 * sizeof(float), s);
   if (e == cudaSuccess) e = paro::launch_sics(q, dtype, g, scores, s);

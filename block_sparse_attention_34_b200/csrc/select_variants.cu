@@ -7,8 +7,7 @@
 //   The candidate blockings are the six axis orders of [F, H, W] with the
 //   call's block size; one CTA reduces one block of one order of one
 //   (batch, head) and adds its value to scores[b, h, order].  Rows are read
-//   at their natural positions (no permuted copy): each warp takes a run of
-//   rows, one 16-byte-or-smaller slice of a row per lane.
+//   at their natural positions (no permuted copy), 16 bytes per lane.
 //
 // * hybrid_kernel — the union of the diagonal block, a local window
 //   |i - j| <= w, the Top-K set (diagonal + k-1 largest others, ties to the
@@ -26,46 +25,67 @@ namespace {
 
 constexpr int kSicsThreads = 128;
 
+// Rows are read 16 bytes per lane: a row of d elements takes L = d *
+// sizeof(T) / 16 lanes (8 for d=64 bf16, 16 for d=128 bf16, 32 for d=128
+// f32), so a warp reads 32 / L rows per load, two loads in flight.  Each
+// lane keeps the running sum of its 16-byte slice of xh; |xh|^2 of a row is
+// ss / ss (one value per row, no second pass).
 template <typename T>
 __global__ void __launch_bounds__(kSicsThreads)
     sics_kernel(const T* __restrict__ x, const __grid_constant__ Grid g,
                 float* __restrict__ scores) {
-  // d <= 256: each lane holds d / 32 <= 8 elements of a row
+  constexpr int kE = 16 / sizeof(T);  // elements per 16-byte slice
   __shared__ float part[kSicsThreads / 32][256];
   __shared__ float diag_part[kSicsThreads / 32];
   const int i = blockIdx.x, order = blockIdx.y;
   const int64_t bh = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int per = g.d / 32;  // elements per lane (d is a multiple of 32)
-  float acc[8], dsum = 0.f;
+  const int L = g.d * (int)sizeof(T) / 16;  // lanes per row: 4, 8, 16 or 32
+  const int rows_per_load = 32 / L;
+  const int slot = lane % L, sub = lane / L;  // slice within the row, row within the load
+  float acc[kE], dsum = 0.f;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  for (int e = 0; e < kE; ++e) acc[e] = 0.f;
   const T* head = x + bh * (int64_t)g.N * g.d;
-  for (int r = warp; r < g.block; r += kSicsThreads / 32) {
-    const int p = i * g.block + r;
-    if (p >= g.N) break;  // pad rows are zero: no direction
-    const T* row = head + (int64_t)natural_index(g, order, p) * g.d + lane * per;
-    float v[8], ss = 0.f;
+  const int step = rows_per_load * (kSicsThreads / 32);
+  for (int r0 = warp * rows_per_load; r0 < g.block; r0 += 2 * step) {
+    uint4 raw[2];
+    bool have[2];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      v[e] = e < per ? to_float(row[e]) : 0.f;
-      ss = fmaf(v[e], v[e], ss);
+    for (int u = 0; u < 2; ++u) {
+      const int p = i * g.block + r0 + u * step + sub;
+      have[u] = r0 + u * step + sub < g.block && p < g.N;
+      raw[u] = have[u] ? __ldg(reinterpret_cast<const uint4*>(
+                             head + (int64_t)natural_index(g, order, p) * g.d) + slot)
+                       : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (ss > 0.f) {
-      const float inv = 1.f / sqrtf(ss);
+    for (int u = 0; u < 2; ++u) {
+      float v[kE];
+      Chunk<T>::unpack(raw[u], v);
+      float ss = 0.f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float h = v[e] * inv;
-        acc[e] += h;
-        dsum = fmaf(h, h, dsum);
+      for (int e = 0; e < kE; ++e) ss = fmaf(v[e], v[e], ss);
+      for (int o = L >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (have[u] && ss > 0.f) {
+        const float inv = rsqrtf(ss);
+#pragma unroll
+        for (int e = 0; e < kE; ++e) acc[e] = fmaf(v[e], inv, acc[e]);
+        if (slot == 0) dsum += ss * inv * inv;
       }
     }
   }
+  // fold the rows-per-load groups of the warp (lanes with the same slot)
+  for (int o = L; o < 32; o <<= 1) {
+#pragma unroll
+    for (int e = 0; e < kE; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
-  for (int e = 0; e < per; ++e) part[warp][lane * per + e] = acc[e];
+  if (lane < L) {
+#pragma unroll
+    for (int e = 0; e < kE; ++e) part[warp][slot * kE + e] = acc[e];
+  }
   if (lane == 0) diag_part[warp] = dsum;
   __syncthreads();
   if (warp == 0) {

@@ -5,7 +5,8 @@ Launch sequence of :meth:`Pipeline.run` (every step through the C ABI, on the
 current torch stream):
 
   bf16:  reorder+pool(q), reorder+pool(k), reorder(v)  -- one HBM pass each
-         score_pooled -> select_topk -> block_sparse_attn(permuted tiles)
+         score_pooled -> select_topk (or select_hybrid: diagonal, window,
+         Top-K and Top-P with per-row counts) -> block_sparse_attn(permuted tiles)
   int8:  quantize+pool(q), quantize+pool(k), quantize(v)
          score_pooled -> select_topk -> block_sparse_attn(int8)
 
@@ -22,12 +23,18 @@ from . import paro
 
 class Pipeline:
     def __init__(self, B, heads, grid, d, block, perms, density, dtype=torch.bfloat16,
-                 device="cuda", int8=False, baseline=False):
+                 device="cuda", int8=False, baseline=False, selection="topk", top_p=0.0,
+                 window=-1):
         self.pr = paro.Problem(B, heads, grid, d, block, perms)
         pr = self.pr
         self.k = paro.k_for_density(pr.NB, density)
         self.int8 = int8
         self.baseline = baseline
+        if selection not in ("topk", "hybrid"):
+            raise ValueError(f"selection {selection!r}: topk or hybrid")
+        self.selection = selection
+        self.top_p = float(top_p)
+        self.window = int(window)
         dev = torch.device(device)
         if int8:
             self.xq = [torch.empty((B, heads, pr.N_p, d), dtype=torch.int8, device=dev) for _ in range(3)]
@@ -37,7 +44,12 @@ class Pipeline:
         self.q_pool = torch.empty((B, heads, pr.NB, d), dtype=torch.float32, device=dev)
         self.k_pool = torch.empty_like(self.q_pool)
         self.scores = torch.empty((B, heads, pr.NB, pr.NB), dtype=torch.float32, device=dev)
-        self.idx = torch.empty((B, heads, pr.NB, self.k), dtype=torch.int32, device=dev)
+        if selection == "hybrid":  # variable counts: rows padded to NB
+            self.idx = torch.empty((B, heads, pr.NB, pr.NB), dtype=torch.int32, device=dev)
+            self.counts = torch.empty((B, heads, pr.NB), dtype=torch.int32, device=dev)
+        else:
+            self.idx = torch.empty((B, heads, pr.NB, self.k), dtype=torch.int32, device=dev)
+            self.counts = None
         out_dtype = torch.bfloat16 if int8 else dtype
         self.out = torch.empty((B, heads, pr.N, d), dtype=out_dtype, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -61,19 +73,31 @@ class Pipeline:
             paro.reorder(k, pr, out=self.xp[1], pool=self.k_pool)
             paro.reorder(v, pr, out=self.xp[2])
             paro.score_pooled(self.q_pool, self.k_pool, pr, scores=self.scores)
-        paro.select_topk(self.scores, pr, self.k, self.idx)
+        if self.selection == "hybrid":
+            paro.select_hybrid(self.scores, pr, self.k, self.top_p, self.window, self.idx,
+                               self.counts)
+        else:
+            paro.select_topk(self.scores, pr, self.k, self.idx)
 
     def attend(self, q, k, v):
         pr = self.pr
         if self.int8:
-            paro.block_sparse_attn(*self.xq, pr, self.idx, scales=tuple(self.sc), out=self.out,
-                                   status=self.status)
+            paro.block_sparse_attn(*self.xq, pr, self.idx, self.counts, scales=tuple(self.sc),
+                                   out=self.out, status=self.status)
         elif self.baseline:
-            paro.block_sparse_attn(q, k, v, pr, self.idx, out=self.out, status=self.status,
-                                   baseline=True)
+            paro.block_sparse_attn(q, k, v, pr, self.idx, self.counts, out=self.out,
+                                   status=self.status, baseline=True)
         else:
-            paro.block_sparse_attn(*self.xp, pr, self.idx, out=self.out, status=self.status,
-                                   permuted=True)
+            paro.block_sparse_attn(*self.xp, pr, self.idx, self.counts, out=self.out,
+                                   status=self.status, permuted=True)
+
+    def kept_tiles(self) -> int:
+        """Kept (query block, key block) tiles of the last selection (reads
+        the per-row counts back for the hybrid filter)."""
+        pr = self.pr
+        if self.counts is not None:
+            return int(self.counts.sum().item())
+        return pr.B * pr.heads * pr.NB * self.k
 
     def run(self, q, k, v):
         self.select(q, k, v)

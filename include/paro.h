@@ -160,8 +160,8 @@ PA_API pa_status pa_select_hybrid(const float* scores, pa_shape shape, int32_t k
  * order table above) and every (b,h):
  *   scores[b,h,o] = sum over the blocks of order o (runs of `block`
  *                   permuted tokens) of SICS(q's rows) + SICS(k's rows).
- * q, k natural order [B,heads,N,d] (PA_F32 or PA_BF16), d a multiple of 32
- * and <= 256; scores [B,heads,6] float, overwritten (accumulated in fp32
+ * q, k natural order [B,heads,N,d] (PA_F32 or PA_BF16), 16-byte aligned;
+ * scores [B,heads,6] float, overwritten (accumulated in fp32
  * with atomics, so the last bits vary between runs).  The order with the
  * largest score is SPADE's pick for the head. */
 PA_API pa_status pa_sics_scores(const void* q, const void* k, pa_dtype dtype, pa_shape shape,
