@@ -302,16 +302,19 @@ def attention_rows(q, k, v, grid, perms, block, idx, rows, counts=None):
 
 # ------------------------------------------------------------------ INT8 --
 
-def quantize_int8(xp: np.ndarray, N: int, block: int):
+def quantize_int8(xp: np.ndarray, N: int, block: int, qmax: int = 127):
     """Per-block symmetric INT8 quantisation (PAROAttention review,
     key_machinery: block-wise INT8 with groups aligned to the FlashAttention
-    block; QK^T in INT8 as in its SageAttention baseline).
+    block; QK^T in INT8 as in its SageAttention baseline).  ``qmax = 7`` is
+    the 4-bit variant (INT4 PV, same review: block-wise INT8/INT4
+    quantisation of the post-softmax map and PV), codes in [-7, 7].
 
-    Defined in float32 with IEEE round-to-nearest on every operation:
+    Defined in float32 with IEEE round-to-nearest on every operation
+    (Q = qmax):
       absmax = max |x| over the block's valid rows,
-      inv    = fl32(127 / absmax),
-      q      = clamp(round_half_even(fl32(x * inv)), -127, 127),
-      scale  = fl32(absmax / 127);
+      inv    = fl32(Q / absmax),
+      q      = clamp(round_half_even(fl32(x * inv)), -Q, Q),
+      scale  = fl32(absmax / Q);
     a block with absmax 0 gets q = 0 and scale 0.  Pad rows quantise to 0.
     xp: [B, h, N_p, d] permuted (values exactly representable in float32).
     Returns q [B, h, N_p, d] int8 and scales [B, h, NB] float32.
@@ -329,14 +332,15 @@ def quantize_int8(xp: np.ndarray, N: int, block: int):
                 amax = np.float32(np.abs(blk).max()) if hi > lo else np.float32(0)
                 if amax == 0:
                     continue
-                inv = np.float32(np.float32(127.0) / amax)
+                qf = np.float32(qmax)
+                inv = np.float32(qf / amax)
                 y = np.rint(blk * inv)  # float32 multiply, then half-even
-                q[b, h, lo:hi] = np.clip(y, -127, 127).astype(np.int8)
-                sc[b, h, i] = np.float32(amax / np.float32(127.0))
+                q[b, h, lo:hi] = np.clip(y, -qmax, qmax).astype(np.int8)
+                sc[b, h, i] = np.float32(amax / qf)
     return q, sc
 
 
-def _int8_query_rows(qi, ki, vi, sq_i, sk, sv, N, block, kept, mode, quantize_p):
+def _int8_query_rows(qi, ki, vi, sq_i, sk, sv, N, block, kept, mode, quantize_p, p_levels=127):
     """INT8 attention of some query rows of one query block (int64 codes
     ``qi`` [r, d], block scale ``sq_i``) over the kept key blocks, in the
     order listed.  Every step is row-wise, so any subset of a block's rows
@@ -367,7 +371,7 @@ def _int8_query_rows(qi, ki, vi, sq_i, sk, sv, N, block, kept, mode, quantize_p)
             m_new = m_row
             alpha = np.ones((rows, 1))
         pt = np.exp(s - m_new)
-        pq = np.rint(127.0 * pt) / 127.0 if quantize_p else pt
+        pq = np.rint(p_levels * pt) / p_levels if quantize_p else pt
         l = l * alpha + pt.sum(axis=1, keepdims=True)
         acc = acc * alpha + (pq @ vi[klo:khi].astype(np.float64)) * float(sv[j])
         m = m_new
@@ -375,7 +379,7 @@ def _int8_query_rows(qi, ki, vi, sq_i, sk, sv, N, block, kept, mode, quantize_p)
 
 
 def attention_int8(q8, k8, v8, sq, sk, sv, N: int, block: int, idx, counts=None,
-                   mode: str = "online", quantize_p: bool = True):
+                   mode: str = "online", quantize_p: bool = True, p_levels: int = 127):
     """INT8 block-sparse attention in the permuted domain, one head.
 
     S = (Q8 K8^T exact in integers) * s_q[i] * s_k[j] / sqrt(d) per tile.
@@ -392,6 +396,9 @@ def attention_int8(q8, k8, v8, sq, sk, sv, N: int, block: int, idx, counts=None,
     an online softmax) -- the order the pages describe.
     mode "rowmax": P_tilde = exp(s - m_row) with the row's final max.
     ``quantize_p=False`` skips the P rounding (P used exactly).
+    ``p_levels = 7`` quantises P to 4 bits, p4 = round_half_even(7 * P_tilde),
+    contributing (p4 V) * s_v[j] / 7 (the INT4 PV variant, with V from
+    quantize_int8(..., qmax=7)).
 
     q8/k8/v8 [Np, d] int8, sq/sk/sv [NB] float32, idx [NB, k]; returns
     [Np, d] float64 (pad rows zero).
@@ -409,12 +416,13 @@ def attention_int8(q8, k8, v8, sq, sk, sv, N: int, block: int, idx, counts=None,
         c = idx.shape[1] if counts is None else int(counts[i])
         kept = [int(j) for j in idx[i, :c]]
         out[lo:hi] = _int8_query_rows(qi[lo:hi], ki, vi, sq[i], sk, sv, N, block, kept, mode,
-                                      quantize_p)
+                                      quantize_p, p_levels)
     return out
 
 
 def attention_int8_rows(q8, k8, v8, sq, sk, sv, N: int, block: int, idx, positions,
-                        counts=None, mode: str = "online", quantize_p: bool = True):
+                        counts=None, mode: str = "online", quantize_p: bool = True,
+                        p_levels: int = 127):
     """Rows of :func:`attention_int8` at the given permuted positions only
     (one head), for full-size checks where the whole head is too costly.
     Returns [len(positions), d] float64."""
@@ -427,5 +435,5 @@ def attention_int8_rows(q8, k8, v8, sq, sk, sv, N: int, block: int, idx, positio
         c = idx.shape[1] if counts is None else int(counts[i])
         kept = [int(j) for j in idx[i, :c]]
         res[r] = _int8_query_rows(qi[p:p + 1], ki, vi, sq[i], sk, sv, N, block, kept, mode,
-                                  quantize_p)[0]
+                                  quantize_p, p_levels)[0]
     return res

@@ -149,3 +149,48 @@ def test_row_subset_matches_whole_head():
         rows = ref.attention_int8_rows(*args, pos, counts=counts, mode=mode)
         assert np.abs(rows - whole[pos]).max() < 1e-12
         assert (rows[3] == 0).all() and (rows[4] == 0).all()  # block 3: empty list
+
+
+def test_int4_codes_hand_example():
+    # absmax 7 -> inv = 1, scale = 1: the codes are the rounded values, |q| <= 7
+    blk = np.array([[7.0, 2.5, 3.5, -2.5], [-0.5, 0.5, 1.5, -7.0]], dtype=np.float32)
+    q, s = ref.quantize_int8(blk.reshape(1, 1, 2, 4), 2, 2, qmax=7)
+    assert q[0, 0].tolist() == [[7, 2, 4, -2], [0, 0, 2, -7]]
+    assert s[0, 0, 0] == np.float32(1.0)
+    # a general block: float32 arithmetic with Q = 7
+    x = np.array([[0.3, -0.1], [0.2, 0.05]], dtype=np.float32).reshape(1, 1, 2, 2)
+    q, s = ref.quantize_int8(x, 2, 2, qmax=7)
+    inv = np.float32(np.float32(7.0) / np.float32(0.3))
+    assert s[0, 0, 0] == np.float32(np.float32(0.3) / np.float32(7.0))
+    assert (q[0, 0] == np.clip(np.rint(x[0, 0] * inv), -7, 7)).all() and np.abs(q).max() == 7
+
+
+def test_int4_pv_exact_when_representable_and_bounded_otherwise():
+    rng = np.random.default_rng(17)
+    block, nb, d = 4, 3, 8
+    N = Np = block * nb
+    idx = np.tile(np.arange(nb, dtype=np.int32), (nb, 1))
+    # V with values on the 4-bit grid (absmax 7 per block) dequantises exactly;
+    # with P rounding off the INT4-PV oracle equals the float attention
+    xs = [rng.integers(-6, 7, size=(Np, d)).astype(np.float32) for _ in range(3)]
+    for x in xs:
+        for i in range(nb):
+            x[i * block, 0] = 7.0
+    q8, sq = ref.quantize_int8((xs[0] * 0.125).reshape(1, 1, Np, d), N, block)
+    k8, sk = ref.quantize_int8((xs[1] * 0.125).reshape(1, 1, Np, d), N, block)
+    v4, sv = ref.quantize_int8(xs[2].reshape(1, 1, Np, d), N, block, qmax=7)
+    assert (sv == 1).all() and (v4[0, 0] == xs[2]).all() and np.abs(v4).max() == 7
+    args = (q8[0, 0], k8[0, 0], v4[0, 0], sq[0, 0], sk[0, 0], sv[0, 0], N, block, idx)
+    exact = ref.attention_int8(*args, quantize_p=False, p_levels=7)
+    qd = q8[0, 0].astype(np.float64) * np.repeat(sq[0, 0], block)[:, None]
+    kd = k8[0, 0].astype(np.float64) * np.repeat(sk[0, 0], block)[:, None]
+    want = ref.attention_permuted(qd, kd, xs[2].astype(np.float64), N, block, idx)
+    assert np.abs(exact - want).max() < 1e-10
+    # 4-bit P: |dO_r| <= sum_c |dP_rc| |v_c| / l_r with |dP| <= 1/14, l_r >= 1
+    quant = ref.attention_int8(*args, p_levels=7)
+    bound = np.abs(xs[2].astype(np.float64)).sum(axis=0)[None, :] / 14.0
+    assert (np.abs(quant - exact) <= bound + 1e-12).all()
+    assert np.abs(quant - exact).max() > 0
+    # the 4-bit P codes are coarser than the 8-bit ones on the same inputs
+    p8 = ref.attention_int8(*args)
+    assert np.abs(quant - exact).max() > np.abs(p8 - exact).max()
