@@ -419,9 +419,12 @@ def run_sweep(a):
     for name, w in ([] if a.selection_only else WORKLOADS.items()):
         q, k, v, perms = make_inputs(w)
         qkv = [t.to(device) for t in (q, k, v)]
-        for precision in (["bf16", "int8"] if w.int8 else [w.dtype]):
-            int8 = precision == "int8"
+        for precision in (["bf16", "int8", "int4pv"] if w.int8 else [w.dtype]):
+            int8 = precision in ("int8", "int4pv")
             pipe = make_pipeline(w, perms, w.density, a.kernel, device, int8=int8)
+            if precision == "int4pv":
+                pipe = Pipeline(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, perms, w.density,
+                                device=device, int4_pv=True)
             for _ in range(10):
                 step(pipe, qkv)
             torch.cuda.synchronize()
@@ -440,7 +443,7 @@ def run_sweep(a):
                 raise RuntimeError(f"{name}: device status {int(pipe.status.item())}")
             flops = w.flops(pipe.k)
             pa, pt = percentiles(attn), percentiles(total)
-            dt = "int8" if int8 else w.dtype
+            dt = precision if int8 else w.dtype
             peak = tensor_peak(peaks, "int8" if int8 else "bf16", "bf16_tflops")
             print(json.dumps({
                 "workload": name, "precision": dt, "B": w.B, "heads": w.heads,

@@ -13,7 +13,8 @@ namespace paro {
 cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, pa_dtype dt,
                               const Grid& g, const int32_t* idx, const int32_t* counts,
                               int k_max, const float* qs, const float* ks, const float* vs,
-                              void* out, int32_t* status, bool permuted, cudaStream_t s);
+                              float p_levels, void* out, int32_t* status, bool permuted,
+                              cudaStream_t s);
 bool attn_sm100_supports(pa_dtype dt, const Grid& g);
 }  // namespace paro
 
@@ -234,16 +235,28 @@ pa_status pa_compact_mask(const uint32_t* bitmask, pa_shape shape, int32_t* idx,
                      "pa_compact_mask launch");
 }
 
-pa_status pa_quantize_int8(const void* x, pa_dtype dtype, pa_shape shape, const int8_t* perms,
-                           int8_t* x_q, float* scales, float* pool, void* stream) {
+static pa_status quantize_common(const void* x, pa_dtype dtype, pa_shape shape,
+                                 const int8_t* perms, int8_t* x_q, float* scales, float* pool,
+                                 int qmax, void* stream) {
   paro::Grid g;
   pa_status st = check_float_dtype(dtype);
   if (st != PA_OK) return st;
   if ((st = make_grid(shape, perms, true, &g)) != PA_OK) return st;
   PA_REQUIRE(x && x_q && scales, "x, x_q and scales must be non-NULL");
   PA_REQUIRE(aligned16(x) && aligned16(x_q), "x and x_q must be 16-byte aligned");
-  return cuda_status(paro::launch_quantize(x, dtype, g, x_q, scales, pool, (cudaStream_t)stream),
-                     "pa_quantize_int8 launch");
+  return cuda_status(
+      paro::launch_quantize(x, dtype, g, x_q, scales, pool, qmax, (cudaStream_t)stream),
+      "pa_quantize launch");
+}
+
+pa_status pa_quantize_int8(const void* x, pa_dtype dtype, pa_shape shape, const int8_t* perms,
+                           int8_t* x_q, float* scales, float* pool, void* stream) {
+  return quantize_common(x, dtype, shape, perms, x_q, scales, pool, 127, stream);
+}
+
+pa_status pa_quantize_int4(const void* x, pa_dtype dtype, pa_shape shape, const int8_t* perms,
+                           int8_t* x_q, float* scales, float* pool, void* stream) {
+  return quantize_common(x, dtype, shape, perms, x_q, scales, pool, 7, stream);
 }
 
 static pa_status attn_common(const void* q, const void* k, const void* v, pa_dtype dtype,
@@ -262,7 +275,9 @@ static pa_status attn_common(const void* q, const void* k, const void* v, pa_dty
   if (dtype == PA_I8) {
     PA_REQUIRE(q_scale && k_scale && v_scale, "INT8 attention needs q_scale, k_scale, v_scale");
   }
-  PA_REQUIRE((flags & ~PA_ATTN_PERMUTED) == 0, "unknown flags 0x%x", flags);
+  PA_REQUIRE((flags & ~(PA_ATTN_PERMUTED | PA_ATTN_P4)) == 0, "unknown flags 0x%x", flags);
+  PA_REQUIRE(!(flags & PA_ATTN_P4) || dtype == PA_I8, "PA_ATTN_P4 needs dtype PA_I8");
+  const float p_levels = (flags & PA_ATTN_P4) ? 7.f : 127.f;
   const bool permuted = dtype == PA_I8 || (flags & PA_ATTN_PERMUTED) != 0;
   cudaStream_t s = (cudaStream_t)stream;
   const bool sm100 = !force_mma && paro::attn_sm100_supports(dtype, g);
@@ -277,7 +292,7 @@ static pa_status attn_common(const void* q, const void* k, const void* v, pa_dty
   cudaError_t e;
   if (sm100)
     e = paro::launch_attn_sm100(q, k, v, dtype, g, idx, counts, k_max, q_scale, k_scale, v_scale,
-                                out, dev_status, permuted, s);
+                                p_levels, out, dev_status, permuted, s);
   else
     e = paro::launch_attn_mma(q, k, v, dtype, g, idx, counts, k_max, out, dev_status, permuted, s);
   return cuda_status(e, "pa_block_sparse_attn launch");

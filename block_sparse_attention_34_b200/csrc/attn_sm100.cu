@@ -517,10 +517,11 @@ bool attn_sm100_supports(pa_dtype dt, const Grid& g) {
 cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, pa_dtype dt,
                               const Grid& g, const int32_t* idx, const int32_t* counts,
                               int k_max, const float* qs, const float* ks, const float* vs,
-                              void* out, int32_t* status, bool permuted, cudaStream_t s) {
+                              float p_levels, void* out, int32_t* status, bool permuted,
+                              cudaStream_t s) {
   if (!attn_sm100_supports(dt, g)) return cudaErrorInvalidValue;
   if (dt == PA_I8)
-    return launch_attn_i8(q, k, v, g, idx, counts, k_max, qs, ks, vs, out, status, s);
+    return launch_attn_i8(q, k, v, g, idx, counts, k_max, qs, ks, vs, p_levels, out, status, s);
   CUtensorMap mq{}, mk{}, mv{};
   if (permuted) {
     const uint64_t rows = (uint64_t)g.B * g.heads * g.Np;

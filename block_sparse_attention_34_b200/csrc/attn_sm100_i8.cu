@@ -13,6 +13,8 @@
 //   P8     = round_half_even(127 P~)           (the tile's symmetric scale 1/127)
 //   l      = l 2^(m_old - m) + sum P~
 //   O      = O 2^(m_old - m) + (P8 V8_j, exact int32) * s_v[j] / 127
+// (with 4-bit P, the INT4 PV variant: 7 in place of 127, and V codes in
+// [-7, 7] from pa_quantize_int4; the integer MMAs are unchanged)
 // and O / l is stored at the natural positions of the block's tokens.
 //
 // One CTA per (query block, head); 14 warps in four roles:
@@ -128,14 +130,15 @@ __device__ __forceinline__ float2 exact_float2(uint32_t a, uint32_t b) {
                make_float2(-kMagic, -kMagic));
 }
 
-// P~ = 2^(s - m) <= 1 for 64 columns of one row, P8 = rne(127 P~) as the
-// low byte of the float 127 P~ + 1.5 * 2^23 (one rounding to the nearest
-// integer, ties to even), packed 4 per 32-bit word; row sums of P~ in rs.
+// P~ = 2^(s - m) <= 1 for 64 columns of one row, P codes = rne(L P~) (L =
+// levels: 127, or 7 for 4-bit P) as the low byte of the float L P~ + 1.5 *
+// 2^23 (one rounding to the nearest integer, ties to even), packed 4 per
+// 32-bit word; row sums of P~ in rs.
 template <bool kRagged>
 __device__ __forceinline__ void tile_exp(const uint32_t (&sr)[64], float2 cq2, float2 nm2,
                                          int valid, float2& rs0, float2& rs1,
-                                         uint32_t (&pk)[16]) {
-  const float2 k127 = make_float2(127.f, 127.f), mg2 = make_float2(kMagic, kMagic);
+                                         uint32_t (&pk)[16], float levels) {
+  const float2 k127 = make_float2(levels, levels), mg2 = make_float2(kMagic, kMagic);
 #pragma unroll
   for (int c = 0; c < 16; ++c) {
     const float2 t0 = ffma2(exact_float2(sr[4 * c], sr[4 * c + 1]), cq2, nm2);
@@ -163,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap map_v, const __grid_constant__ Grid g,
                    const int32_t* __restrict__ idx, const int32_t* __restrict__ counts, int k_max,
                    const float* __restrict__ q_scale, const float* __restrict__ k_scale,
-                   const float* __restrict__ v_scale, float log2e_over_sqrt_d,
+                   const float* __restrict__ v_scale, float log2e_over_sqrt_d, float p_levels,
                    __nv_bfloat16* __restrict__ out, int32_t* __restrict__ status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t base = smem_u32(smem_raw);
@@ -465,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // completed before P V(j - 2) was issued, and so before QK(j)
         const int sl = j & (kScaleSlots - 1);
         s_alpha[sl * 128 + r] = alpha;
-        s_cv[sl * 128 + r] = vsc * (1.f / 127.f);
+        s_cv[sl * 128 + r] = __fdiv_rn(vsc, p_levels);
         mbar_arrive(bar(BSC0 + sl));
       }
       // P~ = 2^(s - m) <= 1, P8 = rne(127 P~): the low byte of the float
@@ -474,9 +477,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       float2 rs0 = make_float2(0.f, 0.f), rs1 = make_float2(0.f, 0.f);
       uint32_t pk[16];
       if (valid >= 64)
-        tile_exp<false>(sr, cq2, nm2, valid, rs0, rs1, pk);
+        tile_exp<false>(sr, cq2, nm2, valid, rs0, rs1, pk, p_levels);
       else
-        tile_exp<true>(sr, cq2, nm2, valid, rs0, rs1, pk);
+        tile_exp<true>(sr, cq2, nm2, valid, rs0, rs1, pk, p_levels);
       const float2 rs = fadd2(rs0, rs1);
       l2 = ffma2(l2, make_float2(alpha, alpha), rs);
       // this half row of P8 (64 bytes = 4 chunks of 16) into the swizzled
@@ -511,8 +514,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_attn_i8(const void* q, const void* k, const void* v, const Grid& g,
                            const int32_t* idx, const int32_t* counts, int k_max, const float* qs,
-                           const float* ks, const float* vs, void* out, int32_t* status,
-                           cudaStream_t s) {
+                           const float* ks, const float* vs, float p_levels, void* out,
+                           int32_t* status, cudaStream_t s) {
   if (g.d != kD || g.block != kBlock) return cudaErrorInvalidValue;
   const uint64_t rows = (uint64_t)g.B * g.heads * g.Np;
   CUtensorMap mq{}, mk{}, mv{};
@@ -526,7 +529,8 @@ cudaError_t launch_attn_i8(const void* q, const void* k, const void* v, const Gr
   const float c = (float)(1.4426950408889634 / sqrt((double)kD));
   dim3 grid(g.NB, g.B * g.heads);
   attn_i8_kernel<<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, g, idx, counts, k_max, qs, ks, vs,
-                                                    c, static_cast<__nv_bfloat16*>(out), status);
+                                                    c, p_levels, static_cast<__nv_bfloat16*>(out),
+                                                    status);
   return cudaGetLastError();
 }
 

@@ -93,8 +93,9 @@ cudaError_t launch_score(const float* qp, const float* kp, const Grid& g, float*
 cudaError_t launch_topk(const float* scores, const Grid& g, int k, int32_t* idx, cudaStream_t s);
 cudaError_t launch_compact(const uint32_t* bm, const Grid& g, int32_t* idx, int32_t* counts,
                            cudaStream_t s);
+// qmax: 127 for INT8 codes, 7 for 4-bit codes (one per byte)
 cudaError_t launch_quantize(const void* x, pa_dtype dt, const Grid& g, int8_t* xq, float* scales,
-                            float* pool, cudaStream_t s);
+                            float* pool, int qmax, cudaStream_t s);
 cudaError_t launch_attn_mma(const void* q, const void* k, const void* v, pa_dtype dt,
                             const Grid& g, const int32_t* idx, const int32_t* counts, int k_max,
                             void* out, int32_t* status, bool permuted, cudaStream_t s);
@@ -103,8 +104,9 @@ cudaError_t launch_sics(const void* x, pa_dtype dt, const Grid& g, float* scores
 cudaError_t launch_hybrid(const float* scores, const Grid& g, int k, double p, int w,
                           int32_t* idx, int32_t* counts, cudaStream_t s);
 // INT8 tcgen05 attention (d = 128, block = 128, permuted int8 inputs)
+// p_levels: P codes round_half_even(p_levels * P~); 127 (INT8) or 7 (4-bit)
 cudaError_t launch_attn_i8(const void* q, const void* k, const void* v, const Grid& g,
                            const int32_t* idx, const int32_t* counts, int k_max, const float* qs,
-                           const float* ks, const float* vs, void* out, int32_t* status,
-                           cudaStream_t s);
+                           const float* ks, const float* vs, float p_levels, void* out,
+                           int32_t* status, cudaStream_t s);
 }  // namespace paro

@@ -245,7 +245,7 @@ template <typename T, int D, int BLOCK>
 __global__ void __launch_bounds__(kThreads) quant_kernel(const T* __restrict__ x, const __grid_constant__ Grid g,
                                                          int8_t* __restrict__ xq,
                                                          float* __restrict__ scales,
-                                                         float* __restrict__ pool) {
+                                                         float* __restrict__ pool, int qmax) {
   constexpr int E = Chunk<T>::n;
   constexpr int VPR = D / E;
   constexpr int GROUPS = kThreads / VPR;
@@ -294,7 +294,8 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const T* __restrict__ x
   amax = 0.f;
 #pragma unroll
   for (int w = 0; w < kThreads / 32; ++w) amax = fmaxf(amax, red[w]);
-  const float inv = amax > 0.f ? __fdiv_rn(127.f, amax) : 0.f;
+  const float qf = (float)qmax;
+  const float inv = amax > 0.f ? __fdiv_rn(qf, amax) : 0.f;
   int8_t* outb = xq + (bh * (int64_t)g.Np + p0) * D;
 #pragma unroll
   for (int u = 0; u < RPT; ++u) {
@@ -306,7 +307,7 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const T* __restrict__ x
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
         int qv = __float2int_rn(__fmul_rn(v[u][e4 * 4 + b], inv));
-        qv = max(-127, min(127, qv));
+        qv = max(-qmax, min(qmax, qv));
         wv |= (uint32_t)(qv & 0xFF) << (8 * b);
       }
       packed[e4] = wv;
@@ -318,7 +319,7 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const T* __restrict__ x
       *reinterpret_cast<uint32_t*>(dst) = packed[0];
     }
   }
-  if (threadIdx.x == 0) scales[bh * g.NB + i] = amax > 0.f ? __fdiv_rn(amax, 127.f) : 0.f;
+  if (threadIdx.x == 0) scales[bh * g.NB + i] = amax > 0.f ? __fdiv_rn(amax, qf) : 0.f;
   if (pool != nullptr) {
     for (int col = threadIdx.x; col < D; col += kThreads) {
       float s = 0.f;
@@ -395,20 +396,21 @@ cudaError_t launch_compact(const uint32_t* bm, const Grid& g, int32_t* idx, int3
 
 template <typename T, int D, int BLOCK>
 static void quant_launch(const void* x, const Grid& g, int8_t* xq, float* sc, float* pool,
-                         cudaStream_t s) {
+                         int qmax, cudaStream_t s) {
   dim3 grid(g.NB, g.B * g.heads);
-  quant_kernel<T, D, BLOCK><<<grid, kThreads, 0, s>>>(static_cast<const T*>(x), g, xq, sc, pool);
+  quant_kernel<T, D, BLOCK><<<grid, kThreads, 0, s>>>(static_cast<const T*>(x), g, xq, sc, pool,
+                                                      qmax);
 }
 
 cudaError_t launch_quantize(const void* x, pa_dtype dt, const Grid& g, int8_t* xq, float* scales,
-                            float* pool, cudaStream_t s) {
+                            float* pool, int qmax, cudaStream_t s) {
   const bool bf = dt == PA_BF16;
 #define PARO_Q(D, BL)                                                        \
   if (g.d == D && g.block == BL) {                                           \
     if (bf)                                                                  \
-      quant_launch<__nv_bfloat16, D, BL>(x, g, xq, scales, pool, s);         \
+      quant_launch<__nv_bfloat16, D, BL>(x, g, xq, scales, pool, qmax, s);   \
     else                                                                     \
-      quant_launch<float, D, BL>(x, g, xq, scales, pool, s);                 \
+      quant_launch<float, D, BL>(x, g, xq, scales, pool, qmax, s);           \
     return cudaGetLastError();                                               \
   }
   PARO_Q(64, 64)

@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libparo.so")
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_TIMEOUT, PA_ERR_DEVICE_CHECK = range(6)
 PA_F32, PA_BF16, PA_I8 = 0, 1, 2
 PA_ATTN_PERMUTED = 1
+PA_ATTN_P4 = 2  # with int8 inputs: 4-bit P codes (INT4 PV)
 STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_CUDA",
                 4: "PA_ERR_TIMEOUT", 5: "PA_ERR_DEVICE_CHECK"}
 ORDER_IDS = {"FHW": 0, "FWH": 1, "HFW": 2, "HWF": 3, "WFH": 4, "WHF": 5}
@@ -63,6 +64,7 @@ def load():
         "pa_select_hybrid": ([_P, PaShape, _I, ctypes.c_double, _I, _P, _P, _P], _I),
         "pa_sics_scores": ([_P, _P, _I, PaShape, _P, _P], _I),
         "pa_quantize_int8": ([_P, _I, PaShape, _P, _P, _P, _P, _P], _I),
+        "pa_quantize_int4": ([_P, _I, PaShape, _P, _P, _P, _P, _P], _I),
         "pa_block_sparse_attn": ([_P, _P, _P, _I, ctypes.c_uint32, PaShape, _P, _P, _P, _I, _P, _P, _P,
                                   _P, _P, _P], _I),
         "pa_block_sparse_attn_mma": ([_P, _P, _P, _I, ctypes.c_uint32, PaShape, _P, _P, _P, _I, _P, _P,
@@ -215,20 +217,25 @@ def sics_scores(q, k, pr: Problem, scores=None):
     return scores
 
 
-def quantize_int8(x, pr: Problem, with_pool=False, x_q=None, scales=None, pool=None):
+def quantize_int8(x, pr: Problem, with_pool=False, x_q=None, scales=None, pool=None, bits=8):
+    """Per-block symmetric quantisation in the permuted order: 8-bit codes
+    (levels +-127), or ``bits=4`` (levels +-7, one code per byte)."""
     _need_cuda(x)
     dev = x.device
     x_q = x_q if x_q is not None else torch.empty((pr.B, pr.heads, pr.N_p, pr.d), dtype=torch.int8, device=dev)
     scales = scales if scales is not None else torch.empty((pr.B, pr.heads, pr.NB), dtype=torch.float32, device=dev)
     if with_pool and pool is None:
         pool = torch.empty((pr.B, pr.heads, pr.NB, pr.d), dtype=torch.float32, device=dev)
-    _check(load().pa_quantize_int8(_ptr(x), _dtype_code(x), pr.shape, pr.perms_ptr, _ptr(x_q),
+    if bits not in (4, 8):
+        raise ValueError(f"bits={bits}: 4 or 8")
+    fn = load().pa_quantize_int8 if bits == 8 else load().pa_quantize_int4
+    _check(fn(_ptr(x), _dtype_code(x), pr.shape, pr.perms_ptr, _ptr(x_q),
                                    _ptr(scales), _ptr(pool), _stream()))
     return (x_q, scales, pool) if with_pool else (x_q, scales)
 
 
 def block_sparse_attn(q, k, v, pr: Problem, idx, counts=None, scales=None, out=None,
-                      status=None, baseline=False, permuted=False):
+                      status=None, baseline=False, permuted=False, p4=False):
     """O = block-sparse attention over the kept tiles, natural token order.
 
     ``permuted``: q, k, v are [B, heads, N_p, d] from :func:`reorder`.
@@ -240,7 +247,7 @@ def block_sparse_attn(q, k, v, pr: Problem, idx, counts=None, scales=None, out=N
     out_dtype = torch.bfloat16 if code == PA_I8 else q.dtype
     out = out if out is not None else torch.empty((pr.B, pr.heads, pr.N, pr.d), dtype=out_dtype, device=q.device)
     k_max = int(idx.shape[-1])
-    flags = PA_ATTN_PERMUTED if permuted else 0
+    flags = (PA_ATTN_PERMUTED if permuted else 0) | (PA_ATTN_P4 if p4 else 0)
     lib = load()
     if baseline:
         st = lib.pa_block_sparse_attn_mma(_ptr(q), _ptr(k), _ptr(v), code, flags, pr.shape,
@@ -256,7 +263,7 @@ def block_sparse_attn(q, k, v, pr: Problem, idx, counts=None, scales=None, out=N
 
 
 def attention(q, k, v, grid, perms, block, density, int8=False, baseline=False, status=None,
-              permuted=True):
+              permuted=True, int4_pv=False):
     """The whole path for one call: reorder with block means (one read of
     q, k, v) -> pooled block scores -> top-k kept blocks -> block-sparse
     attention over the permuted tiles, stored back in natural order.
@@ -268,10 +275,11 @@ def attention(q, k, v, grid, perms, block, density, int8=False, baseline=False, 
     if int8:
         q8, qs, qp = quantize_int8(q, pr, with_pool=True)
         k8, ks, kp = quantize_int8(k, pr, with_pool=True)
-        v8, vs = quantize_int8(v, pr)
+        v8, vs = quantize_int8(v, pr, bits=4 if int4_pv else 8)
         scores = score_pooled(qp, kp, pr)
         idx = select_topk(scores, pr, kk)
-        return block_sparse_attn(q8, k8, v8, pr, idx, scales=(qs, ks, vs), status=status), idx
+        return block_sparse_attn(q8, k8, v8, pr, idx, scales=(qs, ks, vs), status=status,
+                                 p4=int4_pv), idx
     if permuted and not baseline:
         qp, q_pool = reorder(q, pr, with_pool=True)
         kp, k_pool = reorder(k, pr, with_pool=True)

@@ -7,8 +7,8 @@ current torch stream):
   bf16:  reorder+pool(q), reorder+pool(k), reorder(v)  -- one HBM pass each
          score_pooled -> select_topk (or select_hybrid: diagonal, window,
          Top-K and Top-P with per-row counts) -> block_sparse_attn(permuted tiles)
-  int8:  quantize+pool(q), quantize+pool(k), quantize(v)
-         score_pooled -> select_topk -> block_sparse_attn(int8)
+  int8:  quantize+pool(q), quantize+pool(k), quantize(v)  (v to 4 bits with int4_pv)
+         score_pooled -> select_topk -> block_sparse_attn(int8; 4-bit P with int4_pv)
 
 The output is written in natural token order; the inverse reorder is the
 attention kernel's store.
@@ -24,11 +24,12 @@ from . import paro
 class Pipeline:
     def __init__(self, B, heads, grid, d, block, perms, density, dtype=torch.bfloat16,
                  device="cuda", int8=False, baseline=False, selection="topk", top_p=0.0,
-                 window=-1):
+                 window=-1, int4_pv=False):
         self.pr = paro.Problem(B, heads, grid, d, block, perms)
         pr = self.pr
         self.k = paro.k_for_density(pr.NB, density)
-        self.int8 = int8
+        self.int8 = int8 or int4_pv
+        self.int4_pv = int4_pv
         self.baseline = baseline
         if selection not in ("topk", "hybrid"):
             raise ValueError(f"selection {selection!r}: topk or hybrid")
@@ -36,7 +37,7 @@ class Pipeline:
         self.top_p = float(top_p)
         self.window = int(window)
         dev = torch.device(device)
-        if int8:
+        if self.int8:
             self.xq = [torch.empty((B, heads, pr.N_p, d), dtype=torch.int8, device=dev) for _ in range(3)]
             self.sc = [torch.empty((B, heads, pr.NB), dtype=torch.float32, device=dev) for _ in range(3)]
         elif not baseline:
@@ -50,7 +51,7 @@ class Pipeline:
         else:
             self.idx = torch.empty((B, heads, pr.NB, self.k), dtype=torch.int32, device=dev)
             self.counts = None
-        out_dtype = torch.bfloat16 if int8 else dtype
+        out_dtype = torch.bfloat16 if self.int8 else dtype
         self.out = torch.empty((B, heads, pr.N, d), dtype=out_dtype, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
 
@@ -64,7 +65,8 @@ class Pipeline:
         if self.int8:
             paro.quantize_int8(q, pr, x_q=self.xq[0], scales=self.sc[0], pool=self.q_pool)
             paro.quantize_int8(k, pr, x_q=self.xq[1], scales=self.sc[1], pool=self.k_pool)
-            paro.quantize_int8(v, pr, x_q=self.xq[2], scales=self.sc[2])
+            paro.quantize_int8(v, pr, x_q=self.xq[2], scales=self.sc[2],
+                               bits=4 if self.int4_pv else 8)
             paro.score_pooled(self.q_pool, self.k_pool, pr, scores=self.scores)
         elif self.baseline:
             paro.block_score(q, k, pr, self.q_pool, self.k_pool, self.scores)
@@ -83,7 +85,7 @@ class Pipeline:
         pr = self.pr
         if self.int8:
             paro.block_sparse_attn(*self.xq, pr, self.idx, self.counts, scales=tuple(self.sc),
-                                   out=self.out, status=self.status)
+                                   out=self.out, status=self.status, p4=self.int4_pv)
         elif self.baseline:
             paro.block_sparse_attn(q, k, v, pr, self.idx, self.counts, out=self.out,
                                    status=self.status, baseline=True)

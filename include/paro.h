@@ -189,6 +189,12 @@ PA_API pa_status pa_compact_mask(const uint32_t* bitmask, pa_shape shape, int32_
 PA_API pa_status pa_quantize_int8(const void* x, pa_dtype dtype, pa_shape shape, const int8_t* perms,
                            int8_t* x_q, float* scales, float* pool, void* stream);
 
+/* The same quantisation with 4-bit levels (the INT4 PV variant): 7 in place
+ * of 127 everywhere above, codes in [-7, 7], one per int8 byte (the tensor
+ * cores take them as int8 operands, so the products stay exact). */
+PA_API pa_status pa_quantize_int4(const void* x, pa_dtype dtype, pa_shape shape, const int8_t* perms,
+                           int8_t* x_q, float* scales, float* pool, void* stream);
+
 /* Step 4 + fused step 5 (SPADE review, key_machinery (iii): flash
  * block-sparse attention with an online softmax; the inverse reorder is
  * the output store).  For every valid query token n of head (b,h), with
@@ -223,6 +229,12 @@ PA_API pa_status pa_quantize_int8(const void* x, pa_dtype dtype, pa_shape shape,
  * PA_I8 inputs are always permuted (the flag is implied).  The output is
  * always natural order. */
 #define PA_ATTN_PERMUTED 1u
+/* With PA_I8: P is quantised to 4 bits, p4 = round_half_even(7 P~), and the
+ * tile contributes (p4 V) * v_scale / 7 — the INT4 PV variant
+ * (PAROAttention review: block-wise INT8/INT4 quantisation of the
+ * post-softmax map and PV), with v (and its scales) from pa_quantize_int4;
+ * q and k stay INT8. */
+#define PA_ATTN_P4 2u
 
 PA_API pa_status pa_block_sparse_attn(const void* q, const void* k, const void* v, pa_dtype dtype,
                                uint32_t flags, pa_shape shape, const int8_t* perms, const int32_t* idx,

@@ -123,3 +123,15 @@ def test_selection_variant_validation(lib):
     # SICS: float inputs only, non-null buffers
     assert lib.pa_sics_scores(FAKE, FAKE, paro.PA_I8, good, FAKE, None) == paro.PA_ERR_INVALID_ARG
     assert lib.pa_sics_scores(FAKE, None, paro.PA_BF16, good, FAKE, None) == paro.PA_ERR_INVALID_ARG
+
+
+def test_p4_flag_validation(lib):
+    good = paro.PaShape(1, 2, 4, 8, 8, 64, 64)
+    keep, pp = perms_of(0, 5)
+    # PA_ATTN_P4 needs int8 inputs; unknown bits are refused
+    assert lib.pa_block_sparse_attn(FAKE, FAKE, FAKE, paro.PA_BF16, paro.PA_ATTN_P4, good, pp, FAKE,
+                                    None, 1, None, None, None, FAKE, None, None) == paro.PA_ERR_INVALID_ARG
+    assert b"P4" in lib.pa_last_error()
+    assert lib.pa_block_sparse_attn(FAKE, FAKE, FAKE, paro.PA_BF16, 4, good, pp, FAKE,
+                                    None, 1, None, None, None, FAKE, None, None) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_quantize_int4(FAKE, paro.PA_I8, good, pp, FAKE, FAKE, None, None) == paro.PA_ERR_INVALID_ARG

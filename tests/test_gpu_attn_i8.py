@@ -34,23 +34,24 @@ def problem(w, perms, heads=None):
     return paro.Problem(w.B, heads or w.heads, (w.F, w.H, w.W), w.d, w.block, perms)
 
 
-def quantized(w, pr, perms, *xs):
-    """GPU codes/scales of each input, checked bit-exact against the
-    oracle's quantisation of the same permuted float32 values; returns
-    ([(x8, scale)] on the device, [(x8, scale)] of the oracle)."""
+def quantized(w, pr, perms, *xs, bits=(8, 8, 8)):
+    """GPU codes/scales of each input (8-bit, or 4-bit where bits says so),
+    checked bit-exact against the oracle's quantisation of the same permuted
+    float32 values; returns ([(x8, scale)] on the device, [(x8, scale)] of
+    the oracle)."""
     dev, host = [], []
-    for x in xs:
+    for x, nbits in zip(xs, bits):
         (xd,) = to_dev(x)
-        x8, sc = paro.quantize_int8(xd, pr)
+        x8, sc = paro.quantize_int8(xd, pr, bits=nbits)
         xp = ref.reorder(x.float().numpy(), (w.F, w.H, w.W), perms, w.block)
-        want8, want_sc = ref.quantize_int8(xp, w.N, w.block)
+        want8, want_sc = ref.quantize_int8(xp, w.N, w.block, qmax=127 if nbits == 8 else 7)
         assert (x8.cpu().numpy() == want8).all() and (sc.cpu().numpy() == want_sc).all()
         dev.append((x8, sc))
         host.append((want8, want_sc))
     return dev, host
 
 
-def oracle_int8(w, perms, host, idx, counts=None):
+def oracle_int8(w, perms, host, idx, counts=None, p_levels=127):
     """Oracle INT8 attention of every head, mapped to natural order."""
     (q8, sq), (k8, sk), (v8, sv) = host
     B, nh = q8.shape[:2]
@@ -59,16 +60,17 @@ def oracle_int8(w, perms, host, idx, counts=None):
         for h in range(nh):
             outp[b, h] = ref.attention_int8(q8[b, h], k8[b, h], v8[b, h], sq[b, h], sk[b, h],
                                             sv[b, h], w.N, w.block, idx[b, h],
-                                            None if counts is None else counts[b, h])
+                                            None if counts is None else counts[b, h],
+                                            p_levels=p_levels)
     return ref.inverse_reorder(outp, (w.F, w.H, w.W), perms)
 
 
-def run_i8(pr, dev, idx, counts=None, out=None):
+def run_i8(pr, dev, idx, counts=None, out=None, p4=False):
     (q8, sq), (k8, sk), (v8, sv) = dev
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = paro.block_sparse_attn(q8, k8, v8, pr, torch.as_tensor(idx).cuda(),
                                  None if counts is None else torch.as_tensor(counts).cuda(),
-                                 scales=(sq, sk, sv), out=out, status=status)
+                                 scales=(sq, sk, sv), out=out, status=status, p4=p4)
     torch.cuda.synchronize()
     return out, status.item()
 
@@ -198,3 +200,36 @@ def test_i8_longclip_full_size_sampled():
         errs.append(np.abs(got - want))
     err = np.concatenate(errs)
     assert err.max() <= INT8_MAX_ABS and err.mean() <= INT8_MEAN_ABS, (err.max(), err.mean())
+
+
+@pytest.mark.parametrize("w", CASES[:3], ids=lambda w: w.name)
+def test_int4_pv_small(w):
+    """INT4 PV: q, k 8-bit, v 4-bit codes (bit-exact against the oracle's
+    quantiser), P to 4 bits in the kernel; against the oracle's INT4-PV
+    semantics."""
+    q, k, v, perms = inputs(w)
+    pr = problem(w, perms)
+    dev, host = quantized(w, pr, perms, q, k, v, bits=(8, 8, 4))
+    assert int(dev[2][0].abs().max().item()) <= 7
+    idx_ref, _, _ = oracle_topk(q, k, w, perms)
+    out, st = run_i8(pr, dev, idx_ref, p4=True)
+    assert st == 0
+    compare(out, oracle_int8(w, perms, host, idx_ref, p_levels=7), INT8_MAX_ABS, INT8_MEAN_ABS)
+
+
+def test_int4_pv_whole_path():
+    w = CASES[1]
+    q, k, v, perms = inputs(w)
+    pr = problem(w, perms)
+    qd, kd, vd = to_dev(q, k, v)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, idx = paro.attention(qd, kd, vd, (w.F, w.H, w.W), perms, w.block, w.density, int8=True,
+                              int4_pv=True, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    idx_ref, s_ref, _ = oracle_topk(q, k, w, perms)
+    agree = selection_agreement(idx.cpu().numpy(), idx_ref, s_ref)
+    _, host = quantized(w, pr, perms, q, k, v, bits=(8, 8, 4))
+    want = oracle_int8(w, perms, host, idx_ref, p_levels=7)
+    compare_rows(out, want, token_mask(agree, (w.F, w.H, w.W), perms, w.block), INT8_MAX_ABS,
+                 INT8_MEAN_ABS)
