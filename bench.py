@@ -460,6 +460,7 @@ def run_sweep(a):
             del pipe
         del qkv
     run_sweep_selection(device, peaks, peak_src, a.heads)
+    run_sweep_offline(device, peaks, peak_src, a.heads)
 
 
 def timed_calls(fn, reps=20, warm=5):
@@ -527,6 +528,36 @@ def run_sweep_selection(device, peaks, peak_src, heads=None):
         "frac_of_burst_peak_p50": flops / (pa["p50"] / 1e3) / 1e12 / peak,
         "peak_source": f"{peak_src} bf16_tflops", "kernel": attn_kernel_name(pipe),
         "steps": len(attn), "warmup": 10,
+    }), flush=True)
+
+
+def run_sweep_offline(device, peaks, peak_src, heads=None):
+    """PAROAttention's offline stage on the 480p layer: the dense map's row
+    softmax (one pass) and block statistics of all six orders (six passes),
+    metric and choice, and the static masks: every pass is a dense QK^T
+    (2 b^2 d FLOP per tile) plus one exp2 per map entry."""
+    w = WORKLOADS["480p_21x30x52"]
+    q, k, _, _ = make_inputs(w, heads=heads)
+    if heads is not None:
+        w = dataclasses.replace(w, heads=heads)
+    qd, kd = q.to(device), k.to(device)
+    grid = (w.F, w.H, w.W)
+    res = {}
+    ms = timed_calls(lambda: res.update(paro.paro_offline(qd, kd, grid, w.block)), reps=5, warm=2)
+    pm = percentiles(ms)
+    nb = -(-w.N // w.block)
+    tiles = 7 * w.B * w.heads * nb * nb  # 1 row-softmax pass + 6 block-statistics passes
+    flops = 2.0 * w.block * w.block * w.d * tiles
+    peak = tensor_peak(peaks, "bf16", "bf16_tflops")
+    print(json.dumps({
+        "workload": w.name, "what": "PARO offline stage: row softmax + 6 orders' block statistics,"
+        " metric, order choice, static masks (sigma 0.9)", "heads": w.heads,
+        "ms": pm, "tiles": tiles, "qk_flops": flops, "tflops_p50": flops / (pm["p50"] / 1e3) / 1e12,
+        "frac_of_burst_peak_p50": flops / (pm["p50"] / 1e3) / 1e12 / peak,
+        "exp2_per_s_p50": tiles * w.block * w.block / (pm["p50"] / 1e3),
+        "orders_chosen": res["orders"].cpu().flatten().tolist(),
+        "mask_density": float(res["counts"].sum().item()) / (w.B * w.heads * nb * nb),
+        "peak_source": f"{peak_src} bf16_tflops", "steps": len(ms),
     }), flush=True)
 
 

@@ -110,7 +110,7 @@ pa_status check_float_dtype(pa_dtype dt) {
 
 extern "C" {
 
-int32_t pa_abi_version(void) { return 3; }
+int32_t pa_abi_version(void) { return 4; }
 
 const char* pa_last_error(void) { return g_error.c_str(); }
 
@@ -223,6 +223,82 @@ pa_status pa_sics_scores(const void* q, const void* k, pa_dtype dtype, pa_shape 
   if (e == cudaSuccess) e = paro::launch_sics(q, dtype, g, scores, s);
   if (e == cudaSuccess) e = paro::launch_sics(k, dtype, g, scores, s);
   return cuda_status(e, "pa_sics_scores launch");
+}
+
+static pa_status map_common(const void* qp, const void* kp, pa_shape shape, int32_t order,
+                            paro::Grid* g) {
+  pa_status st = make_grid(shape, nullptr, false, g);
+  if (st != PA_OK) return st;
+  PA_REQUIRE(qp && kp, "q_perm and k_perm must be non-NULL");
+  PA_REQUIRE(aligned16(qp) && aligned16(kp), "q_perm and k_perm must be 16-byte aligned");
+  PA_REQUIRE(order >= 0 && order < 6, "order=%d must be in [0, 6)", order);
+  if (g->d != 128 || g->block != 128)
+    return fail(PA_ERR_UNSUPPORTED, "the map statistics need d=128, block=128 (tcgen05 kernel)");
+  if ((int64_t)g->B * g->heads * g->Np >= ((int64_t)1 << 31))
+    return fail(PA_ERR_UNSUPPORTED, "B*heads*N_p exceeds 2^31 rows");
+  return PA_OK;
+}
+
+pa_status pa_map_row_stats(const void* q_perm, const void* k_perm, pa_shape shape, int32_t order,
+                           float* row_max, float* row_sum, int32_t* dev_status, void* stream) {
+  paro::Grid g;
+  pa_status st = map_common(q_perm, k_perm, shape, order, &g);
+  if (st != PA_OK) return st;
+  PA_REQUIRE(row_max && row_sum, "row_max and row_sum must be non-NULL");
+  return cuda_status(paro::launch_map_stats(q_perm, k_perm, g, order, false, row_max, row_sum,
+                                            0.f, nullptr, nullptr, nullptr, dev_status,
+                                            (cudaStream_t)stream),
+                     "pa_map_row_stats launch");
+}
+
+pa_status pa_map_block_stats(const void* q_perm, const void* k_perm, pa_shape shape,
+                             int32_t order, const float* row_max, const float* row_sum, float eps,
+                             float* count, float* total, float* peak, float* log_total,
+                             int32_t* dev_status, void* stream) {
+  paro::Grid g;
+  pa_status st = map_common(q_perm, k_perm, shape, order, &g);
+  if (st != PA_OK) return st;
+  PA_REQUIRE(row_max && row_sum && count && total && peak,
+             "row_max, row_sum, count, total and peak must be non-NULL");
+  PA_REQUIRE(std::isfinite(eps), "eps must be finite");
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t n = (size_t)g.B * g.heads * g.NB * g.NB;
+  cudaError_t e = cudaMemsetAsync(count, 0, n * sizeof(float), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(total, 0, n * sizeof(float), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(peak, 0, n * sizeof(float), s);
+  if (e == cudaSuccess)
+    e = paro::launch_map_stats(q_perm, k_perm, g, order, true, const_cast<float*>(row_max),
+                               const_cast<float*>(row_sum), eps, count, total, peak, dev_status,
+                               s);
+  if (e == cudaSuccess && log_total != nullptr)
+    e = paro::launch_log_total(total, log_total, (int64_t)n, s);
+  return cuda_status(e, "pa_map_block_stats launch");
+}
+
+pa_status pa_paro_metric(const float* count, const float* total, const float* peak,
+                         pa_shape shape, int32_t order, float rho, float* sparse_frac,
+                         float* incoherence, void* stream) {
+  paro::Grid g;
+  pa_status st = make_grid(shape, nullptr, false, &g);
+  if (st != PA_OK) return st;
+  PA_REQUIRE(count && total && peak && sparse_frac && incoherence, "NULL argument");
+  PA_REQUIRE(order >= 0 && order < 6, "order=%d must be in [0, 6)", order);
+  PA_REQUIRE(std::isfinite(rho), "rho must be finite");
+  return cuda_status(paro::launch_paro_metric(count, total, peak, g, order, rho, sparse_frac,
+                                              incoherence, (cudaStream_t)stream),
+                     "pa_paro_metric launch");
+}
+
+pa_status pa_paro_choose(const float* sparse_frac, const float* incoherence, pa_shape shape,
+                         float alpha, float* metric, int8_t* orders, void* stream) {
+  paro::Grid g;
+  pa_status st = make_grid(shape, nullptr, false, &g);
+  if (st != PA_OK) return st;
+  PA_REQUIRE(sparse_frac && incoherence && metric && orders, "NULL argument");
+  PA_REQUIRE(std::isfinite(alpha), "alpha must be finite");
+  return cuda_status(paro::launch_paro_choose(sparse_frac, incoherence, (int64_t)g.B * g.heads,
+                                              alpha, metric, orders, (cudaStream_t)stream),
+                     "pa_paro_choose launch");
 }
 
 pa_status pa_compact_mask(const uint32_t* bitmask, pa_shape shape, int32_t* idx, int32_t* counts,

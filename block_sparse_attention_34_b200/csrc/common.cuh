@@ -103,6 +103,17 @@ cudaError_t launch_attn_mma(const void* q, const void* k, const void* v, pa_dtyp
 cudaError_t launch_sics(const void* x, pa_dtype dt, const Grid& g, float* scores, cudaStream_t s);
 cudaError_t launch_hybrid(const float* scores, const Grid& g, int k, double p, int w,
                           int32_t* idx, int32_t* counts, cudaStream_t s);
+// PAROAttention offline stage (paro_offline.cu)
+cudaError_t launch_map_stats(const void* qp, const void* kp, const Grid& g, int order,
+                             bool block_stats, float* row_max, float* row_sum, float eps,
+                             float* count, float* total, float* peak, int32_t* status,
+                             cudaStream_t s);
+cudaError_t launch_log_total(const float* total, float* log_total, int64_t n, cudaStream_t s);
+cudaError_t launch_paro_metric(const float* count, const float* total, const float* peak,
+                               const Grid& g, int order, float rho, float* sparse_frac,
+                               float* incoh, cudaStream_t s);
+cudaError_t launch_paro_choose(const float* sparse_frac, const float* incoh, int64_t rows,
+                               float alpha, float* metric, int8_t* orders, cudaStream_t s);
 // INT8 tcgen05 attention (d = 128, block = 128, permuted int8 inputs)
 // p_levels: P codes round_half_even(p_levels * P~); 127 (INT8) or 7 (4-bit)
 cudaError_t launch_attn_i8(const void* q, const void* k, const void* v, const Grid& g,

@@ -63,6 +63,11 @@ def load():
         "pa_compact_mask": ([_P, PaShape, _P, _P, _P], _I),
         "pa_select_hybrid": ([_P, PaShape, _I, ctypes.c_double, _I, _P, _P, _P], _I),
         "pa_sics_scores": ([_P, _P, _I, PaShape, _P, _P], _I),
+        "pa_map_row_stats": ([_P, _P, PaShape, _I, _P, _P, _P, _P], _I),
+        "pa_map_block_stats": ([_P, _P, PaShape, _I, _P, _P, ctypes.c_float, _P, _P, _P, _P, _P,
+                                _P], _I),
+        "pa_paro_metric": ([_P, _P, _P, PaShape, _I, ctypes.c_float, _P, _P, _P], _I),
+        "pa_paro_choose": ([_P, _P, PaShape, ctypes.c_float, _P, _P, _P], _I),
         "pa_quantize_int8": ([_P, _I, PaShape, _P, _P, _P, _P, _P], _I),
         "pa_quantize_int4": ([_P, _I, PaShape, _P, _P, _P, _P, _P], _I),
         "pa_block_sparse_attn": ([_P, _P, _P, _I, ctypes.c_uint32, PaShape, _P, _P, _P, _I, _P, _P, _P,
@@ -215,6 +220,71 @@ def sics_scores(q, k, pr: Problem, scores=None):
     scores = scores if scores is not None else torch.empty((pr.B, pr.heads, 6), dtype=torch.float32, device=q.device)
     _check(load().pa_sics_scores(_ptr(q), _ptr(k), _dtype_code(q), pr.shape, _ptr(scores), _stream()))
     return scores
+
+
+def map_row_stats(q_perm, k_perm, pr: Problem, order: int, status=None):
+    """Row softmax (log2 max, sum) of every token of the dense map, from
+    copies of q, k permuted by ``order`` -> ([B,h,N], [B,h,N])."""
+    _need_cuda(q_perm, k_perm)
+    dev = q_perm.device
+    m = torch.empty((pr.B, pr.heads, pr.N), dtype=torch.float32, device=dev)
+    l = torch.empty_like(m)
+    _check(load().pa_map_row_stats(_ptr(q_perm), _ptr(k_perm), pr.shape, int(order), _ptr(m),
+                                   _ptr(l), _ptr(status), _stream()))
+    return m, l
+
+
+def map_block_stats(q_perm, k_perm, pr: Problem, order: int, row_max, row_sum, eps=1e-3,
+                    with_log=True, status=None):
+    """Per block of the map in ``order``: dict of [B,h,NB,NB] count / total
+    / peak (and log_total)."""
+    _need_cuda(q_perm, k_perm, row_max, row_sum)
+    dev = q_perm.device
+    out = {key: torch.empty((pr.B, pr.heads, pr.NB, pr.NB), dtype=torch.float32, device=dev)
+           for key in ("count", "total", "peak")}
+    out["log_total"] = torch.empty_like(out["total"]) if with_log else None
+    _check(load().pa_map_block_stats(_ptr(q_perm), _ptr(k_perm), pr.shape, int(order),
+                                     _ptr(row_max), _ptr(row_sum), float(eps), _ptr(out["count"]),
+                                     _ptr(out["total"]), _ptr(out["peak"]),
+                                     _ptr(out["log_total"]), _ptr(status), _stream()))
+    return out
+
+
+def paro_offline(q, k, grid, block, eps=1e-3, rho=0.9, alpha=0.5, sigma=0.9, status=None):
+    """PAROAttention's offline stage for natural-order q, k (bf16, d = 128,
+    block = 128): the six orders' block statistics of the dense map, the
+    per-head metric and order, and the static mask of each head's chosen
+    order by block-sum thresholding at ``sigma``.  Returns a dict: orders
+    [B,h] int8, metric / sparse_frac / incoherence [B,h,6], idx [B,h,NB,NB]
+    and counts [B,h,NB] (the chosen order's mask, per head)."""
+    B, heads = q.shape[:2]
+    dev = q.device
+    probs = [Problem(B, heads, grid, q.shape[-1], block, [o] * heads) for o in range(6)]
+    pr0 = probs[0]
+    sf = torch.empty((B, heads, 6), dtype=torch.float32, device=dev)
+    inc = torch.empty_like(sf)
+    idx_all = torch.empty((6, B, heads, pr0.NB, pr0.NB), dtype=torch.int32, device=dev)
+    cnt_all = torch.empty((6, B, heads, pr0.NB), dtype=torch.int32, device=dev)
+    row_max = row_sum = None
+    for o, pr in enumerate(probs):
+        qp, kp = reorder(q, pr), reorder(k, pr)
+        if row_max is None:
+            row_max, row_sum = map_row_stats(qp, kp, pr, o, status)
+        st = map_block_stats(qp, kp, pr, o, row_max, row_sum, eps, True, status)
+        _check(load().pa_paro_metric(_ptr(st["count"]), _ptr(st["total"]), _ptr(st["peak"]),
+                                     pr.shape, o, float(rho), _ptr(sf), _ptr(inc), _stream()))
+        select_hybrid(st["log_total"], pr, 0, sigma, -1, idx_all[o], cnt_all[o])
+        del qp, kp, st
+    metric = torch.empty_like(sf)
+    orders = torch.empty((B, heads), dtype=torch.int8, device=dev)
+    _check(load().pa_paro_choose(_ptr(sf), _ptr(inc), pr0.shape, float(alpha), _ptr(metric),
+                                 _ptr(orders), _stream()))
+    # each head's mask in its chosen order (a gather of the six candidates)
+    pick = orders.long()
+    bi = torch.arange(B, device=dev)[:, None]
+    hi = torch.arange(heads, device=dev)[None, :]
+    return {"orders": orders, "metric": metric, "sparse_frac": sf, "incoherence": inc,
+            "idx": idx_all[pick, bi, hi], "counts": cnt_all[pick, bi, hi]}
 
 
 def quantize_int8(x, pr: Problem, with_pool=False, x_q=None, scales=None, pool=None, bits=8):

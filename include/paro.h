@@ -80,7 +80,7 @@ typedef struct {
   int32_t B, heads, F, H, W, d, block;
 } pa_shape;
 
-/* Version of this ABI (bumped on any signature change): 3. */
+/* Version of this ABI (bumped on any signature change): 4. */
 PA_API int32_t pa_abi_version(void);
 
 /* Message of the last failed call on this thread ("" if none). */
@@ -166,6 +166,54 @@ PA_API pa_status pa_select_hybrid(const float* scores, pa_shape shape, int32_t k
  * largest score is SPADE's pick for the head. */
 PA_API pa_status pa_sics_scores(const void* q, const void* k, pa_dtype dtype, pa_shape shape,
                          float* scores, void* stream);
+
+/* PAROAttention's offline stage (PAROAttention review, key_machinery: the
+ * per-head order is chosen offline by a metric balancing block
+ * sparsifiability against block incoherence; static masks by block-sum
+ * thresholding; referee note on Eq. (1): n^{<eps}_{ij}).  Every entry walks
+ * all NB x NB tiles of the dense map P = softmax(q k^T / sqrt(d)) of one
+ * head on the tensor cores.  q_perm, k_perm: [B,heads,N_p,d] bf16 copies
+ * permuted by one order for every head (pa_reorder with perms all = order);
+ * d = 128, block = 128.  dev_status as for pa_block_sparse_attn.
+ *
+ * Row softmax of every token (no order changes it): with
+ * s_c = q.k_c log2(e) / sqrt(d), row_max[b,h,n] = max_c s_c and
+ * row_sum[b,h,n] = sum_c 2^(s_c - row_max), indexed by natural token n;
+ * [B,heads,N] float outputs. */
+PA_API pa_status pa_map_row_stats(const void* q_perm, const void* k_perm, pa_shape shape,
+                           int32_t order, float* row_max, float* row_sum, int32_t* dev_status,
+                           void* stream);
+
+/* Block statistics of the map in one order, from the row softmax above:
+ * for block (i, j) of the permuted map (its valid rows and columns), with
+ * p = 2^(s - row_max) / row_sum,
+ *   count[b,h,i,j] = #{p < eps},  total[...] = sum p,  peak[...] = max p
+ * ([B,heads,NB,NB] float, overwritten), and when log_total is not NULL,
+ * log_total = log(total) (-inf for 0): the scores whose pa_select_hybrid
+ * Top-P set (k = 0, top_p = sigma, window = -1) is the static mask by
+ * block-sum thresholding at sigma.  total and count are summed with
+ * atomics, so their last bits vary between runs. */
+PA_API pa_status pa_map_block_stats(const void* q_perm, const void* k_perm, pa_shape shape,
+                             int32_t order, const float* row_max, const float* row_sum,
+                             float eps, float* count, float* total, float* peak,
+                             float* log_total, int32_t* dev_status, void* stream);
+
+/* Per (b,h), for the statistics of one order:
+ *   sparse_frac[b,h,order] = fraction of blocks with count >= rho * size,
+ *   incoherence[b,h,order] = mean over blocks of positive mean of
+ *                            peak / (total / size)
+ * (size = valid rows x valid columns of the block); [B,heads,6] float,
+ * only slot `order` written. */
+PA_API pa_status pa_paro_metric(const float* count, const float* total, const float* peak,
+                         pa_shape shape, int32_t order, float rho, float* sparse_frac,
+                         float* incoherence, void* stream);
+
+/* Per (b,h) from all six orders' slots: metric[o] = alpha (1 - sf[o]) /
+ * max_o (1 - sf) + (1 - alpha) inc[o] / max_o inc (a term that is 0 for
+ * every order adds 0); orders[b,h] = argmin, ties to the lower id (int8).
+ * metric [B,heads,6] float, orders [B,heads] int8. */
+PA_API pa_status pa_paro_choose(const float* sparse_frac, const float* incoherence, pa_shape shape,
+                         float alpha, float* metric, int8_t* orders, void* stream);
 
 /* Step 3, static (PAROAttention review, key_machinery: static masks stored
  * as bitmasks).  bitmask [B,heads,NB,ceil(NB/32)] uint32, bit (j % 32) of

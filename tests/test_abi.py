@@ -34,7 +34,7 @@ def test_exports_every_declared_symbol(lib):
     assert len(names) >= 12
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.pa_abi_version() == 3
+    assert lib.pa_abi_version() == 4
 
 
 def test_k_for_density_matches_oracle(lib):
@@ -135,3 +135,15 @@ def test_p4_flag_validation(lib):
     assert lib.pa_block_sparse_attn(FAKE, FAKE, FAKE, paro.PA_BF16, 4, good, pp, FAKE,
                                     None, 1, None, None, None, FAKE, None, None) == paro.PA_ERR_INVALID_ARG
     assert lib.pa_quantize_int4(FAKE, paro.PA_I8, good, pp, FAKE, FAKE, None, None) == paro.PA_ERR_INVALID_ARG
+
+
+def test_offline_stage_validation(lib):
+    good = paro.PaShape(1, 2, 4, 8, 8, 128, 128)
+    small = paro.PaShape(1, 2, 4, 8, 8, 64, 64)
+    assert lib.pa_map_row_stats(FAKE, FAKE, good, 6, FAKE, FAKE, None, None) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_map_row_stats(FAKE, FAKE, small, 0, FAKE, FAKE, None, None) == paro.PA_ERR_UNSUPPORTED
+    assert lib.pa_map_row_stats(FAKE, None, good, 0, FAKE, FAKE, None, None) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_map_block_stats(FAKE, FAKE, good, 0, FAKE, FAKE, float("nan"), FAKE, FAKE, FAKE,
+                                  None, None, None) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_paro_metric(FAKE, FAKE, FAKE, good, -1, 0.9, FAKE, FAKE, None) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_paro_choose(FAKE, FAKE, good, float("inf"), FAKE, FAKE, None) == paro.PA_ERR_INVALID_ARG
