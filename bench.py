@@ -410,7 +410,7 @@ def run_sweep(a):
     """Every workload of the configs table on one GPU: per-step device times
     of the attention kernel and of the whole step (selection included) after
     10 warm-up steps, as p10 / p50 / p90 over the timed steps, one JSON line
-    per workload.  Not the default contract line (that is the default run)."""
+    per workload, besides the single summary line of the default run."""
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (there is no CPU path)")
     device = torch.device("cuda", 0)

@@ -10,7 +10,7 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 and the built CUDA library")
-    config.addinivalue_line("markers", "slow: full-size parity on the GPU box")
+    config.addinivalue_line("markers", "slow: full-size parity (minutes on one GPU)")
 
 
 @pytest.fixture(scope="session")
