@@ -332,31 +332,60 @@ def block_sparse_attn(q, k, v, pr: Problem, idx, counts=None, scales=None, out=N
     return out
 
 
+def choose_orders_sics(q, k, grid, block):
+    """SPADE's blocking choice per head: the axis order whose blocks have the
+    largest SICS of q and k (ties to the lower id) -> list of order ids."""
+    B, heads = q.shape[:2]
+    pr = Problem(B, heads, grid, q.shape[-1], block, [0] * heads)
+    sc = sics_scores(q, k, pr)
+    # one order per head: the batch's summed score (a head has one order)
+    return [int(o) for o in torch.argmax(sc.sum(dim=0), dim=-1).tolist()]
+
+
 def attention(q, k, v, grid, perms, block, density, int8=False, baseline=False, status=None,
-              permuted=True, int4_pv=False):
+              permuted=True, int4_pv=False, selection="topk", top_p=0.0, window=-1):
     """The whole path for one call: reorder with block means (one read of
-    q, k, v) -> pooled block scores -> top-k kept blocks -> block-sparse
-    attention over the permuted tiles, stored back in natural order.
-    ``permuted=False`` skips the reorder pass: the block means are taken
-    from the natural layout and the attention kernel gathers token rows.
-    Returns (out, idx)."""
+    q, k, v) -> pooled block scores -> kept blocks -> block-sparse attention
+    over the permuted tiles, stored back in natural order.
+
+    ``perms``: one axis-order id per head, or "sics" to pick each head's
+    order by the SICS blocking score (SPADE).  ``selection``: "topk" (the
+    diagonal plus the k-1 best blocks, k from ``density``) or "hybrid" (the
+    union of that Top-K, the Top-P set at ``top_p`` and the local window
+    |i - j| <= ``window``, with per-row counts).  ``int8`` runs the INT8
+    kernel (``int4_pv``: 4-bit P and V).  ``permuted=False`` skips the
+    reorder pass (the kernel gathers token rows); ``baseline=True`` runs the
+    mma.sync comparison kernel.  Returns (out, idx) — with the hybrid
+    filter, idx is (idx, counts)."""
+    if isinstance(perms, str):
+        if perms != "sics":
+            raise ValueError(f"perms={perms!r}: order ids or 'sics'")
+        perms = choose_orders_sics(q, k, grid, block)
     pr = Problem.from_qkv(q, grid, perms, block)
     kk = k_for_density(pr.NB, density)
+
+    def select(scores):
+        if selection == "hybrid":
+            return select_hybrid(scores, pr, kk, top_p, window)
+        if selection != "topk":
+            raise ValueError(f"selection={selection!r}: topk or hybrid")
+        return select_topk(scores, pr, kk), None
+
     if int8:
         q8, qs, qp = quantize_int8(q, pr, with_pool=True)
         k8, ks, kp = quantize_int8(k, pr, with_pool=True)
         v8, vs = quantize_int8(v, pr, bits=4 if int4_pv else 8)
-        scores = score_pooled(qp, kp, pr)
-        idx = select_topk(scores, pr, kk)
-        return block_sparse_attn(q8, k8, v8, pr, idx, scales=(qs, ks, vs), status=status,
-                                 p4=int4_pv), idx
-    if permuted and not baseline:
+        idx, counts = select(score_pooled(qp, kp, pr))
+        out = block_sparse_attn(q8, k8, v8, pr, idx, counts, scales=(qs, ks, vs), status=status,
+                                p4=int4_pv)
+    elif permuted and not baseline:
         qp, q_pool = reorder(q, pr, with_pool=True)
         kp, k_pool = reorder(k, pr, with_pool=True)
         vp = reorder(v, pr)
-        scores = score_pooled(q_pool, k_pool, pr)
-        idx = select_topk(scores, pr, kk)
-        return block_sparse_attn(qp, kp, vp, pr, idx, status=status, permuted=True), idx
-    _, _, scores = block_score(q, k, pr)
-    idx = select_topk(scores, pr, kk)
-    return block_sparse_attn(q, k, v, pr, idx, baseline=baseline, status=status), idx
+        idx, counts = select(score_pooled(q_pool, k_pool, pr))
+        out = block_sparse_attn(qp, kp, vp, pr, idx, counts, status=status, permuted=True)
+    else:
+        _, _, scores = block_score(q, k, pr)
+        idx, counts = select(scores)
+        out = block_sparse_attn(q, k, v, pr, idx, counts, baseline=baseline, status=status)
+    return out, (idx if counts is None else (idx, counts))

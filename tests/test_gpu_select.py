@@ -168,3 +168,31 @@ def test_hybrid_attention_end_to_end():
     want = ref.attention(as_f64(q), as_f64(k), as_f64(v), (w.F, w.H, w.W), perms, w.block,
                          idx_ref, cnt_ref)
     compare_rows(out, want, token_mask(agree, (w.F, w.H, w.W), perms, w.block))
+
+
+def test_attention_api_sics_orders_and_hybrid_lists():
+    """paro.attention(perms="sics", selection="hybrid"): each head's order
+    is the oracle's SICS pick (where it is clear), and the output equals the
+    oracle's attention over the oracle's hybrid lists for that order."""
+    w = custom("api_780", 1, 3, 128, (6, 10, 13), 128, "bf16", 0.3, perms=(0, 0, 0))
+    q, k, v, _ = inputs(w)
+    grid = (w.F, w.H, w.W)
+    qd, kd, vd = to_dev(q, k, v)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, (idx, cnt) = paro.attention(qd, kd, vd, grid, "sics", w.block, w.density, status=status,
+                                     selection="hybrid", top_p=0.5, window=1)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    want_scores = sel.sics_scores(as_f64(q), as_f64(k), grid, w.block)[0]
+    perms = paro.choose_orders_sics(qd, kd, grid, w.block)
+    for h in range(w.heads):
+        top2 = np.sort(want_scores[h])[-2:]
+        if top2[1] - top2[0] > 1e-3 * abs(top2[1]):
+            assert perms[h] == int(np.argmax(want_scores[h]))
+    kk = ref.k_for_density(w.NB, w.density)
+    _, _, s_ref = ref.pooled_scores(as_f64(q), as_f64(k), grid, perms, w.block)
+    idx_ref, cnt_ref = sel.hybrid_select(s_ref, kk, 0.5, 1)
+    agree = (idx.cpu().numpy() == idx_ref).all(axis=-1) & (cnt.cpu().numpy() == cnt_ref)
+    assert agree.mean() >= 0.9
+    want = ref.attention(as_f64(q), as_f64(k), as_f64(v), grid, perms, w.block, idx_ref, cnt_ref)
+    compare_rows(out, want, token_mask(agree, grid, perms, w.block))
