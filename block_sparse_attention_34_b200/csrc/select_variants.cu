@@ -24,6 +24,7 @@ namespace paro {
 namespace {
 
 constexpr int kSicsThreads = 128;
+static_assert(kSicsThreads >= 128, "one thread per row of a block (block <= 128)");
 
 // Rows are read 16 bytes per lane: a row of d elements takes L = d *
 // sizeof(T) / 16 lanes (8 for d=64 bf16, 16 for d=128 bf16, 32 for d=128
@@ -37,8 +38,15 @@ __global__ void __launch_bounds__(kSicsThreads)
   constexpr int kE = 16 / sizeof(T);  // elements per 16-byte slice
   __shared__ float part[kSicsThreads / 32][256];
   __shared__ float diag_part[kSicsThreads / 32];
+  __shared__ int nat[kSicsThreads];  // natural row of each of the block's rows, -1 past N
   const int i = blockIdx.x, order = blockIdx.y;
   const int64_t bh = blockIdx.z;
+  // one index computation per row (block <= 128 rows), not one per lane
+  if ((int)threadIdx.x < g.block) {
+    const int p = i * g.block + (int)threadIdx.x;
+    nat[threadIdx.x] = p < g.N ? natural_index(g, order, p) : -1;
+  }
+  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int L = g.d * (int)sizeof(T) / 16;  // lanes per row: 4, 8, 16 or 32
   const int rows_per_load = 32 / L;
@@ -53,10 +61,10 @@ __global__ void __launch_bounds__(kSicsThreads)
     bool have[2];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const int p = i * g.block + r0 + u * step + sub;
-      have[u] = r0 + u * step + sub < g.block && p < g.N;
-      raw[u] = have[u] ? __ldg(reinterpret_cast<const uint4*>(
-                             head + (int64_t)natural_index(g, order, p) * g.d) + slot)
+      const int r = r0 + u * step + sub;
+      const int n = r < g.block ? nat[r] : -1;
+      have[u] = n >= 0;
+      raw[u] = have[u] ? __ldg(reinterpret_cast<const uint4*>(head + (int64_t)n * g.d) + slot)
                        : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
