@@ -22,7 +22,8 @@
 // taken on the float bits, all p >= 0).  Warp 8 allocates TMEM and issues
 // QK^T into a double-buffered S (two 128-column buffers), so the MMA of
 // tile j+1 runs while tile j is read; warp 9 streams Q once and the K tiles
-// through a four-stage ring with TMA.  Every wait is bounded as in the
+// through a two-stage ring with TMA (two CTAs per SM share the tensor
+// core and hide each other's waits).  Every wait is bounded as in the
 // attention kernels (PA_ERR_TIMEOUT).
 #include "sm100.cuh"
 #include "tmem.cuh"
@@ -34,7 +35,7 @@ using namespace sm100;
 
 constexpr int kBlock = 128;
 constexpr int kD = 128;
-constexpr int kStages = 4;
+constexpr int kStages = 2;  // two CTAs per SM (shared memory, TMEM 2 x 256 columns)
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;
 constexpr int kThreads = 10 * 32;
@@ -46,7 +47,8 @@ constexpr uint32_t kOffSlot = 256;
 constexpr uint32_t kOffMerge = 512;  // pass-1 merge: [2 halves][2][128] f32 = 2 KB
 constexpr uint32_t kOffQ = 3072;
 constexpr uint32_t kOffK = kOffQ + kTile;
-constexpr uint32_t kSmemBytes = kOffK + kStages * kTile;  // 166,912 B
+constexpr uint32_t kSmemBytes = kOffK + kStages * kTile;  // 101,376 B
+static_assert(2 * (kSmemBytes + 1024) <= 232448, "two CTAs per SM");
 static_assert(kOffQ % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 constexpr uint32_t kTmemCols = 256;
 
@@ -63,7 +65,7 @@ enum : uint32_t {
 static_assert(NBAR * 8 <= kOffSlot, "barrier region");
 
 template <bool kBlockStats>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     map_stats_kernel(const __grid_constant__ CUtensorMap map_q,
                      const __grid_constant__ CUtensorMap map_k, const __grid_constant__ Grid g,
                      int order, float scale_log2, float* __restrict__ row_max,
@@ -180,23 +182,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(BSF0 + b));
       const int valid = min(64, g.N - j * kBlock - hc * 64);  // may be <= 0
+      // full 64-column halves take an unpredicated loop with four partial
+      // accumulators (short dependency chains); only the tail tile masks
       if (!kBlockStats) {
         float mt = -INFINITY;
+        if (valid >= 64) {
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c < valid) mt = fmaxf(mt, __uint_as_float(sr[c]) * scale_log2);
+          for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sr[c]));
+          mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * scale_log2;
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c < valid) mt = fmaxf(mt, __uint_as_float(sr[c]) * scale_log2);
+        }
         const float m_new = fmaxf(m, mt);
         if (m_new != -INFINITY) {
           float acc = 0.f;
+          if (valid >= 64) {
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (c < valid) acc += ex2(fmaf(__uint_as_float(sr[c]), scale_log2, -m_new));
+            for (int c = 0; c < 64; ++c)
+              a4[c & 3] += ex2(fmaf(__uint_as_float(sr[c]), scale_log2, -m_new));
+            acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (c < valid) acc += ex2(fmaf(__uint_as_float(sr[c]), scale_log2, -m_new));
+          }
           l = (m == -INFINITY ? 0.f : l * ex2(m - m_new)) + acc;
           m = m_new;
         }
       } else {
         float cnt = 0.f, sum = 0.f, mx = 0.f;
-        if (row_ok) {
+        if (row_ok && valid >= 64) {
+          float c4[4] = {0.f, 0.f, 0.f, 0.f}, s4[4] = {0.f, 0.f, 0.f, 0.f};
+          float x4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const float pv = ex2(fmaf(__uint_as_float(sr[c]), scale_log2, -m_row)) * inv_l;
+            c4[c & 3] += pv < eps ? 1.f : 0.f;
+            s4[c & 3] += pv;
+            x4[c & 3] = fmaxf(x4[c & 3], pv);
+          }
+          cnt = (c4[0] + c4[1]) + (c4[2] + c4[3]);
+          sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+          mx = fmaxf(fmaxf(x4[0], x4[1]), fmaxf(x4[2], x4[3]));
+        } else if (row_ok) {
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
             if (c < valid) {
