@@ -16,7 +16,7 @@ Sources (PAROAttention, arXiv 2506.16054, Pith verdict page):
   block (i, j) below eps; the report gives eps = 1e-3 and sigma = 90% as the
   example values, and leaves the weight alpha of Eq. (3) unstated.
 
-Readings where the page is silent (each also listed in the design doc):
+Readings where the page is silent:
 
 R1. The map is P = softmax(Q K^T / sqrt(d)) over the N valid tokens of a
     head, rows and columns both permuted by the candidate order; block

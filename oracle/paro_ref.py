@@ -22,7 +22,7 @@ blocking, fusion or reordering beyond what the step itself states.  Sources:
 * PASA (arXiv 2604.12219), Pith page, Figure 2 caption: each query block
   attends to at most k key blocks, cost O(S k) instead of O(S^2).
 
-Readings where the pages are silent (each one also listed in the design doc):
+Readings where the pages are silent:
 
 1. An order's letters list the axes outermost -> innermost; FHW is the
    natural flattening n = f*H*W + h*W + w.  Ids: 0 FHW, 1 FWH, 2 HFW,

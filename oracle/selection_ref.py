@@ -17,7 +17,7 @@ Sources (SPADE, arXiv 2608.03335, Pith verdict page):
 * core_discovery: only blocks that pass a head-wise Top-K / Top-P and
   local-window filter are attended.
 
-Readings where the page is silent (each also listed in the design doc):
+Readings where the page is silent:
 
 S1. Candidate blockings are the six axis orders of [F, H, W] with the
     executor's block size (runs of ``block`` consecutive tokens of the
