@@ -416,6 +416,9 @@ def run_sweep(a):
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     peaks, peak_src = load_peaks()
+    if a.pasa_only:
+        run_sweep_pasa(device, peaks, peak_src, a.heads)
+        return
     for name, w in ([] if a.selection_only else WORKLOADS.items()):
         q, k, v, perms = make_inputs(w)
         qkv = [t.to(device) for t in (q, k, v)]
@@ -461,6 +464,8 @@ def run_sweep(a):
         del qkv
     run_sweep_selection(device, peaks, peak_src, a.heads)
     run_sweep_offline(device, peaks, peak_src, a.heads)
+    if not a.selection_only:
+        run_sweep_pasa(device, peaks, peak_src, a.heads)
 
 
 def timed_calls(fn, reps=20, warm=5):
@@ -561,6 +566,56 @@ def run_sweep_offline(device, peaks, peak_src, heads=None):
     }), flush=True)
 
 
+def run_sweep_pasa(device, peaks, peak_src, heads=None):
+    """PASA's grouped first-order compensation on the 480p layer (top-k at
+    the workload density): the compensated kernel (mma.sync, kept tiles plus
+    every unselected block as one pooled key row) against the same kernel
+    without compensation and the tcgen05 kernel, on the same kept lists.
+    Algorithmic FLOP: 4 b^2 d per kept tile plus 4 b d per (query block,
+    pooled key block) pair."""
+    w = WORKLOADS["480p_21x30x52"]
+    q, k, v, perms = make_inputs(w, heads=heads)
+    if heads is not None:
+        w = dataclasses.replace(w, heads=heads)
+    qd, kd, vd = (t.to(device) for t in (q, k, v))
+    pr = paro.Problem(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, perms)
+    qp, q_pool = paro.reorder(qd, pr, with_pool=True)
+    kp, k_pool = paro.reorder(kd, pr, with_pool=True)
+    vp, v_pool = paro.reorder(vd, pr, with_pool=True)
+    kk = paro.k_for_density(pr.NB, w.density)
+    idx = paro.select_topk(paro.score_pooled(q_pool, k_pool, pr), pr, kk)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    out = torch.empty((w.B, w.heads, w.N, w.d), dtype=qd.dtype, device=device)
+    runs = {
+        "compensated_mma": lambda: paro.block_sparse_attn_compensated(
+            qp, kp, vp, pr, idx, k_pool, v_pool, out=out, status=status, permuted=True),
+        "plain_mma": lambda: paro.block_sparse_attn(qp, kp, vp, pr, idx, out=out, status=status,
+                                                    baseline=True, permuted=True),
+        "plain_tcgen05": lambda: paro.block_sparse_attn(qp, kp, vp, pr, idx, out=out,
+                                                        status=status, permuted=True),
+    }
+    ms = {name: percentiles(timed_calls(fn)) for name, fn in runs.items()}
+    if int(status.item()) != 0:
+        raise RuntimeError(f"pasa: device status {int(status.item())}")
+    kept = w.B * w.heads * pr.NB * kk
+    pooled_pairs = w.B * w.heads * pr.NB * (pr.NB - kk)
+    flops = 4.0 * w.block * w.block * w.d * kept + 4.0 * w.block * w.d * pooled_pairs
+    plain_flops = 4.0 * w.block * w.block * w.d * kept
+    print(json.dumps({
+        "workload": w.name, "what": "PASA grouped first-order compensation of the unselected"
+        " blocks (top-k at the workload density)", "heads": w.heads, "k": kk, "NB": pr.NB,
+        "ms": ms, "flops_compensated": flops,
+        "tflops_compensated_p50": flops / (ms["compensated_mma"]["p50"] / 1e3) / 1e12,
+        "tflops_plain_mma_p50": plain_flops / (ms["plain_mma"]["p50"] / 1e3) / 1e12,
+        "tflops_plain_tcgen05_p50": plain_flops / (ms["plain_tcgen05"]["p50"] / 1e3) / 1e12,
+        "overhead_vs_plain_mma": ms["compensated_mma"]["p50"] / ms["plain_mma"]["p50"],
+        "peak_source": f"{peak_src} bf16_tflops",
+        "frac_of_burst_peak_p50": flops / (ms["compensated_mma"]["p50"] / 1e3) / 1e12
+        / tensor_peak(peaks, "bf16", "bf16_tflops"),
+        "kernel": "attn_mma_kernel<comp>", "steps": 20, "warmup": 5,
+    }), flush=True)
+
+
 def run_reference(a):
     """The reference arm: the float64 oracle on the host cores (rank 0 only),
     each step a bounded sample of the same workload."""
@@ -614,6 +669,8 @@ def main(argv=None):
                     help="per-workload latency percentiles, one JSON line per workload")
     ap.add_argument("--selection-only", action="store_true",
                     help="with --sweep: only the selection-variant lines")
+    ap.add_argument("--pasa-only", action="store_true",
+                    help="with --sweep: only the PASA compensation line")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

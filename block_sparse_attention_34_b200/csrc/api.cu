@@ -110,7 +110,7 @@ pa_status check_float_dtype(pa_dtype dt) {
 
 extern "C" {
 
-int32_t pa_abi_version(void) { return 4; }
+int32_t pa_abi_version(void) { return 5; }
 
 const char* pa_last_error(void) { return g_error.c_str(); }
 
@@ -390,6 +390,31 @@ pa_status pa_block_sparse_attn_mma(const void* q, const void* k, const void* v, 
   PA_REQUIRE(dtype != PA_I8, "the mma.sync baseline takes PA_F32 or PA_BF16");
   return attn_common(q, k, v, dtype, flags, shape, perms, idx, counts, k_max, nullptr, nullptr,
                      nullptr, out, dev_status, stream, true);
+}
+
+pa_status pa_block_sparse_attn_compensated(const void* q, const void* k, const void* v,
+                                           pa_dtype dtype, uint32_t flags, pa_shape shape,
+                                           const int8_t* perms, const int32_t* idx,
+                                           const int32_t* counts, int32_t k_max,
+                                           const float* k_pool, const float* v_pool, void* out,
+                                           int32_t* dev_status, void* stream) {
+  paro::Grid g;
+  pa_status st = make_grid(shape, perms, true, &g);
+  if (st != PA_OK) return st;
+  PA_REQUIRE(dtype == PA_F32 || dtype == PA_BF16,
+             "dtype %d: pa_block_sparse_attn_compensated takes PA_F32 or PA_BF16", (int)dtype);
+  PA_REQUIRE(q && k && v && out && idx && k_pool && v_pool,
+             "q, k, v, idx, k_pool, v_pool and out must be non-NULL");
+  PA_REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out) &&
+                 aligned16(k_pool) && aligned16(v_pool),
+             "q, k, v, k_pool, v_pool and out must be 16-byte aligned");
+  PA_REQUIRE(k_max >= 0 && k_max <= g.NB, "k_max=%d must be in [0, NB=%d]", k_max, g.NB);
+  PA_REQUIRE((flags & ~PA_ATTN_PERMUTED) == 0, "unknown flags 0x%x", flags);
+  if (g.NB > 4096) return fail(PA_ERR_UNSUPPORTED, "NB=%d above 4096 (one bit per block in shared memory)", g.NB);
+  const bool permuted = (flags & PA_ATTN_PERMUTED) != 0;
+  return cuda_status(paro::launch_attn_mma(q, k, v, dtype, g, idx, counts, k_max, out, dev_status,
+                                           permuted, (cudaStream_t)stream, k_pool, v_pool),
+                     "pa_block_sparse_attn_compensated launch");
 }
 
 }  // extern "C"

@@ -96,9 +96,13 @@ cudaError_t launch_compact(const uint32_t* bm, const Grid& g, int32_t* idx, int3
 // qmax: 127 for INT8 codes, 7 for 4-bit codes (one per byte)
 cudaError_t launch_quantize(const void* x, pa_dtype dt, const Grid& g, int8_t* xq, float* scales,
                             float* pool, int qmax, cudaStream_t s);
+// k_pool, v_pool [B*heads, NB, d] float (both or neither): the block means of
+// k and v; with them every unselected key block enters as one pooled key
+// row of weight n_j (PASA's grouped first-order compensation), NB <= 4096.
 cudaError_t launch_attn_mma(const void* q, const void* k, const void* v, pa_dtype dt,
                             const Grid& g, const int32_t* idx, const int32_t* counts, int k_max,
-                            void* out, int32_t* status, bool permuted, cudaStream_t s);
+                            void* out, int32_t* status, bool permuted, cudaStream_t s,
+                            const float* k_pool = nullptr, const float* v_pool = nullptr);
 // Selection variants (select_variants.cu)
 cudaError_t launch_sics(const void* x, pa_dtype dt, const Grid& g, float* scores, cudaStream_t s);
 cudaError_t launch_hybrid(const float* scores, const Grid& g, int k, double p, int w,

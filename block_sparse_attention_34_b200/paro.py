@@ -74,6 +74,8 @@ def load():
                                   _P, _P, _P], _I),
         "pa_block_sparse_attn_mma": ([_P, _P, _P, _I, ctypes.c_uint32, PaShape, _P, _P, _P, _I, _P, _P,
                                       _P], _I),
+        "pa_block_sparse_attn_compensated": ([_P, _P, _P, _I, ctypes.c_uint32, PaShape, _P, _P, _P, _I,
+                                              _P, _P, _P, _P, _P], _I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -332,6 +334,25 @@ def block_sparse_attn(q, k, v, pr: Problem, idx, counts=None, scales=None, out=N
     return out
 
 
+def block_sparse_attn_compensated(q, k, v, pr: Problem, idx, k_pool, v_pool, counts=None,
+                                  out=None, status=None, permuted=False):
+    """Block-sparse attention in which every unselected key block still
+    enters the softmax as one pooled key row (mean key, mean value, weight
+    = its valid keys): PASA's grouped first-order compensation.  k_pool,
+    v_pool [B, heads, NB, d] float32 block means (from :func:`reorder` with
+    ``with_pool`` or :func:`block_score`).  bf16 or fp32 q, k, v; output
+    natural order, q's dtype."""
+    _need_cuda(q, k, v, idx, counts, k_pool, v_pool)
+    out = out if out is not None else torch.empty((pr.B, pr.heads, pr.N, pr.d), dtype=q.dtype,
+                                                  device=q.device)
+    st = load().pa_block_sparse_attn_compensated(
+        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), PA_ATTN_PERMUTED if permuted else 0, pr.shape,
+        pr.perms_ptr, _ptr(idx), _ptr(counts), int(idx.shape[-1]), _ptr(k_pool), _ptr(v_pool),
+        _ptr(out), _ptr(status), _stream())
+    _check(st)
+    return out
+
+
 def choose_orders_sics(q, k, grid, block):
     """SPADE's blocking choice per head: the axis order whose blocks have the
     largest SICS of q and k (ties to the lower id) -> list of order ids."""
@@ -343,7 +364,8 @@ def choose_orders_sics(q, k, grid, block):
 
 
 def attention(q, k, v, grid, perms, block, density, int8=False, baseline=False, status=None,
-              permuted=True, int4_pv=False, selection="topk", top_p=0.0, window=-1):
+              permuted=True, int4_pv=False, selection="topk", top_p=0.0, window=-1,
+              compensate=False):
     """The whole path for one call: reorder with block means (one read of
     q, k, v) -> pooled block scores -> kept blocks -> block-sparse attention
     over the permuted tiles, stored back in natural order.
@@ -355,8 +377,10 @@ def attention(q, k, v, grid, perms, block, density, int8=False, baseline=False, 
     |i - j| <= ``window``, with per-row counts).  ``int8`` runs the INT8
     kernel (``int4_pv``: 4-bit P and V).  ``permuted=False`` skips the
     reorder pass (the kernel gathers token rows); ``baseline=True`` runs the
-    mma.sync comparison kernel.  Returns (out, idx) — with the hybrid
-    filter, idx is (idx, counts)."""
+    mma.sync comparison kernel.  ``compensate`` adds PASA's grouped
+    first-order compensation of the unselected blocks (bf16 / fp32 only;
+    :func:`block_sparse_attn_compensated`).  Returns (out, idx) — with the
+    hybrid filter, idx is (idx, counts)."""
     if isinstance(perms, str):
         if perms != "sics":
             raise ValueError(f"perms={perms!r}: order ids or 'sics'")
@@ -371,7 +395,16 @@ def attention(q, k, v, grid, perms, block, density, int8=False, baseline=False, 
             raise ValueError(f"selection={selection!r}: topk or hybrid")
         return select_topk(scores, pr, kk), None
 
-    if int8:
+    if compensate:
+        if int8:
+            raise ValueError("compensate runs on bf16 / fp32 inputs")
+        qp, q_pool = reorder(q, pr, with_pool=True)
+        kp, k_pool = reorder(k, pr, with_pool=True)
+        vp, v_pool = reorder(v, pr, with_pool=True)
+        idx, counts = select(score_pooled(q_pool, k_pool, pr))
+        out = block_sparse_attn_compensated(qp, kp, vp, pr, idx, k_pool, v_pool, counts,
+                                            status=status, permuted=True)
+    elif int8:
         q8, qs, qp = quantize_int8(q, pr, with_pool=True)
         k8, ks, kp = quantize_int8(k, pr, with_pool=True)
         v8, vs = quantize_int8(v, pr, bits=4 if int4_pv else 8)

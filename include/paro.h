@@ -80,7 +80,7 @@ typedef struct {
   int32_t B, heads, F, H, W, d, block;
 } pa_shape;
 
-/* Version of this ABI (bumped on any signature change): 4. */
+/* Version of this ABI (bumped on any signature change): 5. */
 PA_API int32_t pa_abi_version(void);
 
 /* Message of the last failed call on this thread ("" if none). */
@@ -301,6 +301,36 @@ PA_API pa_status pa_block_sparse_attn_mma(const void* q, const void* k, const vo
                                    uint32_t flags, pa_shape shape, const int8_t* perms, const int32_t* idx,
                                    const int32_t* counts, int32_t k_max, void* out,
                                    int32_t* dev_status, void* stream);
+
+/* Block-sparse attention with PASA's grouped first-order compensation of
+ * the unselected key blocks (PASA review, Figure 2 caption: the key blocks
+ * outside a query's kept set get a grouped first-order compensation instead
+ * of being dropped; section 3.3: a Taylor expansion approximation).  The
+ * page prints no formula; the reading implemented: exp(q.k_c / sqrt(d)) is
+ * expanded to first order about the block's mean score q.kbar_j / sqrt(d),
+ * whose linear term sums to zero over the block, and the block's values are
+ * grouped the same way, so for every valid query token n (query block i):
+ *   out[n] = (sum_{c kept} e^{s_c} v_c + sum_{j in U_i} n_j e^{sbar_j} vbar_j)
+ *          / (sum_{c kept} e^{s_c} + sum_{j in U_i} n_j e^{sbar_j}),
+ *   s_c = q_n.k_c / sqrt(d),  sbar_j = q_n.kbar_j / sqrt(d),
+ * where U_i = the key blocks with at least one valid key that are not in
+ * idx row (b,h,i), n_j = the valid keys of block j, and kbar_j, vbar_j are
+ * the means of those keys and values.
+ *
+ * Arguments, layouts, ownership and errors as pa_block_sparse_attn_mma
+ * (dtype PA_F32 or PA_BF16, flags 0 or PA_ATTN_PERMUTED; k_max = 0 is
+ * allowed and gives the compensation alone), plus:
+ *   k_pool, v_pool  [B,heads,NB,d] float, 16-byte aligned, read only: the
+ *                   means of the valid rows of each permuted block of k and
+ *                   v (the pool output of pa_reorder or pa_block_score).
+ * Runs on the mma.sync kernel (pooled blocks are rounded to bf16 like the
+ * K and V tiles).  NB <= 4096 (PA_ERR_UNSUPPORTED above). */
+PA_API pa_status pa_block_sparse_attn_compensated(const void* q, const void* k, const void* v,
+                                           pa_dtype dtype, uint32_t flags, pa_shape shape,
+                                           const int8_t* perms, const int32_t* idx,
+                                           const int32_t* counts, int32_t k_max,
+                                           const float* k_pool, const float* v_pool, void* out,
+                                           int32_t* dev_status, void* stream);
 
 #ifdef __cplusplus
 }

@@ -34,7 +34,7 @@ def test_exports_every_declared_symbol(lib):
     assert len(names) >= 12
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.pa_abi_version() == 4
+    assert lib.pa_abi_version() == 5
 
 
 def test_k_for_density_matches_oracle(lib):
@@ -147,3 +147,27 @@ def test_offline_stage_validation(lib):
                                   None, None, None) == paro.PA_ERR_INVALID_ARG
     assert lib.pa_paro_metric(FAKE, FAKE, FAKE, good, -1, 0.9, FAKE, FAKE, None) == paro.PA_ERR_INVALID_ARG
     assert lib.pa_paro_choose(FAKE, FAKE, good, float("inf"), FAKE, FAKE, None) == paro.PA_ERR_INVALID_ARG
+
+
+def test_compensated_attention_validation(lib):
+    good = paro.PaShape(1, 2, 4, 8, 8, 64, 64)  # NB = 4
+    keep, pp = perms_of(0, 5)
+    fn = lib.pa_block_sparse_attn_compensated
+    # the pooled summaries are required and 16-byte aligned
+    assert fn(FAKE, FAKE, FAKE, paro.PA_BF16, 0, good, pp, FAKE, None, 2, None, FAKE, FAKE, None,
+              None) == paro.PA_ERR_INVALID_ARG
+    assert b"k_pool" in lib.pa_last_error()
+    assert fn(FAKE, FAKE, FAKE, paro.PA_BF16, 0, good, pp, FAKE, None, 2, FAKE,
+              ctypes.c_void_p(4100), FAKE, None, None) == paro.PA_ERR_INVALID_ARG
+    # bf16 / fp32 only, no INT4 flag, k_max within [0, NB]
+    assert fn(FAKE, FAKE, FAKE, paro.PA_I8, 0, good, pp, FAKE, None, 2, FAKE, FAKE, FAKE, None,
+              None) == paro.PA_ERR_INVALID_ARG
+    assert fn(FAKE, FAKE, FAKE, paro.PA_BF16, paro.PA_ATTN_P4, good, pp, FAKE, None, 2, FAKE, FAKE,
+              FAKE, None, None) == paro.PA_ERR_INVALID_ARG
+    assert fn(FAKE, FAKE, FAKE, paro.PA_BF16, 0, good, pp, FAKE, None, 5, FAKE, FAKE, FAKE, None,
+              None) == paro.PA_ERR_INVALID_ARG
+    # one bit per key block in shared memory: NB <= 4096
+    big = paro.PaShape(1, 2, 65, 64, 64, 64, 64)  # NB = 4160
+    assert fn(FAKE, FAKE, FAKE, paro.PA_BF16, 0, big, pp, FAKE, None, 2, FAKE, FAKE, FAKE, None,
+              None) == paro.PA_ERR_UNSUPPORTED
+    assert b"4096" in lib.pa_last_error()

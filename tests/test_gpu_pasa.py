@@ -1,0 +1,122 @@
+"""GPU parity of block-sparse attention with PASA's grouped first-order
+compensation of the unselected key blocks (PASA, arXiv 2604.12219, Pith
+review page, Figure 2 caption) against the float64 oracle
+(oracle/pasa_ref.py), through the C ABI.
+
+The kept lists are the oracle's own top-k (or variable-length prefixes of
+it, empty rows included), so both sides compute the same definition; the
+GPU's pooled keys and values are fp32 means of the bf16 rows, rounded to
+bf16 in the kernel like the K and V tiles.  Tolerance: the bf16 one
+(2e-2 max-abs, 2e-3 mean-abs)."""
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_34_b200 import paro
+from block_sparse_attention_34_b200.synth import as_f64
+from oracle import paro_ref as ref
+from oracle import pasa_ref as pasa
+
+from helpers import compare, compare_rows, custom, inputs, oracle_topk, selection_agreement, \
+    to_dev, token_mask
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    custom("pasa_512", 1, 2, 128, (4, 8, 16), 128, "bf16", 0.5, perms=(0, 5)),
+    custom("pasa_ragged_315", 1, 3, 128, (5, 7, 9), 128, "bf16", 0.34, perms=(1, 3, 4)),
+    custom("pasa_d64_b64_240", 2, 2, 64, (4, 6, 10), 64, "bf16", 0.5, perms=(2, 0)),
+    custom("pasa_f32_384", 1, 2, 128, (3, 8, 16), 128, "f32", 0.34, perms=(4, 1)),
+    # more key blocks than one pooled tile holds (NB = 144 > 128, NB = 80 > 64)
+    custom("pasa_nb144", 1, 1, 128, (8, 32, 72), 128, "bf16", 0.1, perms=(3,)),
+    custom("pasa_b64_nb80", 1, 2, 64, (4, 32, 40), 64, "bf16", 0.15, perms=(5, 2)),
+]
+
+
+def problem(w, perms):
+    return paro.Problem(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, perms)
+
+
+def run_gpu(w, q, k, v, perms, idx, counts, permuted):
+    pr = problem(w, perms)
+    qd, kd, vd = to_dev(q, k, v)
+    qp, _ = paro.reorder(qd, pr, with_pool=True)
+    kp, k_pool = paro.reorder(kd, pr, with_pool=True)
+    vp, v_pool = paro.reorder(vd, pr, with_pool=True)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    idx_d = torch.from_numpy(np.ascontiguousarray(idx, dtype=np.int32)).cuda()
+    cnt_d = None if counts is None else torch.from_numpy(
+        np.ascontiguousarray(counts, dtype=np.int32)).cuda()
+    if permuted:
+        out = paro.block_sparse_attn_compensated(qp, kp, vp, pr, idx_d, k_pool, v_pool, cnt_d,
+                                                 status=status, permuted=True)
+    else:
+        out = paro.block_sparse_attn_compensated(qd, kd, vd, pr, idx_d, k_pool, v_pool, cnt_d,
+                                                 status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    return out
+
+
+@pytest.mark.parametrize("permuted", [True, False], ids=["permuted", "natural"])
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_compensated_matches_oracle(w, permuted):
+    q, k, v, perms = inputs(w)
+    idx, _, _ = oracle_topk(q, k, w, perms)
+    out = run_gpu(w, q, k, v, perms, idx, None, permuted)
+    want = pasa.attention_compensated(as_f64(q), as_f64(k), as_f64(v), (w.F, w.H, w.W), perms,
+                                      w.block, idx)
+    compare(out, want)
+    # the compensation is not a no-op on these inputs (unless every block is kept)
+    plain = ref.attention(as_f64(q), as_f64(k), as_f64(v), (w.F, w.H, w.W), perms, w.block, idx)
+    if idx.shape[-1] < w.NB:
+        assert np.abs(want - plain).max() > 1e-3
+
+
+def test_variable_counts_and_empty_rows():
+    w = CASES[1]
+    q, k, v, perms = inputs(w)
+    idx, _, kk = oracle_topk(q, k, w, perms, density=1.0)  # all NB blocks, ascending
+    rng = np.random.default_rng(5)
+    counts = rng.integers(0, w.NB + 1, size=idx.shape[:-1]).astype(np.int32)
+    counts[0, 0, 0] = 0  # a query block with no kept block: compensation alone
+    counts[0, 1, 1] = w.NB  # and one with every block kept: plain dense rows
+    idx = idx.copy()
+    for b in range(w.B):
+        for h in range(w.heads):
+            for i in range(w.NB):
+                # a kept list is any ascending subset; take a seeded one
+                pick = np.sort(rng.choice(w.NB, counts[b, h, i], replace=False))
+                idx[b, h, i, :] = -1
+                idx[b, h, i, :pick.size] = pick
+    out = run_gpu(w, q, k, v, perms, idx, counts, permuted=False)
+    want = pasa.attention_compensated(as_f64(q), as_f64(k), as_f64(v), (w.F, w.H, w.W), perms,
+                                      w.block, idx, counts)
+    compare(out, want)
+
+
+def test_api_compensate_flag():
+    w = CASES[0]
+    q, k, v, perms = inputs(w)
+    qd, kd, vd = to_dev(q, k, v)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, idx = paro.attention(qd, kd, vd, (w.F, w.H, w.W), perms, w.block, w.density,
+                              status=status, compensate=True)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    idx_ref, s_ref, _ = oracle_topk(q, k, w, perms)
+    agree = selection_agreement(idx.cpu().numpy(), idx_ref, s_ref)
+    assert agree.mean() >= 0.95
+    want = pasa.attention_compensated(as_f64(q), as_f64(k), as_f64(v), (w.F, w.H, w.W), perms,
+                                      w.block, idx_ref)
+    compare_rows(out, want, token_mask(agree, (w.F, w.H, w.W), perms, w.block))
+
+
+def test_every_block_kept_equals_plain_attention():
+    w = custom("pasa_dense_780", 1, 2, 128, (6, 10, 13), 128, "bf16", 1.0, perms=(4, 0))
+    q, k, v, perms = inputs(w)
+    idx, _, _ = oracle_topk(q, k, w, perms)
+    out = run_gpu(w, q, k, v, perms, idx, None, permuted=True)
+    want = ref.attention(as_f64(q), as_f64(k), as_f64(v), (w.F, w.H, w.W), perms, w.block, idx)
+    compare(out, want)
