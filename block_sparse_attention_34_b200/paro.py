@@ -18,6 +18,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libparo.so")
 
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_TIMEOUT, PA_ERR_DEVICE_CHECK = range(6)
+ABI_VERSION = 5  # the pa_abi_version() these signatures describe
 PA_F32, PA_BF16, PA_I8 = 0, 1, 2
 PA_ATTN_PERMUTED = 1
 PA_ATTN_P4 = 2  # with int8 inputs: 4-bit P codes (INT4 PV)
@@ -77,6 +78,11 @@ def load():
         "pa_block_sparse_attn_compensated": ([_P, _P, _P, _I, ctypes.c_uint32, PaShape, _P, _P, _P, _I,
                                               _P, _P, _P, _P, _P], _I),
     }
+    lib.pa_abi_version.restype = _I
+    if lib.pa_abi_version() != ABI_VERSION:
+        raise RuntimeError(f"{LIB_PATH} has ABI version {lib.pa_abi_version()}, this binding "
+                           f"needs {ABI_VERSION}: rebuild it with "
+                           "`python -m block_sparse_attention_34_b200.build`")
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
         fn.argtypes = args

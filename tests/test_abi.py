@@ -34,7 +34,7 @@ def test_exports_every_declared_symbol(lib):
     assert len(names) >= 12
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.pa_abi_version() == 5
+    assert lib.pa_abi_version() == paro.ABI_VERSION == 5
 
 
 def test_k_for_density_matches_oracle(lib):
