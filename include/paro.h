@@ -20,6 +20,12 @@
  *                                     PAROAttention review, key_machinery);
  *   5. inverse reorder of the output (fused into step 4's store).
  *
+ * Around it: SPADE's selection variants (pa_sics_scores, pa_select_hybrid),
+ * INT4 P V (pa_quantize_int4 with PA_ATTN_P4), PAROAttention's offline stage
+ * (pa_map_row_stats, pa_map_block_stats, pa_paro_metric, pa_paro_choose) and
+ * PASA's compensation of the unselected blocks
+ * (pa_block_sparse_attn_compensated).
+ *
  * Conventions shared by every entry point
  * ---------------------------------------
  * - N = F*H*W tokens per head; NB = ceil(N / block) blocks; N_p = NB*block.
