@@ -109,3 +109,50 @@ def attention_compensated(q, k, v, grid, perms, block, idx, counts=None):
             op = compensated_permuted(qp, kp, vp, N, block, idx[b, h], cnt)
             out[b, h] = ref.inverse_reorder_head(op, grid, perms[h])
     return out
+
+
+def compensated_rows(q, k, v, grid, perms, block, idx, rows, counts=None):
+    """Outputs of selected natural-order query rows only: ``rows`` is a list
+    of (b, h, n).  The same definition as :func:`attention_compensated`
+    (readings P1-P3), one row at a time, for full-size checks where the
+    whole output is too costly.  Block means are taken per (b, h) once."""
+    F, H, W = grid
+    N = F * H * W
+    d = np.asarray(q[0, 0, 0]).shape[-1]
+    nb = -(-N // block)
+    n = block_counts(N, block, nb)
+    res = np.zeros((len(rows), d), dtype=np.float64)
+    perm_cache, pool_cache = {}, {}
+    for r, (b, h, tok) in enumerate(rows):
+        pid = int(perms[h])
+        if pid not in perm_cache:
+            perm_rows = ref.reorder_head(np.arange(N, dtype=np.float64)[:, None], grid, pid,
+                                         block)[:N, 0].astype(np.int64)
+            pos = np.empty(N, dtype=np.int64)
+            pos[perm_rows] = np.arange(N)
+            perm_cache[pid] = (perm_rows, pos)
+        perm_rows, pos = perm_cache[pid]
+        if (b, h) not in pool_cache:
+            kp = ref.reorder_head(np.asarray(k[b, h], dtype=np.float64), grid, pid, block)
+            vp = ref.reorder_head(np.asarray(v[b, h], dtype=np.float64), grid, pid, block)
+            pool_cache[(b, h)] = (ref.block_pool(kp[None, None], N, block)[0, 0],
+                                  ref.block_pool(vp[None, None], N, block)[0, 0])
+        kbar, vbar = pool_cache[(b, h)]
+        i = pos[tok] // block
+        c = idx.shape[-1] if counts is None else int(counts[b, h, i])
+        kept = sorted({int(j) for j in idx[b, h, i, :c] if 0 <= int(j) < nb})
+        unsel = [j for j in range(nb) if j not in kept and n[j] > 0]
+        cols = (perm_rows[np.concatenate([np.arange(j * block, min((j + 1) * block, N))
+                                          for j in kept])]
+                if kept else np.zeros(0, dtype=np.int64))
+        qr = np.asarray(q[b, h, tok], dtype=np.float64)
+        s = np.asarray(k[b, h][cols], dtype=np.float64) @ qr / math.sqrt(d)
+        sb = kbar[unsel] @ qr / math.sqrt(d)
+        m = max(s.max() if s.size else -np.inf, sb.max() if sb.size else -np.inf)
+        if m == -np.inf:
+            continue
+        p = np.exp(s - m)
+        w = n[unsel] * np.exp(sb - m)
+        num = p @ np.asarray(v[b, h][cols], dtype=np.float64) + w @ vbar[unsel]
+        res[r] = num / (p.sum() + w.sum())
+    return res

@@ -14,12 +14,13 @@ import pytest
 import torch
 
 from block_sparse_attention_34_b200 import paro
+from block_sparse_attention_34_b200.configs import WORKLOADS
 from block_sparse_attention_34_b200.synth import as_f64
 from oracle import paro_ref as ref
 from oracle import pasa_ref as pasa
 
-from helpers import compare, compare_rows, custom, inputs, oracle_topk, selection_agreement, \
-    to_dev, token_mask
+from helpers import BF16_MAX_ABS, BF16_MEAN_ABS, compare, compare_rows, custom, inputs, \
+    oracle_topk, selection_agreement, to_dev, token_mask
 
 pytestmark = pytest.mark.gpu
 
@@ -120,3 +121,29 @@ def test_every_block_kept_equals_plain_attention():
     out = run_gpu(w, q, k, v, perms, idx, None, permuted=True)
     want = ref.attention(as_f64(q), as_f64(k), as_f64(v), (w.F, w.H, w.W), perms, w.block, idx)
     compare(out, want)
+
+
+def test_480p_full_size_sampled():
+    """The measured PASA workload (480p layer, 12 heads, top-k at 0.25, the
+    compensated kernel on permuted tiles) with the oracle's kept lists of
+    every head; seeded rows plus each head's last token (ragged tail) are
+    compared with the oracle's row evaluator."""
+    w = WORKLOADS["480p_21x30x52"]
+    q, k, v, perms = inputs(w)
+    grid = (w.F, w.H, w.W)
+    kk = ref.k_for_density(w.NB, w.density)
+    idx = np.zeros((w.B, w.heads, w.NB, kk), dtype=np.int32)
+    for h in range(w.heads):
+        _, _, s = ref.pooled_scores(as_f64(q[:, h:h + 1]), as_f64(k[:, h:h + 1]), grid,
+                                    perms[h:h + 1], w.block)
+        idx[:, h:h + 1] = ref.select_topk(s, kk)
+    out = run_gpu(w, q, k, v, perms, idx, None, permuted=True)
+    rng = np.random.default_rng(13)
+    rows = [(0, int(rng.integers(w.heads)), int(rng.integers(w.N))) for _ in range(96)]
+    rows += [(0, h, w.N - 1) for h in range(w.heads)]
+    want = pasa.compensated_rows(as_f64(q), as_f64(k), as_f64(v), grid, perms, w.block, idx, rows)
+    got = out[0].float().cpu().numpy()
+    got = np.stack([got[h, n] for (_, h, n) in rows]).astype(np.float64)
+    err = np.abs(got - want)
+    assert np.isfinite(got).all()
+    assert err.max() <= BF16_MAX_ABS and err.mean() <= BF16_MEAN_ABS, (err.max(), err.mean())

@@ -167,3 +167,24 @@ def test_underflowing_unselected_blocks_leave_sparse_output():
 def test_block_counts_ragged_tail():
     assert pasa.block_counts(60, 8, 8).tolist() == [8] * 7 + [4]
     assert pasa.block_counts(64, 8, 8).tolist() == [8] * 8
+
+
+@pytest.mark.parametrize("grid,block", [((2, 4, 4), 8), ((3, 2, 5), 7)])
+def test_row_evaluator_matches_whole_head(grid, block):
+    rng = np.random.default_rng(48)
+    N = grid[0] * grid[1] * grid[2]
+    nh, d = 3, 4
+    nb = -(-N // block)
+    q, k, v = (rng.standard_normal((2, nh, N, d)) for _ in range(3))
+    perms = [0, 4, 5]
+    idx = np.full((2, nh, nb, nb), -1, dtype=np.int32)
+    counts = np.zeros((2, nh, nb), dtype=np.int32)
+    for b in range(2):
+        i1, c1 = random_idx(rng, nh, nb, max(1, nb - 2))
+        idx[b], counts[b] = i1[0], c1[0]
+    counts[1, 2, 0] = 0  # an empty kept list: compensation alone
+    whole = pasa.attention_compensated(q, k, v, grid, perms, block, idx, counts)
+    rows = [(b, h, n) for b in range(2) for h in range(nh) for n in range(N)]
+    got = pasa.compensated_rows(q, k, v, grid, perms, block, idx, rows, counts)
+    want = np.stack([whole[b, h, n] for (b, h, n) in rows])
+    assert np.abs(got - want).max() < 1e-12
