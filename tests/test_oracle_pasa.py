@@ -15,7 +15,8 @@ oracle/pasa_ref.py).
 * the error law that makes it first order: with equal values in a block and
   keys spread by eps about their mean, the error is O(eps^2) (halving eps
   quarters it), where an expansion about any other point than the mean
-  would leave an O(eps) term.
+  would leave an O(eps) term;
+* a hand-worked example (tests/golden/pasa_2x1x2_whf.txt): 7/2 - sqrt(2)/2.
 """
 
 import math
@@ -188,3 +189,33 @@ def test_row_evaluator_matches_whole_head(grid, block):
     got = pasa.compensated_rows(q, k, v, grid, perms, block, idx, rows, counts)
     want = np.stack([whole[b, h, n] for (b, h, n) in rows])
     assert np.abs(got - want).max() < 1e-12
+
+
+def test_golden_hand_worked():
+    import os
+    vals = {}
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                        "pasa_2x1x2_whf.txt")
+    with open(path) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            name, *rest = line.split()
+            vals[name] = rest
+    grid = tuple(int(x) for x in vals["grid"])
+    pid = ref.ORDER_NAMES.index(vals["order"][0])
+    block = int(vals["block"][0])
+    N = 4
+    q = np.ones((1, 1, N, 1))
+    k = np.log(np.arange(1, N + 1, dtype=np.float64)).reshape(1, 1, N, 1)
+    v = np.arange(1, N + 1, dtype=np.float64).reshape(1, 1, N, 1)
+    idx = np.full((1, 1, 2, 2), -1, dtype=np.int32)
+    counts = np.zeros((1, 1, 2), dtype=np.int32)
+    for i in range(2):
+        row = [int(x) for x in vals[f"idx{i}"]]
+        idx[0, 0, i, :len(row)] = row
+        counts[0, 0, i] = len(row)
+    got = pasa.attention_compensated(q, k, v, grid, [pid], block, idx, counts)[0, 0, :, 0]
+    want = np.array([float(x) for x in vals["out"]])
+    assert np.abs(got - want).max() < 1e-14
+    assert abs(want[0] - (3.5 - math.sqrt(2) / 2)) < 1e-15
