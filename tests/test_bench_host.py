@@ -120,3 +120,18 @@ def test_percentiles_pick_order_statistics():
     p = bench.percentiles(xs)
     assert p == {"p10": 1.0, "p50": 5.0, "p90": 9.0}
     assert bench.percentiles([2.5]) == {"p10": 2.5, "p50": 2.5, "p90": 2.5}
+
+
+def test_sweep_options_parse_and_refuse_without_cuda():
+    """--sweep with --pasa-only / --selection-only parses, and with no CUDA
+    device the run stops with a message instead of falling back to the CPU."""
+    sys.path.insert(0, ROOT)
+    import pytest
+    import bench
+
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present: the sweep would run")
+    for extra in (["--pasa-only"], ["--selection-only"], []):
+        with pytest.raises(SystemExit) as e:
+            bench.main(["--sweep", *extra])
+        assert "CUDA" in str(e.value)
