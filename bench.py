@@ -283,6 +283,26 @@ def cpu_baseline(w, q, k, v, perms, idx_host, budget_s=12.0, max_blocks=None, in
     return flops / dt / 1e12, dt, f"head 0, query blocks 0..{done - 1} of {w.NB} ({done * kk} kept tiles)"
 
 
+def pasa_cpu_baseline(w, q, k, v, perms):
+    """The compensation oracle, as it stands, on head 0 of the workload (all
+    its query blocks), with the oracle's own top-k at the workload density.
+    Returns TFLOPS of the algorithmic work (kept tiles plus one pooled row per
+    unselected block and query row), seconds, and the sample."""
+    from oracle import paro_ref as ref
+    from oracle import pasa_ref as pasa
+    grid = (w.F, w.H, w.W)
+    q0, k0, v0 = (x[:, :1].double().numpy() for x in (q, k, v))
+    _, _, s = ref.pooled_scores(q0, k0, grid, perms[:1], w.block)
+    kk = ref.k_for_density(w.NB, w.density)
+    idx = ref.select_topk(s, kk)
+    qp, kp, vp = (ref.reorder_head(x[0, 0], grid, perms[0], w.block) for x in (q0, k0, v0))
+    t0 = time.perf_counter()
+    pasa.compensated_permuted(qp, kp, vp, w.N, w.block, idx[0, 0])
+    dt = time.perf_counter() - t0
+    flops = 4.0 * w.block * w.d * w.NB * (w.block * kk + (w.NB - kk))
+    return flops / dt / 1e12, dt, f"head 0, all {w.NB} query blocks (k = {kk})"
+
+
 def cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -597,6 +617,7 @@ def run_sweep_pasa(device, peaks, peak_src, heads=None):
     ms = {name: percentiles(timed_calls(fn)) for name, fn in runs.items()}
     if int(status.item()) != 0:
         raise RuntimeError(f"pasa: device status {int(status.item())}")
+    cpu_tf, cpu_s, cpu_sample = pasa_cpu_baseline(w, q, k, v, perms)
     kept = w.B * w.heads * pr.NB * kk
     pooled_pairs = w.B * w.heads * pr.NB * (pr.NB - kk)
     flops = 4.0 * w.block * w.block * w.d * kept + 4.0 * w.block * w.d * pooled_pairs
@@ -613,6 +634,8 @@ def run_sweep_pasa(device, peaks, peak_src, heads=None):
         "frac_of_burst_peak_p50": flops / (ms["compensated_mma"]["p50"] / 1e3) / 1e12
         / tensor_peak(peaks, "bf16", "bf16_tflops"),
         "kernel": "attn_mma_kernel<comp>", "steps": 20, "warmup": 5,
+        "cpu_baseline": {"value": cpu_tf, "unit": "TFLOPS", "cores": cores(), "kind": "oracle",
+                         "sample": cpu_sample, "seconds": cpu_s},
     }), flush=True)
 
 

@@ -135,3 +135,14 @@ def test_sweep_options_parse_and_refuse_without_cuda():
         with pytest.raises(SystemExit) as e:
             bench.main(["--sweep", *extra])
         assert "CUDA" in str(e.value)
+
+
+def test_pasa_cpu_baseline_runs_the_oracle():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    w = WORKLOADS["small_8x16x16"]
+    q, k, v, perms = make_inputs(w, heads=1)
+    tf, dt, sample = bench.pasa_cpu_baseline(w, q, k, v, perms)
+    assert tf > 0 and dt > 0
+    assert f"all {w.NB} query blocks" in sample
