@@ -303,6 +303,19 @@ def pasa_cpu_baseline(w, q, k, v, perms):
     return flops / dt / 1e12, dt, f"head 0, all {w.NB} query blocks (k = {kk})"
 
 
+def sics_cpu_baseline(w, q, k):
+    """The SICS oracle, as it stands, on head 0 (six orders, q and k).
+    Returns GB/s of the same algorithmic bytes as the kernel's line (every
+    row of q and k read once per order), seconds, and the sample."""
+    from oracle import selection_ref as sel
+    t0 = time.perf_counter()
+    sel.sics_scores(q[:, :1].double().numpy(), k[:, :1].double().numpy(), (w.F, w.H, w.W),
+                    w.block)
+    dt = time.perf_counter() - t0
+    nbytes = 2 * 6 * w.B * w.N * w.d * q.element_size()
+    return nbytes / dt / 1e9, dt, "head 0 of the layer (six orders, q and k)"
+
+
 def cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -519,11 +532,14 @@ def run_sweep_selection(device, peaks, peak_src, heads=None):
     nbytes = 2 * 6 * w.B * w.heads * w.N * w.d * qkv[0].element_size()
     pm = percentiles(ms)
     hbm = float(peaks.get("hbm_gbs", 6650.0))
+    cpu_gbs, cpu_s, cpu_sample = sics_cpu_baseline(w, q, k)
     print(json.dumps({
         "workload": w.name, "kernel": "sics_kernel", "what": "SICS of the six orders, q and k",
         "ms": pm, "bytes": nbytes, "gbs_p50": nbytes / (pm["p50"] / 1e3) / 1e9,
         "frac_of_hbm_p50": nbytes / (pm["p50"] / 1e3) / 1e9 / hbm,
         "peak_source": f"{peak_src} hbm_gbs", "steps": len(ms),
+        "cpu_baseline": {"value": cpu_gbs, "unit": "GB/s", "cores": cores(), "kind": "oracle",
+                         "sample": cpu_sample, "seconds": cpu_s},
     }), flush=True)
     pipe = Pipeline(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, perms, 0.10, device=device,
                     selection="hybrid", top_p=0.5, window=1)

@@ -146,3 +146,13 @@ def test_pasa_cpu_baseline_runs_the_oracle():
     tf, dt, sample = bench.pasa_cpu_baseline(w, q, k, v, perms)
     assert tf > 0 and dt > 0
     assert f"all {w.NB} query blocks" in sample
+
+
+def test_sics_cpu_baseline_runs_the_oracle():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    w = WORKLOADS["small_8x16x16"]
+    q, k, _, _ = make_inputs(w, heads=1)
+    gbs, dt, sample = bench.sics_cpu_baseline(w, q, k)
+    assert gbs > 0 and dt > 0 and "head 0" in sample
