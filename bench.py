@@ -283,6 +283,16 @@ def cpu_baseline(w, q, k, v, perms, idx_host, budget_s=12.0, max_blocks=None, in
     return flops / dt / 1e12, dt, f"head 0, query blocks 0..{done - 1} of {w.NB} ({done * kk} kept tiles)"
 
 
+def oracle_idx_head0(w, q, k, perms, density):
+    """The oracle's own kept lists for head 0 (its float64 pooled scores,
+    top-k at ``density``): [B, 1, NB, k] int32.  The CPU baselines take their
+    work from these, never from the GPU's lists."""
+    from oracle import paro_ref as ref
+    _, _, s = ref.pooled_scores(q[:, :1].double().numpy(), k[:, :1].double().numpy(),
+                                (w.F, w.H, w.W), perms[:1], w.block)
+    return ref.select_topk(s, ref.k_for_density(w.NB, density))
+
+
 def pasa_cpu_baseline(w, q, k, v, perms):
     """The compensation oracle, as it stands, on head 0 of the workload (all
     its query blocks), with the oracle's own top-k at the workload density.
@@ -396,7 +406,7 @@ def run_ours(a):
 
     cpu = None
     if rank == 0 and ws == 1 and not a.no_cpu_baseline:
-        tf, dt, sample = cpu_baseline(w, q, k, v, perms, pipe.idx.cpu().numpy(),
+        tf, dt, sample = cpu_baseline(w, q, k, v, perms, oracle_idx_head0(w, q, k, perms, dens),
                                       budget_s=a.cpu_budget, int8=int8)
         cpu = {"value": tf, "unit": "TFLOPS", "cores": cores(), "kind": "oracle",
                "sample": sample, "seconds": round(dt, 2)}
@@ -661,15 +671,11 @@ def run_reference(a):
     ws, rank, _ = dist_env()
     if rank != 0:
         return
-    from oracle import paro_ref as ref
     w = WORKLOADS[a.workload]
     dens = a.density if a.density is not None else w.density
     q, k, v, perms = make_inputs(w, heads=1)
-    grid = (w.F, w.H, w.W)
-    # the oracle's own selection for head 0 (pooled scores -> top-k)
-    _, _, s = ref.pooled_scores(q.double().numpy(), k.double().numpy(), grid, perms[:1], w.block)
-    kk = ref.k_for_density(w.NB, dens)
-    idx = ref.select_topk(s, kk)
+    idx = oracle_idx_head0(w, q, k, perms, dens)
+    kk = idx.shape[-1]
     blocks = max(1, a.ref_blocks)
     times = []
     for it in range(a.warmup + a.steps):

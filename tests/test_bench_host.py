@@ -156,3 +156,23 @@ def test_sics_cpu_baseline_runs_the_oracle():
     q, k, _, _ = make_inputs(w, heads=1)
     gbs, dt, sample = bench.sics_cpu_baseline(w, q, k)
     assert gbs > 0 and dt > 0 and "head 0" in sample
+
+
+def test_default_line_cpu_baseline_takes_the_oracles_lists():
+    """The default line's CPU baseline, as bench.py builds it: the oracle's
+    own kept lists of head 0 (never the GPU's), then the bounded sample, on
+    the default 720p workload (one query block) and the INT8 long clip."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    for name, int8 in (("720p_21x45x80", False), ("longclip_33x45x80_int8", True)):
+        w = WORKLOADS[name]
+        q, k, v, perms = make_inputs(w, heads=1)
+        idx = bench.oracle_idx_head0(w, q, k, perms, w.density)
+        from oracle import paro_ref as ref
+        assert idx.shape == (w.B, 1, w.NB, ref.k_for_density(w.NB, w.density))
+        assert (idx[..., 0] <= np.arange(w.NB)).all()  # ascending lists that hold the diagonal
+        assert all(i in idx[0, 0, i] for i in range(w.NB))
+        tf, dt, sample = bench.cpu_baseline(w, q, k, v, perms, idx, budget_s=1e9, max_blocks=1,
+                                            int8=int8)
+        assert tf > 0 and "query blocks 0..0" in sample
