@@ -119,16 +119,18 @@ def test_offline_stage_matches_oracle():
         metric, sf, inc = off.permutation_metric(as_f64(q)[0, h], as_f64(k)[0, h], grid, w.block)
         assert np.abs(res["sparse_frac"][0, h].cpu().numpy() - sf).max() <= 1.0 / (w.NB ** 2) + 1e-6
         assert np.abs(res["incoherence"][0, h].cpu().numpy() / np.maximum(inc, 1e-30) - 1).max() < 1e-3
-        srt = np.sort(metric)
-        if srt[1] - srt[0] > 1e-3:
-            assert int(res["orders"][0, h].item()) == off.choose_order(metric)
-        o = int(res["orders"][0, h].item())
+        # the oracle's candidates: its pick and every order within 1e-3 of it
+        # (orders whose blocks hold the same token sets tie exactly)
+        ties = [o for o in range(6) if metric[o] - metric.min() <= 1e-3]
+        assert off.choose_order(metric) in ties
+        assert int(res["orders"][0, h].item()) in ties
+        # the GPU's static masks are the block-sum thresholding of one of them
         pmap = off.attention_map(as_f64(q)[0, h], as_f64(k)[0, h])
-        tot = off.block_stats(pmap, grid, o, w.block)["total"]
         idx = res["idx"][0, h].cpu().numpy()
         cnt = res["counts"][0, h].cpu().numpy()
-        for i in range(w.NB):
-            assert valid_mask_rows(tot[i], i, 0.9, idx[i, :cnt[i]].tolist())
+        rows = [idx[i, :cnt[i]].tolist() for i in range(w.NB)]
+        assert any(all(valid_mask_rows(tot[i], i, 0.9, rows[i]) for i in range(w.NB))
+                   for tot in (off.block_stats(pmap, grid, o, w.block)["total"] for o in ties))
 
 
 def test_frame_local_map_picks_frame_order_and_diagonal_masks():
