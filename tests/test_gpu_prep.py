@@ -105,7 +105,8 @@ def test_topk_on_pooled_scores(w):
     s32 = s.astype(np.float32)
     heads = q.shape[1]
     pr = paro.Problem(w.B, heads, (w.F, w.H, w.W), w.d, w.block, perms)
-    kk = paro.k_for_density(pr.NB, w.density)
+    kk = ref.k_for_density(pr.NB, w.density)
+    assert paro.k_for_density(pr.NB, w.density) == kk
     idx = paro.select_topk(torch.from_numpy(s32).cuda(), pr, kk).cpu().numpy()
     want = ref.select_topk(s32.astype(np.float64), kk)
     assert (idx == want).all()
