@@ -194,7 +194,7 @@ def test_720p_full_size_sampled(c720, density):
                                             (w.F, w.H, w.W), perms[hh:hh + 1], w.block)
             got_s = pipe.scores[:, hh:hh + 1].cpu().double().numpy()
             assert np.abs(got_s - s_ref).max() < 1e-4 * max(1.0, np.abs(s_ref).max())
-            idx_ref[:, hh:hh + 1] = ref.select_topk(s_ref, pipe.k)
+            idx_ref[:, hh:hh + 1] = ref.select_topk(s_ref, ref.k_for_density(w.NB, density))
             agree[:, hh:hh + 1] = selection_agreement(idx_h[:, hh:hh + 1], idx_ref[:, hh:hh + 1],
                                                       s_ref)
         tok_ok = token_mask(agree, (w.F, w.H, w.W), perms, w.block)

@@ -172,6 +172,7 @@ def test_i8_longclip_full_size_sampled():
     torch.cuda.synchronize()
     assert pipe.status.item() == 0
     assert torch.isfinite(out).all()
+    assert pipe.k == ref.k_for_density(w.NB, w.density)
     idx_h = pipe.idx.cpu().numpy()
     grid = (w.F, w.H, w.W)
     rng = np.random.default_rng(21)
@@ -185,7 +186,7 @@ def test_i8_longclip_full_size_sampled():
             assert (dev8[:, sl].cpu().numpy() == x8).all()
             assert (dev_sc[:, sl].cpu().numpy() == sc).all()
         _, _, s_ref = ref.pooled_scores(as_f64(q[:, sl]), as_f64(k[:, sl]), grid, ph, w.block)
-        idx_ref = ref.select_topk(s_ref, pipe.k)
+        idx_ref = ref.select_topk(s_ref, ref.k_for_density(w.NB, w.density))
         agree = selection_agreement(idx_h[:, sl], idx_ref, s_ref)[0, 0]
         # sampled permuted positions whose query block agrees, plus the tail
         pos = [int(p) for p in rng.integers(0, w.N, 64) if agree[int(p) // w.block]]
