@@ -37,7 +37,12 @@ Readings where the pages are silent:
    -inf.  Selected indices are returned in ascending order.
 5. Pad keys are masked with -inf; pad query rows are never output.
 6. Softmax scale 1/sqrt(d).
-7. INT8: see :func:`quantize_int8` and :func:`attention_int8`.
+7. INT8: Q, K, V per-block symmetric codes (:func:`quantize_int8`); P read
+   as the pages state it, the exactly normalised post-softmax map quantised
+   per (query block, key block) tile with the tile's own absmax / 127
+   (:func:`attention_int8`, mode "tile", the default).  The one-pass
+   replays of a flash kernel's order ("online", "rowmax") are kept as
+   named diagnostics.
 
 Parity status: every function here is pinned by the tests under
 ``tests/test_oracle_*.py`` (brute force, library routines, closed forms);
@@ -340,11 +345,12 @@ def quantize_int8(xp: np.ndarray, N: int, block: int, qmax: int = 127):
     return q, sc
 
 
-def _int8_query_rows(qi, ki, vi, sq_i, sk, sv, N, block, kept, mode, quantize_p, p_levels=127):
-    """INT8 attention of some query rows of one query block (int64 codes
-    ``qi`` [r, d], block scale ``sq_i``) over the kept key blocks, in the
-    order listed.  Every step is row-wise, so any subset of a block's rows
-    gets the same values as the whole block.  Returns [r, d] float64."""
+def _int8_tiles(qi, ki, sq_i, sk, N, block, kept):
+    """Score tiles of some query rows (integer codes ``qi`` [r, d] as float64,
+    block scale ``sq_i``) against the kept key blocks, in the order listed:
+    [(j, klo, khi, s)] with s = (q8 k8^T, exact) * s_q * s_k[j] / sqrt(d).
+    The integer products are summed in float64, exactly: |q8 k8| <= 127^2
+    per term, so every partial sum stays far below 2^53."""
     d = qi.shape[1]
     inv_sqrt_d = 1.0 / math.sqrt(d)
     tiles = []
@@ -353,8 +359,48 @@ def _int8_query_rows(qi, ki, vi, sq_i, sk, sv, N, block, kept, mode, quantize_p,
         if khi <= klo:
             continue
         s_int = qi @ ki[klo:khi].T
-        s = s_int.astype(np.float64) * (float(sq_i) * float(sk[j]) * inv_sqrt_d)
-        tiles.append((j, klo, khi, s))
+        tiles.append((j, klo, khi, s_int * (float(sq_i) * float(sk[j]) * inv_sqrt_d)))
+    return tiles
+
+
+def _int8_block_tilewise(qi, ki, vi, sq_i, sk, sv, N, block, kept, quantize_p, p_levels):
+    """Mode "tile" for all valid rows of one query block (the rows share each
+    tile's P scale, so they are evaluated together).
+
+    P is the exactly normalised softmax of every row over all its kept keys;
+    then each (query block, key block) tile of P is quantised symmetrically
+    with its own scale absmax/p_levels (absmax over the tile's valid rows and
+    keys), codes round_half_even(P / scale); the tile contributes
+    (codes V8) * scale * s_v[j].  A tile whose P is all zero contributes 0."""
+    rows = qi.shape[0]
+    tiles = _int8_tiles(qi, ki, sq_i, sk, N, block, kept)
+    if not tiles:
+        return np.zeros((rows, vi.shape[1]), dtype=np.float64)
+    m = np.max([t[3].max(axis=1) for t in tiles], axis=0)[:, None]
+    l = np.zeros((rows, 1))
+    for (_, _, _, s) in tiles:
+        l = l + np.exp(s - m).sum(axis=1, keepdims=True)
+    out = np.zeros((rows, vi.shape[1]))
+    for (j, klo, khi, s) in tiles:
+        p = np.exp(s - m) / l
+        if quantize_p:
+            amax = p.max()
+            if amax == 0.0:
+                continue
+            scale = amax / p_levels
+            codes = np.clip(np.rint(p / scale), -p_levels, p_levels)
+            out = out + (codes @ vi[klo:khi]) * (scale * float(sv[j]))
+        else:
+            out = out + (p @ vi[klo:khi]) * float(sv[j])
+    return out
+
+
+def _int8_query_rows(qi, ki, vi, sq_i, sk, sv, N, block, kept, mode, quantize_p, p_levels=127):
+    """Modes "online" and "rowmax" of INT8 attention for some query rows of
+    one query block, over the kept key blocks in the order listed.  Every
+    step is row-wise, so any subset of a block's rows gets the same values
+    as the whole block.  Returns [r, d] float64."""
+    tiles = _int8_tiles(qi, ki, sq_i, sk, N, block, kept)
     rows = qi.shape[0]
     if not tiles:
         return np.zeros((rows, vi.shape[1]), dtype=np.float64)
@@ -373,67 +419,100 @@ def _int8_query_rows(qi, ki, vi, sq_i, sk, sv, N, block, kept, mode, quantize_p,
         pt = np.exp(s - m_new)
         pq = np.rint(p_levels * pt) / p_levels if quantize_p else pt
         l = l * alpha + pt.sum(axis=1, keepdims=True)
-        acc = acc * alpha + (pq @ vi[klo:khi].astype(np.float64)) * float(sv[j])
+        acc = acc * alpha + (pq @ vi[klo:khi]) * float(sv[j])
         m = m_new
     return acc / l
 
 
+INT8_MODES = ("tile", "online", "rowmax")
+
+
+def _int8_block(qi, ki, vi, sq, sk, sv, N, block, i, kept, mode, quantize_p, p_levels):
+    lo, hi = i * block, min((i + 1) * block, N)
+    if mode == "tile":
+        return _int8_block_tilewise(qi[lo:hi], ki, vi, sq[i], sk, sv, N, block, kept,
+                                    quantize_p, p_levels)
+    return _int8_query_rows(qi[lo:hi], ki, vi, sq[i], sk, sv, N, block, kept, mode, quantize_p,
+                            p_levels)
+
+
 def attention_int8(q8, k8, v8, sq, sk, sv, N: int, block: int, idx, counts=None,
-                   mode: str = "online", quantize_p: bool = True, p_levels: int = 127):
+                   mode: str = "tile", quantize_p: bool = True, p_levels: int = 127):
     """INT8 block-sparse attention in the permuted domain, one head.
 
-    S = (Q8 K8^T exact in integers) * s_q[i] * s_k[j] / sqrt(d) per tile.
-    P is quantised per (query block, key block) tile with a symmetric scale
-    (PAROAttention review, core_discovery: block-wise INT8 quantisation of
-    the post-softmax map).  The softmax numerator of a tile is bounded by 1
-    after max subtraction, so the tile's symmetric scale is 1/127:
-    p8 = round_half_even(127 * P_tilde), and the tile contributes
-    (p8 V8) * s_v[j] / 127.  The normaliser sums the unquantised P_tilde.
+    S = (Q8 K8^T exact in integers) * s_q[i] * s_k[j] / sqrt(d) per tile
+    (PAROAttention review, key_machinery: block-wise INT8 Q/K with groups
+    aligned to the attention block).
 
-    mode "online": kept tiles in ascending order with a running row max,
-    P_tilde = exp(s - m_run), earlier sums rescaled by exp(m_old - m_new)
-    (SPADE review, key_machinery (iii): flash block-sparse attention with
-    an online softmax) -- the order the pages describe.
-    mode "rowmax": P_tilde = exp(s - m_row) with the row's final max.
-    ``quantize_p=False`` skips the P rounding (P used exactly).
-    ``p_levels = 7`` quantises P to 4 bits, p4 = round_half_even(7 * P_tilde),
-    contributing (p4 V) * s_v[j] / 7 (the INT4 PV variant, with V from
-    quantize_int8(..., qmax=7)).
+    P, in the default mode "tile" (PAROAttention review, key_machinery and
+    core_discovery: block-wise quantisation of the post-softmax attention
+    map, groups aligned to the FlashAttention block): the exactly normalised
+    softmax P of each row over all its kept keys, quantised per (query
+    block, key block) tile with that tile's own symmetric scale
+    absmax(P_tile) / 127, codes round_half_even(P / scale); the tile
+    contributes (codes V8) * scale * s_v[j].  This result does not depend
+    on the order in which the kept tiles are visited.
+
+    Two diagnostic modes replay the one-pass order of a flash kernel (SPADE
+    review, key_machinery (iii): online softmax), where the normaliser is
+    not known while a tile is quantised; there the un-normalised tile
+    numerator P~ = exp(s - m) <= 1 is rounded with the fixed scale 1/127,
+    p8 = round_half_even(127 P~), the tile contributes (p8 V8) * s_v[j] / 127
+    and the normaliser sums the unrounded P~:
+      "online": kept tiles in the listed (ascending) order, m the running
+                row max, earlier sums rescaled by exp(m_old - m_new);
+      "rowmax": m the row's final max.
+    ``quantize_p=False`` skips the P rounding (P used exactly; all modes
+    then agree).  ``p_levels = 7`` quantises P to 4 bits (levels +-7) in
+    every mode: the INT4 PV variant, with V from quantize_int8(..., qmax=7).
 
     q8/k8/v8 [Np, d] int8, sq/sk/sv [NB] float32, idx [NB, k]; returns
     [Np, d] float64 (pad rows zero).
     """
+    if mode not in INT8_MODES:
+        raise ValueError(f"mode {mode!r}: one of {INT8_MODES}")
     Np, d = q8.shape
     nb = Np // block
     out = np.zeros((Np, v8.shape[1]), dtype=np.float64)
-    qi = q8.astype(np.int64)
-    ki = k8.astype(np.int64)
-    vi = v8.astype(np.int64)
+    qi = q8.astype(np.float64)
+    ki = k8.astype(np.float64)
+    vi = v8.astype(np.float64)
     for i in range(nb):
         lo, hi = i * block, min((i + 1) * block, N)
         if hi <= lo:
             continue
         c = idx.shape[1] if counts is None else int(counts[i])
         kept = [int(j) for j in idx[i, :c]]
-        out[lo:hi] = _int8_query_rows(qi[lo:hi], ki, vi, sq[i], sk, sv, N, block, kept, mode,
-                                      quantize_p, p_levels)
+        out[lo:hi] = _int8_block(qi, ki, vi, sq, sk, sv, N, block, i, kept, mode, quantize_p,
+                                 p_levels)
     return out
 
 
 def attention_int8_rows(q8, k8, v8, sq, sk, sv, N: int, block: int, idx, positions,
-                        counts=None, mode: str = "online", quantize_p: bool = True,
+                        counts=None, mode: str = "tile", quantize_p: bool = True,
                         p_levels: int = 127):
     """Rows of :func:`attention_int8` at the given permuted positions only
     (one head), for full-size checks where the whole head is too costly.
+    In mode "tile" each position's whole query block is evaluated (its rows
+    share the tiles' P scales) and the requested row taken.
     Returns [len(positions), d] float64."""
-    qi = q8.astype(np.int64)
-    ki = k8.astype(np.int64)
-    vi = v8.astype(np.int64)
+    if mode not in INT8_MODES:
+        raise ValueError(f"mode {mode!r}: one of {INT8_MODES}")
+    qi = q8.astype(np.float64)
+    ki = k8.astype(np.float64)
+    vi = v8.astype(np.float64)
     res = np.zeros((len(positions), v8.shape[1]), dtype=np.float64)
+    cache = {}
     for r, p in enumerate(positions):
         i = int(p) // block
         c = idx.shape[1] if counts is None else int(counts[i])
         kept = [int(j) for j in idx[i, :c]]
-        res[r] = _int8_query_rows(qi[p:p + 1], ki, vi, sq[i], sk, sv, N, block, kept, mode,
-                                  quantize_p, p_levels)[0]
+        if mode == "tile":
+            if i not in cache:
+                cache[i] = _int8_block(qi, ki, vi, sq, sk, sv, N, block, i, kept, mode,
+                                       quantize_p, p_levels)
+            res[r] = cache[i][int(p) - i * block]
+        else:
+            res[r] = _int8_query_rows(qi[p:p + 1], ki, vi, sq[i], sk, sv, N, block, kept, mode,
+                                      quantize_p, p_levels)[0]
     return res

@@ -9,9 +9,18 @@ aligned to the attention block, for QK^T and for the post-softmax map P).
   attention of the same values;
 * analytic bound on the effect of rounding P;
 * online and row-max modes coincide when a row keeps a single block.
+
+The default P reading, mode "tile" (the exactly normalised P quantised per
+(query block, key block) tile with the tile's own absmax / 127), is pinned
+by a hand-worked example (tests/golden/int8_tile_n4_b2.txt), a pure-Python
+brute force on tiny inputs (loops, Python's half-even round()), a closed
+form (equal scores: P = 1/n is exact on the grid, O = the mean of the
+dequantised values), independence from the order of the kept list, the
+whole-block / sampled-row agreement, and the rounding bound.
 """
 
 import math
+import os
 
 import numpy as np
 
@@ -94,7 +103,7 @@ def test_p_rounding_bound():
     k8, sk = ref.quantize_int8(x[1] * 0.5, N, block)
     v8, sv = ref.quantize_int8(x[2], N, block)
     idx = np.tile(np.arange(nb, dtype=np.int32), (nb, 1))
-    for mode in ("online", "rowmax"):
+    for mode in ("tile", "online", "rowmax"):
         exact = ref.attention_int8(q8[0, 0], k8[0, 0], v8[0, 0], sq[0, 0], sk[0, 0], sv[0, 0],
                                    N, block, idx, mode=mode, quantize_p=False)
         quant = ref.attention_int8(q8[0, 0], k8[0, 0], v8[0, 0], sq[0, 0], sk[0, 0], sv[0, 0],
@@ -194,3 +203,141 @@ def test_int4_pv_exact_when_representable_and_bounded_otherwise():
     # the 4-bit P codes are coarser than the 8-bit ones on the same inputs
     p8 = ref.attention_int8(*args)
     assert np.abs(quant - exact).max() > np.abs(p8 - exact).max()
+
+
+def _golden_int8(golden_dir):
+    vals = {}
+    with open(os.path.join(golden_dir, "int8_tile_n4_b2.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                key, *rest = line.split()
+                vals[key] = rest
+    return vals
+
+
+def test_tile_mode_golden_hand_worked(golden_dir):
+    g = _golden_int8(golden_dir)
+    q8, k8, v8 = (np.array([int(x) for x in g[n]], dtype=np.int8)[:, None]
+                  for n in ("q8", "k8", "v8"))
+    one = np.ones(2, dtype=np.float32)
+    idx = np.full((2, 2), -1, dtype=np.int32)
+    counts = np.array([len(g["idx0"]), len(g["idx1"])], dtype=np.int32)
+    idx[0, :counts[0]] = [int(x) for x in g["idx0"]]
+    idx[1, :counts[1]] = [int(x) for x in g["idx1"]]
+    want = np.array([float(x) for x in g["out"]])
+    got = ref.attention_int8(q8, k8, v8, one, one, one, 4, 2, idx, counts)  # default: tile
+    assert np.abs(got[:, 0] - want).max() < 1e-12
+    # the online reading keeps a per-row fixed scale: row 1 comes out exact (2.5)
+    onl = ref.attention_int8(q8, k8, v8, one, one, one, 4, 2, idx, counts, mode="online")
+    assert abs(onl[1, 0] - 2.5) < 1e-12 and abs(got[1, 0] - 2.5) > 2e-3
+    # rows evaluated alone still use their whole block's tile scales
+    rows = ref.attention_int8_rows(q8, k8, v8, one, one, one, 4, 2, idx, [1, 3], counts)
+    assert np.abs(rows[:, 0] - want[[1, 3]]).max() < 1e-12
+
+
+def _brute_tile(q8, k8, v8, sq, sk, sv, N, block, idx, counts, levels):
+    """Pure-Python loops: normalised softmax per row over its kept valid keys,
+    then per tile absmax, codes by Python's round() (half to even)."""
+    Np, d = len(q8), len(q8[0])
+    out = [[0.0] * d for _ in range(Np)]
+    for i in range(Np // block):
+        rows = [r for r in range(i * block, (i + 1) * block) if r < N]
+        kept = [int(j) for j in idx[i][:counts[i]]]
+        keys = {j: [c for c in range(j * block, (j + 1) * block) if c < N] for j in kept}
+        s = {}
+        for r in rows:
+            for j in kept:
+                for c in keys[j]:
+                    dot = sum(int(q8[r][t]) * int(k8[c][t]) for t in range(d))
+                    s[r, c] = dot * float(sq[i]) * float(sk[j]) / math.sqrt(d)
+        p = {}
+        for r in rows:
+            cs = [c for j in kept for c in keys[j]]
+            if not cs:
+                continue
+            m = max(s[r, c] for c in cs)
+            z = sum(math.exp(s[r, c] - m) for c in cs)
+            for c in cs:
+                p[r, c] = math.exp(s[r, c] - m) / z
+        for j in kept:
+            amax = max([p[r, c] for r in rows for c in keys[j]], default=0.0)
+            if amax == 0.0:
+                continue
+            scale = amax / levels
+            for r in rows:
+                for c in keys[j]:
+                    code = round(p[r, c] / scale)
+                    for t in range(d):
+                        out[r][t] += code * int(v8[c][t]) * scale * float(sv[j])
+    return np.array(out)
+
+
+def test_tile_mode_brute_force_loops():
+    rng = np.random.default_rng(31)
+    block, N, d = 4, 11, 3  # a ragged last block
+    nb = -(-N // block)
+    Np = nb * block
+    x = rng.standard_normal((3, 1, 1, Np, d)).astype(np.float32)
+    x[:, :, :, N:] = 0
+    q8, sq = ref.quantize_int8(x[0] * 2, N, block)
+    k8, sk = ref.quantize_int8(x[1] * 2, N, block)
+    v8, sv = ref.quantize_int8(x[2], N, block)
+    idx = np.array([[0, 2, -1], [0, 1, 2], [2, -1, -1]], dtype=np.int32)
+    counts = np.array([2, 3, 1], dtype=np.int32)
+    for levels in (127, 7):
+        want = _brute_tile(q8[0, 0], k8[0, 0], v8[0, 0], sq[0, 0], sk[0, 0], sv[0, 0], N, block,
+                           idx, counts, levels)
+        got = ref.attention_int8(q8[0, 0], k8[0, 0], v8[0, 0], sq[0, 0], sk[0, 0], sv[0, 0], N,
+                                 block, idx, counts, p_levels=levels)
+        assert np.abs(got[:N] - want[:N]).max() < 1e-12
+        assert (got[N:] == 0).all()
+
+
+def test_tile_mode_equal_scores_closed_form():
+    """All-zero key codes: every score is 0, P = 1/n on the n kept valid keys,
+    every tile's codes are 127 and the result is the mean of the dequantised
+    values of the kept keys, exactly."""
+    rng = np.random.default_rng(4)
+    block, N, d = 4, 14, 5
+    nb = -(-N // block)
+    Np = nb * block
+    q8 = rng.integers(-127, 128, size=(Np, d)).astype(np.int8)
+    k8 = np.zeros((Np, d), dtype=np.int8)
+    v8 = rng.integers(-127, 128, size=(Np, d)).astype(np.int8)
+    sq = np.full(nb, 0.5, np.float32)
+    sk = np.full(nb, 0.25, np.float32)
+    sv = rng.uniform(0.1, 1.0, nb).astype(np.float32)
+    idx = np.array([[0, 3], [1, 3], [0, 2], [2, 3]], dtype=np.int32)
+    got = ref.attention_int8(q8, k8, v8, sq, sk, sv, N, block, idx)
+    vdeq = v8.astype(np.float64) * np.repeat(sv.astype(np.float64), block)[:, None]
+    for i in range(nb):
+        cols = [c for j in idx[i] for c in range(j * block, (j + 1) * block) if c < N]
+        want = vdeq[cols].mean(axis=0)
+        assert np.abs(got[i * block:min((i + 1) * block, N)] - want).max() < 1e-12
+
+
+def test_tile_mode_does_not_depend_on_list_order():
+    rng = np.random.default_rng(12)
+    block, nb, d = 8, 5, 16
+    N = Np = block * nb
+    x = rng.standard_normal((3, 1, 1, Np, d)).astype(np.float32)
+    q8, sq = ref.quantize_int8(x[0] * 3, N, block)
+    k8, sk = ref.quantize_int8(x[1] * 3, N, block)
+    v8, sv = ref.quantize_int8(x[2], N, block)
+    idx = np.array([[0, 1, 3], [0, 1, 4], [1, 2, 3], [0, 3, 4], [2, 3, 4]], dtype=np.int32)
+    a = ref.attention_int8(q8[0, 0], k8[0, 0], v8[0, 0], sq[0, 0], sk[0, 0], sv[0, 0], N, block,
+                           idx)
+    b = ref.attention_int8(q8[0, 0], k8[0, 0], v8[0, 0], sq[0, 0], sk[0, 0], sv[0, 0], N, block,
+                           idx[:, ::-1].copy())
+    assert np.abs(a - b).max() < 1e-13
+    # the one-pass replay does depend on it once the running max moves
+    c = ref.attention_int8(q8[0, 0], k8[0, 0], v8[0, 0], sq[0, 0], sk[0, 0], sv[0, 0], N, block,
+                           idx, mode="online")
+    d_ = ref.attention_int8(q8[0, 0], k8[0, 0], v8[0, 0], sq[0, 0], sk[0, 0], sv[0, 0], N, block,
+                            idx[:, ::-1].copy(), mode="online")
+    assert np.abs(c - d_).max() > 1e-6
+    # sampled rows equal the whole-head evaluation
+    pos = [0, 9, 17, 39]
+    rows = ref.attention_int8_rows(q8[0, 0], k8[0, 0], v8[0, 0], sq[0, 0], sk[0, 0], sv[0, 0],
+                                   N, block, idx, pos)
+    assert np.abs(rows - a[pos]).max() < 1e-13
