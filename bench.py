@@ -117,8 +117,12 @@ def ncu_traffic(workload: str, kernel: str):
 NOMINAL_RATIO = {"bf16": 1.0, "int8": 2.0}
 
 
-def tensor_peak(peaks, dtype: str, which: str = "bf16_tflops_sustained") -> float:
-    return float(peaks.get(which, 1400.0)) * NOMINAL_RATIO[dtype]
+def tensor_peak(peaks, dtype: str, which: str = "bf16_tflops") -> float:
+    """The burst GEMM figure by default: the attention kernel is timed in
+    steps of tens of milliseconds, at the clock a short burst runs at (the
+    sustained figure was taken over seconds of back-to-back GEMMs under the
+    power cap, at a lower median clock)."""
+    return float(peaks.get(which, 1590.0)) * NOMINAL_RATIO[dtype]
 
 
 class ClockSampler:
@@ -363,6 +367,8 @@ def run_ours(a):
 
     peaks, peak_src = load_peaks()
     peak = tensor_peak(peaks, dtype)
+    peak_sus = tensor_peak(peaks, dtype, "bf16_tflops_sustained")
+    sus_mhz = (peaks.get("clocks_under_load") or {}).get("sm_mhz_median")
     achieved = flops / (attn_avg / 1e3) / 1e12
 
     # speedup over the same kernel on the dense (density 1.0) layer
@@ -438,8 +444,11 @@ def run_ours(a):
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": ncu_traffic(w.name, kname),
                          "kernel": kname,
-                         "peak_source": (f"{peak_src} bf16_tflops_sustained"
-                                         + (" x 2 (nominal int8/bf16 dense ratio)" if int8 else ""))},
+                         "peak_source": (f"{peak_src} bf16_tflops (burst)"
+                                         + (" x 2 (nominal int8/bf16 dense ratio)" if int8 else "")),
+                         "frac_of_sustained": achieved / peak_sus,
+                         "sustained_peak": peak_sus,
+                         "sustained_peak_clock_mhz": sus_mhz},
             "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": pipe.launches * a.steps,
             "clocks": clocks, "dense": dense, "int8": i8,

@@ -110,7 +110,13 @@ pa_status check_float_dtype(pa_dtype dt) {
 
 extern "C" {
 
-int32_t pa_abi_version(void) { return 5; }
+int32_t pa_abi_version(void) { return 6; }
+
+pa_status pa_clear_status(int32_t* dev_status, void* stream) {
+  PA_REQUIRE(dev_status != nullptr, "dev_status must be non-NULL");
+  return cuda_status(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), (cudaStream_t)stream),
+                     "pa_clear_status memset");
+}
 
 const char* pa_last_error(void) { return g_error.c_str(); }
 
@@ -190,7 +196,9 @@ pa_status pa_select_topk(const float* scores, pa_shape shape, int32_t k, int32_t
   if (st != PA_OK) return st;
   PA_REQUIRE(scores && idx, "scores and idx must be non-NULL");
   PA_REQUIRE(k >= 1 && k <= g.NB, "k=%d must be in [1, NB=%d]", k, g.NB);
-  PA_REQUIRE(g.NB <= 16384, "NB=%d exceeds 16384 (row keys must fit in shared memory)", g.NB);
+  if (g.NB > paro::kTopkMaxNB)
+    return fail(PA_ERR_UNSUPPORTED, "NB=%d exceeds %d (a row's keys must fit in shared memory)",
+                g.NB, paro::kTopkMaxNB);
   return cuda_status(paro::launch_topk(scores, g, k, idx, (cudaStream_t)stream),
                      "pa_select_topk launch");
 }

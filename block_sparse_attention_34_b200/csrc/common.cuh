@@ -13,6 +13,12 @@ namespace paro {
 
 constexpr int kMaxHeads = 1024;
 
+// Top-k selection: warps per CTA, each holding one row of NB 32-bit keys in
+// shared memory, so NB is bounded by the opt-in shared memory per CTA.
+constexpr int kTopkWarps = 4;
+constexpr int kSmemOptIn = 232448;  // bytes of shared memory a CTA may opt into
+constexpr int kTopkMaxNB = kSmemOptIn / (kTopkWarps * 4);  // 14528
+
 // Sizes of one call plus the per-order index tables.  For order o (letters
 // outer -> inner, PAROAttention review: the six orders of [F, H, W]) a
 // permuted position p decomposes as p = (c_out * mid[o] + c_mid) * inn[o] +

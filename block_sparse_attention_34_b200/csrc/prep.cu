@@ -162,7 +162,6 @@ __device__ __forceinline__ uint32_t score_key(float f, bool diag) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-constexpr int kTopkWarps = 4;
 
 // One warp per row (bh, i).  Phase 1 finds, bit by bit from the top, the
 // 32-bit key t of the k-th largest key (counting multiplicity).  Every key

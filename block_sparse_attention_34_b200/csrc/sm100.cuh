@@ -176,16 +176,6 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t tmem, uint32_t cols) {
                : "memory");
 }
 
-// Per-warpgroup register budget (every warp of the warpgroup executes it).
-template <int N>
-__device__ __forceinline__ void regs_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N));
-}
-template <int N>
-__device__ __forceinline__ void regs_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N));
-}
-
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
 }

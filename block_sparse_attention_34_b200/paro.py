@@ -18,7 +18,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libparo.so")
 
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_TIMEOUT, PA_ERR_DEVICE_CHECK = range(6)
-ABI_VERSION = 5  # the pa_abi_version() these signatures describe
+ABI_VERSION = 6  # the pa_abi_version() these signatures describe
 PA_F32, PA_BF16, PA_I8 = 0, 1, 2
 PA_ATTN_PERMUTED = 1
 PA_ATTN_P4 = 2  # with int8 inputs: 4-bit P codes (INT4 PV)
@@ -54,6 +54,7 @@ def load():
     sig = {
         "pa_abi_version": ([], _I),
         "pa_last_error": ([], ctypes.c_char_p),
+        "pa_clear_status": ([_P, _P], _I),
         "pa_num_blocks": ([PaShape], _I),
         "pa_k_for_density": ([_I, ctypes.c_double], _I),
         "pa_reorder": ([_P, _P, _I, PaShape, _P, _P, _P], _I),
@@ -115,12 +116,41 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 
 def _need_cuda(*ts):
+    dev = None
     for t in ts:
         if t is not None:
             if not t.is_cuda:
                 raise ValueError("tensors must be on a CUDA device (no CPU path)")
             if not t.is_contiguous():
                 raise ValueError("tensors must be contiguous")
+            if dev is None:
+                dev = t.device
+            elif t.device != dev:
+                raise ValueError(f"tensors on different devices ({dev} and {t.device})")
+
+
+_FLOAT = (torch.float32, torch.bfloat16)
+
+
+def _expect(t, name, shape, dtypes):
+    """Raise ValueError unless tensor ``t`` has exactly ``shape`` and one of
+    ``dtypes``: the library reads and writes whole buffers of the sizes the
+    shape implies, so a smaller buffer must never reach it."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(int(x) for x in shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if isinstance(dtypes, torch.dtype):
+        dtypes = (dtypes,)
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected one of {dtypes}")
+
+
+def _same_dtype(*named):
+    ts = [(n, t) for n, t in named if t is not None]
+    for n, t in ts[1:]:
+        if t.dtype != ts[0][1].dtype:
+            raise ValueError(f"{n}: dtype {t.dtype} differs from {ts[0][0]}'s {ts[0][1].dtype}")
 
 
 class Problem:
@@ -139,6 +169,26 @@ class Problem:
         self.shape = PaShape(self.B, self.heads, self.F, self.H, self.W, self.d, self.block)
 
     @property
+    def natural(self):
+        return (self.B, self.heads, self.N, self.d)
+
+    @property
+    def permuted(self):
+        return (self.B, self.heads, self.N_p, self.d)
+
+    @property
+    def pooled(self):
+        return (self.B, self.heads, self.NB, self.d)
+
+    @property
+    def square(self):
+        return (self.B, self.heads, self.NB, self.NB)
+
+    @property
+    def per_block(self):
+        return (self.B, self.heads, self.NB)
+
+    @property
     def perms_ptr(self):
         return self._perms.ctypes.data_as(ctypes.c_void_p)
 
@@ -146,6 +196,13 @@ class Problem:
     def from_qkv(cls, q, grid, perms, block):
         B, h, N, d = q.shape
         return cls(B, h, grid, d, block, perms)
+
+
+def clear_status(status):
+    """Enqueue status[0] = PA_OK on the current stream (a memset)."""
+    _need_cuda(status)
+    _expect_status(status)
+    _check(load().pa_clear_status(_ptr(status), _stream()))
 
 
 def k_for_density(nb: int, density: float) -> int:
@@ -156,7 +213,10 @@ def reorder(x, pr: Problem, out=None, pool=None, with_pool=False):
     """Permuted copy [B, heads, N_p, d] of natural-order x; with
     ``with_pool`` (or a given ``pool`` buffer) also the block means, from
     the same read: returns (x_perm, pool)."""
-    _need_cuda(x)
+    _need_cuda(x, out, pool)
+    _expect(x, "x", pr.natural, _FLOAT)
+    _expect(out, "out", pr.permuted, x.dtype)
+    _expect(pool, "pool", pr.pooled, torch.float32)
     out = out if out is not None else torch.empty((pr.B, pr.heads, pr.N_p, pr.d), dtype=x.dtype,
                                                   device=x.device)
     if with_pool and pool is None:
@@ -167,7 +227,9 @@ def reorder(x, pr: Problem, out=None, pool=None, with_pool=False):
 
 
 def inverse_reorder(xp, pr: Problem, out=None):
-    _need_cuda(xp)
+    _need_cuda(xp, out)
+    _expect(xp, "xp", pr.permuted, _FLOAT)
+    _expect(out, "out", pr.natural, xp.dtype)
     out = out if out is not None else torch.empty((pr.B, pr.heads, pr.N, pr.d), dtype=xp.dtype,
                                                   device=xp.device)
     _check(load().pa_inverse_reorder(_ptr(xp), _ptr(out), _dtype_code(xp), pr.shape, pr.perms_ptr,
@@ -176,7 +238,12 @@ def inverse_reorder(xp, pr: Problem, out=None):
 
 
 def block_score(q, k, pr: Problem, q_pool=None, k_pool=None, scores=None):
-    _need_cuda(q, k)
+    _need_cuda(q, k, q_pool, k_pool, scores)
+    _expect(q, "q", pr.natural, _FLOAT)
+    _expect(k, "k", pr.natural, q.dtype)
+    _expect(q_pool, "q_pool", pr.pooled, torch.float32)
+    _expect(k_pool, "k_pool", pr.pooled, torch.float32)
+    _expect(scores, "scores", pr.square, torch.float32)
     dev = q.device
     q_pool = q_pool if q_pool is not None else torch.empty((pr.B, pr.heads, pr.NB, pr.d), dtype=torch.float32, device=dev)
     k_pool = k_pool if k_pool is not None else torch.empty_like(q_pool)
@@ -187,21 +254,29 @@ def block_score(q, k, pr: Problem, q_pool=None, k_pool=None, scores=None):
 
 
 def score_pooled(q_pool, k_pool, pr: Problem, scores=None):
-    _need_cuda(q_pool, k_pool)
+    _need_cuda(q_pool, k_pool, scores)
+    _expect(q_pool, "q_pool", pr.pooled, torch.float32)
+    _expect(k_pool, "k_pool", pr.pooled, torch.float32)
+    _expect(scores, "scores", pr.square, torch.float32)
     scores = scores if scores is not None else torch.empty((pr.B, pr.heads, pr.NB, pr.NB), dtype=torch.float32, device=q_pool.device)
     _check(load().pa_score_pooled(_ptr(q_pool), _ptr(k_pool), pr.shape, _ptr(scores), _stream()))
     return scores
 
 
 def select_topk(scores, pr: Problem, k: int, idx=None):
-    _need_cuda(scores)
+    _need_cuda(scores, idx)
+    _expect(scores, "scores", pr.square, torch.float32)
+    _expect(idx, "idx", pr.per_block + (int(k),), torch.int32)
     idx = idx if idx is not None else torch.empty((pr.B, pr.heads, pr.NB, k), dtype=torch.int32, device=scores.device)
     _check(load().pa_select_topk(_ptr(scores), pr.shape, int(k), _ptr(idx), _stream()))
     return idx
 
 
 def compact_mask(bitmask, pr: Problem, idx=None, counts=None):
-    _need_cuda(bitmask)
+    _need_cuda(bitmask, idx, counts)
+    _expect(bitmask, "bitmask", pr.per_block + (-(-pr.NB // 32),), (torch.int32, torch.uint32))
+    _expect(idx, "idx", pr.square, torch.int32)
+    _expect(counts, "counts", pr.per_block, torch.int32)
     dev = bitmask.device
     idx = idx if idx is not None else torch.empty((pr.B, pr.heads, pr.NB, pr.NB), dtype=torch.int32, device=dev)
     counts = counts if counts is not None else torch.empty((pr.B, pr.heads, pr.NB), dtype=torch.int32, device=dev)
@@ -212,7 +287,10 @@ def compact_mask(bitmask, pr: Problem, idx=None, counts=None):
 def select_hybrid(scores, pr: Problem, k: int, top_p: float, window: int, idx=None, counts=None):
     """Union of the diagonal, a local window, Top-K and Top-P per query-block
     row -> (idx [B,h,NB,NB] ascending, -1 padded; counts [B,h,NB])."""
-    _need_cuda(scores)
+    _need_cuda(scores, idx, counts)
+    _expect(scores, "scores", pr.square, torch.float32)
+    _expect(idx, "idx", pr.square, torch.int32)
+    _expect(counts, "counts", pr.per_block, torch.int32)
     dev = scores.device
     idx = idx if idx is not None else torch.empty((pr.B, pr.heads, pr.NB, pr.NB), dtype=torch.int32, device=dev)
     counts = counts if counts is not None else torch.empty((pr.B, pr.heads, pr.NB), dtype=torch.int32, device=dev)
@@ -224,7 +302,10 @@ def select_hybrid(scores, pr: Problem, k: int, top_p: float, window: int, idx=No
 def sics_scores(q, k, pr: Problem, scores=None):
     """[B,h,6] blocking scores of the six axis orders (SICS of q's and k's
     blocks); the argmax per head is the order SPADE's rule picks."""
-    _need_cuda(q, k)
+    _need_cuda(q, k, scores)
+    _expect(q, "q", pr.natural, _FLOAT)
+    _expect(k, "k", pr.natural, q.dtype)
+    _expect(scores, "scores", (pr.B, pr.heads, 6), torch.float32)
     scores = scores if scores is not None else torch.empty((pr.B, pr.heads, 6), dtype=torch.float32, device=q.device)
     _check(load().pa_sics_scores(_ptr(q), _ptr(k), _dtype_code(q), pr.shape, _ptr(scores), _stream()))
     return scores
@@ -234,6 +315,8 @@ def map_row_stats(q_perm, k_perm, pr: Problem, order: int, status=None):
     """Row softmax (log2 max, sum) of every token of the dense map, from
     copies of q, k permuted by ``order`` -> ([B,h,N], [B,h,N])."""
     _need_cuda(q_perm, k_perm)
+    _expect(q_perm, "q_perm", pr.permuted, torch.bfloat16)
+    _expect(k_perm, "k_perm", pr.permuted, torch.bfloat16)
     dev = q_perm.device
     m = torch.empty((pr.B, pr.heads, pr.N), dtype=torch.float32, device=dev)
     l = torch.empty_like(m)
@@ -247,6 +330,10 @@ def map_block_stats(q_perm, k_perm, pr: Problem, order: int, row_max, row_sum, e
     """Per block of the map in ``order``: dict of [B,h,NB,NB] count / total
     / peak (and log_total)."""
     _need_cuda(q_perm, k_perm, row_max, row_sum)
+    _expect(q_perm, "q_perm", pr.permuted, torch.bfloat16)
+    _expect(k_perm, "k_perm", pr.permuted, torch.bfloat16)
+    _expect(row_max, "row_max", (pr.B, pr.heads, pr.N), torch.float32)
+    _expect(row_sum, "row_sum", (pr.B, pr.heads, pr.N), torch.float32)
     dev = q_perm.device
     out = {key: torch.empty((pr.B, pr.heads, pr.NB, pr.NB), dtype=torch.float32, device=dev)
            for key in ("count", "total", "peak")}
@@ -298,7 +385,11 @@ def paro_offline(q, k, grid, block, eps=1e-3, rho=0.9, alpha=0.5, sigma=0.9, sta
 def quantize_int8(x, pr: Problem, with_pool=False, x_q=None, scales=None, pool=None, bits=8):
     """Per-block symmetric quantisation in the permuted order: 8-bit codes
     (levels +-127), or ``bits=4`` (levels +-7, one code per byte)."""
-    _need_cuda(x)
+    _need_cuda(x, x_q, scales, pool)
+    _expect(x, "x", pr.natural, _FLOAT)
+    _expect(x_q, "x_q", pr.permuted, torch.int8)
+    _expect(scales, "scales", pr.per_block, torch.float32)
+    _expect(pool, "pool", pr.pooled, torch.float32)
     dev = x.device
     x_q = x_q if x_q is not None else torch.empty((pr.B, pr.heads, pr.N_p, pr.d), dtype=torch.int8, device=dev)
     scales = scales if scales is not None else torch.empty((pr.B, pr.heads, pr.NB), dtype=torch.float32, device=dev)
@@ -312,6 +403,21 @@ def quantize_int8(x, pr: Problem, with_pool=False, x_q=None, scales=None, pool=N
     return (x_q, scales, pool) if with_pool else (x_q, scales)
 
 
+def _check_lists(idx, counts, pr: Problem):
+    """idx [B,h,NB,k_max] int32 with 0 <= k_max <= NB; counts [B,h,NB] int32."""
+    if idx is None:
+        raise ValueError("idx is required")
+    if idx.dim() != 4 or tuple(idx.shape[:3]) != pr.per_block or idx.shape[3] > pr.NB:
+        raise ValueError(f"idx: shape {tuple(idx.shape)}, expected {pr.per_block + ('k<=NB',)}")
+    _expect(idx, "idx", tuple(idx.shape), torch.int32)
+    _expect(counts, "counts", pr.per_block, torch.int32)
+
+
+def _expect_status(status):
+    if status is not None and (status.dtype != torch.int32 or status.numel() < 1):
+        raise ValueError("status: an int32 tensor of at least one element")
+
+
 def block_sparse_attn(q, k, v, pr: Problem, idx, counts=None, scales=None, out=None,
                       status=None, baseline=False, permuted=False, p4=False):
     """O = block-sparse attention over the kept tiles, natural token order.
@@ -320,9 +426,21 @@ def block_sparse_attn(q, k, v, pr: Problem, idx, counts=None, scales=None, out=N
     ``scales`` = (q_scale, k_scale, v_scale) for int8 q/k/v from
     :func:`quantize_int8` (output bf16).  ``baseline=True`` runs the
     mma.sync comparison kernel instead of the tcgen05 one."""
-    _need_cuda(q, k, v, idx, counts)
+    _need_cuda(q, k, v, idx, counts, out, status, *(scales or ()))
     code = _dtype_code(q)
+    _same_dtype(("q", q), ("k", k), ("v", v))
+    rows = pr.permuted if (permuted or code == PA_I8) else pr.natural
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _expect(t, name, rows, (torch.float32, torch.bfloat16, torch.int8))
+    _check_lists(idx, counts, pr)
+    if code == PA_I8:
+        if scales is None or len(scales) != 3:
+            raise ValueError("int8 q, k, v need scales=(q_scale, k_scale, v_scale)")
+        for name, t in zip(("q_scale", "k_scale", "v_scale"), scales):
+            _expect(t, name, pr.per_block, torch.float32)
     out_dtype = torch.bfloat16 if code == PA_I8 else q.dtype
+    _expect(out, "out", pr.natural, out_dtype)
+    _expect_status(status)
     out = out if out is not None else torch.empty((pr.B, pr.heads, pr.N, pr.d), dtype=out_dtype, device=q.device)
     k_max = int(idx.shape[-1])
     flags = (PA_ATTN_PERMUTED if permuted else 0) | (PA_ATTN_P4 if p4 else 0)
@@ -348,7 +466,16 @@ def block_sparse_attn_compensated(q, k, v, pr: Problem, idx, k_pool, v_pool, cou
     v_pool [B, heads, NB, d] float32 block means (from :func:`reorder` with
     ``with_pool`` or :func:`block_score`).  bf16 or fp32 q, k, v; output
     natural order, q's dtype."""
-    _need_cuda(q, k, v, idx, counts, k_pool, v_pool)
+    _need_cuda(q, k, v, idx, counts, k_pool, v_pool, out, status)
+    _same_dtype(("q", q), ("k", k), ("v", v))
+    rows = pr.permuted if permuted else pr.natural
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _expect(t, name, rows, _FLOAT)
+    _check_lists(idx, counts, pr)
+    _expect(k_pool, "k_pool", pr.pooled, torch.float32)
+    _expect(v_pool, "v_pool", pr.pooled, torch.float32)
+    _expect(out, "out", pr.natural, q.dtype)
+    _expect_status(status)
     out = out if out is not None else torch.empty((pr.B, pr.heads, pr.N, pr.d), dtype=q.dtype,
                                                   device=q.device)
     st = load().pa_block_sparse_attn_compensated(

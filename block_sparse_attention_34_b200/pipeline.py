@@ -2,7 +2,7 @@
 that repeated calls (a DiT's layers and denoising steps) launch kernels only.
 
 Launch sequence of :meth:`Pipeline.run` (every step through the C ABI, on the
-current torch stream):
+current torch stream; the status word is cleared first, by a memset):
 
   bf16:  reorder+pool(q), reorder+pool(k), reorder(v)  -- one HBM pass each
          score_pooled -> select_topk (or select_hybrid: diagonal, window,
@@ -102,6 +102,9 @@ class Pipeline:
         return pr.B * pr.heads * pr.NB * self.k
 
     def run(self, q, k, v):
+        # one status word for the whole call sequence, cleared per call (a
+        # kernel that finds a timeout recorded there skips its work)
+        paro.clear_status(self.status)
         self.select(q, k, v)
         self.attend(q, k, v)
         return self.out

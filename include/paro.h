@@ -86,11 +86,18 @@ typedef struct {
   int32_t B, heads, F, H, W, d, block;
 } pa_shape;
 
-/* Version of this ABI (bumped on any signature change): 5. */
+/* Version of this ABI (bumped on any signature change): 6. */
 PA_API int32_t pa_abi_version(void);
 
 /* Message of the last failed call on this thread ("" if none). */
 PA_API const char* pa_last_error(void);
+
+/* Enqueue a reset of the device status word *dev_status (one int32, device
+ * memory) to PA_OK on `stream` (a memset; no kernel).  A kernel that finds
+ * PA_ERR_TIMEOUT recorded skips its work, so a caller reusing one status
+ * word across calls clears it before each call sequence.  Not part of the
+ * pages' method: bookkeeping of this library's error reporting. */
+PA_API pa_status pa_clear_status(int32_t* dev_status, void* stream);
 
 /* NB = ceil(F*H*W / block), or -1 for a malformed shape. */
 PA_API int32_t pa_num_blocks(pa_shape shape);
@@ -136,7 +143,9 @@ PA_API pa_status pa_score_pooled(const float* q_pool, const float* k_pool, pa_sh
  * block; SPADE review: Top-K filter).  Row (b,h,i) of scores
  * [B,heads,NB,NB] -> idx[b,h,i,0..k-1] (int32, ascending): block i itself,
  * then the k-1 largest other scores, ties to the lower block index, NaN
- * read as -inf, -0.0 equal to +0.0.  1 <= k <= NB. */
+ * read as -inf, -0.0 equal to +0.0.  1 <= k <= NB; NB <= 14528
+ * (PA_ERR_UNSUPPORTED above: four rows of NB keys share a CTA's shared
+ * memory). */
 PA_API pa_status pa_select_topk(const float* scores, pa_shape shape, int32_t k, int32_t* idx,
                          void* stream);
 

@@ -34,7 +34,7 @@ def test_exports_every_declared_symbol(lib):
     assert len(names) >= 12
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.pa_abi_version() == paro.ABI_VERSION == 5
+    assert lib.pa_abi_version() == paro.ABI_VERSION == 6
 
 
 def test_k_for_density_matches_oracle(lib):
@@ -171,3 +171,115 @@ def test_compensated_attention_validation(lib):
     assert fn(FAKE, FAKE, FAKE, paro.PA_BF16, 0, big, pp, FAKE, None, 2, FAKE, FAKE, FAKE, None,
               None) == paro.PA_ERR_UNSUPPORTED
     assert b"4096" in lib.pa_last_error()
+
+
+def test_topk_nb_limit_is_reported(lib):
+    """NB above the shared-memory bound of the top-k kernel is refused as
+    unsupported before any launch (14528 = 232448 B / (4 rows x 4 B))."""
+    idx = ctypes.c_void_p(4096)
+    # 1 x 1 x 14529 tokens, block 1 is not a supported block; use block 64:
+    # N = 64 * 14529 gives NB = 14529
+    st = lib.pa_select_topk(FAKE, paro.PaShape(1, 1, 1, 1, 64 * 14529, 64, 64), 1, idx, None)
+    assert st == paro.PA_ERR_UNSUPPORTED
+    assert b"14528" in lib.pa_last_error()
+
+
+def test_clear_status_rejects_null(lib):
+    assert lib.pa_clear_status(None, None) == paro.PA_ERR_INVALID_ARG
+
+
+# --- the Python binding refuses mismatched tensors before any library call ---
+
+@pytest.fixture()
+def host_binding(monkeypatch):
+    """The binding with its CUDA-device check disabled and a library that
+    fails the test if it is ever called: every case below must be refused
+    by the binding's own shape and dtype checks."""
+    import torch
+
+    class NoLib:
+        def __getattr__(self, name):
+            raise AssertionError(f"library call {name} reached with a bad argument")
+
+    monkeypatch.setattr(paro, "_need_cuda", lambda *ts: None)
+    monkeypatch.setattr(paro, "load", lambda: NoLib())
+    return torch
+
+
+def test_binding_rejects_bad_shapes(host_binding):
+    torch = host_binding
+    pr = paro.Problem(1, 2, (4, 8, 16), 128, 128, [0, 5])  # N 512, NB 4, N_p 512
+    pr_r = paro.Problem(1, 2, (3, 5, 9), 128, 128, [0, 5])  # N 135, NB 2, N_p 256
+    nat = torch.zeros(pr_r.natural, dtype=torch.bfloat16)
+    perm = torch.zeros(pr_r.permuted, dtype=torch.bfloat16)
+    idx = torch.zeros(pr_r.per_block + (2,), dtype=torch.int32)
+    bad = [
+        # permuted=True with natural-order tensors: a tiled load would read
+        # past the allocation
+        lambda: paro.block_sparse_attn(nat, nat, nat, pr_r, idx, permuted=True),
+        # natural-order call with permuted tensors
+        lambda: paro.block_sparse_attn(perm, perm, perm, pr_r, idx),
+        # k and v of another dtype than q
+        lambda: paro.block_sparse_attn(nat, nat.float(), nat, pr_r, idx),
+        # kept lists wider than NB, or of another row count
+        lambda: paro.block_sparse_attn(nat, nat, nat, pr_r,
+                                       torch.zeros(pr_r.per_block + (3,), dtype=torch.int32)),
+        lambda: paro.block_sparse_attn(nat, nat, nat, pr_r,
+                                       torch.zeros((1, 2, 3, 2), dtype=torch.int32)),
+        lambda: paro.block_sparse_attn(nat, nat, nat, pr_r, idx.long()),
+        # counts of the wrong length, output of the wrong shape or dtype
+        lambda: paro.block_sparse_attn(nat, nat, nat, pr_r, idx,
+                                       torch.zeros((1, 2, 3), dtype=torch.int32)),
+        lambda: paro.block_sparse_attn(nat, nat, nat, pr_r, idx, out=torch.zeros(pr_r.permuted)),
+        lambda: paro.block_sparse_attn(nat, nat, nat, pr_r, idx,
+                                       out=torch.zeros(pr_r.natural, dtype=torch.float32)),
+        # int8 without scales, or with scales of the wrong length
+        lambda: paro.block_sparse_attn(*(torch.zeros(pr_r.permuted, dtype=torch.int8),) * 3,
+                                       pr_r, idx),
+        lambda: paro.block_sparse_attn(*(torch.zeros(pr_r.permuted, dtype=torch.int8),) * 3,
+                                       pr_r, idx, scales=(torch.zeros(3),) * 3),
+        # top-k output narrower than k
+        lambda: paro.select_topk(torch.zeros(pr.square), pr, 3,
+                                 torch.zeros(pr.per_block + (2,), dtype=torch.int32)),
+        lambda: paro.select_topk(torch.zeros(pr.square, dtype=torch.float64), pr, 2),
+        # reorder into a buffer without the tail padding
+        lambda: paro.reorder(nat, pr_r, out=torch.zeros(pr_r.natural, dtype=torch.bfloat16)),
+        lambda: paro.reorder(nat, pr_r, pool=torch.zeros((1, 2, 2, 64))),
+        lambda: paro.inverse_reorder(nat, pr_r),
+        lambda: paro.quantize_int8(nat, pr_r, x_q=torch.zeros(pr_r.natural, dtype=torch.int8)),
+        lambda: paro.score_pooled(torch.zeros(pr.pooled), torch.zeros(pr.pooled), pr,
+                                  torch.zeros((1, 2, 4, 5))),
+        lambda: paro.compact_mask(torch.zeros((1, 2, 4, 2), dtype=torch.int32), pr),
+        lambda: paro.block_score(nat, nat.float(), pr_r),
+        lambda: paro.block_sparse_attn_compensated(nat, nat, nat, pr_r, idx,
+                                                   torch.zeros((1, 2, 2, 64)),
+                                                   torch.zeros(pr_r.pooled)),
+    ]
+    for i, call in enumerate(bad):
+        with pytest.raises(ValueError):
+            call()
+
+
+def test_binding_passes_good_shapes_to_the_library(host_binding):
+    """The same calls with well-formed tensors get past the checks (they
+    reach the stand-in library, which raises AssertionError)."""
+    torch = host_binding
+    pr_r = paro.Problem(1, 2, (3, 5, 9), 128, 128, [0, 5])
+    nat = torch.zeros(pr_r.natural, dtype=torch.bfloat16)
+    perm = torch.zeros(pr_r.permuted, dtype=torch.bfloat16)
+    i8 = torch.zeros(pr_r.permuted, dtype=torch.int8)
+    idx = torch.zeros(pr_r.per_block + (2,), dtype=torch.int32)
+    sc = torch.zeros(pr_r.per_block)
+    good = [
+        lambda: paro.block_sparse_attn(nat, nat, nat, pr_r, idx),
+        lambda: paro.block_sparse_attn(perm, perm, perm, pr_r, idx, permuted=True),
+        lambda: paro.block_sparse_attn(i8, i8, i8, pr_r, idx, scales=(sc, sc, sc)),
+        lambda: paro.reorder(nat, pr_r, with_pool=True),
+        lambda: paro.select_topk(torch.zeros(pr_r.square), pr_r, 2),
+        lambda: paro.block_sparse_attn_compensated(perm, perm, perm, pr_r, idx,
+                                                   torch.zeros(pr_r.pooled),
+                                                   torch.zeros(pr_r.pooled), permuted=True),
+    ]
+    for call in good:
+        with pytest.raises(AssertionError, match="library call"):
+            call()

@@ -143,17 +143,39 @@ def test_malformed_list_is_reported_not_fatal(path):
                 assert (got[0, h, rows] == 7.0).all()
 
 
-def test_480p_two_heads_full():
+def oracle_lists(w, q, k, perms, idx_gpu, density=None):
+    """Per head: the oracle's kept lists (top-k of its float64 pooled
+    scores), and the [B,h,NB] rows where the GPU's lists equal them (the
+    others must be valid near-tie choices)."""
+    idx_ref = np.zeros_like(idx_gpu)
+    agree = np.ones(idx_gpu.shape[:3], dtype=bool)
+    dens = w.density if density is None else density
+    for hh in range(w.heads):
+        sl = slice(hh, hh + 1)
+        _, _, s_ref = ref.pooled_scores(as_f64(q[:, sl]), as_f64(k[:, sl]), (w.F, w.H, w.W),
+                                        perms[sl], w.block)
+        idx_ref[:, sl] = ref.select_topk(s_ref, ref.k_for_density(w.NB, dens))
+        agree[:, sl] = selection_agreement(idx_gpu[:, sl], idx_ref[:, sl], s_ref)
+    return idx_ref, agree
+
+
+def test_480p_all_heads_full():
+    """The bench's launch sequence (Pipeline) on the whole 480p-shaped layer
+    (21x30x52 tokens, 12 heads, density 0.25): every output row of every
+    head against the oracle over the oracle's kept lists."""
     w = WORKLOADS["480p_21x30x52"]
-    q, k, v, perms = inputs(w, heads=2)
-    pr = problem(w, perms, heads=2)
-    qd, kd, vd = to_dev(q, k, v)
-    status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    out, idx = paro.attention(qd, kd, vd, (w.F, w.H, w.W), perms, w.block, w.density,
-                              status=status)
+    q, k, v, perms = inputs(w)
+    pipe = Pipeline(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, perms, w.density)
+    pipe.out.fill_(float("nan"))  # every row must be written
+    out = pipe.run(*to_dev(q, k, v))
     torch.cuda.synchronize()
-    assert status.item() == 0
-    check_against_oracle_selection(w, q, k, v, perms, out, idx)
+    assert pipe.status.item() == 0
+    assert torch.isfinite(out).all()
+    assert pipe.k == ref.k_for_density(w.NB, w.density)
+    idx_ref, agree = oracle_lists(w, q, k, perms, pipe.idx.cpu().numpy())
+    assert agree.mean() >= 0.95
+    want = ref.attention(as_f64(q), as_f64(k), as_f64(v), (w.F, w.H, w.W), perms, w.block, idx_ref)
+    compare_rows(out, want, token_mask(agree, (w.F, w.H, w.W), perms, w.block))
 
 
 @pytest.fixture(scope="module")
@@ -163,52 +185,59 @@ def c720():
     return w, q, k, v, perms
 
 
-def sampled_rows(w, n, seed):
+def sampled_rows(w, per_head, seed):
+    """per_head seeded rows of every head, plus each head's last token (the
+    ragged tail block)."""
     rng = np.random.default_rng(seed)
-    rows = [(0, int(rng.integers(w.heads)), int(rng.integers(w.N))) for _ in range(n)]
-    # always include the last token of every head (ragged tail block)
-    rows += [(0, h, w.N - 1) for h in range(0, w.heads, 7)]
+    rows = []
+    for h in range(w.heads):
+        rows += [(0, h, int(n)) for n in rng.integers(0, w.N, per_head)]
+        rows.append((0, h, w.N - 1))
     return rows
 
 
-@pytest.mark.parametrize("density", [0.15, 1.0])
-def test_720p_full_size_sampled(c720, density):
-    """The bench's launch sequence (Pipeline) on the full 720p-shaped layer."""
-    w, q, k, v, perms = c720
+def full_size_sampled(w, q, k, v, perms, density, per_head, seed, min_rows):
+    """Pipeline at full size; sampled rows of every head against the oracle
+    row evaluator over the oracle's kept lists."""
     pipe = Pipeline(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, perms, density)
     assert pipe.k == ref.k_for_density(w.NB, density)
-    qkv = to_dev(q, k, v)
-    out = pipe.run(*qkv)
+    pipe.out.fill_(float("nan"))  # every row must be written
+    out = pipe.run(*to_dev(q, k, v))
     torch.cuda.synchronize()
     assert pipe.status.item() == 0
+    assert torch.isfinite(out).all()
     idx_h = pipe.idx.cpu().numpy()
-    rows = sampled_rows(w, 192 if density < 1.0 else 48, seed=11)
-    heads = sorted({h for (_, h, _) in rows})
-    idx_ref = np.zeros_like(idx_h)
+    rows = sampled_rows(w, per_head, seed)
     if density < 1.0:
-        # the kept lists of the sampled heads are the oracle's top-k of its
-        # float64 pooled scores (near ties excepted), and the scores agree
-        agree = np.ones(idx_h.shape[:3], dtype=bool)
-        for hh in heads:
-            _, _, s_ref = ref.pooled_scores(as_f64(q[:, hh:hh + 1]), as_f64(k[:, hh:hh + 1]),
-                                            (w.F, w.H, w.W), perms[hh:hh + 1], w.block)
-            got_s = pipe.scores[:, hh:hh + 1].cpu().double().numpy()
-            assert np.abs(got_s - s_ref).max() < 1e-4 * max(1.0, np.abs(s_ref).max())
-            idx_ref[:, hh:hh + 1] = ref.select_topk(s_ref, ref.k_for_density(w.NB, density))
-            agree[:, hh:hh + 1] = selection_agreement(idx_h[:, hh:hh + 1], idx_ref[:, hh:hh + 1],
-                                                      s_ref)
+        idx_ref, agree = oracle_lists(w, q, k, perms, idx_h, density)
         tok_ok = token_mask(agree, (w.F, w.H, w.W), perms, w.block)
         rows = [r for r in rows if tok_ok[r]]
-        assert len(rows) >= 150
+        assert len(rows) >= min_rows
     else:
-        idx_ref[:] = np.arange(w.NB, dtype=np.int32)
+        idx_ref = np.broadcast_to(np.arange(w.NB, dtype=np.int32), idx_h.shape).copy()
         assert (idx_h == idx_ref).all()
     want = ref.attention_rows(as_f64(q), as_f64(k), as_f64(v), (w.F, w.H, w.W), perms, w.block,
                               idx_ref, rows)
     got = out[0].float().cpu().numpy()
     got = np.stack([got[h, n] for (_, h, n) in rows]).astype(np.float64)
     err = np.abs(got - want)
-    assert np.isfinite(got).all()
     assert err.max() <= BF16_MAX_ABS and err.mean() <= BF16_MEAN_ABS, (err.max(), err.mean())
-    # every output row was written (the buffer came from torch.empty)
-    assert torch.isfinite(out).all()
+    return err
+
+
+@pytest.mark.parametrize("density", [0.15, 1.0])
+def test_720p_full_size_sampled(c720, density):
+    """The bench's launch sequence (Pipeline) on the full 720p-shaped layer
+    (21x45x80 tokens, 40 heads): 5 seeded rows of every head (1 at density
+    1.0) plus every head's last token."""
+    w, q, k, v, perms = c720
+    full_size_sampled(w, q, k, v, perms, density, 5 if density < 1.0 else 1, 11, 200)
+
+
+def test_longclip_bf16_full_size_sampled():
+    """The long-clip shape (33x45x80 tokens, 24 heads, density 0.20) in bf16
+    through the Pipeline: 8 seeded rows of every head plus every head's last
+    token."""
+    w = WORKLOADS["longclip_33x45x80_int8"]
+    q, k, v, perms = inputs(w)
+    full_size_sampled(w, q, k, v, perms, w.density, 8, 13, 180)

@@ -1,6 +1,13 @@
 """GPU parity of the INT8 block-sparse attention (tcgen05 kind::i8) against
-the oracle's INT8 semantics (per-block symmetric Q/K/V codes, P quantised to
-round_half_even(127 P~) per tile, online running max), through the C ABI.
+the oracle's INT8 semantics, through the C ABI.
+
+Primary comparison, at 6e-2 max-abs / 6e-3 mean-abs: the oracle's default
+reading of the pages (per-block symmetric Q/K/V codes; the exactly
+normalised post-softmax P quantised per (query block, key block) tile with
+the tile's own absmax / 127).  The kernel computes P in one pass (the
+un-normalised tile numerator rounded with the fixed scale 1/127 under a
+running row max); the oracle's "online" replay of that order is checked as
+well, at the tighter bf16 tolerance.
 
 The codes and scales the kernel reads come from pa_quantize_int8 and are
 first checked bit-exact against the oracle's quantisation; the kept lists
@@ -17,8 +24,9 @@ from block_sparse_attention_34_b200.pipeline import Pipeline
 from block_sparse_attention_34_b200.synth import as_f64
 from oracle import paro_ref as ref
 
-from helpers import (INT8_MAX_ABS, INT8_MEAN_ABS, compare, compare_rows, custom, inputs,
-                     oracle_topk, selection_agreement, to_dev, token_mask, token_rows)
+from helpers import (BF16_MAX_ABS, BF16_MEAN_ABS, INT8_MAX_ABS, INT8_MEAN_ABS, compare,
+                     compare_rows, custom, inputs, oracle_topk, selection_agreement, to_dev,
+                     token_mask, token_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -51,7 +59,7 @@ def quantized(w, pr, perms, *xs, bits=(8, 8, 8)):
     return dev, host
 
 
-def oracle_int8(w, perms, host, idx, counts=None, p_levels=127):
+def oracle_int8(w, perms, host, idx, counts=None, p_levels=127, mode="tile"):
     """Oracle INT8 attention of every head, mapped to natural order."""
     (q8, sq), (k8, sk), (v8, sv) = host
     B, nh = q8.shape[:2]
@@ -61,7 +69,7 @@ def oracle_int8(w, perms, host, idx, counts=None, p_levels=127):
             outp[b, h] = ref.attention_int8(q8[b, h], k8[b, h], v8[b, h], sq[b, h], sk[b, h],
                                             sv[b, h], w.N, w.block, idx[b, h],
                                             None if counts is None else counts[b, h],
-                                            p_levels=p_levels)
+                                            p_levels=p_levels, mode=mode)
     return ref.inverse_reorder(outp, (w.F, w.H, w.W), perms)
 
 
@@ -84,6 +92,9 @@ def test_i8_topk_small(w):
     out, st = run_i8(pr, dev, idx_ref)
     assert st == 0 and out.dtype == torch.bfloat16
     compare(out, oracle_int8(w, perms, host, idx_ref), INT8_MAX_ABS, INT8_MEAN_ABS)
+    # the kernel's own one-pass order, tighter
+    compare(out, oracle_int8(w, perms, host, idx_ref, mode="online"), BF16_MAX_ABS,
+            BF16_MEAN_ABS)
 
 
 def test_i8_variable_counts_and_edge_rows():
@@ -112,6 +123,8 @@ def test_i8_variable_counts_and_edge_rows():
     assert st == 0
     want = oracle_int8(w, perms, host, idx, counts)
     compare(out, want, INT8_MAX_ABS, INT8_MEAN_ABS)
+    compare(out, oracle_int8(w, perms, host, idx, counts, mode="online"), BF16_MAX_ABS,
+            BF16_MEAN_ABS)
     tok = token_rows((w.F, w.H, w.W), perms[1], w.block)[2 * w.block:3 * w.block]
     assert (out[0, 1, torch.from_numpy(tok).cuda()] == 0).all()
 
@@ -163,21 +176,30 @@ def test_i8_whole_path_small():
 
 def test_i8_longclip_full_size_sampled():
     """The bench's INT8 launch sequence (Pipeline) on the full long-clip
-    layer (33x45x80 tokens, 24 heads), checked on sampled rows of a few
-    heads: quantised codes, kept lists and outputs against the oracle."""
+    layer (33x45x80 tokens, 24 heads), checked on sampled rows of six heads:
+    quantised codes, kept lists and outputs against the oracle's INT8
+    reading (6e-2 / 6e-3; the kernel's one-pass order tighter), and the
+    INT8 output's distance from the float64 attention of the unquantised
+    inputs reported beside the bf16 kernel's on the same rows."""
     w = WORKLOADS["longclip_33x45x80_int8"]
     q, k, v, perms = inputs(w)
-    pipe = Pipeline(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, perms, w.density, int8=True)
-    out = pipe.run(*to_dev(q, k, v))
+    grid = (w.F, w.H, w.W)
+    qd, kd, vd = to_dev(q, k, v)
+    pipe = Pipeline(w.B, w.heads, grid, w.d, w.block, perms, w.density, int8=True)
+    pipe.out.fill_(float("nan"))  # every row must be written
+    out = pipe.run(qd, kd, vd)
     torch.cuda.synchronize()
     assert pipe.status.item() == 0
     assert torch.isfinite(out).all()
     assert pipe.k == ref.k_for_density(w.NB, w.density)
+    pipe16 = Pipeline(w.B, w.heads, grid, w.d, w.block, perms, w.density)
+    out16 = pipe16.run(qd, kd, vd)
+    torch.cuda.synchronize()
+    assert pipe16.status.item() == 0
     idx_h = pipe.idx.cpu().numpy()
-    grid = (w.F, w.H, w.W)
     rng = np.random.default_rng(21)
-    errs = []
-    for hh in (0, 9, w.heads - 1):
+    errs, errs_online, err_f64, err16_f64 = [], [], [], []
+    for hh in (0, 5, 9, 14, 19, w.heads - 1):
         sl = slice(hh, hh + 1)
         ph = perms[sl]
         xp = [ref.reorder(x[:, sl].float().numpy(), grid, ph, w.block) for x in (q, k, v)]
@@ -189,18 +211,35 @@ def test_i8_longclip_full_size_sampled():
         idx_ref = ref.select_topk(s_ref, ref.k_for_density(w.NB, w.density))
         agree = selection_agreement(idx_h[:, sl], idx_ref, s_ref)[0, 0]
         # sampled permuted positions whose query block agrees, plus the tail
-        pos = [int(p) for p in rng.integers(0, w.N, 64) if agree[int(p) // w.block]]
+        pos = [int(p) for p in rng.integers(0, w.N, 24) if agree[int(p) // w.block]]
         if agree[(w.N - 1) // w.block]:
             pos.append(w.N - 1)
-        assert len(pos) >= 48
+        assert len(pos) >= 16
         (q8, sq), (k8, sk), (v8, sv) = host
-        want = ref.attention_int8_rows(q8[0, 0], k8[0, 0], v8[0, 0], sq[0, 0], sk[0, 0],
-                                       sv[0, 0], w.N, w.block, idx_ref[0, 0], pos)
+        args = (q8[0, 0], k8[0, 0], v8[0, 0], sq[0, 0], sk[0, 0], sv[0, 0], w.N, w.block,
+                idx_ref[0, 0], pos)
+        want = ref.attention_int8_rows(*args)
+        want_online = ref.attention_int8_rows(*args, mode="online")
         tok = token_rows(grid, perms[hh], w.block)[pos]
-        got = out[0, hh, torch.from_numpy(tok).cuda()].float().cpu().double().numpy()
+        tok_d = torch.from_numpy(tok).cuda()
+        got = out[0, hh, tok_d].float().cpu().double().numpy()
         errs.append(np.abs(got - want))
+        errs_online.append(np.abs(got - want_online))
+        f64 = ref.attention_rows(as_f64(q[:, sl]), as_f64(k[:, sl]), as_f64(v[:, sl]), grid, ph,
+                                 w.block, idx_ref, [(0, 0, int(n)) for n in tok])
+        err_f64.append(np.abs(got - f64))
+        err16_f64.append(np.abs(out16[0, hh, tok_d].float().cpu().double().numpy() - f64))
     err = np.concatenate(errs)
     assert err.max() <= INT8_MAX_ABS and err.mean() <= INT8_MEAN_ABS, (err.max(), err.mean())
+    err_o = np.concatenate(errs_online)
+    assert err_o.max() <= BF16_MAX_ABS and err_o.mean() <= BF16_MEAN_ABS, (err_o.max(),
+                                                                           err_o.mean())
+    e8, e16 = np.concatenate(err_f64), np.concatenate(err16_f64)
+    print(f"long clip, sampled rows: INT8 vs float64 attention of the unquantised inputs "
+          f"max {e8.max():.3e} mean {e8.mean():.3e}; bf16 kernel max {e16.max():.3e} "
+          f"mean {e16.mean():.3e}")
+    # the INT8 path stays within its own tolerance of unquantised attention
+    assert e8.max() <= INT8_MAX_ABS and e8.mean() <= INT8_MEAN_ABS
 
 
 @pytest.mark.parametrize("w", CASES[:3], ids=lambda w: w.name)
@@ -215,7 +254,8 @@ def test_int4_pv_small(w):
     idx_ref, _, _ = oracle_topk(q, k, w, perms)
     out, st = run_i8(pr, dev, idx_ref, p4=True)
     assert st == 0
-    compare(out, oracle_int8(w, perms, host, idx_ref, p_levels=7), INT8_MAX_ABS, INT8_MEAN_ABS)
+    compare(out, oracle_int8(w, perms, host, idx_ref, p_levels=7, mode="online"), INT8_MAX_ABS,
+            INT8_MEAN_ABS)
 
 
 def test_int4_pv_whole_path():
@@ -231,6 +271,6 @@ def test_int4_pv_whole_path():
     idx_ref, s_ref, _ = oracle_topk(q, k, w, perms)
     agree = selection_agreement(idx.cpu().numpy(), idx_ref, s_ref)
     _, host = quantized(w, pr, perms, q, k, v, bits=(8, 8, 4))
-    want = oracle_int8(w, perms, host, idx_ref, p_levels=7)
+    want = oracle_int8(w, perms, host, idx_ref, p_levels=7, mode="online")
     compare_rows(out, want, token_mask(agree, (w.F, w.H, w.W), perms, w.block), INT8_MAX_ABS,
                  INT8_MEAN_ABS)
