@@ -18,6 +18,13 @@ cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, pa_dt
 bool attn_sm100_supports(pa_dtype dt, const Grid& g);
 }  // namespace paro
 
+namespace paro {
+namespace {
+StallTest g_stall{-1, -1, -1, 0, 1000000000ull};
+}  // namespace
+StallTest stall_test() { return g_stall; }
+}  // namespace paro
+
 namespace {
 
 thread_local std::string g_error;
@@ -119,6 +126,19 @@ pa_status pa_clear_status(int32_t* dev_status, void* stream) {
 }
 
 const char* pa_last_error(void) { return g_error.c_str(); }
+
+pa_status pa_test_inject_v_stall(int32_t query_block, int32_t batch_head, int32_t tile,
+                                 uint64_t wait_limit_ns) {
+  if (tile < 0) {
+    paro::g_stall = paro::StallTest{-1, -1, -1, 0, 1000000000ull};
+    return ok();
+  }
+  PA_REQUIRE(query_block >= 0 && batch_head >= 0, "query_block and batch_head must be >= 0");
+  PA_REQUIRE(wait_limit_ns >= 1000 && wait_limit_ns <= 1000000000ull,
+             "wait_limit_ns=%llu must be in [1 us, 1 s]", (unsigned long long)wait_limit_ns);
+  paro::g_stall = paro::StallTest{query_block, batch_head, tile, 0, wait_limit_ns};
+  return ok();
+}
 
 int32_t pa_num_blocks(pa_shape s) {
   if (s.F < 1 || s.H < 1 || s.W < 1 || s.block < 1) return -1;

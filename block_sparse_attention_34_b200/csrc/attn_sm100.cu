@@ -11,19 +11,23 @@
 // tokens.
 //
 // One CTA per (query block, head); 12 warps with fixed roles:
-//   warps 0-7  softmax, two warpgroups splitting every tile by columns: warp
-//              w owns rows 32*(w%4) .. +31 (its TMEM lane quarter; a warp
-//              may only touch its own quarter) and key columns
-//              64*(w/4) .. +63 of every tile.  Each column half is an exact
-//              split of the row's keys and keeps its own running max, row
-//              sum and O accumulator, so no cross-warp exchange happens per
-//              tile; the halves are merged once at the end:
+//   warps 0-3  softmax group 0: the even-numbered kept tiles (0, 2, 4, ...);
+//   warps 4-7  softmax group 1: the odd-numbered kept tiles.
+//              Warp w of a group owns rows 32*(w%4) .. +31 (its tensor
+//              memory lane quarter), one row per thread, all 128 keys of
+//              the tile.  Each group keeps its own running max, row sum and
+//              O accumulator: the even and the odd tiles are an exact split
+//              of the row's keys, merged once at the end,
 //              O = (O_0 2^(m_0-m) + O_1 2^(m_1-m)) / (l_0 2^(m_0-m) +
-//              l_1 2^(m_1-m)).  A thread reads its 64 scores from TMEM,
-//              writes its 64 probabilities (bf16 pairs) into its half of the
-//              tile's P region of tensor memory (the P V MMA's A operand),
-//              and when its max grows by more than 2^8 rescales its O;
-//   warp 8     allocates TMEM; one lane issues every tcgen05.mma and commit;
+//              l_1 2^(m_1-m)).  The two groups work on consecutive tiles at
+//              the same time, so one group's exponentials overlap the other
+//              group's S read and the tensor cores' QK^T and P V of both.
+//              A thread reads its row of S (128 fp32) from tensor memory,
+//              writes its 128 probabilities as bf16 pairs over the first 64
+//              columns of the same S buffer (the P V MMA's A operand), and
+//              when its max grows by more than 2^8 rescales its O row;
+//   warp 8     allocates tensor memory; one lane issues every tcgen05.mma
+//              and commit;
 //   warp 9     loads Q, then K tiles; warp 10 loads V tiles.  With inputs in
 //              the permuted order (pa_reorder) every tile is 128 contiguous
 //              rows: one lane issues two TMA tiled boxes (one per 64-column
@@ -33,41 +37,23 @@
 //              positions from the head's axis order) and each lane's arrival
 //              on the stage's mbarrier fires when its copies land;
 //   warp 11    validates the kept list, then idles.
-// Tensor memory (512 columns): S at 0, P double buffer (64 columns each)
-// at 128 and 192, O_0 and O_1 at 256 and 384.  Shared memory: Q
-// (32 KB) and three-stage K and V rings (6 x 32 KB) in the canonical
-// K-major / MN-major SWIZZLE_128B layouts the MMA descriptors name.
+// Tensor memory (512 columns): S/P of the even tiles at 0, of the odd tiles
+// at 128; O_0 at 256, O_1 at 384.  Shared memory: Q (32 KB) and three-stage
+// K and V rings (6 x 32 KB) in the canonical K-major / MN-major
+// SWIZZLE_128B layouts the MMA descriptors name.
 //
-// MMA issue order QK(0), QK(1), PV(0), QK(2), PV(1), ...: QK^T of tile j+1
-// is issued as soon as both halves have read S(j) out of tensor memory, so
-// it runs while the softmax warps turn S(j) into P(j).  tcgen05 operations
-// of one thread complete in order, so S(j) being ready implies P V(j-2),
-// the previous reader of P(j)'s buffer, has completed.  A
-// K stage is refilled once its QK^T completes, a V stage once its P V
-// completes.  Every mbarrier wait is bounded (about one second of
-// %globaltimer); on expiry the kernel records PA_ERR_TIMEOUT in the device
-// status word, each role leaves its loop, in-flight copies and MMAs are
-// drained and TMEM is released before the CTA exits.
+// MMA issue order QK(0), QK(1), PV(0), QK(2), PV(1), QK(3), ...: QK^T of
+// tile j+2 reuses the S buffer whose P(j) the P V(j) just issued reads; the
+// tcgen05.mma operations of one thread execute in issue order, so the
+// overwrite follows the read.  A K stage is refilled once its QK^T
+// completes, a V stage once its P V completes.  Every mbarrier wait is
+// bounded (about one second of %globaltimer); on expiry the kernel records
+// PA_ERR_TIMEOUT in the device status word, each role leaves its loop,
+// in-flight copies and MMAs are drained and tensor memory is released
+// before the CTA exits.
 #include "sm100.cuh"
 
 namespace paro {
-
-#ifdef PARO_TRACE
-// Phase trace (debug builds only): clock64() of each role's key events for
-// one CTA, event e of tile j at g_paro_trace[e * 128 + j].
-__device__ long long* g_paro_trace = nullptr;
-__device__ int g_paro_trace_cta = 7;
-#define PARO_T(ev, j)                                                                    \
-  do {                                                                                   \
-    if (g_paro_trace != nullptr && blockIdx.x == g_paro_trace_cta && blockIdx.y == 0 &&  \
-        (j) < 128)                                                                       \
-      g_paro_trace[(ev) * 128 + (j)] = clock64();                                        \
-  } while (0)
-#else
-#define PARO_T(ev, j) \
-  do {                \
-  } while (0)
-#endif
 
 namespace {
 
@@ -81,11 +67,11 @@ constexpr int kKWarp = 9;
 constexpr int kVWarp = 10;
 constexpr int kCheckWarp = 11;
 constexpr int kThreads = 12 * 32;  // 384
-constexpr int kSoftThreads = 256;
+constexpr int kGroupThreads = 128;  // one softmax group
 constexpr uint32_t kTile = kBlock * kD * 2;  // 32 KB
 constexpr uint32_t kHalf = kBlock * 128;     // 16 KB: 64 columns
 // small region first: mbarriers, TMEM slot and flags, the final merge
-// buffer [m, l][2 halves][128 rows] float; the operand tiles start
+// buffer [m, l][2 groups][128 rows] float; the operand tiles start
 // 1024-aligned
 constexpr uint32_t kOffBar = 0;
 constexpr uint32_t kOffSlot = 256;
@@ -97,7 +83,7 @@ constexpr uint32_t kOffV = kOffK + kStages * kTile;  // kStages stages
 constexpr uint32_t kSmemBytes = kOffV + kStages * kTile;  // 232,448 B = 227 KB
 constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold (factor 256)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColP = 128, kColO = 256;
+constexpr uint32_t kColS = 0, kColO = 256;  // + 128 * group
 
 enum : uint32_t {
   BQ = 0,
@@ -105,10 +91,9 @@ enum : uint32_t {
   BV0 = 4,    // V stage full (3)
   BKF0 = 7,   // K stage free (3)
   BVF0 = 10,  // V stage free (3)
-  BS = 13,    // S(j) ready
-  BSF = 14,   // S(j) read by every softmax thread
-  BP0 = 15,   // P(j) written by every softmax thread (2, by j & 1)
-  BPV0 = 17,  // P V(j) complete (2)
+  BS0 = 13,   // S of the group's next tile ready (2, by group)
+  BP0 = 15,   // P written by every thread of the group (2)
+  BPV0 = 17,  // P V of the group's tile complete (2)
   BDRAIN = 19,
   BM = 20,    // final merge exchange
   NBAR = 21
@@ -156,7 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __nv_bfloat16* __restrict__ v, const __grid_constant__ Grid g,
                       const int32_t* __restrict__ idx, const int32_t* __restrict__ counts,
                       int k_max, float scale_log2, __nv_bfloat16* __restrict__ out,
-                      int32_t* __restrict__ status) {
+                      int32_t* __restrict__ status, const StallTest st) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // the operand tiles need 1024-byte alignment (the swizzle pattern repeats
   // every 8 rows of 128 bytes); dynamic shared memory starts at the window
@@ -170,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOffSlot);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile uint32_t* bad_flag = tmem_slot + 2;
-  float* merge = reinterpret_cast<float*>(gbase + kOffMerge);  // [m|l][half][row]
+  float* merge = reinterpret_cast<float*>(gbase + kOffMerge);  // [m|l][group][row]
   auto bar = [&](uint32_t slot) { return base + kOffBar + slot * 8u; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -181,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t row = bh * g.NB + i;
   const int32_t* ids = idx + row * k_max;
   const int cnt = counts != nullptr ? __ldg(counts + row) : k_max;
-  Ctl ctl{abort_flag, status};
+  const Ctl ctl{abort_flag, status, st.limit_ns};
   // a wait of an earlier CTA of this launch already expired: end quickly
   const bool expired =
       status != nullptr && *reinterpret_cast<volatile int32_t*>(status) == PA_ERR_TIMEOUT;
@@ -195,14 +180,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(BKF0 + s), 1);
       mbar_init(bar(BVF0 + s), 1);
     }
-    mbar_init(bar(BS), 1);
-    mbar_init(bar(BSF), kSoftThreads);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(BP0 + b), kSoftThreads);
+      mbar_init(bar(BS0 + b), 1);
+      mbar_init(bar(BP0 + b), kGroupThreads);
       mbar_init(bar(BPV0 + b), 1);
     }
     mbar_init(bar(BDRAIN), 1);
-    mbar_init(bar(BM), kSoftThreads);
+    mbar_init(bar(BM), 2 * kGroupThreads);
     *abort_flag = 0;
     *bad_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -261,9 +245,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (j >= kStages &&
               !warp_wait(bar((is_k ? BKF0 : BVF0) + s), ((j / kStages) - 1) & 1, ctl))
             break;
-          PARO_T(is_k ? 0 : 2, j);
           const int kb = __ldg(ids + j);
           const uint32_t full = bar((is_k ? BK0 : BV0) + s);
+          if (!is_k && j == st.tile && i == st.cta_x && bh == st.cta_y) {
+            issued = j + 1;  // test hook: this tile never arrives
+            continue;
+          }
           if constexpr (kTma) {
             if (lane == 0) {
               mbar_arrive_tx(full, kTile);
@@ -279,9 +266,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // on every path this warp's copies have landed before it leaves
         if constexpr (kTma) {
           if (lane == 0) {
-            if (is_k) drain_phase(bar(BQ), 0);
+            if (is_k) drain_phase(bar(BQ), 0, ctl.limit_ns);
             for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
-              drain_phase(bar((is_k ? BK0 : BV0) + j % kStages), (j / kStages) & 1);
+              drain_phase(bar((is_k ? BK0 : BV0) + j % kStages), (j / kStages) & 1,
+                          ctl.limit_ns);
           }
         } else {
           cp_async_wait_all();
@@ -294,28 +282,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t id_pv = idesc_bf16(kBlock, kD, true);
         bool ok = wait_phase(bar(BQ), 0, ctl);
         fence_async_smem();  // cp.async (generic proxy) writes -> MMA operand reads
-        // QK^T of tile j into S: needs K(j) and, for j >= 1, every softmax
-        // thread to have read S(j-1)
+        // QK^T of tile j into S buffer j & 1: needs K(j); the buffer's
+        // previous contents, P(j-2), are read by P V(j-2), issued before
         auto issue_qk = [&](int j) -> bool {
-          const int s = j % kStages;
+          const int s = j % kStages, b = j & 1;
           if (!wait_phase(bar(BK0 + s), (j / kStages) & 1, ctl)) return false;
-          if (j >= 1 && !wait_phase(bar(BSF), (j - 1) & 1, ctl)) return false;
           fence_async_smem();
           tc_fence_after();
           const uint32_t ka = base + kOffK + s * kTile;
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk) {
             const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-            mma_f16_ss(tmem + kColS, sw128_desc(base + kOffQ + off, 16, 1024),
+            mma_f16_ss(tmem + kColS + b * 128, sw128_desc(base + kOffQ + off, 16, 1024),
                        sw128_desc(ka + off, 16, 1024), id_qk, kk > 0 ? 1u : 0u);
           }
-          mma_commit(bar(BS));
+          mma_commit(bar(BS0 + b));
           mma_commit(bar(BKF0 + s));
-          PARO_T(4, j);
           return true;
         };
-        // O_h += P(j)[:, keys of half h] V(j)[rows of half h], h = 0, 1:
-        // P from tensor memory (bf16 pairs), V from the ring
+        // O_b += P(j) V(j), b = j & 1: P (bf16 pairs) from the first 64
+        // columns of S buffer b, V from the ring
         auto issue_pv = [&](int j) -> bool {
           const int b = j & 1, s = j % kStages;
           if (!wait_phase(bar(BP0 + b), (j >> 1) & 1, ctl)) return false;
@@ -325,70 +311,98 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t va = base + kOffV + s * kTile;
 #pragma unroll
           for (int kk = 0; kk < kBlock / 16; ++kk)
-            mma_f16_ts(tmem + kColO + (kk >> 2) * 128, tmem + kColP + b * 64 + kk * 8,
+            mma_f16_ts(tmem + kColO + b * 128, tmem + kColS + b * 128 + kk * 8,
                        sw128_desc(va + kk * 16 * 128, kHalf, 1024), id_pv,
-                       (j > 0 || (kk & 3) > 0) ? 1u : 0u);
+                       (j >= 2 || kk > 0) ? 1u : 0u);
           mma_commit(bar(BPV0 + b));
           mma_commit(bar(BVF0 + s));
-          PARO_T(5, j);
           return true;
         };
         ok = ok && issue_qk(0);
+        if (ok && n_tiles > 1) ok = issue_qk(1);
         for (int j = 0; ok && j < n_tiles; ++j) {
-          if (j + 1 < n_tiles && !issue_qk(j + 1)) { ok = false; break; }
           if (!issue_pv(j)) { ok = false; break; }
+          if (j + 2 < n_tiles && !issue_qk(j + 2)) { ok = false; break; }
         }
         // drain: every MMA issued above has completed once this commit fires
         mma_commit(bar(BDRAIN));
-        drain_phase(bar(BDRAIN), 0);
+        drain_phase(bar(BDRAIN), 0, ctl.limit_ns);
       }
     }
     __syncwarp();  // reconverge after the lane-0 roles
   } else {
     // ------------------------------------------------------ softmax ----
-    const int hc = warp >> 2;     // column half: keys 64*hc .. 64*hc+63
+    const int grp = warp >> 2;  // 0: even tiles, 1: odd tiles
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // tile row == TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t o_col = kColO + hc * 128;
-    float m_used = -INFINITY, l = 0.f;  // this half's reference max and row sum
+    const uint32_t s_col = kColS + grp * 128;
+    const uint32_t o_col = kColO + grp * 128;
+    float m_used = -INFINITY, l = 0.f;  // this group's reference max and row sum
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      const int b = j & 1;
-      if (!warp_wait(bar(BS), j & 1, ctl)) { ok = false; break; }
-      if (lane == 0 && quarter == 0) PARO_T(6 + 4 * hc, j);
+    for (int t = 0;; ++t) {
+      const int j = 2 * t + grp;
+      if (j >= n_tiles) break;
+      if (!warp_wait(bar(BS0 + grp), t & 1, ctl)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld64(lane_addr + kColS + hc * 64, sr);
-      tc_fence_before();
-      mbar_arrive(bar(BSF));  // S may take QK^T(j+1)
-      if (lane == 0 && quarter == 0) PARO_T(7 + 4 * hc, j);
-      const int valid = g.N - __ldg(ids + j) * kBlock - hc * 64;  // existing keys of my half
-      if (valid < 64) {  // only the ragged last block (warp-uniform)
+      uint32_t sr[128];
+      tmem_ld128(lane_addr + s_col, sr);
+      const int valid = g.N - __ldg(ids + j) * kBlock;  // existing keys of the tile
+      if (valid < kBlock) {  // only the ragged last block (warp-uniform)
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
+        for (int c = 0; c < kBlock; ++c)
           if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
       }
       float mp[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) mp[u] = __uint_as_float(sr[u]);
+      for (int u = 0; u < 8; ++u)
+        mp[u] = fmax3(__uint_as_float(sr[u]), __uint_as_float(sr[u + 8]),
+                      __uint_as_float(sr[u + 16]));
+      // columns 24..127 in steps of 16 (the last step takes 120..127 alone)
 #pragma unroll
-      for (int c = 8; c < 64; ++c) mp[c & 7] = fmaxf(mp[c & 7], __uint_as_float(sr[c]));
-      const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) *
+      for (int c = 24; c < kBlock; c += 16)
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (c + u + 8 < kBlock)
+            mp[u] = fmax3(mp[u], __uint_as_float(sr[c + u]), __uint_as_float(sr[c + u + 8]));
+          else if (c + u < kBlock)
+            mp[u] = fmaxf(mp[u], __uint_as_float(sr[c + u]));
+      const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]),
+                             fmaxf(mp[6], mp[7])) *
                        scale_log2;
-      if (lane == 0 && quarter == 0) PARO_T(8 + 4 * hc, j);
-      // lazy rescale: keep the reference max unless this half's max grew
-      // by more than 2^8 (exact either way: O_h and l share the reference).
-      // A half whose keys are all padding (mx = -inf) keeps its reference.
+      // lazy rescale: keep the reference max unless this row's max grew by
+      // more than 2^8 (exact either way: O and l share the reference)
       const bool first = m_used == -INFINITY;
       const bool need = !first && mx > m_used + kRescaleLog2;
-      if (first && mx != -INFINITY) m_used = mx;
+      const float alpha = need ? ex2(m_used - mx) : 1.f;
+      if (first || need) m_used = mx;  // a tile has at least one existing key
+      // P = 2^(s*scale - m) as bf16 pairs over the first 64 columns of the S
+      // buffer (its fp32 values are all in registers); row sum in 8 chains
+      const float neg_m = -m_used;
+      float rs[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) rs[u] = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int e = 32 * cc + 2 * c;
+          const float e0 = ex2(fmaf(__uint_as_float(sr[e]), scale_log2, neg_m));
+          const float e1 = ex2(fmaf(__uint_as_float(sr[e + 1]), scale_log2, neg_m));
+          rs[e & 7] += e0;
+          rs[(e + 1) & 7] += e1;
+          pk[c] = pack_bf16(e0, e1);
+        }
+        tmem_st16_async(lane_addr + s_col + 16 * cc, pk);
+      }
+      tmem_wait_st();
+      l = l * alpha + (((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7])));
       if (__any_sync(0xffffffffu, need)) {
-        // O_h holds P V up to tile j-1 once that MMA completed
-        if (!warp_wait(bar(BPV0 + ((j - 1) & 1)), ((j - 1) >> 1) & 1, ctl)) { ok = false; break; }
+        // O holds P V up to this group's previous tile once that MMA
+        // completed; P V of this tile is issued after the arrival below
+        if (!warp_wait(bar(BPV0 + grp), (t - 1) & 1, ctl)) { ok = false; break; }
         tc_fence_after();
-        const float alpha = need ? ex2(m_used - mx) : 1.f;
 #pragma unroll 1
         for (int c0 = 0; c0 < 128; c0 += 32) {
           uint32_t orr[32];
@@ -397,49 +411,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
           tmem_st32(lane_addr + o_col + c0, orr);
         }
-        l *= alpha;
-        if (need) m_used = mx;
       }
-      // P = 2^(s*scale - m) as bf16 pairs into my half of P buffer b (free:
-      // S(j) ready means P V(j-2) completed); row sum in 8 chains
-      const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
-      float rs[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) rs[u] = 0.f;
-      uint32_t pk[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float e0 = ex2(fmaf(__uint_as_float(sr[2 * c]), scale_log2, neg_m));
-        const float e1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), scale_log2, neg_m));
-        rs[(2 * c) & 7] += e0;
-        rs[(2 * c + 1) & 7] += e1;
-        pk[c] = pack_bf16(e0, e1);
-      }
-      tmem_st32(lane_addr + kColP + b * 64 + hc * 32, pk);
-      l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
-      if (lane == 0 && quarter == 0) PARO_T(9 + 4 * hc, j);
       tc_fence_before();
-      mbar_arrive(bar(BP0 + b));
+      mbar_arrive(bar(BP0 + grp));
     }
-    // ---- epilogue: merge the halves, then half h writes output columns
-    // 64h .. 64h+63 of the row at the natural position of its token
+    // ---- epilogue: merge the groups, then group g writes output columns
+    // 64g .. 64g+63 of the row at the natural position of its token
     const int p = i * kBlock + r;
     __nv_bfloat16* orow = p < g.N ? out + (bh * (int64_t)g.N + natural_index(g, order, p)) * kD
                                   : nullptr;
     if (run && cnt == 0) {
       if (orow != nullptr)
         for (int c = 0; c < 8; ++c)
-          reinterpret_cast<uint4*>(orow + hc * 64)[c] = make_uint4(0, 0, 0, 0);
+          reinterpret_cast<uint4*>(orow + grp * 64)[c] = make_uint4(0, 0, 0, 0);
     } else if (ok && n_tiles > 0) {
-      merge[(0 * 2 + hc) * 128 + r] = m_used;
-      merge[(1 * 2 + hc) * 128 + r] = l;
+      merge[(0 * 2 + grp) * 128 + r] = m_used;
+      merge[(1 * 2 + grp) * 128 + r] = l;
       mbar_arrive(bar(BM));
       bool okm = all_wait(bar(BM), 0, ctl);
       float f0 = 0.f, f1 = 0.f, lt = 0.f;
       if (okm) {
         const float m0 = merge[r], m1 = merge[128 + r];
         const float m = fmaxf(m0, m1);
-        // a half that saw only padding has l = 0 and an untouched O: weight 0
+        // a group that saw no tile (a one-tile list) has l = 0 and an
+        // unwritten O: weight 0
         f0 = m0 == -INFINITY ? 0.f : ex2(m0 - m);
         f1 = m1 == -INFINITY ? 0.f : ex2(m1 - m);
         lt = merge[256 + r] * f0 + merge[384 + r] * f1;
@@ -453,10 +448,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         f1 *= inv;
 #pragma unroll 1
         for (int c0 = 0; c0 < 64; c0 += 32) {
-          const int col = hc * 64 + c0;
+          const int col = grp * 64 + c0;
           uint32_t oa[32], ob[32];
-          tmem_ld32(lane_addr + kColO + col, oa);
-          tmem_ld32(lane_addr + kColO + 128 + col, ob);
+          tmem_ld32x2(lane_addr + kColO + col, oa, lane_addr + kColO + 128 + col, ob);
           if (orow != nullptr) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -503,7 +497,7 @@ cudaError_t launch_typed(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
   attn_sm100_kernel<kTma><<<grid, kThreads, kSmemBytes, s>>>(
       mq, mk, mv, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
       static_cast<const __nv_bfloat16*>(v), g, idx, counts, k_max, scale_log2,
-      static_cast<__nv_bfloat16*>(out), status);
+      static_cast<__nv_bfloat16*>(out), status, stall_test());
   return cudaGetLastError();
 }
 

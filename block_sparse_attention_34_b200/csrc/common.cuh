@@ -31,6 +31,16 @@ struct Grid {
   int8_t perm[kMaxHeads];
 };
 
+// Test hook of the bounded waits (pa_test_inject_v_stall): the V-tile
+// loader of CTA (cta_x, cta_y) of the tcgen05 bf16 attention kernel skips
+// kept tile `tile` (no copy, no arrival), and every bounded wait of that
+// kernel gives up after limit_ns.  tile < 0: off (limit 1 s).
+struct StallTest {
+  int32_t cta_x, cta_y, tile, pad;
+  uint64_t limit_ns;
+};
+StallTest stall_test();  // host: the current setting
+
 __device__ __forceinline__ int natural_index(const Grid& g, int order, int p) {
   const int inn = g.inn[order], mid = g.mid[order];
   const int ci = p % inn;

@@ -54,14 +54,16 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
-// Abort flag shared by the CTA's roles plus the device status word.
+// Abort flag shared by the CTA's roles, the device status word, and how
+// long a wait may last before it gives up.
 struct Ctl {
   volatile uint32_t* abort;
   int32_t* status;
+  uint64_t limit_ns = kTimeoutNs;
 };
 
 // Bounded wait on one phase of an mbarrier (one thread).  Gives up when the
-// CTA's abort flag is raised, or after kTimeoutNs, raising it and recording
+// CTA's abort flag is raised, or after c.limit_ns, raising it and recording
 // PA_ERR_TIMEOUT.
 __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, Ctl c) {
   if (mbar_try(bar, parity)) return true;
@@ -70,7 +72,7 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, Ctl c)
     if (mbar_try(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*c.abort) return false;
-      if (global_ns() - t0 > kTimeoutNs) {
+      if (global_ns() - t0 > c.limit_ns) {
         *c.abort = 1;
         report(c.status, PA_ERR_TIMEOUT);
         return false;
@@ -81,10 +83,11 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, Ctl c)
 
 // Bounded wait that ignores the abort flag: used on the way out to let this
 // thread's own copies land before the CTA releases its shared memory.
-__device__ __forceinline__ bool drain_phase(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool drain_phase(uint32_t bar, uint32_t parity,
+                                            uint64_t limit_ns = kTimeoutNs) {
   const uint64_t t0 = global_ns();
   while (!mbar_try(bar, parity))
-    if (global_ns() - t0 > kTimeoutNs) return false;
+    if (global_ns() - t0 > limit_ns) return false;
   return true;
 }
 
@@ -236,6 +239,13 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// max of three floats in one instruction (sm_100 three-input max.f32).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 // Paired fp32 arithmetic (sm_100 f32x2 forms): two IEEE round-to-nearest

@@ -55,6 +55,7 @@ def load():
         "pa_abi_version": ([], _I),
         "pa_last_error": ([], ctypes.c_char_p),
         "pa_clear_status": ([_P, _P], _I),
+        "pa_test_inject_v_stall": ([_I, _I, _I, ctypes.c_uint64], _I),
         "pa_num_blocks": ([PaShape], _I),
         "pa_k_for_density": ([_I, ctypes.c_double], _I),
         "pa_reorder": ([_P, _P, _I, PaShape, _P, _P, _P], _I),
@@ -203,6 +204,14 @@ def clear_status(status):
     _need_cuda(status)
     _expect_status(status)
     _check(load().pa_clear_status(_ptr(status), _stream()))
+
+
+def test_inject_v_stall(query_block: int, batch_head: int, tile: int, wait_limit_ns: int):
+    """Failure-path test hook (pa_test_inject_v_stall): the V loader of one
+    CTA of the tcgen05 bf16 kernel skips one kept tile, so a bounded wait
+    runs out after ``wait_limit_ns``; ``tile < 0`` switches it off."""
+    _check(load().pa_test_inject_v_stall(int(query_block), int(batch_head), int(tile),
+                                         int(wait_limit_ns)))
 
 
 def k_for_density(nb: int, density: float) -> int:

@@ -99,6 +99,22 @@ PA_API const char* pa_last_error(void);
  * pages' method: bookkeeping of this library's error reporting. */
 PA_API pa_status pa_clear_status(int32_t* dev_status, void* stream);
 
+/* Test hook of the failure path (not part of the pages' method).  For the
+ * pa_block_sparse_attn launches on the tcgen05 bf16 kernel that follow
+ * (d = 128, block = 128, PA_BF16), the V-tile loader of the CTA of query
+ * block `query_block` and batch-head `batch_head` (b * heads + h) skips kept
+ * tile number `tile` of its list (issues no copy and no arrival), so the
+ * MMA issuer's bounded wait for that tile runs out; every bounded wait of
+ * the kernel then gives up after `wait_limit_ns` (1 us .. 1 s) instead of
+ * 1 s.  The CTA records PA_ERR_TIMEOUT on dev_status, every role leaves its
+ * loop, copies and MMAs in flight are drained and tensor memory is
+ * released; CTAs that start later find the status and skip their work.  No
+ * trap, no fault, nothing left waiting.  tile < 0 switches the hook off
+ * (the default).  Process-wide setting, read at launch; not for concurrent
+ * use. */
+PA_API pa_status pa_test_inject_v_stall(int32_t query_block, int32_t batch_head, int32_t tile,
+                                        uint64_t wait_limit_ns);
+
 /* NB = ceil(F*H*W / block), or -1 for a malformed shape. */
 PA_API int32_t pa_num_blocks(pa_shape shape);
 

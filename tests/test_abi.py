@@ -283,3 +283,11 @@ def test_binding_passes_good_shapes_to_the_library(host_binding):
     for call in good:
         with pytest.raises(AssertionError, match="library call"):
             call()
+
+
+def test_stall_hook_arguments_are_checked(lib):
+    """The failure-path test hook validates its arguments on the host."""
+    assert lib.pa_test_inject_v_stall(0, 0, 1, 10) == paro.PA_ERR_INVALID_ARG  # below 1 us
+    assert lib.pa_test_inject_v_stall(-1, 0, 1, 1_000_000) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_test_inject_v_stall(0, 0, 1, 2_000_000_000) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_test_inject_v_stall(-1, -1, -1, 0) == paro.PA_OK  # off
