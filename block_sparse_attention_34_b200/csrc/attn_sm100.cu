@@ -15,19 +15,21 @@
 //   warps 4-7  softmax group 1: the odd-numbered kept tiles.
 //              Warp w of a group owns rows 32*(w%4) .. +31 (its tensor
 //              memory lane quarter), one row per thread, all 128 keys of
-//              the tile.  Each group keeps its own running max, row sum and
-//              O accumulator: the even and the odd tiles are an exact split
-//              of the row's keys, merged once at the end,
-//              O = (O_0 2^(m_0-m) + O_1 2^(m_1-m)) / (l_0 2^(m_0-m) +
-//              l_1 2^(m_1-m)).  The two groups work on consecutive tiles at
-//              the same time, so one group's exponentials overlap the other
-//              group's S read and the tensor cores' QK^T and P V of both.
-//              A thread reads its row of S (128 fp32) from tensor memory,
-//              writes its 128 probabilities as bf16 pairs over the first 64
-//              columns of the same S buffer (the P V MMA's A operand), and
-//              when its max grows by more than 2^8 rescales its O row;
+//              the tile.  A thread copies its row of S (128 fp32) from the
+//              group's S buffer into registers and releases the buffer, so
+//              QK^T two tiles ahead can start at once; it then writes its
+//              128 probabilities as bf16 pairs into the group's P buffer
+//              (the P V MMA's A operand).  Both groups accumulate into one
+//              O, so every row has one reference max m_j, passed along the
+//              tile order through shared memory: m_j = m_{j-1} unless tile
+//              j's max exceeds it by more than 2^8 (then m_j is that max and
+//              the group rescales O after P V(j-1) and before P V(j): the
+//              rescale is lazy and exact).  Each group keeps its own row
+//              sum relative to the latest reference it used; the two are
+//              added at the end;
 //   warp 8     allocates tensor memory; one lane issues every tcgen05.mma
-//              and commit;
+//              and commit, in the order QK(0), QK(1), then QK(j+2), PV(j)
+//              for j = 0, 1, ...;
 //   warp 9     loads Q, then K tiles; warp 10 loads V tiles.  With inputs in
 //              the permuted order (pa_reorder) every tile is 128 contiguous
 //              rows: one lane issues two TMA tiled boxes (one per 64-column
@@ -35,19 +37,17 @@
 //              natural-order inputs the warp gathers the token rows itself
 //              (16-byte cp.async, 16 lanes per 256-byte row, natural
 //              positions from the head's axis order) and each lane's arrival
-//              on the stage's mbarrier fires when its copies land;
+//              on the stage's mbarrier fires when its copies land.  The kept
+//              block indices are read 32 at a time and passed by shuffle;
 //   warp 11    validates the kept list, then idles.
-// Tensor memory (512 columns): S/P of the even tiles at 0, of the odd tiles
-// at 128; O_0 at 256, O_1 at 384.  Shared memory: Q (32 KB) and three-stage
-// K and V rings (6 x 32 KB) in the canonical K-major / MN-major
-// SWIZZLE_128B layouts the MMA descriptors name.
+// Tensor memory (512 columns): S_0 at 0 and S_1 at 128 (128 columns each),
+// P_0 at 256 and P_1 at 320 (64 columns each), O at 384.  Shared memory: Q
+// (32 KB) and three-stage K and V rings (6 x 32 KB) in the canonical
+// K-major / MN-major SWIZZLE_128B layouts the MMA descriptors name.
 //
-// MMA issue order QK(0), QK(1), PV(0), QK(2), PV(1), QK(3), ...: QK^T of
-// tile j+2 reuses the S buffer whose P(j) the P V(j) just issued reads; the
-// tcgen05.mma operations of one thread execute in issue order, so the
-// overwrite follows the read.  A K stage is refilled once its QK^T
-// completes, a V stage once its P V completes.  Every mbarrier wait is
-// bounded (about one second of %globaltimer); on expiry the kernel records
+// A K stage is refilled once its QK^T completes, a V stage once its P V
+// completes; each MMA group signals its completion with one commit.  Every mbarrier wait is bounded (about one second of
+// %globaltimer, or the limit the launch sets); on expiry the kernel records
 // PA_ERR_TIMEOUT in the device status word, each role leaves its loop,
 // in-flight copies and MMAs are drained and tensor memory is released
 // before the CTA exits.
@@ -62,20 +62,22 @@ using namespace sm100;
 constexpr int kBlock = 128;
 constexpr int kD = 128;
 constexpr int kStages = 3;
-constexpr int kMmaWarp = 8;
+constexpr int kMmaWarp = 8;   // QK^T issuer, tensor memory owner
 constexpr int kKWarp = 9;
 constexpr int kVWarp = 10;
-constexpr int kCheckWarp = 11;
+constexpr int kPvWarp = 11;   // kept-list check
 constexpr int kThreads = 12 * 32;  // 384
 constexpr int kGroupThreads = 128;  // one softmax group
 constexpr uint32_t kTile = kBlock * kD * 2;  // 32 KB
 constexpr uint32_t kHalf = kBlock * 128;     // 16 KB: 64 columns
-// small region first: mbarriers, TMEM slot and flags, the final merge
-// buffer [m, l][2 groups][128 rows] float; the operand tiles start
-// 1024-aligned
+// small region first: mbarriers, TMEM slot and flags, the row sums of the
+// two groups [2][128] float for the final sum, and the reference max of
+// each row after each group's latest tile [2][128] float; the operand
+// tiles start 1024-aligned
 constexpr uint32_t kOffBar = 0;
 constexpr uint32_t kOffSlot = 256;
 constexpr uint32_t kOffMerge = 512;
+constexpr uint32_t kOffRef = kOffMerge + 2 * 128 * 4;
 constexpr uint32_t kSmall = 3072;
 constexpr uint32_t kOffQ = kSmall;
 constexpr uint32_t kOffK = kOffQ + kTile;            // kStages stages
@@ -83,23 +85,29 @@ constexpr uint32_t kOffV = kOffK + kStages * kTile;  // kStages stages
 constexpr uint32_t kSmemBytes = kOffV + kStages * kTile;  // 232,448 B = 227 KB
 constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold (factor 256)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColO = 256;  // + 128 * group
+constexpr uint32_t kColS = 0, kColP = 256, kColO = 384;  // S, P: + 128 / 64 * group
 
+// QK^T(j) and P V(j) each end with one commit, into a ring of 6 barriers
+// (slot j % 6, phase j / 6) that every consumer of that event waits on: the
+// tile's softmax group (S ready; its P buffer free), the loaders (K or V
+// stage free), the O rescale and the epilogue.  No waiter can fall 6 tiles
+// behind, so a slot's phases never alias.
+constexpr int kRing = 6;
 enum : uint32_t {
   BQ = 0,
   BK0 = 1,    // K stage full (3)
   BV0 = 4,    // V stage full (3)
-  BKF0 = 7,   // K stage free (3)
-  BVF0 = 10,  // V stage free (3)
-  BS0 = 13,   // S of the group's next tile ready (2, by group)
-  BP0 = 15,   // P written by every thread of the group (2)
-  BPV0 = 17,  // P V of the group's tile complete (2)
-  BDRAIN = 19,
-  BM = 20,    // final merge exchange
-  NBAR = 21
+  BQK0 = 7,   // QK^T(j) complete (6)
+  BPV0 = 13,  // P V(j) complete (6)
+  BSF0 = 19,  // S copied out by every thread of the group (2)
+  BP0 = 21,   // P written by every thread of the group (2)
+  BMX0 = 23,  // the group's reference max of its tile published (2)
+  BDRAIN = 25,
+  BM = 26,    // final sum exchange
+  NBAR = 27
 };
 static_assert(NBAR * 8 <= kOffSlot, "barrier region");
-static_assert(kOffMerge + 2 * 2 * 128 * 4 <= kSmall, "merge region");
+static_assert(kOffRef + 2 * 128 * 4 <= kSmall, "row sum and reference regions");
 
 // One warp copies a 128 x 128 bf16 tile whose row r is the token at
 // permuted position p0 + r of head `head` (rows past N zero-filled).  Lane l
@@ -155,8 +163,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOffSlot);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile uint32_t* bad_flag = tmem_slot + 2;
-  float* merge = reinterpret_cast<float*>(gbase + kOffMerge);  // [m|l][group][row]
+  float* lsum = reinterpret_cast<float*>(gbase + kOffMerge);  // [group][row]
+  float* mref = reinterpret_cast<float*>(gbase + kOffRef);    // [group][row]
   auto bar = [&](uint32_t slot) { return base + kOffBar + slot * 8u; };
+  auto qk_done = [&](int j) { return bar(BQK0 + j % kRing); };
+  auto pv_done = [&](int j) { return bar(BPV0 + j % kRing); };
+  auto ring_par = [](int j) { return (uint32_t)((j / kRing) & 1); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x;
@@ -177,13 +189,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar(BK0 + s), kLoadArrivals);
       mbar_init(bar(BV0 + s), kLoadArrivals);
-      mbar_init(bar(BKF0 + s), 1);
-      mbar_init(bar(BVF0 + s), 1);
+    }
+    for (int x = 0; x < kRing; ++x) {
+      mbar_init(bar(BQK0 + x), 1);
+      mbar_init(bar(BPV0 + x), 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(BS0 + b), 1);
+      mbar_init(bar(BSF0 + b), kGroupThreads);
       mbar_init(bar(BP0 + b), kGroupThreads);
-      mbar_init(bar(BPV0 + b), 1);
+      mbar_init(bar(BMX0 + b), kGroupThreads);
     }
     mbar_init(bar(BDRAIN), 1);
     mbar_init(bar(BM), 2 * kGroupThreads);
@@ -192,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   if (warp == kMmaWarp) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-  if (warp == kCheckWarp) {
+  if (warp == kPvWarp) {
     // the kept list: count in range, indices ascending in [0, NB)
     bool bad = cnt < 0 || cnt > k_max;
     if (!bad) {
@@ -239,13 +253,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             cp_async_arrive(bar(BQ));
           }
         }
+        int kb_lane = 0;  // kept index j0 + lane of the current chunk of 32
         for (int j = 0; j < n_tiles; ++j) {
           const int s = j % kStages;
+          if ((j & 31) == 0) kb_lane = j + lane < n_tiles ? __ldg(ids + j + lane) : 0;
+          const int kb = __shfl_sync(0xffffffffu, kb_lane, j & 31);
           // the stage is free once QK^T (K) or P V (V) of tile j-3 completed
-          if (j >= kStages &&
-              !warp_wait(bar((is_k ? BKF0 : BVF0) + s), ((j / kStages) - 1) & 1, ctl))
+          if (j >= kStages && !warp_wait(is_k ? qk_done(j - kStages) : pv_done(j - kStages),
+                                         ring_par(j - kStages), ctl))
             break;
-          const int kb = __ldg(ids + j);
           const uint32_t full = bar((is_k ? BK0 : BV0) + s);
           if (!is_k && j == st.tile && i == st.cta_x && bh == st.cta_y) {
             issued = j + 1;  // test hook: this tile never arrives
@@ -277,54 +293,84 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (warp == kMmaWarp) {
       // -------------------------------------------------------- MMA ----
+      // Issue order QK(0), QK(1), then QK(j+2), PV(j) for j = 0, 1, ...:
+      // QK^T(j+2) waits only for S(j) to be copied out (early in group
+      // j & 1's work), and P(j) has the time of QK^T(j+2) and PV(j-1).  The
+      // tensor pipe queues few MMAs, so time this thread spends away from
+      // issuing is lost: each MMA group ends with one commit, and the
+      // barriers of the next group are tested (without blocking) before the
+      // current group is issued, so that a blocking wait is left only when
+      // that test failed.
       if (lane == 0 && n_tiles > 0) {
         constexpr uint32_t id_qk = idesc_bf16(kBlock, kBlock, false);
         constexpr uint32_t id_pv = idesc_bf16(kBlock, kD, true);
-        bool ok = wait_phase(bar(BQ), 0, ctl);
-        fence_async_smem();  // cp.async (generic proxy) writes -> MMA operand reads
-        // QK^T of tile j into S buffer j & 1: needs K(j); the buffer's
-        // previous contents, P(j-2), are read by P V(j-2), issued before
-        auto issue_qk = [&](int j) -> bool {
-          const int s = j % kStages, b = j & 1;
-          if (!wait_phase(bar(BK0 + s), (j / kStages) & 1, ctl)) return false;
-          fence_async_smem();
-          tc_fence_after();
-          const uint32_t ka = base + kOffK + s * kTile;
+        // descriptors of stage 0 / of Q; other stages and k-steps add their
+        // byte offset / 16 to the start-address field (addresses < 256 KB,
+        // so the 14-bit field never carries)
+        const uint64_t dq = sw128_desc(base + kOffQ, 16, 1024);
+        const uint64_t dk0 = sw128_desc(base + kOffK, 16, 1024);
+        const uint64_t dv0 = sw128_desc(base + kOffV, kHalf, 1024);
+        auto issue_qk = [&](int j) {  // S_b = Q K(j)^T, b = j & 1
+          const uint64_t dk = dk0 + (uint64_t)((j % kStages) * (kTile >> 4));
+          const uint32_t d_tmem = tmem + kColS + (j & 1) * 128;
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-            mma_f16_ss(tmem + kColS + b * 128, sw128_desc(base + kOffQ + off, 16, 1024),
-                       sw128_desc(ka + off, 16, 1024), id_qk, kk > 0 ? 1u : 0u);
+            const uint64_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+            mma_f16_ss(d_tmem, dq + off, dk + off, id_qk, kk > 0 ? 1u : 0u);
           }
-          mma_commit(bar(BS0 + b));
-          mma_commit(bar(BKF0 + s));
-          return true;
+          mma_commit(qk_done(j));
         };
-        // O_b += P(j) V(j), b = j & 1: P (bf16 pairs) from the first 64
-        // columns of S buffer b, V from the ring
-        auto issue_pv = [&](int j) -> bool {
-          const int b = j & 1, s = j % kStages;
-          if (!wait_phase(bar(BP0 + b), (j >> 1) & 1, ctl)) return false;
-          if (!wait_phase(bar(BV0 + s), (j / kStages) & 1, ctl)) return false;
-          fence_async_smem();
-          tc_fence_after();
-          const uint32_t va = base + kOffV + s * kTile;
+        auto issue_pv = [&](int j) {  // O += P(j) V(j), P from group (j & 1)'s buffer
+          const uint64_t dv = dv0 + (uint64_t)((j % kStages) * (kTile >> 4));
+          const uint32_t a_tmem = tmem + kColP + (j & 1) * 64;
 #pragma unroll
           for (int kk = 0; kk < kBlock / 16; ++kk)
-            mma_f16_ts(tmem + kColO + b * 128, tmem + kColS + b * 128 + kk * 8,
-                       sw128_desc(va + kk * 16 * 128, kHalf, 1024), id_pv,
-                       (j >= 2 || kk > 0) ? 1u : 0u);
-          mma_commit(bar(BPV0 + b));
-          mma_commit(bar(BVF0 + s));
-          return true;
+            mma_f16_ts(tmem + kColO, a_tmem + kk * 8, dv + (uint64_t)(kk * 128), id_pv,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(pv_done(j));
         };
-        ok = ok && issue_qk(0);
-        if (ok && n_tiles > 1) ok = issue_qk(1);
-        for (int j = 0; ok && j < n_tiles; ++j) {
-          if (!issue_pv(j)) { ok = false; break; }
-          if (j + 2 < n_tiles && !issue_qk(j + 2)) { ok = false; break; }
+        // barriers of QK^T(j): S(j-2) copied out (j >= 2) and K(j) loaded
+        auto qk_ready_test = [&](int j) {
+          return (j < 2 || mbar_test(bar(BSF0 + (j & 1)), ((j >> 1) - 1) & 1)) &&
+                 mbar_test(bar(BK0 + j % kStages), (j / kStages) & 1);
+        };
+        auto qk_wait = [&](int j) {
+          return (j < 2 || wait_phase(bar(BSF0 + (j & 1)), ((j >> 1) - 1) & 1, ctl)) &&
+                 wait_phase(bar(BK0 + j % kStages), (j / kStages) & 1, ctl);
+        };
+        bool ok = wait_phase(bar(BQ), 0, ctl);
+        // cp.async (generic proxy) writes -> MMA operand reads; TMA writes are
+        // async-proxy and ordered by the mbarrier they complete
+        if constexpr (!kTma) fence_async_smem();
+        for (int j = 0; ok && j < 2 && j < n_tiles; ++j) {
+          ok = qk_wait(j);
+          if (!ok) break;
+          if constexpr (!kTma) fence_async_smem();
+          tc_fence_after();
+          issue_qk(j);
         }
-        // drain: every MMA issued above has completed once this commit fires
+        bool qk_ready = false;  // QK^T(j+2)'s barriers, tested one step early
+        for (int j = 0; ok && j < n_tiles; ++j) {
+          // P(j) and V(j): tested now, used after QK^T(j+2) is issued
+          const bool p_ready = mbar_test(bar(BP0 + (j & 1)), (j >> 1) & 1);
+          const bool v_ready = mbar_test(bar(BV0 + j % kStages), (j / kStages) & 1);
+          if (j + 2 < n_tiles) {
+            if (!qk_ready && !qk_wait(j + 2)) { ok = false; break; }
+            if constexpr (!kTma) fence_async_smem();
+            tc_fence_after();
+            issue_qk(j + 2);
+          }
+          qk_ready = j + 3 < n_tiles && qk_ready_test(j + 3);
+          if (!p_ready && !wait_phase(bar(BP0 + (j & 1)), (j >> 1) & 1, ctl)) { ok = false; break; }
+          if (!v_ready && !wait_phase(bar(BV0 + j % kStages), (j / kStages) & 1, ctl)) {
+            ok = false;
+            break;
+          }
+          if constexpr (!kTma) fence_async_smem();
+          tc_fence_after();
+          issue_pv(j);
+        }
+        // every MMA issued above has completed once this commit fires
         mma_commit(bar(BDRAIN));
         drain_phase(bar(BDRAIN), 0, ctl.limit_ns);
       }
@@ -337,21 +383,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = quarter * 32 + lane;  // tile row == TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     const uint32_t s_col = kColS + grp * 128;
-    const uint32_t o_col = kColO + grp * 128;
-    float m_used = -INFINITY, l = 0.f;  // this group's reference max and row sum
+    const uint32_t p_col = kColP + grp * 64;
+    // the kept list is ascending, so only its last entry can be the ragged
+    // last block of the head
+    const int tail_keys = g.N - (g.NB - 1) * kBlock;
+    const bool ragged_last =
+        n_tiles > 0 && tail_keys < kBlock && __ldg(ids + n_tiles - 1) == g.NB - 1;
+    float m_mine = -INFINITY, l = 0.f;  // this group's row sum, relative to m_mine
     bool ok = true;
     for (int t = 0;; ++t) {
       const int j = 2 * t + grp;
       if (j >= n_tiles) break;
-      if (!warp_wait(bar(BS0 + grp), t & 1, ctl)) { ok = false; break; }
+      if (!warp_wait(qk_done(j), ring_par(j), ctl)) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[128];
       tmem_ld128(lane_addr + s_col, sr);
-      const int valid = g.N - __ldg(ids + j) * kBlock;  // existing keys of the tile
-      if (valid < kBlock) {  // only the ragged last block (warp-uniform)
+      tc_fence_before();
+      mbar_arrive(bar(BSF0 + grp));  // S_grp may take QK^T two tiles ahead
+      if (ragged_last && j == n_tiles - 1) {  // warp-uniform
 #pragma unroll
         for (int c = 0; c < kBlock; ++c)
-          if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
+          if (c >= tail_keys) sr[c] = __float_as_uint(-INFINITY);
       }
       float mp[8];
 #pragma unroll
@@ -370,15 +422,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]),
                              fmaxf(mp[6], mp[7])) *
                        scale_log2;
-      // lazy rescale: keep the reference max unless this row's max grew by
-      // more than 2^8 (exact either way: O and l share the reference)
-      const bool first = m_used == -INFINITY;
-      const bool need = !first && mx > m_used + kRescaleLog2;
-      const float alpha = need ? ex2(m_used - mx) : 1.f;
-      if (first || need) m_used = mx;  // a tile has at least one existing key
-      // P = 2^(s*scale - m) as bf16 pairs over the first 64 columns of the S
-      // buffer (its fp32 values are all in registers); row sum in 8 chains
-      const float neg_m = -m_used;
+      // the reference after tile j-1 (published by the other group), then
+      // this tile's: kept unless this tile's max exceeds it by more than 2^8
+      float m_prev = -INFINITY;
+      if (j >= 1) {
+        if (!warp_wait(bar(BMX0 + (grp ^ 1)), ((j - 1) >> 1) & 1, ctl)) { ok = false; break; }
+        m_prev = mref[(grp ^ 1) * 128 + r];
+      }
+      const float m_j = (m_prev == -INFINITY || mx > m_prev + kRescaleLog2) ? mx : m_prev;
+      mref[grp * 128 + r] = m_j;
+      mbar_arrive(bar(BMX0 + grp));  // release: the store above is visible to the waiter
+      if (m_mine != -INFINITY) l *= ex2(m_mine - m_j);  // this group's sum, to m_j
+      m_mine = m_j;
+      // the group's P buffer is free once P V of its previous tile completed
+      if (j >= 2 && !warp_wait(pv_done(j - 2), ring_par(j - 2), ctl)) { ok = false; break; }
+      tc_fence_after();
+      // P = 2^(s*scale - m_j) as bf16 pairs into the group's P buffer; row
+      // sum in 8 chains
+      const float neg_m = -m_j;
       float rs[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) rs[u] = 0.f;
@@ -394,29 +455,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           rs[(e + 1) & 7] += e1;
           pk[c] = pack_bf16(e0, e1);
         }
-        tmem_st16_async(lane_addr + s_col + 16 * cc, pk);
+        tmem_st16_async(lane_addr + p_col + 16 * cc, pk);
       }
       tmem_wait_st();
-      l = l * alpha + (((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7])));
+      l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
+      // O holds P V up to tile j-1 relative to m_prev: rescale it before
+      // P V(j) once that MMA completed (rare: the reference moved)
+      const bool need = m_prev != -INFINITY && m_j != m_prev;
       if (__any_sync(0xffffffffu, need)) {
-        // O holds P V up to this group's previous tile once that MMA
-        // completed; P V of this tile is issued after the arrival below
-        if (!warp_wait(bar(BPV0 + grp), (t - 1) & 1, ctl)) { ok = false; break; }
+        if (!warp_wait(pv_done(j - 1), ring_par(j - 1), ctl)) { ok = false; break; }
         tc_fence_after();
+        const float alpha = need ? ex2(m_prev - m_j) : 1.f;
 #pragma unroll 1
         for (int c0 = 0; c0 < 128; c0 += 32) {
           uint32_t orr[32];
-          tmem_ld32(lane_addr + o_col + c0, orr);
+          tmem_ld32(lane_addr + kColO + c0, orr);
 #pragma unroll
           for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
-          tmem_st32(lane_addr + o_col + c0, orr);
+          tmem_st32(lane_addr + kColO + c0, orr);
         }
       }
       tc_fence_before();
       mbar_arrive(bar(BP0 + grp));
     }
-    // ---- epilogue: merge the groups, then group g writes output columns
-    // 64g .. 64g+63 of the row at the natural position of its token
+    // ---- epilogue: add the groups' row sums (each relative to its own
+    // latest reference; O is relative to the last tile's, the larger), then
+    // group g writes output columns 64g .. 64g+63 of the row at the natural
+    // position of its token
     const int p = i * kBlock + r;
     __nv_bfloat16* orow = p < g.N ? out + (bh * (int64_t)g.N + natural_index(g, order, p)) * kD
                                   : nullptr;
@@ -425,47 +490,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 8; ++c)
           reinterpret_cast<uint4*>(orow + grp * 64)[c] = make_uint4(0, 0, 0, 0);
     } else if (ok && n_tiles > 0) {
-      merge[(0 * 2 + grp) * 128 + r] = m_used;
-      merge[(1 * 2 + grp) * 128 + r] = l;
+      lsum[grp * 128 + r] = l;
+      mref[grp * 128 + r] = m_mine;  // -inf for a group that saw no tile
       mbar_arrive(bar(BM));
       bool okm = all_wait(bar(BM), 0, ctl);
-      float f0 = 0.f, f1 = 0.f, lt = 0.f;
+      float inv = 0.f;
       if (okm) {
-        const float m0 = merge[r], m1 = merge[128 + r];
+        const float m0 = mref[r], m1 = mref[128 + r];
         const float m = fmaxf(m0, m1);
-        // a group that saw no tile (a one-tile list) has l = 0 and an
-        // unwritten O: weight 0
-        f0 = m0 == -INFINITY ? 0.f : ex2(m0 - m);
-        f1 = m1 == -INFINITY ? 0.f : ex2(m1 - m);
-        lt = merge[256 + r] * f0 + merge[384 + r] * f1;
+        const float lt = (m0 == -INFINITY ? 0.f : lsum[r] * ex2(m0 - m)) +
+                         (m1 == -INFINITY ? 0.f : lsum[128 + r] * ex2(m1 - m));
+        inv = lt > 0.f ? 1.f / lt : 0.f;
       }
-      // every P V has completed once the MMA lane's drain commit fired
-      if (okm) okm = warp_wait(bar(BDRAIN), 0, ctl);
+      // every P V has completed once the last one's commit fired
+      if (okm) okm = warp_wait(pv_done(n_tiles - 1), ring_par(n_tiles - 1), ctl);
       if (okm) {
         tc_fence_after();
-        const float inv = lt > 0.f ? 1.f / lt : 0.f;
-        f0 *= inv;
-        f1 *= inv;
 #pragma unroll 1
         for (int c0 = 0; c0 < 64; c0 += 32) {
           const int col = grp * 64 + c0;
-          uint32_t oa[32], ob[32];
-          tmem_ld32x2(lane_addr + kColO + col, oa, lane_addr + kColO + 128 + col, ob);
+          uint32_t oa[32];
+          tmem_ld32(lane_addr + kColO + col, oa);
           if (orow != nullptr) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-              float vv[8];
-#pragma unroll
-              for (int u = 0; u < 8; ++u) {
-                const float a0 = f0 != 0.f ? __uint_as_float(oa[c * 8 + u]) * f0 : 0.f;
-                const float a1 = f1 != 0.f ? __uint_as_float(ob[c * 8 + u]) * f1 : 0.f;
-                vv[u] = a0 + a1;
-              }
               uint4 w;
-              w.x = pack_bf16(vv[0], vv[1]);
-              w.y = pack_bf16(vv[2], vv[3]);
-              w.z = pack_bf16(vv[4], vv[5]);
-              w.w = pack_bf16(vv[6], vv[7]);
+              w.x = pack_bf16(__uint_as_float(oa[c * 8 + 0]) * inv, __uint_as_float(oa[c * 8 + 1]) * inv);
+              w.y = pack_bf16(__uint_as_float(oa[c * 8 + 2]) * inv, __uint_as_float(oa[c * 8 + 3]) * inv);
+              w.z = pack_bf16(__uint_as_float(oa[c * 8 + 4]) * inv, __uint_as_float(oa[c * 8 + 5]) * inv);
+              w.w = pack_bf16(__uint_as_float(oa[c * 8 + 6]) * inv, __uint_as_float(oa[c * 8 + 7]) * inv);
               reinterpret_cast<uint4*>(orow + col)[c] = w;
             }
           }
