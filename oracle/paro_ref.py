@@ -58,6 +58,33 @@ import numpy as np
 # Axis letters of each order id, outermost first.
 ORDER_NAMES = ("FHW", "FWH", "HFW", "HWF", "WFH", "WHF")
 
+# Order ids 6 .. 11: SPADE's 3D blockings (SPADE, arXiv 2608.03335, Pith
+# verdict page, key_machinery (i): spatial, temporal and mixed 3D blocking
+# candidates of the token grid).  Reading: a blocking by tiles of
+# tf x th x tw tokens (tf*th*tw = the block size) orders the tokens tile by
+# tile -- tiles in (f, h, w) order of their tile coordinates, tokens inside a
+# tile in (f, h, w) order -- and the executor's blocks are runs of ``block``
+# consecutive positions of that order (tiles on the far edges of a grid that
+# the tile does not divide are partial, so blocks then straddle tiles).  Two
+# of each kind per block size: spatial (tf = 1), mixed, temporal (tf >= 8).
+TILE_SHAPES = {
+    128: ((1, 8, 16), (1, 16, 8), (2, 8, 8), (4, 4, 8), (8, 4, 4), (16, 2, 4)),
+    64: ((1, 8, 8), (1, 4, 16), (2, 4, 8), (4, 4, 4), (8, 2, 4), (16, 2, 2)),
+}
+N_ORDERS = 12  # ids 0-5 axis orders, 6-11 tile blockings (blocks 64 and 128)
+
+
+def n_candidates(block: int) -> int:
+    """Blocking candidates of a block size: the six axis orders, plus the six
+    tile blockings where a tile table exists."""
+    return N_ORDERS if block in TILE_SHAPES else 6
+
+
+def order_name(perm_id: int, block: int) -> str:
+    if perm_id < 6:
+        return ORDER_NAMES[perm_id]
+    return "T%dx%dx%d" % TILE_SHAPES[block][perm_id - 6]
+
 
 # ---------------------------------------------------------------- reorder --
 
@@ -66,26 +93,54 @@ def order_axes(perm_id: int) -> tuple:
     return tuple("FHW".index(c) for c in ORDER_NAMES[int(perm_id)])
 
 
+def tile_order(grid: tuple, shape: tuple) -> np.ndarray:
+    """Natural indices n = f*H*W + h*W + w of the tokens in tile-major order
+    for tiles of ``shape`` = (tf, th, tw): tiles in (f, h, w) order, tokens
+    inside a tile in (f, h, w) order, partial tiles at the far edges."""
+    F, H, W = grid
+    tf, th, tw = shape
+    seq = []
+    for f0 in range(0, F, tf):
+        for h0 in range(0, H, th):
+            for w0 in range(0, W, tw):
+                for f in range(f0, min(f0 + tf, F)):
+                    for h in range(h0, min(h0 + th, H)):
+                        for w in range(w0, min(w0 + tw, W)):
+                            seq.append(f * H * W + h * W + w)
+    return np.asarray(seq, dtype=np.int64)
+
+
 def reorder_head(x: np.ndarray, grid: tuple, perm_id: int, block: int) -> np.ndarray:
     """One head's [N, d] rows in natural FHW order -> [N_p, d] in the head's
     order, zero rows appended at the tail (PAROAttention review,
-    key_machinery: the six axis orders of [F, H, W])."""
+    key_machinery: the six axis orders of [F, H, W]; ids 6-11: SPADE's 3D
+    tile blockings, see TILE_SHAPES)."""
     F, H, W = grid
     N, d = x.shape
     assert N == F * H * W
-    ax = order_axes(perm_id)
-    y = x.reshape(F, H, W, d).transpose(ax + (3,)).reshape(N, d)
+    if int(perm_id) < 6:
+        ax = order_axes(perm_id)
+        y = x.reshape(F, H, W, d).transpose(ax + (3,)).reshape(N, d)
+    else:
+        y = x[tile_order(grid, TILE_SHAPES[block][int(perm_id) - 6])]
     nb = -(-N // block)
     out = np.zeros((nb * block, d), dtype=x.dtype)
     out[:N] = y
     return out
 
 
-def inverse_reorder_head(xp: np.ndarray, grid: tuple, perm_id: int) -> np.ndarray:
-    """Inverse of :func:`reorder_head`: drop the pad rows, undo the order."""
+def inverse_reorder_head(xp: np.ndarray, grid: tuple, perm_id: int,
+                         block: int | None = None) -> np.ndarray:
+    """Inverse of :func:`reorder_head`: drop the pad rows, undo the order
+    (``block`` names the tile shape of ids 6-11)."""
     F, H, W = grid
     N = F * H * W
     d = xp.shape[1]
+    if int(perm_id) >= 6:
+        order = tile_order(grid, TILE_SHAPES[block][int(perm_id) - 6])
+        out = np.zeros((N, d), dtype=xp.dtype)
+        out[order] = xp[:N]
+        return out
     ax = order_axes(perm_id)
     sizes = tuple((F, H, W)[a] for a in ax)
     y = xp[:N].reshape(sizes + (d,))
@@ -104,14 +159,14 @@ def reorder(x: np.ndarray, grid: tuple, perms, block: int) -> np.ndarray:
     return out
 
 
-def inverse_reorder(xp: np.ndarray, grid: tuple, perms) -> np.ndarray:
+def inverse_reorder(xp: np.ndarray, grid: tuple, perms, block: int | None = None) -> np.ndarray:
     """[B, h, N_p, d] -> [B, h, N, d]."""
     B, nh, _, d = xp.shape
     N = grid[0] * grid[1] * grid[2]
     out = np.zeros((B, nh, N, d), dtype=xp.dtype)
     for b in range(B):
         for h in range(nh):
-            out[b, h] = inverse_reorder_head(xp[b, h], grid, perms[h])
+            out[b, h] = inverse_reorder_head(xp[b, h], grid, perms[h], block)
     return out
 
 
@@ -267,7 +322,7 @@ def attention(q, k, v, grid, perms, block, idx, counts=None):
             vp = reorder_head(v[b, h], grid, perms[h], block)
             cnt = None if counts is None else counts[b, h]
             op = attention_permuted(qp, kp, vp, N, block, idx[b, h], cnt)
-            out[b, h] = inverse_reorder_head(op, grid, perms[h])
+            out[b, h] = inverse_reorder_head(op, grid, perms[h], block)
     return out
 
 

@@ -107,7 +107,7 @@ def attention_compensated(q, k, v, grid, perms, block, idx, counts=None):
             vp = ref.reorder_head(v[b, h], grid, perms[h], block)
             cnt = None if counts is None else counts[b, h]
             op = compensated_permuted(qp, kp, vp, N, block, idx[b, h], cnt)
-            out[b, h] = ref.inverse_reorder_head(op, grid, perms[h])
+            out[b, h] = ref.inverse_reorder_head(op, grid, perms[h], block)
     return out
 
 

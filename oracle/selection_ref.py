@@ -19,14 +19,18 @@ Sources (SPADE, arXiv 2608.03335, Pith verdict page):
 
 Readings where the page is silent:
 
-S1. Candidate blockings are the six axis orders of [F, H, W] with the
-    executor's block size (runs of ``block`` consecutive tokens of the
-    permuted order, the blocks the attention kernel runs).
+S1. Candidate blockings: the six axis orders of [F, H, W] and six 3D tile
+    blockings (key_machinery (i): spatial, temporal and mixed candidates),
+    ids 6-11, tiles of tf x th x tw = block tokens in tile-major order
+    (oracle/paro_ref.py TILE_SHAPES: for block 128 spatial 1x8x16 and
+    1x16x8, mixed 2x8x8 and 4x4x8, temporal 8x4x4 and 16x2x4); in every
+    case the blocks are runs of ``block`` consecutive tokens of the
+    candidate's order (the blocks the attention kernel runs).
 S2. "Pairwise" counts ordered pairs s != t (the identity above); a zero row
     has no direction and contributes nothing (xh = 0).  Pad rows are zero.
-S3. The score of an order is SICS over Q's blocks plus SICS over K's blocks
-    (the same token sets); the selected order is the argmax, ties to the
-    lower order id.
+S3. The score of a candidate is SICS over Q's blocks plus SICS over K's
+    blocks (the same token sets); the selected one is the argmax, ties to
+    the lower id; a head's pick sums its score over the batch.
 S4. Top-P on a query-block row: weights w_j = exp(s_j - max_j s_j) over all
     key blocks (NaN scores weigh 0 and sort as -inf); blocks in order of
     decreasing score, ties to the lower index; keep the shortest prefix
@@ -74,24 +78,33 @@ def sics_order(x: np.ndarray, grid: tuple, perm_id: int, block: int) -> float:
 
 
 def sics_scores(q, k, grid: tuple, block: int) -> np.ndarray:
-    """[B, h, N, d] q, k -> [B, h, 6] scores, SICS(Q) + SICS(K) per order
-    (reading S3)."""
+    """[B, h, N, d] q, k -> [B, h, 12] scores, SICS(Q) + SICS(K) per
+    candidate blocking: the six axis orders and the six 3D tile blockings
+    (readings S1, S3)."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     B, nh = q.shape[:2]
-    out = np.zeros((B, nh, 6), dtype=np.float64)
+    nc = ref.n_candidates(block)
+    out = np.zeros((B, nh, nc), dtype=np.float64)
     for b in range(B):
         for h in range(nh):
-            for o in range(6):
+            for o in range(nc):
                 out[b, h, o] = (sics_order(q[b, h], grid, o, block)
                                 + sics_order(k[b, h], grid, o, block))
     return out
 
 
 def select_orders(scores: np.ndarray) -> np.ndarray:
-    """[B, h, 6] -> [B, h] int8 argmax order ids, ties to the lower id
+    """[B, h, C] -> [B, h] int8 argmax candidate ids, ties to the lower id
     (np.argmax returns the first maximum)."""
     return np.argmax(np.asarray(scores), axis=-1).astype(np.int8)
+
+
+def head_picks(scores: np.ndarray) -> np.ndarray:
+    """[B, h, C] -> [h] int8: each head's blocking, the argmax of its score
+    summed over the batch (a head has one blocking), ties to the lower id
+    (reading S3)."""
+    return np.argmax(np.asarray(scores, dtype=np.float64).sum(axis=0), axis=-1).astype(np.int8)
 
 
 # ------------------------------------------------------------ filters --
