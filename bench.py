@@ -318,7 +318,7 @@ def pasa_cpu_baseline(w, q, k, v, perms):
 
 
 def sics_cpu_baseline(w, q, k):
-    """The SICS oracle, as it stands, on head 0 (six orders, q and k).
+    """The SICS oracle, as it stands, on head 0 (all 12 candidates, q and k).
     Returns GB/s of the same algorithmic bytes as the kernel's line (every
     row of q and k read once per order), seconds, and the sample."""
     from oracle import selection_ref as sel
@@ -326,8 +326,8 @@ def sics_cpu_baseline(w, q, k):
     sel.sics_scores(q[:, :1].double().numpy(), k[:, :1].double().numpy(), (w.F, w.H, w.W),
                     w.block)
     dt = time.perf_counter() - t0
-    nbytes = 2 * 6 * w.B * w.N * w.d * q.element_size()
-    return nbytes / dt / 1e9, dt, "head 0 of the layer (six orders, q and k)"
+    nbytes = 2 * 12 * w.B * w.N * w.d * q.element_size()
+    return nbytes / dt / 1e9, dt, "head 0 of the layer (12 candidates, q and k)"
 
 
 def cores():
@@ -537,29 +537,64 @@ def timed_calls(fn, reps=20, warm=5):
 
 def run_sweep_selection(device, peaks, peak_src, heads=None):
     """The selection variants on the 720p layer: the SICS blocking score of
-    the six orders (HBM-bound: q and k read once per order) and a layer
-    whose kept lists come from the hybrid filter (diagonal, window 1,
-    Top-K at density 0.10, Top-P 0.5)."""
+    the 12 candidate blockings (HBM-bound: q and k read once per candidate),
+    the layer (top-k at the workload density) run on the blockings SICS
+    picked, and a layer whose kept lists come from the hybrid filter
+    (diagonal, window 1, Top-K at density 0.10, Top-P 0.5)."""
     w = WORKLOADS["720p_21x45x80"]
     q, k, v, perms = make_inputs(w, heads=heads)
     if heads is not None:
         w = dataclasses.replace(w, heads=heads)
     qkv = [t.to(device) for t in (q, k, v)]
     pr = paro.Problem(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, [0] * w.heads)
-    sc = torch.empty((w.B, w.heads, 6), dtype=torch.float32, device=device)
-    ms = timed_calls(lambda: paro.sics_scores(qkv[0], qkv[1], pr, sc))
-    nbytes = 2 * 6 * w.B * w.heads * w.N * w.d * qkv[0].element_size()
+    sc = torch.empty((w.B, w.heads, paro.N_ORDERS), dtype=torch.float32, device=device)
+    picks = torch.empty((w.heads,), dtype=torch.int8, device=device)
+    ms = timed_calls(lambda: paro.sics_scores(qkv[0], qkv[1], pr, sc, picks))
+    nbytes = 2 * paro.N_ORDERS * w.B * w.heads * w.N * w.d * qkv[0].element_size()
     pm = percentiles(ms)
     hbm = float(peaks.get("hbm_gbs", 6650.0))
     cpu_gbs, cpu_s, cpu_sample = sics_cpu_baseline(w, q, k)
     print(json.dumps({
-        "workload": w.name, "kernel": "sics_kernel", "what": "SICS of the six orders, q and k",
+        "workload": w.name, "kernel": "sics_kernel", "what": "SICS of the 12 candidate blockings (6 axis orders, 6 3D tiles), q and k, with the per-head pick",
         "ms": pm, "bytes": nbytes, "gbs_p50": nbytes / (pm["p50"] / 1e3) / 1e9,
         "frac_of_hbm_p50": nbytes / (pm["p50"] / 1e3) / 1e9 / hbm,
         "peak_source": f"{peak_src} hbm_gbs", "steps": len(ms),
         "cpu_baseline": {"value": cpu_gbs, "unit": "GB/s", "cores": cores(), "kind": "oracle",
                          "sample": cpu_sample, "seconds": cpu_s},
     }), flush=True)
+    # the layer on SICS's per-head blockings (reorder + pool on those
+    # orders, scores, top-k, attention over the permuted tiles)
+    sics_perms = [int(o) for o in picks.cpu().tolist()]
+    spipe = Pipeline(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, sics_perms, w.density,
+                     device=device)
+    s_attn, s_total = [], []
+    for it in range(25):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record()
+        spipe.select(*qkv)
+        e[1].record()
+        spipe.attend(*qkv)
+        e[2].record()
+        torch.cuda.synchronize()
+        if it >= 5:
+            s_attn.append(e[1].elapsed_time(e[2]))
+            s_total.append(e[0].elapsed_time(e[2]))
+    if int(spipe.status.item()) != 0:
+        raise RuntimeError(f"sics layer: device status {int(spipe.status.item())}")
+    sflops = w.flops(spipe.k)
+    sa, st = percentiles(s_attn), percentiles(s_total)
+    print(json.dumps({
+        "workload": w.name, "precision": "bf16", "selection": "top-k on SICS-picked blockings",
+        "picks": {str(o): sics_perms.count(o) for o in sorted(set(sics_perms))},
+        "k": spipe.k, "NB": spipe.pr.NB, "attn_ms": sa, "step_ms": st,
+        "select_ms_p50": st["p50"] - sa["p50"],
+        "tflops_p50": sflops / (sa["p50"] / 1e3) / 1e12,
+        "frac_of_burst_peak_p50": sflops / (sa["p50"] / 1e3) / 1e12
+        / tensor_peak(peaks, "bf16", "bf16_tflops"),
+        "peak_source": f"{peak_src} bf16_tflops", "kernel": attn_kernel_name(spipe),
+        "steps": len(s_attn), "warmup": 5,
+    }), flush=True)
+    del spipe
     pipe = Pipeline(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, perms, 0.10, device=device,
                     selection="hybrid", top_p=0.5, window=1)
     attn, total = [], []
@@ -623,11 +658,12 @@ def run_sweep_offline(device, peaks, peak_src, heads=None):
 
 def run_sweep_pasa(device, peaks, peak_src, heads=None):
     """PASA's grouped first-order compensation on the 480p layer (top-k at
-    the workload density): the compensated kernel (mma.sync, kept tiles plus
-    every unselected block as one pooled key row) against the same kernel
-    without compensation and the tcgen05 kernel, on the same kept lists.
-    Algorithmic FLOP: 4 b^2 d per kept tile plus 4 b d per (query block,
-    pooled key block) pair."""
+    the workload density): the compensated tcgen05 kernel (kept tiles, then
+    every unselected block as one pooled key row) with bf16 block means
+    (rounded once per call; the rounding is inside the timed call) and with
+    fp32 means (rounded by the loader warps), against the same kernel
+    without compensation, on the same kept lists.  Algorithmic FLOP: 4 b^2 d
+    per kept tile plus 4 b d per (query block, pooled key block) pair."""
     w = WORKLOADS["480p_21x30x52"]
     q, k, v, perms = make_inputs(w, heads=heads)
     if heads is not None:
@@ -641,13 +677,23 @@ def run_sweep_pasa(device, peaks, peak_src, heads=None):
     idx = paro.select_topk(paro.score_pooled(q_pool, k_pool, pr), pr, kk)
     status = torch.zeros(1, dtype=torch.int32, device=device)
     out = torch.empty((w.B, w.heads, w.N, w.d), dtype=qd.dtype, device=device)
+    kb = torch.empty(k_pool.shape, dtype=torch.bfloat16, device=device)
+    vb = torch.empty_like(kb)
+
+    def compensated_bf16_means():
+        paro.round_bf16(k_pool, kb)
+        paro.round_bf16(v_pool, vb)
+        return paro.block_sparse_attn_compensated(qp, kp, vp, pr, idx, kb, vb, out=out,
+                                                  status=status, permuted=True)
+
     runs = {
-        "compensated_mma": lambda: paro.block_sparse_attn_compensated(
+        "compensated_tcgen05": compensated_bf16_means,
+        "compensated_tcgen05_f32_means": lambda: paro.block_sparse_attn_compensated(
             qp, kp, vp, pr, idx, k_pool, v_pool, out=out, status=status, permuted=True),
-        "plain_mma": lambda: paro.block_sparse_attn(qp, kp, vp, pr, idx, out=out, status=status,
-                                                    baseline=True, permuted=True),
         "plain_tcgen05": lambda: paro.block_sparse_attn(qp, kp, vp, pr, idx, out=out,
                                                         status=status, permuted=True),
+        "plain_mma": lambda: paro.block_sparse_attn(qp, kp, vp, pr, idx, out=out, status=status,
+                                                    baseline=True, permuted=True),
     }
     ms = {name: percentiles(timed_calls(fn)) for name, fn in runs.items()}
     if int(status.item()) != 0:
@@ -661,14 +707,16 @@ def run_sweep_pasa(device, peaks, peak_src, heads=None):
         "workload": w.name, "what": "PASA grouped first-order compensation of the unselected"
         " blocks (top-k at the workload density)", "heads": w.heads, "k": kk, "NB": pr.NB,
         "ms": ms, "flops_compensated": flops,
-        "tflops_compensated_p50": flops / (ms["compensated_mma"]["p50"] / 1e3) / 1e12,
-        "tflops_plain_mma_p50": plain_flops / (ms["plain_mma"]["p50"] / 1e3) / 1e12,
+        "tflops_compensated_p50": flops / (ms["compensated_tcgen05"]["p50"] / 1e3) / 1e12,
         "tflops_plain_tcgen05_p50": plain_flops / (ms["plain_tcgen05"]["p50"] / 1e3) / 1e12,
-        "overhead_vs_plain_mma": ms["compensated_mma"]["p50"] / ms["plain_mma"]["p50"],
+        "tflops_plain_mma_p50": plain_flops / (ms["plain_mma"]["p50"] / 1e3) / 1e12,
+        "overhead_vs_plain_tcgen05": ms["compensated_tcgen05"]["p50"] / ms["plain_tcgen05"]["p50"],
+        "overhead_f32_means_vs_plain_tcgen05": ms["compensated_tcgen05_f32_means"]["p50"]
+        / ms["plain_tcgen05"]["p50"],
         "peak_source": f"{peak_src} bf16_tflops",
-        "frac_of_burst_peak_p50": flops / (ms["compensated_mma"]["p50"] / 1e3) / 1e12
+        "frac_of_burst_peak_p50": flops / (ms["compensated_tcgen05"]["p50"] / 1e3) / 1e12
         / tensor_peak(peaks, "bf16", "bf16_tflops"),
-        "kernel": "attn_mma_kernel<comp>", "steps": 20, "warmup": 5,
+        "kernel": "attn_sm100_kernel<comp>", "steps": 20, "warmup": 5,
         "cpu_baseline": {"value": cpu_tf, "unit": "TFLOPS", "cores": cores(), "kind": "oracle",
                          "sample": cpu_sample, "seconds": cpu_s},
     }), flush=True)

@@ -14,7 +14,8 @@ cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, pa_dt
                               const Grid& g, const int32_t* idx, const int32_t* counts,
                               int k_max, const float* qs, const float* ks, const float* vs,
                               float p_levels, void* out, int32_t* status, bool permuted,
-                              cudaStream_t s);
+                              cudaStream_t s, const void* k_pool = nullptr,
+                              const void* v_pool = nullptr, pa_dtype pool_dtype = PA_F32);
 bool attn_sm100_supports(pa_dtype dt, const Grid& g);
 }  // namespace paro
 
@@ -91,11 +92,24 @@ pa_status make_grid(const pa_shape& s, const int8_t* perms, bool need_perms, par
     g->sm[o] = stride[axes[o][1]];
     g->si[o] = stride[axes[o][2]];
   }
+  // the 3D tile blockings of ids 6-11 (tf, th, tw; volume = block): two
+  // spatial (tf = 1), two mixed, two temporal
+  static const int tiles128[6][3] = {{1, 8, 16}, {1, 16, 8}, {2, 8, 8},
+                                     {4, 4, 8},  {8, 4, 4},  {16, 2, 4}};
+  static const int tiles64[6][3] = {{1, 8, 8}, {1, 4, 16}, {2, 4, 8},
+                                    {4, 4, 4}, {8, 2, 4},  {16, 2, 2}};
+  for (int t = 0; t < 6; ++t) {
+    const int* sh = s.block == 128 ? tiles128[t] : tiles64[t];
+    g->tf[t] = sh[0];
+    g->th[t] = sh[1];
+    g->tw[t] = sh[2];
+  }
   if (need_perms) {
     if (perms == nullptr) return fail(PA_ERR_INVALID_ARG, "perms is NULL");
     for (int h = 0; h < s.heads; ++h) {
-      if (perms[h] < 0 || perms[h] > 5)
-        return fail(PA_ERR_INVALID_ARG, "perms[%d]=%d is not an order id 0..5", h, (int)perms[h]);
+      if (perms[h] < 0 || perms[h] >= paro::kOrders)
+        return fail(PA_ERR_INVALID_ARG, "perms[%d]=%d is not an order id 0..%d", h,
+                    (int)perms[h], paro::kOrders - 1);
       g->perm[h] = perms[h];
     }
   }
@@ -117,7 +131,7 @@ pa_status check_float_dtype(pa_dtype dt) {
 
 extern "C" {
 
-int32_t pa_abi_version(void) { return 6; }
+int32_t pa_abi_version(void) { return 8; }
 
 pa_status pa_clear_status(int32_t* dev_status, void* stream) {
   PA_REQUIRE(dev_status != nullptr, "dev_status must be non-NULL");
@@ -238,7 +252,7 @@ pa_status pa_select_hybrid(const float* scores, pa_shape shape, int32_t k, doubl
 }
 
 pa_status pa_sics_scores(const void* q, const void* k, pa_dtype dtype, pa_shape shape,
-                         float* scores, void* stream) {
+                         float* scores, int8_t* orders, void* stream) {
   paro::Grid g;
   pa_status st = make_grid(shape, nullptr, false, &g);
   if (st != PA_OK) return st;
@@ -247,9 +261,11 @@ pa_status pa_sics_scores(const void* q, const void* k, pa_dtype dtype, pa_shape 
   PA_REQUIRE(q && k && scores, "q, k and scores must be non-NULL");
   PA_REQUIRE(aligned16(q) && aligned16(k), "q and k must be 16-byte aligned");
   cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = cudaMemsetAsync(scores, 0, (size_t)g.B * g.heads * 6 * sizeof(float), s);
+  cudaError_t e =
+      cudaMemsetAsync(scores, 0, (size_t)g.B * g.heads * paro::kOrders * sizeof(float), s);
   if (e == cudaSuccess) e = paro::launch_sics(q, dtype, g, scores, s);
   if (e == cudaSuccess) e = paro::launch_sics(k, dtype, g, scores, s);
+  if (e == cudaSuccess && orders != nullptr) e = paro::launch_sics_pick(scores, g, orders, s);
   return cuda_status(e, "pa_sics_scores launch");
 }
 
@@ -424,8 +440,9 @@ pa_status pa_block_sparse_attn_compensated(const void* q, const void* k, const v
                                            pa_dtype dtype, uint32_t flags, pa_shape shape,
                                            const int8_t* perms, const int32_t* idx,
                                            const int32_t* counts, int32_t k_max,
-                                           const float* k_pool, const float* v_pool, void* out,
-                                           int32_t* dev_status, void* stream) {
+                                           const void* k_pool, const void* v_pool,
+                                           pa_dtype pool_dtype, void* out, int32_t* dev_status,
+                                           void* stream) {
   paro::Grid g;
   pa_status st = make_grid(shape, perms, true, &g);
   if (st != PA_OK) return st;
@@ -438,11 +455,34 @@ pa_status pa_block_sparse_attn_compensated(const void* q, const void* k, const v
              "q, k, v, k_pool, v_pool and out must be 16-byte aligned");
   PA_REQUIRE(k_max >= 0 && k_max <= g.NB, "k_max=%d must be in [0, NB=%d]", k_max, g.NB);
   PA_REQUIRE((flags & ~PA_ATTN_PERMUTED) == 0, "unknown flags 0x%x", flags);
+  PA_REQUIRE(pool_dtype == PA_F32 || pool_dtype == PA_BF16,
+             "pool_dtype %d: the block means are PA_F32 or PA_BF16", (int)pool_dtype);
+  const bool sm100 = dtype == PA_BF16 && paro::attn_sm100_supports(dtype, g);
+  if (pool_dtype == PA_BF16 && !sm100)
+    return fail(PA_ERR_UNSUPPORTED,
+                "bf16 block means need the tcgen05 kernel (PA_BF16, d=128, block=128)");
   if (g.NB > 4096) return fail(PA_ERR_UNSUPPORTED, "NB=%d above 4096 (one bit per block in shared memory)", g.NB);
   const bool permuted = (flags & PA_ATTN_PERMUTED) != 0;
+  cudaStream_t s = (cudaStream_t)stream;
+  // the tcgen05 kernel for bf16, d = 128, block = 128; the mma.sync one otherwise
+  if (sm100)
+    return cuda_status(paro::launch_attn_sm100(q, k, v, dtype, g, idx, counts, k_max, nullptr,
+                                               nullptr, nullptr, 127.f, out, dev_status, permuted,
+                                               s, k_pool, v_pool, pool_dtype),
+                       "pa_block_sparse_attn_compensated launch");
   return cuda_status(paro::launch_attn_mma(q, k, v, dtype, g, idx, counts, k_max, out, dev_status,
-                                           permuted, (cudaStream_t)stream, k_pool, v_pool),
+                                           permuted, s, static_cast<const float*>(k_pool),
+                                           static_cast<const float*>(v_pool)),
                      "pa_block_sparse_attn_compensated launch");
+}
+
+pa_status pa_round_bf16(const float* x, void* y, int64_t n, void* stream) {
+  PA_REQUIRE(n >= 0, "n=%lld must be >= 0", (long long)n);
+  if (n == 0) return PA_OK;
+  PA_REQUIRE(x && y, "x and y must be non-NULL");
+  PA_REQUIRE(aligned16(x) && aligned16(y), "x and y must be 16-byte aligned");
+  PA_REQUIRE(n <= ((int64_t)1 << 40), "n=%lld too large", (long long)n);
+  return cuda_status(paro::launch_round_bf16(x, y, n, (cudaStream_t)stream), "pa_round_bf16 launch");
 }
 
 }  // extern "C"

@@ -45,12 +45,25 @@
 // (32 KB) and three-stage K and V rings (6 x 32 KB) in the canonical
 // K-major / MN-major SWIZZLE_128B layouts the MMA descriptors name.
 //
+// With PASA's compensation (kComp; PASA, arXiv 2604.12219, Figure 2 caption
+// and section 3.3: the key blocks outside a query block's kept set enter
+// through a grouped first-order term), ceil(NB/128) pooled tiles follow the
+// kept tiles of every row: row c of pooled tile p is block b = 128p + c's
+// mean key and mean value (fp32 block means, rounded to bf16 by the loader
+// warps into the same swizzled stage layout), and the softmax adds log2 of
+// the block's valid key count to its score and gives kept blocks and
+// columns past NB the score -inf.  So block b adds n_b e^{q.kbar_b/sqrt(d)}
+// to the normaliser and that times vbar_b to the numerator, in the same
+// online softmax.
+//
 // A K stage is refilled once its QK^T completes, a V stage once its P V
 // completes; each MMA group signals its completion with one commit.  Every mbarrier wait is bounded (about one second of
 // %globaltimer, or the limit the launch sets); on expiry the kernel records
 // PA_ERR_TIMEOUT in the device status word, each role leaves its loop,
 // in-flight copies and MMAs are drained and tensor memory is released
 // before the CTA exits.
+#include <type_traits>
+
 #include "sm100.cuh"
 
 namespace paro {
@@ -78,6 +91,8 @@ constexpr uint32_t kOffBar = 0;
 constexpr uint32_t kOffSlot = 256;
 constexpr uint32_t kOffMerge = 512;
 constexpr uint32_t kOffRef = kOffMerge + 2 * 128 * 4;
+constexpr uint32_t kOffBits = kOffRef + 2 * 128 * 4;  // kComp: the kept list as NB bits
+constexpr int kCompMaxNB = 4096;
 constexpr uint32_t kSmall = 3072;
 constexpr uint32_t kOffQ = kSmall;
 constexpr uint32_t kOffK = kOffQ + kTile;            // kStages stages
@@ -107,7 +122,61 @@ enum : uint32_t {
   NBAR = 27
 };
 static_assert(NBAR * 8 <= kOffSlot, "barrier region");
-static_assert(kOffRef + 2 * 128 * 4 <= kSmall, "row sum and reference regions");
+static_assert(kOffBits + kCompMaxNB / 8 <= kSmall, "row sum, reference and bitset regions");
+
+// Rows t0 .. t0+127 of a [nb, 128] float block-mean array, rounded to bf16,
+// into a stage in the SWIZZLE_128B layout of copy_tile (rows >= nb zero),
+// by one warp with generic-proxy stores.  Lane l converts the 16-byte
+// chunks e = l + 32m (row e / 16, chunk e % 16), m = 0..63, in four batches
+// of 16 whose 32 global loads are all issued before any is used (the
+// block means sit in L2; the batches hide its latency).
+__device__ __forceinline__ void pool_tile(unsigned char* stage, const float* __restrict__ src,
+                                          int t0, int nb, int lane) {
+  constexpr int kBatch = 16;
+#pragma unroll 1
+  for (int m0 = 0; m0 < kBlock * 16 / 32; m0 += kBatch) {
+    float4 a[kBatch], b[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int e = lane + 32 * (m0 + u);
+      const int r = e >> 4, c16 = e & 15;
+      if (t0 + r < nb) {
+        const float4* f = reinterpret_cast<const float4*>(src + (int64_t)(t0 + r) * kD + c16 * 8);
+        a[u] = __ldg(f);
+        b[u] = __ldg(f + 1);
+      } else {
+        a[u] = b[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int e = lane + 32 * (m0 + u);
+      const int r = e >> 4, c16 = e & 15, half = c16 >> 3, c = c16 & 7;
+      uint4 w;
+      w.x = pack_bf16(a[u].x, a[u].y);
+      w.y = pack_bf16(a[u].z, a[u].w);
+      w.z = pack_bf16(b[u].x, b[u].y);
+      w.w = pack_bf16(b[u].z, b[u].w);
+      *reinterpret_cast<uint4*>(stage + half * kHalf + sw128_off(r, c)) = w;
+    }
+  }
+}
+
+// One warp copies rows r0 .. r0+127 of a [rows, 128] bf16 array into a
+// stage in the SWIZZLE_128B layout (16-byte cp.async, 16 lanes per row);
+// rows at or past `valid` (relative to r0) are zero-filled.
+__device__ __forceinline__ void copy_rows(uint32_t tile, const __nv_bfloat16* __restrict__ src,
+                                          int64_t r0, int valid, int lane) {
+  const int c16 = lane & 15, half = c16 >> 3, c = c16 & 7;
+  const char* src0 = reinterpret_cast<const char*>(src + r0 * kD) + c16 * 16;
+#pragma unroll 8
+  for (int m = 0; m < kBlock / 2; ++m) {
+    const int r = 2 * m + (lane >> 4);
+    const bool ok = r < valid;
+    cp_async16(tile + half * kHalf + sw128_off(r, c), src0 + (ok ? (int64_t)r * (kD * 2) : 0),
+               ok ? 16u : 0u);
+  }
+}
 
 // One warp copies a 128 x 128 bf16 tile whose row r is the token at
 // permuted position p0 + r of head `head` (rows past N zero-filled).  Lane l
@@ -140,16 +209,26 @@ __device__ __forceinline__ void copy_tile(uint32_t tile, const __nv_bfloat16* __
 // pa_reorder): every tile is 128 contiguous rows, loaded with two TMA tiled
 // boxes (one per 64-column half) by one lane.  Otherwise q, k, v are in the
 // natural order and the copy warps gather the rows with cp.async.
-template <bool kTma>
+// kComp: PASA's compensation from the block means k_pool, v_pool
+// ([B*heads, NB, d]): float (rounded to bf16 by the loader warps), or, with
+// pool_bf16, already bf16 and loaded like the kept tiles (map_kp, map_vp
+// over the [B*heads*NB, d] rows; rows past a head's NB belong to the next
+// head and are masked like the blocks past NB, rows past the array's end
+// read as zero).
+template <bool kTma, bool kComp>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                       const __grid_constant__ CUtensorMap map_k,
                       const __grid_constant__ CUtensorMap map_v,
+                      const __grid_constant__ CUtensorMap map_kp,
+                      const __grid_constant__ CUtensorMap map_vp,
                       const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                       const __nv_bfloat16* __restrict__ v, const __grid_constant__ Grid g,
                       const int32_t* __restrict__ idx, const int32_t* __restrict__ counts,
                       int k_max, float scale_log2, __nv_bfloat16* __restrict__ out,
-                      int32_t* __restrict__ status, const StallTest st) {
+                      int32_t* __restrict__ status, const StallTest st,
+                      const void* __restrict__ k_pool, const void* __restrict__ v_pool,
+                      int pool_bf16) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // the operand tiles need 1024-byte alignment (the swizzle pattern repeats
   // every 8 rows of 128 bytes); dynamic shared memory starts at the window
@@ -220,13 +299,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       *bad_flag = 1;
       report(status, PA_ERR_DEVICE_CHECK);
     }
+    if constexpr (kComp) {
+      uint32_t* bits = reinterpret_cast<uint32_t*>(gbase + kOffBits);
+      for (int x = lane; x < kCompMaxNB / 32; x += 32) bits[x] = 0u;
+      __syncwarp();
+      if (!__any_sync(0xffffffffu, bad))  // a malformed list is never used
+        for (int e = lane; e < cnt; e += 32) {
+          const int jb = __ldg(ids + e);
+          atomicOr(bits + (jb >> 5), 1u << (jb & 31));
+        }
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const bool run = *bad_flag == 0 && !expired;
-  const int n_tiles = run ? cnt : 0;
+  const int n_pool = kComp ? (g.NB + kBlock - 1) / kBlock : 0;  // pooled tiles
+  const int n_tiles = run ? cnt + n_pool : 0;
   const __nv_bfloat16* qh = q + bh * (int64_t)g.N * kD;
   const __nv_bfloat16* kh = k + bh * (int64_t)g.N * kD;
   const __nv_bfloat16* vh = v + bh * (int64_t)g.N * kD;
@@ -256,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int kb_lane = 0;  // kept index j0 + lane of the current chunk of 32
         for (int j = 0; j < n_tiles; ++j) {
           const int s = j % kStages;
-          if ((j & 31) == 0) kb_lane = j + lane < n_tiles ? __ldg(ids + j + lane) : 0;
+          if ((j & 31) == 0) kb_lane = j + lane < cnt ? __ldg(ids + j + lane) : 0;
           const int kb = __shfl_sync(0xffffffffu, kb_lane, j & 31);
           // the stage is free once QK^T (K) or P V (V) of tile j-3 completed
           if (j >= kStages && !warp_wait(is_k ? qk_done(j - kStages) : pv_done(j - kStages),
@@ -265,6 +355,44 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t full = bar((is_k ? BK0 : BV0) + s);
           if (!is_k && j == st.tile && i == st.cta_x && bh == st.cta_y) {
             issued = j + 1;  // test hook: this tile never arrives
+            continue;
+          }
+          if (kComp && j >= cnt) {
+            const int p0 = (j - cnt) * kBlock;  // first pooled block of the tile
+            if (pool_bf16) {
+              // bf16 block means: 128 contiguous rows, like a kept tile
+              if constexpr (kTma) {
+                if (lane == 0) {
+                  const CUtensorMap* pmap = is_k ? &map_kp : &map_vp;
+                  const int prow = (int)(bh * g.NB) + p0;
+                  mbar_arrive_tx(full, kTile);
+                  tma_load_2d(ring + s * kTile, pmap, 0, prow, full);
+                  tma_load_2d(ring + s * kTile + kHalf, pmap, 64, prow, full);
+                }
+              } else {
+                copy_rows(ring + s * kTile,
+                          static_cast<const __nv_bfloat16*>(is_k ? k_pool : v_pool),
+                          bh * (int64_t)g.NB + p0, g.NB - p0, lane);
+                cp_async_arrive(full);
+              }
+            } else {
+              // float block means, converted by this warp's generic stores;
+              // ordered after the stage's previous async-proxy reads and
+              // before the tensor core's
+              fence_async_smem();
+              pool_tile(gbase + (ring - base) + s * kTile,
+                        static_cast<const float*>(is_k ? k_pool : v_pool) +
+                            bh * (int64_t)g.NB * kD,
+                        p0, g.NB, lane);
+              fence_async_smem();
+              __syncwarp();
+              if (kTma) {
+                if (lane == 0) mbar_arrive(full);
+              } else {
+                mbar_arrive(full);
+              }
+            }
+            issued = j + 1;
             continue;
           }
           if constexpr (kTma) {
@@ -388,19 +516,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     // last block of the head
     const int tail_keys = g.N - (g.NB - 1) * kBlock;
     const bool ragged_last =
-        n_tiles > 0 && tail_keys < kBlock && __ldg(ids + n_tiles - 1) == g.NB - 1;
+        run && cnt > 0 && tail_keys < kBlock && __ldg(ids + cnt - 1) == g.NB - 1;
+    // pooled tiles: a full block's weight 2^7 enters as +7 in the exponent
+    // (log2 units); the ragged last block's as log2(tail_keys), i.e. a raw
+    // score offset d_last relative to the full blocks'
+    const float lb_full = kComp ? log2f((float)kBlock) : 0.f;
+    const float d_last =
+        kComp ? (log2f((float)tail_keys) - log2f((float)kBlock)) / scale_log2 : 0.f;
     float m_mine = -INFINITY, l = 0.f;  // this group's row sum, relative to m_mine
-    bool ok = true;
-    for (int t = 0;; ++t) {
-      const int j = 2 * t + grp;
-      if (j >= n_tiles) break;
-      if (!warp_wait(qk_done(j), ring_par(j), ctl)) { ok = false; break; }
+    // the group's tiles: the kept ones, then (kComp) the pooled ones, in two
+    // loops so that the hot one carries no pooled-tile code
+    auto step = [&](int j, auto pooled) -> bool {
+      if (!warp_wait(qk_done(j), ring_par(j), ctl)) return false;
       tc_fence_after();
       uint32_t sr[128];
       tmem_ld128(lane_addr + s_col, sr);
       tc_fence_before();
       mbar_arrive(bar(BSF0 + grp));  // S_grp may take QK^T two tiles ahead
-      if (ragged_last && j == n_tiles - 1) {  // warp-uniform
+      float bias = 0.f;  // added to every score of the tile in log2 units
+      if constexpr (decltype(pooled)::value) {
+        // pooled tile: column c is key block p0 + c, used unless it is kept
+        // or past NB (p0 is a multiple of 128 and p0 + 127 < 4096: four
+        // whole bitset words); every used column's weight is 2^7 (bias),
+        // the ragged last block's tail_keys (d_last on its score)
+        const uint32_t* bits = reinterpret_cast<const uint32_t*>(gbase + kOffBits);
+        const int p0 = (j - cnt) * kBlock;
+        uint32_t uw[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const int n_in = g.NB - (p0 + 32 * x);  // blocks of this word below NB
+          const uint32_t valid = n_in >= 32 ? ~0u : (n_in <= 0 ? 0u : (1u << n_in) - 1u);
+          uw[x] = ~bits[(p0 >> 5) + x] & valid;
+        }
+        bias = lb_full;
+        const int c_last = g.NB - 1 - p0;
+        if (tail_keys < kBlock && c_last < kBlock) {  // warp-uniform
+#pragma unroll
+          for (int c = 0; c < kBlock; ++c) {
+            const float sv = __uint_as_float(sr[c]) + (c == c_last ? d_last : 0.f);
+            sr[c] = (uw[c >> 5] >> (c & 31)) & 1u ? __float_as_uint(sv)
+                                                   : __float_as_uint(-INFINITY);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < kBlock; ++c)
+            if (!((uw[c >> 5] >> (c & 31)) & 1u)) sr[c] = __float_as_uint(-INFINITY);
+        }
+      } else if (ragged_last && j == cnt - 1) {  // warp-uniform
 #pragma unroll
         for (int c = 0; c < kBlock; ++c)
           if (c >= tail_keys) sr[c] = __float_as_uint(-INFINITY);
@@ -421,25 +583,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             mp[u] = fmaxf(mp[u], __uint_as_float(sr[c + u]));
       const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]),
                              fmaxf(mp[6], mp[7])) *
-                       scale_log2;
+                           scale_log2 +
+                       bias;
       // the reference after tile j-1 (published by the other group), then
       // this tile's: kept unless this tile's max exceeds it by more than 2^8
       float m_prev = -INFINITY;
       if (j >= 1) {
-        if (!warp_wait(bar(BMX0 + (grp ^ 1)), ((j - 1) >> 1) & 1, ctl)) { ok = false; break; }
+        if (!warp_wait(bar(BMX0 + (grp ^ 1)), ((j - 1) >> 1) & 1, ctl)) return false;
         m_prev = mref[(grp ^ 1) * 128 + r];
       }
+      // (a pooled tile whose blocks are all kept has mx = -inf and keeps
+      // the reference)
       const float m_j = (m_prev == -INFINITY || mx > m_prev + kRescaleLog2) ? mx : m_prev;
       mref[grp * 128 + r] = m_j;
       mbar_arrive(bar(BMX0 + grp));  // release: the store above is visible to the waiter
       if (m_mine != -INFINITY) l *= ex2(m_mine - m_j);  // this group's sum, to m_j
       m_mine = m_j;
       // the group's P buffer is free once P V of its previous tile completed
-      if (j >= 2 && !warp_wait(pv_done(j - 2), ring_par(j - 2), ctl)) { ok = false; break; }
+      if (j >= 2 && !warp_wait(pv_done(j - 2), ring_par(j - 2), ctl)) return false;
       tc_fence_after();
       // P = 2^(s*scale - m_j) as bf16 pairs into the group's P buffer; row
       // sum in 8 chains
-      const float neg_m = -m_j;
+      const float neg_m = (m_j == -INFINITY ? 0.f : -m_j) + bias;
       float rs[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) rs[u] = 0.f;
@@ -463,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P V(j) once that MMA completed (rare: the reference moved)
       const bool need = m_prev != -INFINITY && m_j != m_prev;
       if (__any_sync(0xffffffffu, need)) {
-        if (!warp_wait(pv_done(j - 1), ring_par(j - 1), ctl)) { ok = false; break; }
+        if (!warp_wait(pv_done(j - 1), ring_par(j - 1), ctl)) return false;
         tc_fence_after();
         const float alpha = need ? ex2(m_prev - m_j) : 1.f;
 #pragma unroll 1
@@ -477,7 +642,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(bar(BP0 + grp));
-    }
+      return true;
+    };
+    bool ok = true;
+    int jg = grp;
+    for (; ok && jg < n_tiles && (!kComp || jg < cnt); jg += 2) ok = step(jg, std::false_type{});
+    if constexpr (kComp)
+      for (; ok && jg < n_tiles; jg += 2) ok = step(jg, std::true_type{});
     // ---- epilogue: add the groups' row sums (each relative to its own
     // latest reference; O is relative to the last tile's, the larger), then
     // group g writes output columns 64g .. 64g+63 of the row at the natural
@@ -485,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int p = i * kBlock + r;
     __nv_bfloat16* orow = p < g.N ? out + (bh * (int64_t)g.N + natural_index(g, order, p)) * kD
                                   : nullptr;
-    if (run && cnt == 0) {
+    if (run && n_tiles == 0) {
       if (orow != nullptr)
         for (int c = 0; c < 8; ++c)
           reinterpret_cast<uint4*>(orow + grp * 64)[c] = make_uint4(0, 0, 0, 0);
@@ -537,20 +708,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <bool kTma>
+template <bool kTma, bool kComp>
 cudaError_t launch_typed(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                         const void* q, const void* k, const void* v, const Grid& g,
-                         const int32_t* idx, const int32_t* counts, int k_max, void* out,
-                         int32_t* status, cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel<kTma>,
+                         const CUtensorMap& mkp, const CUtensorMap& mvp, const void* q,
+                         const void* k, const void* v, const Grid& g, const int32_t* idx,
+                         const int32_t* counts, int k_max, void* out, int32_t* status,
+                         cudaStream_t s, const void* k_pool, const void* v_pool, int pool_bf16) {
+  if (kComp && g.NB > kCompMaxNB) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel<kTma, kComp>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)kD));
   dim3 grid(g.NB, g.B * g.heads);
-  attn_sm100_kernel<kTma><<<grid, kThreads, kSmemBytes, s>>>(
-      mq, mk, mv, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+  attn_sm100_kernel<kTma, kComp><<<grid, kThreads, kSmemBytes, s>>>(
+      mq, mk, mv, mkp, mvp, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
       static_cast<const __nv_bfloat16*>(v), g, idx, counts, k_max, scale_log2,
-      static_cast<__nv_bfloat16*>(out), status, stall_test());
+      static_cast<__nv_bfloat16*>(out), status, stall_test(), k_pool, v_pool, pool_bf16);
   return cudaGetLastError();
 }
 
@@ -565,20 +738,36 @@ cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, pa_dt
                               const Grid& g, const int32_t* idx, const int32_t* counts,
                               int k_max, const float* qs, const float* ks, const float* vs,
                               float p_levels, void* out, int32_t* status, bool permuted,
-                              cudaStream_t s) {
+                              cudaStream_t s, const void* k_pool, const void* v_pool,
+                              pa_dtype pool_dtype) {
   if (!attn_sm100_supports(dt, g)) return cudaErrorInvalidValue;
+  const bool comp = k_pool != nullptr && v_pool != nullptr;
+  if (comp && dt != PA_BF16) return cudaErrorInvalidValue;
   if (dt == PA_I8)
     return launch_attn_i8(q, k, v, g, idx, counts, k_max, qs, ks, vs, p_levels, out, status, s);
-  CUtensorMap mq{}, mk{}, mv{};
+  CUtensorMap mq{}, mk{}, mv{}, mkp{}, mvp{};
+  const int pool_bf16 = comp && pool_dtype == PA_BF16 ? 1 : 0;
+  if (pool_bf16 && permuted) {
+    const uint64_t prow = (uint64_t)g.B * g.heads * g.NB;
+    if (!encode_tile_map(&mkp, k_pool, prow, kD, 2, 64, kBlock) ||
+        !encode_tile_map(&mvp, v_pool, prow, kD, 2, 64, kBlock))
+      return cudaErrorInvalidValue;
+  }
   if (permuted) {
     const uint64_t rows = (uint64_t)g.B * g.heads * g.Np;
     if (!encode_tile_map(&mq, q, rows, kD, 2, 64, kBlock) ||
         !encode_tile_map(&mk, k, rows, kD, 2, 64, kBlock) ||
         !encode_tile_map(&mv, v, rows, kD, 2, 64, kBlock))
       return cudaErrorInvalidValue;
-    return launch_typed<true>(mq, mk, mv, q, k, v, g, idx, counts, k_max, out, status, s);
+    return comp ? launch_typed<true, true>(mq, mk, mv, mkp, mvp, q, k, v, g, idx, counts, k_max,
+                                           out, status, s, k_pool, v_pool, pool_bf16)
+                : launch_typed<true, false>(mq, mk, mv, mkp, mvp, q, k, v, g, idx, counts, k_max,
+                                            out, status, s, nullptr, nullptr, 0);
   }
-  return launch_typed<false>(mq, mk, mv, q, k, v, g, idx, counts, k_max, out, status, s);
+  return comp ? launch_typed<false, true>(mq, mk, mv, mkp, mvp, q, k, v, g, idx, counts, k_max,
+                                          out, status, s, k_pool, v_pool, pool_bf16)
+              : launch_typed<false, false>(mq, mk, mv, mkp, mvp, q, k, v, g, idx, counts, k_max,
+                                           out, status, s, nullptr, nullptr, 0);
 }
 
 }  // namespace paro

@@ -19,15 +19,25 @@ constexpr int kTopkWarps = 4;
 constexpr int kSmemOptIn = 232448;  // bytes of shared memory a CTA may opt into
 constexpr int kTopkMaxNB = kSmemOptIn / (kTopkWarps * 4);  // 14528
 
-// Sizes of one call plus the per-order index tables.  For order o (letters
-// outer -> inner, PAROAttention review: the six orders of [F, H, W]) a
-// permuted position p decomposes as p = (c_out * mid[o] + c_mid) * inn[o] +
-// c_in, and the token's natural index is c_out*so[o] + c_mid*sm[o] +
-// c_in*si[o] (natural strides: F -> H*W, H -> W, W -> 1).
+// Token orders: ids 0-5 are the six axis orders of [F, H, W] (PAROAttention
+// review), ids 6-11 SPADE's 3D tile blockings (SPADE review,
+// key_machinery (i): spatial, temporal and mixed blocking candidates): tiles
+// of tf x th x tw tokens (tf*th*tw = the block size), tiles in (f, h, w)
+// order, tokens inside a tile in (f, h, w) order, partial tiles at the far
+// edges of a grid the tile does not divide.
+constexpr int kAxisOrders = 6;
+constexpr int kOrders = 12;
+
+// Sizes of one call plus the per-order index tables.  For an axis order o
+// (letters outer -> inner) a permuted position p decomposes as p = (c_out *
+// mid[o] + c_mid) * inn[o] + c_in, and the token's natural index is
+// c_out*so[o] + c_mid*sm[o] + c_in*si[o] (natural strides: F -> H*W, H -> W,
+// W -> 1).  Tile order 6 + t has the tile shape (tf[t], th[t], tw[t]).
 struct Grid {
   int32_t B, heads, F, H, W, d, block;
   int32_t N, NB, Np;
   int32_t mid[6], inn[6], so[6], sm[6], si[6];
+  int32_t tf[6], th[6], tw[6];
   int8_t perm[kMaxHeads];
 };
 
@@ -42,12 +52,34 @@ struct StallTest {
 StallTest stall_test();  // host: the current setting
 
 __device__ __forceinline__ int natural_index(const Grid& g, int order, int p) {
-  const int inn = g.inn[order], mid = g.mid[order];
-  const int ci = p % inn;
-  const int t = p / inn;
-  const int cm = t % mid;
-  const int co = t / mid;
-  return co * g.so[order] + cm * g.sm[order] + ci * g.si[order];
+  if (order < kAxisOrders) {
+    const int inn = g.inn[order], mid = g.mid[order];
+    const int ci = p % inn;
+    const int t = p / inn;
+    const int cm = t % mid;
+    const int co = t / mid;
+    return co * g.so[order] + cm * g.sm[order] + ci * g.si[order];
+  }
+  // tile-major order: the slab of tile rows a (frames a*tf ..), the row of
+  // tiles b (heights b*th ..) inside it, the tile c (widths c*tw ..), then
+  // the token inside the (possibly partial) tile
+  const int t = order - kAxisOrders;
+  const int tf = g.tf[t], th = g.th[t], tw = g.tw[t];
+  const int HW = g.H * g.W;
+  const int a = p / (tf * HW);
+  int rem = p - a * tf * HW;
+  const int sf = min(tf, g.F - a * tf);
+  const int b = rem / (sf * th * g.W);
+  rem -= b * sf * th * g.W;
+  const int sh = min(th, g.H - b * th);
+  const int c = rem / (sf * sh * tw);
+  rem -= c * sf * sh * tw;
+  const int sw = min(tw, g.W - c * tw);
+  const int f1 = rem / (sh * sw);
+  rem -= f1 * sh * sw;
+  const int h1 = rem / sw;
+  const int w1 = rem - h1 * sw;
+  return (a * tf + f1) * HW + (b * th + h1) * g.W + c * tw + w1;
 }
 
 // First error wins; never traps.
@@ -121,6 +153,9 @@ cudaError_t launch_attn_mma(const void* q, const void* k, const void* v, pa_dtyp
                             const float* k_pool = nullptr, const float* v_pool = nullptr);
 // Selection variants (select_variants.cu)
 cudaError_t launch_sics(const void* x, pa_dtype dt, const Grid& g, float* scores, cudaStream_t s);
+cudaError_t launch_sics_pick(const float* scores, const Grid& g, int8_t* orders, cudaStream_t s);
+// y[i] = bf16(x[i]) for n floats (x, y 16-byte aligned)
+cudaError_t launch_round_bf16(const float* x, void* y, int64_t n, cudaStream_t s);
 cudaError_t launch_hybrid(const float* scores, const Grid& g, int k, double p, int w,
                           int32_t* idx, int32_t* counts, cudaStream_t s);
 // PAROAttention offline stage (paro_offline.cu)

@@ -420,4 +420,32 @@ cudaError_t launch_quantize(const void* x, pa_dtype dt, const Grid& g, int8_t* x
   return cudaErrorInvalidValue;
 }
 
+namespace {
+// y[i] = x[i] rounded to bf16 (round-to-nearest-even), 8 elements per thread.
+__global__ void round_bf16_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ y,
+                                  int64_t n) {
+  const int64_t i0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  if (i0 + 8 <= n) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(x + i0));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(x + i0) + 1);
+    uint4 w;
+    __nv_bfloat162 t;
+    t = __floats2bfloat162_rn(a.x, a.y); w.x = *reinterpret_cast<uint32_t*>(&t);
+    t = __floats2bfloat162_rn(a.z, a.w); w.y = *reinterpret_cast<uint32_t*>(&t);
+    t = __floats2bfloat162_rn(b.x, b.y); w.z = *reinterpret_cast<uint32_t*>(&t);
+    t = __floats2bfloat162_rn(b.z, b.w); w.w = *reinterpret_cast<uint32_t*>(&t);
+    *reinterpret_cast<uint4*>(y + i0) = w;
+  } else {
+    for (int64_t i = i0; i < n; ++i) y[i] = __float2bfloat16_rn(x[i]);
+  }
+}
+}  // namespace
+
+cudaError_t launch_round_bf16(const float* x, void* y, int64_t n, cudaStream_t s) {
+  const int64_t threads = (n + 7) / 8;
+  const unsigned blocks = (unsigned)((threads + 255) / 256);
+  round_bf16_kernel<<<blocks, 256, 0, s>>>(x, static_cast<__nv_bfloat16*>(y), n);
+  return cudaGetLastError();
+}
+
 }  // namespace paro

@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(kSicsThreads)
       float dg = 0.f;
 #pragma unroll
       for (int w = 0; w < kSicsThreads / 32; ++w) dg += diag_part[w];
-      atomicAdd(scores + bh * 6 + order, sq - dg);
+      atomicAdd(scores + bh * kOrders + order, sq - dg);
     }
   }
 }
@@ -262,7 +262,31 @@ __global__ void __launch_bounds__(kHybThreads)
   if (t == 0) counts[row] = cnt;
 }
 
+// One thread per head: the argmax over the candidates of the head's score
+// summed over the batch (a head has one blocking), ties to the lower id.
+__global__ void sics_pick_kernel(const float* __restrict__ scores, const __grid_constant__ Grid g,
+                                 int8_t* __restrict__ orders) {
+  const int h = blockIdx.x * blockDim.x + threadIdx.x;
+  if (h >= g.heads) return;
+  int best = 0;
+  float best_v = -INFINITY;
+  for (int o = 0; o < kOrders; ++o) {
+    float v = 0.f;
+    for (int b = 0; b < g.B; ++b) v += scores[((int64_t)b * g.heads + h) * kOrders + o];
+    if (v > best_v) {
+      best_v = v;
+      best = o;
+    }
+  }
+  orders[h] = (int8_t)best;
+}
+
 }  // namespace
+
+cudaError_t launch_sics_pick(const float* scores, const Grid& g, int8_t* orders, cudaStream_t s) {
+  sics_pick_kernel<<<(g.heads + 127) / 128, 128, 0, s>>>(scores, g, orders);
+  return cudaGetLastError();
+}
 
 size_t hybrid_smem_bytes(int nb) {
   int m = 1;
@@ -272,7 +296,7 @@ size_t hybrid_smem_bytes(int nb) {
 
 cudaError_t launch_sics(const void* x, pa_dtype dt, const Grid& g, float* scores,
                         cudaStream_t s) {
-  dim3 grid(g.NB, 6, g.B * g.heads);
+  dim3 grid(g.NB, kOrders, g.B * g.heads);
   if (dt == PA_BF16)
     sics_kernel<__nv_bfloat16><<<grid, kSicsThreads, 0, s>>>(
         static_cast<const __nv_bfloat16*>(x), g, scores);

@@ -18,13 +18,19 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libparo.so")
 
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_TIMEOUT, PA_ERR_DEVICE_CHECK = range(6)
-ABI_VERSION = 6  # the pa_abi_version() these signatures describe
+ABI_VERSION = 8  # the pa_abi_version() these signatures describe
 PA_F32, PA_BF16, PA_I8 = 0, 1, 2
 PA_ATTN_PERMUTED = 1
 PA_ATTN_P4 = 2  # with int8 inputs: 4-bit P codes (INT4 PV)
 STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_CUDA",
                 4: "PA_ERR_TIMEOUT", 5: "PA_ERR_DEVICE_CHECK"}
 ORDER_IDS = {"FHW": 0, "FWH": 1, "HFW": 2, "HWF": 3, "WFH": 4, "WHF": 5}
+# ids 6-11: 3D tile blockings (tf, th, tw) of the block size (include/paro.h)
+TILE_IDS = {128: {"T1x8x16": 6, "T1x16x8": 7, "T2x8x8": 8, "T4x4x8": 9, "T8x4x4": 10,
+                  "T16x2x4": 11},
+            64: {"T1x8x8": 6, "T1x4x16": 7, "T2x4x8": 8, "T4x4x4": 9, "T8x2x4": 10,
+                 "T16x2x2": 11}}
+N_ORDERS = 12
 
 
 class PaShape(ctypes.Structure):
@@ -65,7 +71,7 @@ def load():
         "pa_select_topk": ([_P, PaShape, _I, _P, _P], _I),
         "pa_compact_mask": ([_P, PaShape, _P, _P, _P], _I),
         "pa_select_hybrid": ([_P, PaShape, _I, ctypes.c_double, _I, _P, _P, _P], _I),
-        "pa_sics_scores": ([_P, _P, _I, PaShape, _P, _P], _I),
+        "pa_sics_scores": ([_P, _P, _I, PaShape, _P, _P, _P], _I),
         "pa_map_row_stats": ([_P, _P, PaShape, _I, _P, _P, _P, _P], _I),
         "pa_map_block_stats": ([_P, _P, PaShape, _I, _P, _P, ctypes.c_float, _P, _P, _P, _P, _P,
                                 _P], _I),
@@ -78,7 +84,8 @@ def load():
         "pa_block_sparse_attn_mma": ([_P, _P, _P, _I, ctypes.c_uint32, PaShape, _P, _P, _P, _I, _P, _P,
                                       _P], _I),
         "pa_block_sparse_attn_compensated": ([_P, _P, _P, _I, ctypes.c_uint32, PaShape, _P, _P, _P, _I,
-                                              _P, _P, _P, _P, _P], _I),
+                                              _P, _P, _I, _P, _P, _P], _I),
+        "pa_round_bf16": ([_P, _P, ctypes.c_int64, _P], _I),
     }
     lib.pa_abi_version.restype = _I
     if lib.pa_abi_version() != ABI_VERSION:
@@ -308,16 +315,21 @@ def select_hybrid(scores, pr: Problem, k: int, top_p: float, window: int, idx=No
     return idx, counts
 
 
-def sics_scores(q, k, pr: Problem, scores=None):
-    """[B,h,6] blocking scores of the six axis orders (SICS of q's and k's
-    blocks); the argmax per head is the order SPADE's rule picks."""
-    _need_cuda(q, k, scores)
+def sics_scores(q, k, pr: Problem, scores=None, orders=None):
+    """Blocking scores of the 12 candidates (six axis orders, six 3D tile
+    blockings): SICS of q's and k's blocks -> (scores [B,h,12], orders
+    [heads] int8, each head's pick by the library: the largest score summed
+    over the batch, ties to the lower id)."""
+    _need_cuda(q, k, scores, orders)
     _expect(q, "q", pr.natural, _FLOAT)
     _expect(k, "k", pr.natural, q.dtype)
-    _expect(scores, "scores", (pr.B, pr.heads, 6), torch.float32)
-    scores = scores if scores is not None else torch.empty((pr.B, pr.heads, 6), dtype=torch.float32, device=q.device)
-    _check(load().pa_sics_scores(_ptr(q), _ptr(k), _dtype_code(q), pr.shape, _ptr(scores), _stream()))
-    return scores
+    _expect(scores, "scores", (pr.B, pr.heads, N_ORDERS), torch.float32)
+    _expect(orders, "orders", (pr.heads,), torch.int8)
+    scores = scores if scores is not None else torch.empty((pr.B, pr.heads, N_ORDERS), dtype=torch.float32, device=q.device)
+    orders = orders if orders is not None else torch.empty((pr.heads,), dtype=torch.int8, device=q.device)
+    _check(load().pa_sics_scores(_ptr(q), _ptr(k), _dtype_code(q), pr.shape, _ptr(scores),
+                                 _ptr(orders), _stream()))
+    return scores, orders
 
 
 def map_row_stats(q_perm, k_perm, pr: Problem, order: int, status=None):
@@ -472,17 +484,21 @@ def block_sparse_attn_compensated(q, k, v, pr: Problem, idx, k_pool, v_pool, cou
     """Block-sparse attention in which every unselected key block still
     enters the softmax as one pooled key row (mean key, mean value, weight
     = its valid keys): PASA's grouped first-order compensation.  k_pool,
-    v_pool [B, heads, NB, d] float32 block means (from :func:`reorder` with
-    ``with_pool`` or :func:`block_score`).  bf16 or fp32 q, k, v; output
-    natural order, q's dtype."""
+    v_pool [B, heads, NB, d] block means (from :func:`reorder` with
+    ``with_pool`` or :func:`block_score`), both float32, or both bfloat16
+    (:func:`round_bf16`; bf16 q, k, v with d = block = 128 only, the faster
+    form).  bf16 or fp32 q, k, v; output natural order, q's dtype."""
     _need_cuda(q, k, v, idx, counts, k_pool, v_pool, out, status)
     _same_dtype(("q", q), ("k", k), ("v", v))
     rows = pr.permuted if permuted else pr.natural
     for name, t in (("q", q), ("k", k), ("v", v)):
         _expect(t, name, rows, _FLOAT)
     _check_lists(idx, counts, pr)
-    _expect(k_pool, "k_pool", pr.pooled, torch.float32)
-    _expect(v_pool, "v_pool", pr.pooled, torch.float32)
+    pool_dt = k_pool.dtype if k_pool is not None else torch.float32
+    if pool_dt not in (torch.float32, torch.bfloat16):
+        raise ValueError(f"k_pool dtype {pool_dt}: float32 or bfloat16")
+    _expect(k_pool, "k_pool", pr.pooled, pool_dt)
+    _expect(v_pool, "v_pool", pr.pooled, pool_dt)
     _expect(out, "out", pr.natural, q.dtype)
     _expect_status(status)
     out = out if out is not None else torch.empty((pr.B, pr.heads, pr.N, pr.d), dtype=q.dtype,
@@ -490,19 +506,35 @@ def block_sparse_attn_compensated(q, k, v, pr: Problem, idx, k_pool, v_pool, cou
     st = load().pa_block_sparse_attn_compensated(
         _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), PA_ATTN_PERMUTED if permuted else 0, pr.shape,
         pr.perms_ptr, _ptr(idx), _ptr(counts), int(idx.shape[-1]), _ptr(k_pool), _ptr(v_pool),
-        _ptr(out), _ptr(status), _stream())
+        _dtype_code(k_pool), _ptr(out), _ptr(status), _stream())
     _check(st)
     return out
 
 
+def round_bf16(x, out=None):
+    """x (float32, CUDA, contiguous) rounded to bfloat16 by the library's
+    kernel: the bf16 block means :func:`block_sparse_attn_compensated`
+    loads with the K and V tiles' copy engine."""
+    _need_cuda(x, out)
+    if x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 tensor")
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device)
+    elif out.dtype != torch.bfloat16 or out.shape != x.shape or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous bfloat16 tensor of shape {tuple(x.shape)}")
+    _check(load().pa_round_bf16(_ptr(x), _ptr(out), x.numel(), _stream()))
+    return out
+
+
 def choose_orders_sics(q, k, grid, block):
-    """SPADE's blocking choice per head: the axis order whose blocks have the
-    largest SICS of q and k (ties to the lower id) -> list of order ids."""
+    """SPADE's blocking choice per head, made by the library: the candidate
+    (axis order or 3D tile blocking) whose blocks have the largest SICS of q
+    and k -> list of order ids (copied to the host: the calls that follow
+    take the order ids as host data)."""
     B, heads = q.shape[:2]
     pr = Problem(B, heads, grid, q.shape[-1], block, [0] * heads)
-    sc = sics_scores(q, k, pr)
-    # one order per head: the batch's summed score (a head has one order)
-    return [int(o) for o in torch.argmax(sc.sum(dim=0), dim=-1).tolist()]
+    _, orders = sics_scores(q, k, pr)
+    return [int(o) for o in orders.cpu().tolist()]
 
 
 def attention(q, k, v, grid, perms, block, density, int8=False, baseline=False, status=None,
@@ -544,6 +576,9 @@ def attention(q, k, v, grid, perms, block, density, int8=False, baseline=False, 
         kp, k_pool = reorder(k, pr, with_pool=True)
         vp, v_pool = reorder(v, pr, with_pool=True)
         idx, counts = select(score_pooled(q_pool, k_pool, pr))
+        if q.dtype == torch.bfloat16 and pr.d == 128 and pr.block == 128:
+            # the tcgen05 kernel loads bf16 means like K and V tiles
+            k_pool, v_pool = round_bf16(k_pool), round_bf16(v_pool)
         out = block_sparse_attn_compensated(qp, kp, vp, pr, idx, k_pool, v_pool, counts,
                                             status=status, permuted=True)
     elif int8:

@@ -39,7 +39,11 @@ AXES = "FHW"
 
 
 def axis_order(perm_id: int) -> tuple:
-    """Axis indices (0=F, 1=H, 2=W) of an order id, outermost first."""
+    """Axis indices (0=F, 1=H, 2=W) of an order id, outermost first.  Ids
+    6-11 (3D tile blockings) walk the tokens inside a tile in F, H, W order,
+    so their innermost axis is W."""
+    if perm_id >= 6:
+        return (0, 1, 2)
     names = ("FHW", "FWH", "HFW", "HWF", "WFH", "WHF")[perm_id]
     return tuple(AXES.index(c) for c in names)
 

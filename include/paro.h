@@ -32,9 +32,15 @@
  * - Order ids (one int8 per head, HOST memory, length shape.heads, the same
  *   for every batch index): 0 FHW, 1 FWH, 2 HFW, 3 HWF, 4 WFH, 5 WHF, the
  *   letters listing the axes outermost -> innermost.  FHW is the natural
- *   flattening n = f*H*W + h*W + w.  Token n of a head sits at position
- *   pos(n) of that head's order; block i holds positions [i*block,
- *   (i+1)*block); positions >= N are zero padding.
+ *   flattening n = f*H*W + h*W + w.  Ids 6-11 are SPADE's 3D tile blockings
+ *   (SPADE review, key_machinery (i)): tiles of tf x th x tw tokens, tiles
+ *   in (f, h, w) order of their tile coordinates, tokens inside a tile in
+ *   (f, h, w) order, partial tiles at the far edges; (tf, th, tw) for
+ *   block 128: 6 (1,8,16), 7 (1,16,8), 8 (2,8,8), 9 (4,4,8), 10 (8,4,4),
+ *   11 (16,2,4); for block 64: 6 (1,8,8), 7 (1,4,16), 8 (2,4,8), 9 (4,4,4),
+ *   10 (8,2,4), 11 (16,2,2).  Token n of a head sits at position pos(n) of
+ *   that head's order; block i holds positions [i*block, (i+1)*block);
+ *   positions >= N are zero padding.
  * - Q, K, V and the attention output are [B, heads, N, d] row-major in the
  *   natural order, contiguous, device memory, base 16-byte aligned.
  *   INT8 tensors and pooled summaries are in the permuted order.
@@ -86,7 +92,7 @@ typedef struct {
   int32_t B, heads, F, H, W, d, block;
 } pa_shape;
 
-/* Version of this ABI (bumped on any signature change): 6. */
+/* Version of this ABI (bumped on any signature change): 8. */
 PA_API int32_t pa_abi_version(void);
 
 /* Message of the last failed call on this thread ("" if none). */
@@ -187,16 +193,21 @@ PA_API pa_status pa_select_hybrid(const float* scores, pa_shape shape, int32_t k
 /* Blocking-scheme score (SPADE review, key_machinery (ii): the Sum of
  * Intra-block Cosine Similarities, one pass per block by the identity
  * sum_{s != t} cos(x_s, x_t) = |sum_t xh_t|^2 - sum_t |xh_t|^2, xh = x/|x|,
- * zero rows adding nothing).  For every axis order o (0..5, the ids of the
- * order table above) and every (b,h):
- *   scores[b,h,o] = sum over the blocks of order o (runs of `block`
- *                   permuted tokens) of SICS(q's rows) + SICS(k's rows).
+ * zero rows adding nothing) of every candidate blocking (key_machinery
+ * (i): spatial, temporal and mixed 3D blockings; the ids of the order table
+ * above, 0-11: the six axis orders and the six tile blockings).  For every
+ * candidate o and every (b,h):
+ *   scores[b,h,o] = sum over the blocks of candidate o (runs of `block`
+ *                   positions of its token order) of SICS(q's rows) +
+ *                   SICS(k's rows).
  * q, k natural order [B,heads,N,d] (PA_F32 or PA_BF16), 16-byte aligned;
- * scores [B,heads,6] float, overwritten (accumulated in fp32
- * with atomics, so the last bits vary between runs).  The order with the
- * largest score is SPADE's pick for the head. */
+ * scores [B,heads,12] float, overwritten (accumulated in fp32 with atomics,
+ * so the last bits vary between runs).  orders, if not NULL, [heads] int8
+ * device memory, receives each head's pick: the candidate with the largest
+ * score summed over the batch (a head has one blocking), ties to the lower
+ * id -- SPADE's choice, to pass as the head's order id. */
 PA_API pa_status pa_sics_scores(const void* q, const void* k, pa_dtype dtype, pa_shape shape,
-                         float* scores, void* stream);
+                         float* scores, int8_t* orders, void* stream);
 
 /* PAROAttention's offline stage (PAROAttention review, key_machinery: the
  * per-head order is chosen offline by a metric balancing block
@@ -351,17 +362,35 @@ PA_API pa_status pa_block_sparse_attn_mma(const void* q, const void* k, const vo
  * Arguments, layouts, ownership and errors as pa_block_sparse_attn_mma
  * (dtype PA_F32 or PA_BF16, flags 0 or PA_ATTN_PERMUTED; k_max = 0 is
  * allowed and gives the compensation alone), plus:
- *   k_pool, v_pool  [B,heads,NB,d] float, 16-byte aligned, read only: the
+ *   k_pool, v_pool  [B,heads,NB,d], 16-byte aligned, read only: the
  *                   means of the valid rows of each permuted block of k and
- *                   v (the pool output of pa_reorder or pa_block_score).
- * Runs on the mma.sync kernel (pooled blocks are rounded to bf16 like the
- * K and V tiles).  NB <= 4096 (PA_ERR_UNSUPPORTED above). */
+ *                   v (the pool output of pa_reorder or pa_block_score),
+ *                   element type pool_dtype.
+ *   pool_dtype      PA_F32, or PA_BF16 for the same means rounded to bf16
+ *                   (pa_round_bf16); PA_BF16 needs the tcgen05 kernel
+ *                   (PA_ERR_UNSUPPORTED otherwise).
+ * PA_BF16 with d = 128 and block = 128 runs on the tcgen05 kernel: after a
+ * row's kept tiles come ceil(NB/128) tiles of pooled key rows (128 blocks'
+ * means each), in the same online softmax; float means are rounded to bf16
+ * by the kernel's loader warps, bf16 means are loaded like the K and V
+ * tiles (the faster form).  Other shapes and PA_F32 run on the mma.sync
+ * kernel, which rounds pooled blocks to bf16 like the K and V tiles.
+ * NB <= 4096 (PA_ERR_UNSUPPORTED above: the kept list is held as one bit
+ * per block in shared memory). */
 PA_API pa_status pa_block_sparse_attn_compensated(const void* q, const void* k, const void* v,
                                            pa_dtype dtype, uint32_t flags, pa_shape shape,
                                            const int8_t* perms, const int32_t* idx,
                                            const int32_t* counts, int32_t k_max,
-                                           const float* k_pool, const float* v_pool, void* out,
+                                           const void* k_pool, const void* v_pool,
+                                           pa_dtype pool_dtype, void* out,
                                            int32_t* dev_status, void* stream);
+
+/* y[i] = x[i] rounded to bf16 (round to nearest even) for i < n: the bf16
+ * block means that pa_block_sparse_attn_compensated takes with pool_dtype
+ * PA_BF16.  x: n floats, y: n bf16, device memory, 16-byte aligned, not
+ * overlapping; n = 0 does nothing.  Not an operation of the pages: a
+ * storage conversion, so that the attention kernel moves 2-byte means. */
+PA_API pa_status pa_round_bf16(const float* x, void* y, int64_t n, void* stream);
 
 #ifdef __cplusplus
 }

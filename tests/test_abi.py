@@ -34,7 +34,7 @@ def test_exports_every_declared_symbol(lib):
     assert len(names) >= 12
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.pa_abi_version() == paro.ABI_VERSION == 6
+    assert lib.pa_abi_version() == paro.ABI_VERSION == 8
 
 
 def test_k_for_density_matches_oracle(lib):
@@ -72,9 +72,11 @@ def test_host_validation(lib):
     # wrong dtype for reorder
     assert lib.pa_reorder(FAKE, FAKE, paro.PA_I8, good, pp, None, None) == paro.PA_ERR_INVALID_ARG
     # bad order id
-    keep2, bad = perms_of(0, 6)
+    keep2, bad = perms_of(0, 12)  # ids 0-11 are valid (axis orders, tile blockings)
     assert lib.pa_reorder(FAKE, FAKE, paro.PA_BF16, good, bad, None, None) == paro.PA_ERR_INVALID_ARG
-    assert b"perms[1]=6" in lib.pa_last_error()
+    assert b"perms[1]=12" in lib.pa_last_error()
+    keep3, neg = perms_of(-1, 0)
+    assert lib.pa_reorder(FAKE, FAKE, paro.PA_BF16, good, neg, None, None) == paro.PA_ERR_INVALID_ARG
     # NULL perms / pointers / misaligned pointers
     assert lib.pa_reorder(FAKE, FAKE, paro.PA_BF16, good, None, None, None) == paro.PA_ERR_INVALID_ARG
     assert lib.pa_reorder(None, FAKE, paro.PA_BF16, good, pp, None, None) == paro.PA_ERR_INVALID_ARG
@@ -121,8 +123,8 @@ def test_selection_variant_validation(lib):
     big = paro.PaShape(1, 1, 1, 1, 4097 * 64, 64, 64)  # NB = 4097
     assert lib.pa_select_hybrid(FAKE, big, 2, 0.5, 1, FAKE, FAKE, None) == paro.PA_ERR_UNSUPPORTED
     # SICS: float inputs only, non-null buffers
-    assert lib.pa_sics_scores(FAKE, FAKE, paro.PA_I8, good, FAKE, None) == paro.PA_ERR_INVALID_ARG
-    assert lib.pa_sics_scores(FAKE, None, paro.PA_BF16, good, FAKE, None) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_sics_scores(FAKE, FAKE, paro.PA_I8, good, FAKE, None, None) == paro.PA_ERR_INVALID_ARG
+    assert lib.pa_sics_scores(FAKE, None, paro.PA_BF16, good, FAKE, None, None) == paro.PA_ERR_INVALID_ARG
 
 
 def test_p4_flag_validation(lib):
@@ -154,23 +156,42 @@ def test_compensated_attention_validation(lib):
     keep, pp = perms_of(0, 5)
     fn = lib.pa_block_sparse_attn_compensated
     # the pooled summaries are required and 16-byte aligned
-    assert fn(FAKE, FAKE, FAKE, paro.PA_BF16, 0, good, pp, FAKE, None, 2, None, FAKE, FAKE, None,
+    assert fn(FAKE, FAKE, FAKE, paro.PA_BF16, 0, good, pp, FAKE, None, 2, None, FAKE, paro.PA_F32, FAKE, None,
               None) == paro.PA_ERR_INVALID_ARG
     assert b"k_pool" in lib.pa_last_error()
     assert fn(FAKE, FAKE, FAKE, paro.PA_BF16, 0, good, pp, FAKE, None, 2, FAKE,
-              ctypes.c_void_p(4100), FAKE, None, None) == paro.PA_ERR_INVALID_ARG
+              ctypes.c_void_p(4100), paro.PA_F32, FAKE, None, None) == paro.PA_ERR_INVALID_ARG
     # bf16 / fp32 only, no INT4 flag, k_max within [0, NB]
-    assert fn(FAKE, FAKE, FAKE, paro.PA_I8, 0, good, pp, FAKE, None, 2, FAKE, FAKE, FAKE, None,
+    assert fn(FAKE, FAKE, FAKE, paro.PA_I8, 0, good, pp, FAKE, None, 2, FAKE, FAKE, paro.PA_F32, FAKE, None,
               None) == paro.PA_ERR_INVALID_ARG
-    assert fn(FAKE, FAKE, FAKE, paro.PA_BF16, paro.PA_ATTN_P4, good, pp, FAKE, None, 2, FAKE, FAKE,
+    assert fn(FAKE, FAKE, FAKE, paro.PA_BF16, paro.PA_ATTN_P4, good, pp, FAKE, None, 2, FAKE, FAKE, paro.PA_F32,
               FAKE, None, None) == paro.PA_ERR_INVALID_ARG
-    assert fn(FAKE, FAKE, FAKE, paro.PA_BF16, 0, good, pp, FAKE, None, 5, FAKE, FAKE, FAKE, None,
+    assert fn(FAKE, FAKE, FAKE, paro.PA_BF16, 0, good, pp, FAKE, None, 5, FAKE, FAKE, paro.PA_F32, FAKE, None,
               None) == paro.PA_ERR_INVALID_ARG
     # one bit per key block in shared memory: NB <= 4096
     big = paro.PaShape(1, 2, 65, 64, 64, 64, 64)  # NB = 4160
-    assert fn(FAKE, FAKE, FAKE, paro.PA_BF16, 0, big, pp, FAKE, None, 2, FAKE, FAKE, FAKE, None,
+    assert fn(FAKE, FAKE, FAKE, paro.PA_BF16, 0, big, pp, FAKE, None, 2, FAKE, FAKE, paro.PA_F32, FAKE, None,
               None) == paro.PA_ERR_UNSUPPORTED
     assert b"4096" in lib.pa_last_error()
+    # the means are float or bf16; bf16 means need the tcgen05 kernel (d = 128,
+    # block = 128, PA_BF16), so this d = 64 shape is unsupported
+    assert fn(FAKE, FAKE, FAKE, paro.PA_BF16, 0, good, pp, FAKE, None, 2, FAKE, FAKE, paro.PA_I8,
+              FAKE, None, None) == paro.PA_ERR_INVALID_ARG
+    assert fn(FAKE, FAKE, FAKE, paro.PA_BF16, 0, good, pp, FAKE, None, 2, FAKE, FAKE,
+              paro.PA_BF16, FAKE, None, None) == paro.PA_ERR_UNSUPPORTED
+    assert b"tcgen05" in lib.pa_last_error()
+    wide = paro.PaShape(1, 2, 4, 8, 16, 128, 128)
+    assert fn(FAKE, FAKE, FAKE, paro.PA_F32, 0, wide, pp, FAKE, None, 2, FAKE, FAKE,
+              paro.PA_BF16, FAKE, None, None) == paro.PA_ERR_UNSUPPORTED
+
+
+def test_round_bf16_validation(lib):
+    fn = lib.pa_round_bf16
+    assert fn(None, None, 0, None) == paro.PA_OK  # nothing to do
+    assert fn(FAKE, FAKE, -1, None) == paro.PA_ERR_INVALID_ARG
+    assert fn(None, FAKE, 8, None) == paro.PA_ERR_INVALID_ARG
+    assert fn(FAKE, ctypes.c_void_p(4100), 8, None) == paro.PA_ERR_INVALID_ARG
+    assert b"aligned" in lib.pa_last_error()
 
 
 def test_topk_nb_limit_is_reported(lib):
@@ -254,6 +275,15 @@ def test_binding_rejects_bad_shapes(host_binding):
         lambda: paro.block_sparse_attn_compensated(nat, nat, nat, pr_r, idx,
                                                    torch.zeros((1, 2, 2, 64)),
                                                    torch.zeros(pr_r.pooled)),
+        # k_pool and v_pool of different dtypes, or an integer dtype
+        lambda: paro.block_sparse_attn_compensated(nat, nat, nat, pr_r, idx,
+                                                   torch.zeros(pr_r.pooled, dtype=torch.bfloat16),
+                                                   torch.zeros(pr_r.pooled)),
+        lambda: paro.block_sparse_attn_compensated(nat, nat, nat, pr_r, idx,
+                                                   torch.zeros(pr_r.pooled, dtype=torch.int32),
+                                                   torch.zeros(pr_r.pooled, dtype=torch.int32)),
+        lambda: paro.round_bf16(torch.zeros(8, dtype=torch.bfloat16)),
+        lambda: paro.round_bf16(torch.zeros(8), out=torch.zeros(8, dtype=torch.bfloat16)[:4]),
     ]
     for i, call in enumerate(bad):
         with pytest.raises(ValueError):
@@ -279,6 +309,10 @@ def test_binding_passes_good_shapes_to_the_library(host_binding):
         lambda: paro.block_sparse_attn_compensated(perm, perm, perm, pr_r, idx,
                                                    torch.zeros(pr_r.pooled),
                                                    torch.zeros(pr_r.pooled), permuted=True),
+        lambda: paro.block_sparse_attn_compensated(
+            perm, perm, perm, pr_r, idx, torch.zeros(pr_r.pooled, dtype=torch.bfloat16),
+            torch.zeros(pr_r.pooled, dtype=torch.bfloat16), permuted=True),
+        lambda: paro.round_bf16(torch.zeros(8)),
     ]
     for call in good:
         with pytest.raises(AssertionError, match="library call"):

@@ -46,6 +46,8 @@ TC_CASES = [
     custom("ragged_780", 2, 3, 128, (6, 10, 13), 128, "bf16", 0.6, perms=(5, 2, 4)),
     custom("multi_tile_2048", 1, 2, 128, (8, 16, 16), 128, "bf16", 0.75, perms=(3, 1)),
     custom("dense_780", 1, 2, 128, (6, 10, 13), 128, "bf16", 1.0, perms=(4, 0)),
+    # 3D tile blockings (ids 6-11) on a grid no tile divides
+    custom("tiles_1800", 1, 6, 128, (5, 18, 20), 128, "bf16", 0.5, perms=(6, 7, 8, 9, 10, 11)),
 ]
 
 

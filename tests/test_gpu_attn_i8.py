@@ -35,6 +35,7 @@ CASES = [
     custom("ragged_780", 2, 3, 128, (6, 10, 13), 128, "bf16", 0.6, perms=(5, 2, 4)),
     custom("multi_tile_2048", 1, 2, 128, (8, 16, 16), 128, "bf16", 0.75, perms=(3, 1)),
     custom("dense_780", 1, 2, 128, (6, 10, 13), 128, "bf16", 1.0, perms=(4, 0)),
+    custom("tiles_1800", 1, 3, 128, (5, 18, 20), 128, "bf16", 0.5, perms=(6, 8, 10)),
 ]
 
 
@@ -70,7 +71,7 @@ def oracle_int8(w, perms, host, idx, counts=None, p_levels=127, mode="tile"):
                                             sv[b, h], w.N, w.block, idx[b, h],
                                             None if counts is None else counts[b, h],
                                             p_levels=p_levels, mode=mode)
-    return ref.inverse_reorder(outp, (w.F, w.H, w.W), perms)
+    return ref.inverse_reorder(outp, (w.F, w.H, w.W), perms, w.block)
 
 
 def run_i8(pr, dev, idx, counts=None, out=None, p4=False):

@@ -16,11 +16,15 @@ from helpers import custom, inputs, to_dev
 
 pytestmark = pytest.mark.gpu
 
-# small grids with ragged tails, every order, both dtypes and head dims
+# small grids with ragged tails, every order (axis orders and tile
+# blockings), both dtypes and head dims
 CASES = [
     custom("ragged_f32", 1, 6, 64, (3, 5, 7), 64, "f32", 0.5, perms=(0, 1, 2, 3, 4, 5)),
     custom("ragged_bf16", 2, 6, 128, (5, 7, 9), 128, "bf16", 0.5, perms=(5, 4, 3, 2, 1, 0)),
     custom("ragged_bf16_b64", 1, 3, 128, (2, 9, 11), 64, "bf16", 0.5, perms=(1, 3, 5)),
+    # the 3D tile blockings (ids 6-11), ragged edges, both block sizes
+    custom("tiles_bf16", 1, 6, 128, (5, 18, 20), 128, "bf16", 0.5, perms=(6, 7, 8, 9, 10, 11)),
+    custom("tiles_f32_b64", 2, 6, 64, (19, 6, 11), 64, "f32", 0.5, perms=(11, 10, 9, 8, 7, 6)),
     WORKLOADS["tiny_4x8x8"],
     WORKLOADS["small_8x16x16"],
 ]
