@@ -197,7 +197,7 @@ def percentiles(xs):
 
 def attn_kernel_name(pipe) -> str:
     if pipe.int8:
-        return "attn_i8_kernel"
+        return "attn_i8_kernel<tile>" if pipe.p_tile else "attn_i8_kernel"
     return "attn_mma_kernel" if pipe.baseline else "attn_sm100_kernel"
 
 
@@ -471,15 +471,23 @@ def run_sweep(a):
     if a.pasa_only:
         run_sweep_pasa(device, peaks, peak_src, a.heads)
         return
-    for name, w in ([] if a.selection_only else WORKLOADS.items()):
+    names = a.sweep_workloads.split(",") if a.sweep_workloads else list(WORKLOADS)
+    for name in ([] if a.selection_only else names):
+        w = WORKLOADS[name]
         q, k, v, perms = make_inputs(w)
         qkv = [t.to(device) for t in (q, k, v)]
-        for precision in (["bf16", "int8", "int4pv"] if w.int8 else [w.dtype]):
-            int8 = precision in ("int8", "int4pv")
-            pipe = make_pipeline(w, perms, w.density, a.kernel, device, int8=int8)
-            if precision == "int4pv":
+        # int8: one-pass P (fixed scale 1/127); int8_tile: normalised P with a
+        # scale per tile (two passes); int4pv: 4-bit P and V, tile reading
+        # (two passes); int4pv_onepass: the one-pass 4-bit form
+        precisions = ["bf16", "int8", "int8_tile", "int4pv", "int4pv_onepass"]
+        for precision in (precisions if w.int8 else [w.dtype]):
+            int8 = precision != "bf16" and precision != w.dtype
+            if int8:
                 pipe = Pipeline(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, perms, w.density,
-                                device=device, int4_pv=True)
+                                device=device, int8=True, int4_pv=precision.startswith("int4"),
+                                p_tile=precision in ("int8_tile", "int4pv"))
+            else:
+                pipe = make_pipeline(w, perms, w.density, a.kernel, device, int8=False)
             for _ in range(10):
                 step(pipe, qkv)
             torch.cuda.synchronize()
@@ -514,9 +522,11 @@ def run_sweep(a):
             }), flush=True)
             del pipe
         del qkv
+    if a.sweep_workloads:
+        return
     run_sweep_selection(device, peaks, peak_src, a.heads)
     run_sweep_offline(device, peaks, peak_src, a.heads)
-    if not a.selection_only:
+    if not a.selection_only and not a.sweep_workloads:
         run_sweep_pasa(device, peaks, peak_src, a.heads)
 
 
@@ -771,6 +781,8 @@ def main(argv=None):
                     help="per-workload latency percentiles, one JSON line per workload")
     ap.add_argument("--selection-only", action="store_true",
                     help="with --sweep: only the selection-variant lines")
+    ap.add_argument("--sweep-workloads", default="",
+                    help="with --sweep: comma-separated workload names (default: all)")
     ap.add_argument("--pasa-only", action="store_true",
                     help="with --sweep: only the PASA compensation line")
     ap.add_argument("--no-dense", action="store_true")

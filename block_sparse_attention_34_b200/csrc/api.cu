@@ -395,8 +395,10 @@ static pa_status attn_common(const void* q, const void* k, const void* v, pa_dty
   if (dtype == PA_I8) {
     PA_REQUIRE(q_scale && k_scale && v_scale, "INT8 attention needs q_scale, k_scale, v_scale");
   }
-  PA_REQUIRE((flags & ~(PA_ATTN_PERMUTED | PA_ATTN_P4)) == 0, "unknown flags 0x%x", flags);
+  PA_REQUIRE((flags & ~(PA_ATTN_PERMUTED | PA_ATTN_P4 | PA_ATTN_P_TILE)) == 0,
+             "unknown flags 0x%x", flags);
   PA_REQUIRE(!(flags & PA_ATTN_P4) || dtype == PA_I8, "PA_ATTN_P4 needs dtype PA_I8");
+  PA_REQUIRE(!(flags & PA_ATTN_P_TILE) || dtype == PA_I8, "PA_ATTN_P_TILE needs dtype PA_I8");
   const float p_levels = (flags & PA_ATTN_P4) ? 7.f : 127.f;
   const bool permuted = dtype == PA_I8 || (flags & PA_ATTN_PERMUTED) != 0;
   cudaStream_t s = (cudaStream_t)stream;
@@ -410,7 +412,10 @@ static pa_status attn_common(const void* q, const void* k, const void* v, pa_dty
                        "pa_block_sparse_attn memset");
   }
   cudaError_t e;
-  if (sm100)
+  if (dtype == PA_I8)
+    e = paro::launch_attn_i8(q, k, v, g, idx, counts, k_max, q_scale, k_scale, v_scale, p_levels,
+                             (flags & PA_ATTN_P_TILE) != 0, out, dev_status, s);
+  else if (sm100)
     e = paro::launch_attn_sm100(q, k, v, dtype, g, idx, counts, k_max, q_scale, k_scale, v_scale,
                                 p_levels, out, dev_status, permuted, s);
   else

@@ -743,8 +743,7 @@ cudaError_t launch_attn_sm100(const void* q, const void* k, const void* v, pa_dt
   if (!attn_sm100_supports(dt, g)) return cudaErrorInvalidValue;
   const bool comp = k_pool != nullptr && v_pool != nullptr;
   if (comp && dt != PA_BF16) return cudaErrorInvalidValue;
-  if (dt == PA_I8)
-    return launch_attn_i8(q, k, v, g, idx, counts, k_max, qs, ks, vs, p_levels, out, status, s);
+  if (dt == PA_I8) return cudaErrorInvalidValue;  // launch_attn_i8
   CUtensorMap mq{}, mk{}, mv{}, mkp{}, mvp{};
   const int pool_bf16 = comp && pool_dtype == PA_BF16 ? 1 : 0;
   if (pool_bf16 && permuted) {

@@ -17,6 +17,17 @@
 // [-7, 7] from pa_quantize_int4; the integer MMAs are unchanged)
 // and O / l is stored at the natural positions of the block's tokens.
 //
+// kTwoPass: the post-softmax map is quantised per tile after it
+// is normalised, each tile with its own scale.  Pass 1 runs Q K^T over the
+// kept tiles for the exact row max m and sum l (each 64-column half keeps
+// its own pair, merged once); pass 2 runs Q K^T again and, per tile,
+//   P      = 2^(S log2 e - m) / l             (the normalised map)
+//   a      = max of P over the tile's valid rows and keys (shared by the
+//            eight softmax warps through shared memory)
+//   P8     = round_half_even(L P / a)           (L = 127, or 7 for 4 bits)
+//   O      = O + (P8 V8_j, exact int32) * (a / L) s_v[j]
+// so O needs no rescale and no final division.
+//
 // One CTA per (query block, head); 14 warps in four roles:
 //   warps 0-7   softmax: warp w serves tile rows 32 (w & 3) .. +31 (its
 //               TMEM lane quarter) and S columns 64 (w >> 2) .. +63.  Per
@@ -86,6 +97,7 @@ constexpr int kCorrThreads = 4 * 32;
 constexpr int kScaleSlots = 4;
 constexpr uint32_t kTile = kBlock * kD;  // 16 KB: one 128-byte-swizzled panel
 constexpr uint32_t kOffBar = 0;
+constexpr uint32_t kOffAmx = 384;  // kTwoPass: per-warp tile maxima [2 parity][8 warps] f32
 constexpr uint32_t kOffSlot = 512;
 constexpr uint32_t kOffX = 1024;   // row-max exchange [2 parity][2 half][128] f32
 constexpr uint32_t kOffA = 3072;   // rescale factor alpha [4 slots][128] f32
@@ -118,9 +130,12 @@ enum : uint32_t {
   BX0 = BPVF0 + 2,        // row-max exchange of lane quarter q (4)
   BL = BX0 + 4,           // final row sums written
   BDRAIN,
-  NBAR
+  BMG,                    // kTwoPass: pass-1 half statistics written
+  BAM0,                   // kTwoPass: warp maxima of tile j written, slot j & 1 (2)
+  NBAR = BAM0 + 2
 };
-static_assert(NBAR * 8 <= kOffSlot, "barrier region");
+static_assert(NBAR * 8 <= kOffAmx, "barrier region");
+static_assert(kOffAmx + 16 * 4 <= kOffSlot, "tile maxima region");
 
 // float of an int32 |x| < 2^22 held in the bits of a 32-bit register (two
 // such values at once: the subtraction is one paired instruction)
@@ -160,6 +175,26 @@ __device__ __forceinline__ void tile_exp(const uint32_t (&sr)[64], float2 cq2, f
   }
 }
 
+// Largest int32 score among the first `valid` of 64 columns (INT32_MIN if
+// none): the order of S, since its scale is positive.
+__device__ __forceinline__ int32_t half_max(const uint32_t (&sr)[64], int valid) {
+  int32_t mi = INT32_MIN;
+  if (valid >= 64) {
+    int32_t mp[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) mp[u] = INT32_MIN;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) mp[c & 7] = max(mp[c & 7], (int32_t)sr[c]);
+    mi = max(max(max(mp[0], mp[1]), max(mp[2], mp[3])), max(max(mp[4], mp[5]), max(mp[6], mp[7])));
+  } else {
+#pragma unroll
+    for (int c = 0; c < 64; ++c)
+      if (c < valid) mi = max(mi, (int32_t)sr[c]);
+  }
+  return mi;
+}
+
+template <bool kTwoPass>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_i8_kernel(const __grid_constant__ CUtensorMap map_q,
                    const __grid_constant__ CUtensorMap map_k,
@@ -168,6 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const float* __restrict__ q_scale, const float* __restrict__ k_scale,
                    const float* __restrict__ v_scale, float log2e_over_sqrt_d, float p_levels,
                    __nv_bfloat16* __restrict__ out, int32_t* __restrict__ status) {
+  static_assert(kTile == kBlock * kD, "kTile names the tile's byte size here");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t base = smem_u32(smem_raw);
   if ((base & 1023u) != 0) {
@@ -214,6 +250,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int q = 0; q < 4; ++q) mbar_init(bar(BX0 + q), 64);
     mbar_init(bar(BL), kSoftThreads);
     mbar_init(bar(BDRAIN), 1);
+    mbar_init(bar(BMG), kSoftThreads);
+    for (int b = 0; b < 2; ++b) mbar_init(bar(BAM0 + b), kSoftWarps);
     *abort_flag = 0;
     *bad_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -246,19 +284,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (n_tiles > 0 && lane == 0) {
       mbar_arrive_tx(bar(BQ), kTile);
       tma_load_2d(base + kOffQ, &map_q, 0, row0 + i * kBlock, bar(BQ));
+      // K tile t of the kept entry j (kTwoPass: t < n_tiles is pass 1, K only;
+      // pass 2 loads K again with V); the K ring counts t, the V ring j
       int nk = 0, nv = 0;  // K and V tiles issued
-      for (int j = 0; j < n_tiles; ++j) {
-        const int s = j % kStages;
+      const int n_k = kTwoPass ? 2 * n_tiles : n_tiles;
+      for (int t = 0; t < n_k; ++t) {
+        const bool pass1 = kTwoPass && t < n_tiles;
+        const int j = kTwoPass && !pass1 ? t - n_tiles : t;
+        const int s = t % kStages;
         const int y = row0 + __ldg(ids + j) * kBlock;
-        if (j >= kStages && !wait_phase(bar(BKF0 + s), ((j / kStages) - 1) & 1, ctl)) break;
-        PARO_T8(0, j);
+        if (t >= kStages && !wait_phase(bar(BKF0 + s), ((t / kStages) - 1) & 1, ctl)) break;
+        PARO_T8(0, t);
         mbar_arrive_tx(bar(BK0 + s), kTile);
         tma_load_2d(base + kOffK + s * kTile, &map_k, 0, y, bar(BK0 + s));
-        nk = j + 1;
-        if (j >= kStages && !wait_phase(bar(BVF0 + s), ((j / kStages) - 1) & 1, ctl)) break;
+        nk = t + 1;
+        if (pass1) continue;
+        const int sv = j % kStages;
+        if (j >= kStages && !wait_phase(bar(BVF0 + sv), ((j / kStages) - 1) & 1, ctl)) break;
         PARO_T8(11, j);
-        mbar_arrive_tx(bar(BV0 + s), kTile);
-        tma_load_2d(base + kOffV + s * kTile, &map_v, 0, y, bar(BV0 + s));
+        mbar_arrive_tx(bar(BV0 + sv), kTile);
+        tma_load_2d(base + kOffV + sv * kTile, &map_v, 0, y, bar(BV0 + sv));
         nv = j + 1;
       }
       // copies still in flight land before the CTA exits
@@ -306,9 +351,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(bar(BVF0 + s));
         return true;
       };
-      ok = ok && issue_qk(0);
+      // kTwoPass: pass 1 is Q K^T alone over the kept tiles; pass 2's Q K^T
+      // count on from n_tiles (the K ring and S handshakes continue)
+      const int t0 = kTwoPass ? n_tiles : 0;
+      for (int t = 0; ok && t < t0; ++t) ok = issue_qk(t);
+      ok = ok && issue_qk(t0);
       for (int j = 0; ok && j < n_tiles; ++j) {
-        if (j + 1 < n_tiles && !issue_qk(j + 1)) break;
+        if (j + 1 < n_tiles && !issue_qk(t0 + j + 1)) break;
         if (!issue_pv(j)) break;
       }
       mma_commit(bar(BDRAIN));
@@ -413,90 +462,186 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_run = -INFINITY;
     float2 l2 = make_float2(0.f, 0.f);
     bool ok = true;
-    // kept index and block scales of the current tile, read a tile ahead
-    int kb_next = 0;
-    float ks_next = 0.f, vs_next = 0.f;
-    if (n_tiles > 0) {
-      kb_next = __ldg(ids);
-      ks_next = __ldg(k_scale + bh * g.NB + kb_next);
-      vs_next = __ldg(v_scale + bh * g.NB + kb_next);
-    }
-    for (int j = 0; j < n_tiles; ++j) {
-      const int kb = kb_next;
-      const float ksc = ks_next, vsc = vs_next;
-      if (j + 1 < n_tiles) {
-        kb_next = __ldg(ids + j + 1);
+    if constexpr (kTwoPass) {
+      // ---- pass 1: exact row max and sum of this half (S read only)
+      float m_h = -INFINITY, l_h = 0.f;
+      for (int t = 0; t < n_tiles; ++t) {
+        const int kb = __ldg(ids + t);
+        const float cq = sq * __ldg(k_scale + bh * g.NB + kb);
+        if (!warp_wait(bar(BS), t & 1, ctl)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sr[64];
+        tmem_ld64(lane_addr + kColS + hc * 64, sr);
+        tc_fence_before();
+        mbar_arrive(bar(BSF));  // S may take the next Q K^T
+        const int valid = g.N - kb * kBlock - hc * 64;
+        const int32_t mi = half_max(sr, valid);
+        if (mi == INT32_MIN) continue;  // no valid key in this half
+        const float m_new = fmaxf(m_h, (__int_as_float(mi + kMagicBits) - kMagic) * cq);
+        const float alpha = m_h == -INFINITY ? 0.f : ex2(m_h - m_new);
+        float2 rs0 = make_float2(0.f, 0.f), rs1 = make_float2(0.f, 0.f);
+        uint32_t pk[16];
+        const float2 cq2 = make_float2(cq, cq), nm2 = make_float2(-m_new, -m_new);
+        if (valid >= 64)
+          tile_exp<false>(sr, cq2, nm2, valid, rs0, rs1, pk, 1.f);
+        else
+          tile_exp<true>(sr, cq2, nm2, valid, rs0, rs1, pk, 1.f);
+        const float2 rs = fadd2(rs0, rs1);
+        l_h = l_h * alpha + (rs.x + rs.y);
+        m_h = m_new;
+      }
+      // ---- merge the two halves' (m, l): both partner warps form the same
+      // row statistics
+      float m = -INFINITY, inv_l = 0.f;
+      if (ok && n_tiles > 0) {
+        xch[hc * 128 + r] = m_h;
+        xch[256 + hc * 128 + r] = l_h;
+        mbar_arrive(bar(BMG));
+        if (!all_wait(bar(BMG), 0, ctl)) ok = false;
+        if (ok) {
+          const float m_o = xch[(1 - hc) * 128 + r], l_o = xch[256 + (1 - hc) * 128 + r];
+          m = fmaxf(m_h, m_o);
+          const float l = (m_h == -INFINITY ? 0.f : l_h * ex2(m_h - m)) +
+                          (m_o == -INFINITY ? 0.f : l_o * ex2(m_o - m));
+          inv_l = l > 0.f ? 1.f / l : 0.f;
+        }
+      }
+      // pad query rows (past N) take no part in a tile's maximum
+      const bool row_valid = i * kBlock + r < g.N;
+      float* amx = reinterpret_cast<float*>(smem_raw + kOffAmx);
+      // ---- pass 2: normalised P, its per-tile maximum, codes, P V
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int t = n_tiles + j;
+        const int kb = __ldg(ids + j);
+        const float cq = sq * __ldg(k_scale + bh * g.NB + kb);
+        const float vsc = __ldg(v_scale + bh * g.NB + kb);
+        if (!warp_wait(bar(BS), t & 1, ctl)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sr[64];
+        tmem_ld64(lane_addr + kColS + hc * 64, sr);
+        tc_fence_before();
+        mbar_arrive(bar(BSF));
+        const int valid = g.N - kb * kBlock - hc * 64;
+        const int32_t mi = half_max(sr, valid);
+        // this row's largest P in the half: the same arithmetic as its
+        // element's (below), so no code exceeds L
+        float pmax = 0.f;
+        if (row_valid && mi != INT32_MIN)
+          pmax = ex2(fmaf(__int_as_float(mi + kMagicBits) - kMagic, cq, -m)) * inv_l;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) pmax = fmaxf(pmax, __shfl_xor_sync(0xffffffffu, pmax, o));
+        if (lane == 0) {
+          amx[(j & 1) * 8 + warp] = pmax;
+          mbar_arrive(bar(BAM0 + (j & 1)));
+        }
+        // slot j & 1 is rewritten for tile j + 2 only after every warp
+        // arrived for tile j + 1, i.e. after it read tile j's values
+        if (!all_wait(bar(BAM0 + (j & 1)), (j >> 1) & 1, ctl)) { ok = false; break; }
+        float a = amx[(j & 1) * 8];
+#pragma unroll
+        for (int w = 1; w < kSoftWarps; ++w) a = fmaxf(a, amx[(j & 1) * 8 + w]);
+        if (hc == 0) {
+          // O = O + (a / L) s_v (P8 V8): no rescale in this mode
+          const int sl = j & (kScaleSlots - 1);
+          s_alpha[sl * 128 + r] = 1.f;
+          s_cv[sl * 128 + r] = __fdiv_rn(a, p_levels) * vsc;
+          mbar_arrive(bar(BSC0 + sl));
+        }
+        // codes rne(L P / a) = rne(2^(s - m) * (L / (a l))); pad rows 0
+        const float kq = a > 0.f && row_valid ? inv_l * __fdiv_rn(p_levels, a) : 0.f;
+        const float2 cq2 = make_float2(cq, cq), nm2 = make_float2(-m, -m);
+        float2 rs0 = make_float2(0.f, 0.f), rs1 = make_float2(0.f, 0.f);
+        uint32_t pk[16];
+        if (valid >= 64)
+          tile_exp<false>(sr, cq2, nm2, valid, rs0, rs1, pk, kq);
+        else
+          tile_exp<true>(sr, cq2, nm2, valid, rs0, rs1, pk, kq);
+        unsigned char* prow = smem_raw + kOffP + (j & 1) * kTile + r * 128;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          *reinterpret_cast<uint4*>(prow + (((hc * 4 + u) ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        fence_async_smem();
+        mbar_arrive(bar(BP0 + (j & 1)));
+      }
+      if (ok && n_tiles > 0) {
+        // O is already normalised: the epilogue divides by 1 + 0
+        s_l[hc * 128 + r] = hc == 0 ? 1.f : 0.f;
+        mbar_arrive(bar(BL));
+      }
+    } else {
+      // kept index and block scales of the current tile, read a tile ahead
+      int kb_next = 0;
+      float ks_next = 0.f, vs_next = 0.f;
+      if (n_tiles > 0) {
+        kb_next = __ldg(ids);
         ks_next = __ldg(k_scale + bh * g.NB + kb_next);
         vs_next = __ldg(v_scale + bh * g.NB + kb_next);
       }
-      if (!warp_wait(bar(BS), j & 1, ctl)) { ok = false; break; }
-      if (lane == 0 && quarter == 0) PARO_T8(3 + 3 * hc, j);
-      tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld64(lane_addr + kColS + hc * 64, sr);
-      tc_fence_before();
-      mbar_arrive(bar(BSF));  // S may take QK^T(j+1)
-      const int valid = g.N - kb * kBlock - hc * 64;  // valid columns of this half
-      const float cq = sq * ksc;
-      // row max of this half in integers (cq >= 0 keeps the order)
-      int32_t mi = INT32_MIN;
-      if (valid >= 64) {
-        int32_t mp[8];
+      for (int j = 0; j < n_tiles; ++j) {
+        const int kb = kb_next;
+        const float ksc = ks_next, vsc = vs_next;
+        if (j + 1 < n_tiles) {
+          kb_next = __ldg(ids + j + 1);
+          ks_next = __ldg(k_scale + bh * g.NB + kb_next);
+          vs_next = __ldg(v_scale + bh * g.NB + kb_next);
+        }
+        if (!warp_wait(bar(BS), j & 1, ctl)) { ok = false; break; }
+        if (lane == 0 && quarter == 0) PARO_T8(3 + 3 * hc, j);
+        tc_fence_after();
+        uint32_t sr[64];
+        tmem_ld64(lane_addr + kColS + hc * 64, sr);
+        tc_fence_before();
+        mbar_arrive(bar(BSF));  // S may take QK^T(j+1)
+        const int valid = g.N - kb * kBlock - hc * 64;  // valid columns of this half
+        const float cq = sq * ksc;
+        // row max of this half in integers (cq >= 0 keeps the order)
+        const int32_t mi = half_max(sr, valid);
+        const float m_half =
+            mi == INT32_MIN ? -INFINITY : (__int_as_float(mi + kMagicBits) - kMagic) * cq;
+        // trade the half maxima with the partner warp (same rows, other half)
+        float* xs = xch + (j & 1) * 256;
+        xs[hc * 128 + r] = m_half;
+        mbar_arrive(xbar);
+        if (!all_wait(xbar, j & 1, ctl)) { ok = false; break; }
+        if (lane == 0 && quarter == 0) PARO_T8(4 + 3 * hc, j);
+        const float m_new = fmaxf(m_run, fmaxf(m_half, xs[(1 - hc) * 128 + r]));
+        const float alpha = m_run == -INFINITY ? 0.f : ex2(m_run - m_new);
+        if (hc == 0) {
+          // slot j % 4 was last read by the correction of tile j - 4, which
+          // completed before P V(j - 2) was issued, and so before QK(j)
+          const int sl = j & (kScaleSlots - 1);
+          s_alpha[sl * 128 + r] = alpha;
+          s_cv[sl * 128 + r] = __fdiv_rn(vsc, p_levels);
+          mbar_arrive(bar(BSC0 + sl));
+        }
+        // P~ = 2^(s - m) <= 1, P8 = rne(127 P~): the low byte of the float
+        // 127 P~ + 1.5 * 2^23 (one rounding, to the nearest integer, ties even)
+        const float2 cq2 = make_float2(cq, cq), nm2 = make_float2(-m_new, -m_new);
+        float2 rs0 = make_float2(0.f, 0.f), rs1 = make_float2(0.f, 0.f);
+        uint32_t pk[16];
+        if (valid >= 64)
+          tile_exp<false>(sr, cq2, nm2, valid, rs0, rs1, pk, p_levels);
+        else
+          tile_exp<true>(sr, cq2, nm2, valid, rs0, rs1, pk, p_levels);
+        const float2 rs = fadd2(rs0, rs1);
+        l2 = ffma2(l2, make_float2(alpha, alpha), rs);
+        // this half row of P8 (64 bytes = 4 chunks of 16) into the swizzled
+        // tile; the async proxy (the MMA) reads it after the fence
+        unsigned char* prow = smem_raw + kOffP + (j & 1) * kTile + r * 128;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) mp[u] = INT32_MIN;
-#pragma unroll
-        for (int c = 0; c < 64; ++c) mp[c & 7] = max(mp[c & 7], (int32_t)sr[c]);
-        mi = max(max(max(mp[0], mp[1]), max(mp[2], mp[3])),
-                 max(max(mp[4], mp[5]), max(mp[6], mp[7])));
-      } else {
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c < valid) mi = max(mi, (int32_t)sr[c]);
+        for (int t = 0; t < 4; ++t)
+          *reinterpret_cast<uint4*>(prow + (((hc * 4 + t) ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+        fence_async_smem();
+        mbar_arrive(bar(BP0 + (j & 1)));
+        if (lane == 0 && quarter == 0) PARO_T8(5 + 3 * hc, j);
+        m_run = m_new;
       }
-      const float m_half =
-          mi == INT32_MIN ? -INFINITY : (__int_as_float(mi + kMagicBits) - kMagic) * cq;
-      // trade the half maxima with the partner warp (same rows, other half)
-      float* xs = xch + (j & 1) * 256;
-      xs[hc * 128 + r] = m_half;
-      mbar_arrive(xbar);
-      if (!all_wait(xbar, j & 1, ctl)) { ok = false; break; }
-      if (lane == 0 && quarter == 0) PARO_T8(4 + 3 * hc, j);
-      const float m_new = fmaxf(m_run, fmaxf(m_half, xs[(1 - hc) * 128 + r]));
-      const float alpha = m_run == -INFINITY ? 0.f : ex2(m_run - m_new);
-      if (hc == 0) {
-        // slot j % 4 was last read by the correction of tile j - 4, which
-        // completed before P V(j - 2) was issued, and so before QK(j)
-        const int sl = j & (kScaleSlots - 1);
-        s_alpha[sl * 128 + r] = alpha;
-        s_cv[sl * 128 + r] = __fdiv_rn(vsc, p_levels);
-        mbar_arrive(bar(BSC0 + sl));
+      if (ok && n_tiles > 0) {
+        s_l[hc * 128 + r] = l2.x + l2.y;
+        mbar_arrive(bar(BL));
       }
-      // P~ = 2^(s - m) <= 1, P8 = rne(127 P~): the low byte of the float
-      // 127 P~ + 1.5 * 2^23 (one rounding, to the nearest integer, ties even)
-      const float2 cq2 = make_float2(cq, cq), nm2 = make_float2(-m_new, -m_new);
-      float2 rs0 = make_float2(0.f, 0.f), rs1 = make_float2(0.f, 0.f);
-      uint32_t pk[16];
-      if (valid >= 64)
-        tile_exp<false>(sr, cq2, nm2, valid, rs0, rs1, pk, p_levels);
-      else
-        tile_exp<true>(sr, cq2, nm2, valid, rs0, rs1, pk, p_levels);
-      const float2 rs = fadd2(rs0, rs1);
-      l2 = ffma2(l2, make_float2(alpha, alpha), rs);
-      // this half row of P8 (64 bytes = 4 chunks of 16) into the swizzled
-      // tile; the async proxy (the MMA) reads it after the fence
-      unsigned char* prow = smem_raw + kOffP + (j & 1) * kTile + r * 128;
-#pragma unroll
-      for (int t = 0; t < 4; ++t)
-        *reinterpret_cast<uint4*>(prow + (((hc * 4 + t) ^ (r & 7)) << 4)) =
-            make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
-      fence_async_smem();
-      mbar_arrive(bar(BP0 + (j & 1)));
-      if (lane == 0 && quarter == 0) PARO_T8(5 + 3 * hc, j);
-      m_run = m_new;
-    }
-    if (ok && n_tiles > 0) {
-      s_l[hc * 128 + r] = l2.x + l2.y;
-      mbar_arrive(bar(BL));
     }
     __syncwarp();
   }
@@ -514,8 +659,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_attn_i8(const void* q, const void* k, const void* v, const Grid& g,
                            const int32_t* idx, const int32_t* counts, int k_max, const float* qs,
-                           const float* ks, const float* vs, float p_levels, void* out,
-                           int32_t* status, cudaStream_t s) {
+                           const float* ks, const float* vs, float p_levels, bool p_tile,
+                           void* out, int32_t* status, cudaStream_t s) {
   if (g.d != kD || g.block != kBlock) return cudaErrorInvalidValue;
   const uint64_t rows = (uint64_t)g.B * g.heads * g.Np;
   CUtensorMap mq{}, mk{}, mv{};
@@ -523,14 +668,14 @@ cudaError_t launch_attn_i8(const void* q, const void* k, const void* v, const Gr
       !encode_tile_map(&mk, k, rows, kD, 1, 128, kBlock) ||
       !encode_tile_map(&mv, v, rows, kD, 1, 128, kBlock))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(attn_i8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSmemBytes);
+  auto kernel = p_tile ? attn_i8_kernel<true> : attn_i8_kernel<false>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   const float c = (float)(1.4426950408889634 / sqrt((double)kD));
   dim3 grid(g.NB, g.B * g.heads);
-  attn_i8_kernel<<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, g, idx, counts, k_max, qs, ks, vs,
-                                                    c, p_levels, static_cast<__nv_bfloat16*>(out),
-                                                    status);
+  kernel<<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, g, idx, counts, k_max, qs, ks, vs, c,
+                                            p_levels, static_cast<__nv_bfloat16*>(out), status);
   return cudaGetLastError();
 }
 

@@ -170,9 +170,10 @@ cudaError_t launch_paro_metric(const float* count, const float* total, const flo
 cudaError_t launch_paro_choose(const float* sparse_frac, const float* incoh, int64_t rows,
                                float alpha, float* metric, int8_t* orders, cudaStream_t s);
 // INT8 tcgen05 attention (d = 128, block = 128, permuted int8 inputs)
-// p_levels: P codes round_half_even(p_levels * P~); 127 (INT8) or 7 (4-bit)
+// p_levels: P code levels, 127 (INT8) or 7 (4-bit); p_tile: the two-pass
+// form (normalised P, one scale per tile) instead of rne(p_levels * P~)
 cudaError_t launch_attn_i8(const void* q, const void* k, const void* v, const Grid& g,
                            const int32_t* idx, const int32_t* counts, int k_max, const float* qs,
-                           const float* ks, const float* vs, float p_levels, void* out,
-                           int32_t* status, cudaStream_t s);
+                           const float* ks, const float* vs, float p_levels, bool p_tile,
+                           void* out, int32_t* status, cudaStream_t s);
 }  // namespace paro

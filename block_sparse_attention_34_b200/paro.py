@@ -22,6 +22,7 @@ ABI_VERSION = 8  # the pa_abi_version() these signatures describe
 PA_F32, PA_BF16, PA_I8 = 0, 1, 2
 PA_ATTN_PERMUTED = 1
 PA_ATTN_P4 = 2  # with int8 inputs: 4-bit P codes (INT4 PV)
+PA_ATTN_P_TILE = 4  # with int8 inputs: normalised P, one scale per tile (two passes)
 STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_CUDA",
                 4: "PA_ERR_TIMEOUT", 5: "PA_ERR_DEVICE_CHECK"}
 ORDER_IDS = {"FHW": 0, "FWH": 1, "HFW": 2, "HWF": 3, "WFH": 4, "WHF": 5}
@@ -440,13 +441,16 @@ def _expect_status(status):
 
 
 def block_sparse_attn(q, k, v, pr: Problem, idx, counts=None, scales=None, out=None,
-                      status=None, baseline=False, permuted=False, p4=False):
+                      status=None, baseline=False, permuted=False, p4=False, p_tile=False):
     """O = block-sparse attention over the kept tiles, natural token order.
 
     ``permuted``: q, k, v are [B, heads, N_p, d] from :func:`reorder`.
     ``scales`` = (q_scale, k_scale, v_scale) for int8 q/k/v from
-    :func:`quantize_int8` (output bf16).  ``baseline=True`` runs the
-    mma.sync comparison kernel instead of the tcgen05 one."""
+    :func:`quantize_int8` (output bf16); with them ``p4`` quantises P to 4
+    bits and ``p_tile`` quantises the normalised P with one scale per tile
+    (two passes over the kept tiles) instead of the one-pass fixed scale.
+    ``baseline=True`` runs the mma.sync comparison kernel instead of the
+    tcgen05 one."""
     _need_cuda(q, k, v, idx, counts, out, status, *(scales or ()))
     code = _dtype_code(q)
     _same_dtype(("q", q), ("k", k), ("v", v))
@@ -464,7 +468,8 @@ def block_sparse_attn(q, k, v, pr: Problem, idx, counts=None, scales=None, out=N
     _expect_status(status)
     out = out if out is not None else torch.empty((pr.B, pr.heads, pr.N, pr.d), dtype=out_dtype, device=q.device)
     k_max = int(idx.shape[-1])
-    flags = (PA_ATTN_PERMUTED if permuted else 0) | (PA_ATTN_P4 if p4 else 0)
+    flags = ((PA_ATTN_PERMUTED if permuted else 0) | (PA_ATTN_P4 if p4 else 0)
+             | (PA_ATTN_P_TILE if p_tile else 0))
     lib = load()
     if baseline:
         st = lib.pa_block_sparse_attn_mma(_ptr(q), _ptr(k), _ptr(v), code, flags, pr.shape,
@@ -539,7 +544,7 @@ def choose_orders_sics(q, k, grid, block):
 
 def attention(q, k, v, grid, perms, block, density, int8=False, baseline=False, status=None,
               permuted=True, int4_pv=False, selection="topk", top_p=0.0, window=-1,
-              compensate=False):
+              compensate=False, p_tile=None):
     """The whole path for one call: reorder with block means (one read of
     q, k, v) -> pooled block scores -> kept blocks -> block-sparse attention
     over the permuted tiles, stored back in natural order.
@@ -549,7 +554,10 @@ def attention(q, k, v, grid, perms, block, density, int8=False, baseline=False, 
     diagonal plus the k-1 best blocks, k from ``density``) or "hybrid" (the
     union of that Top-K, the Top-P set at ``top_p`` and the local window
     |i - j| <= ``window``, with per-row counts).  ``int8`` runs the INT8
-    kernel (``int4_pv``: 4-bit P and V).  ``permuted=False`` skips the
+    kernel (``int4_pv``: 4-bit P and V; ``p_tile``: P normalised and
+    quantised per tile, the pages' reading, by default with ``int4_pv``
+    only, since at 8 bits the one-pass form stays within the INT8
+    tolerance of it).  ``permuted=False`` skips the
     reorder pass (the kernel gathers token rows); ``baseline=True`` runs the
     mma.sync comparison kernel.  ``compensate`` adds PASA's grouped
     first-order compensation of the unselected blocks (bf16 / fp32 only;
@@ -587,7 +595,7 @@ def attention(q, k, v, grid, perms, block, density, int8=False, baseline=False, 
         v8, vs = quantize_int8(v, pr, bits=4 if int4_pv else 8)
         idx, counts = select(score_pooled(qp, kp, pr))
         out = block_sparse_attn(q8, k8, v8, pr, idx, counts, scales=(qs, ks, vs), status=status,
-                                p4=int4_pv)
+                                p4=int4_pv, p_tile=int4_pv if p_tile is None else p_tile)
     elif permuted and not baseline:
         qp, q_pool = reorder(q, pr, with_pool=True)
         kp, k_pool = reorder(k, pr, with_pool=True)

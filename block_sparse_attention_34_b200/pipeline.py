@@ -8,7 +8,8 @@ current torch stream; the status word is cleared first, by a memset):
          score_pooled -> select_topk (or select_hybrid: diagonal, window,
          Top-K and Top-P with per-row counts) -> block_sparse_attn(permuted tiles)
   int8:  quantize+pool(q), quantize+pool(k), quantize(v)  (v to 4 bits with int4_pv)
-         score_pooled -> select_topk -> block_sparse_attn(int8; 4-bit P with int4_pv)
+         score_pooled -> select_topk -> block_sparse_attn(int8; 4-bit P with int4_pv;
+         P normalised and quantised per tile with p_tile, by default with int4_pv)
 
 The output is written in natural token order; the inverse reorder is the
 attention kernel's store.
@@ -24,12 +25,13 @@ from . import paro
 class Pipeline:
     def __init__(self, B, heads, grid, d, block, perms, density, dtype=torch.bfloat16,
                  device="cuda", int8=False, baseline=False, selection="topk", top_p=0.0,
-                 window=-1, int4_pv=False):
+                 window=-1, int4_pv=False, p_tile=None):
         self.pr = paro.Problem(B, heads, grid, d, block, perms)
         pr = self.pr
         self.k = paro.k_for_density(pr.NB, density)
         self.int8 = int8 or int4_pv
         self.int4_pv = int4_pv
+        self.p_tile = int4_pv if p_tile is None else bool(p_tile)
         self.baseline = baseline
         if selection not in ("topk", "hybrid"):
             raise ValueError(f"selection {selection!r}: topk or hybrid")
@@ -85,7 +87,8 @@ class Pipeline:
         pr = self.pr
         if self.int8:
             paro.block_sparse_attn(*self.xq, pr, self.idx, self.counts, scales=tuple(self.sc),
-                                   out=self.out, status=self.status, p4=self.int4_pv)
+                                   out=self.out, status=self.status, p4=self.int4_pv,
+                                   p_tile=self.p_tile)
         elif self.baseline:
             paro.block_sparse_attn(q, k, v, pr, self.idx, self.counts, out=self.out,
                                    status=self.status, baseline=True)

@@ -325,6 +325,17 @@ PA_API pa_status pa_quantize_int4(const void* x, pa_dtype dtype, pa_shape shape,
  * post-softmax map and PV), with v (and its scales) from pa_quantize_int4;
  * q and k stay INT8. */
 #define PA_ATTN_P4 2u
+/* With PA_I8 (alone or with PA_ATTN_P4): the post-softmax map is quantised
+ * after it is normalised, one symmetric scale per (query block, key block)
+ * tile (PAROAttention review, key_machinery and core_discovery: block-wise
+ * quantisation of the attention map, groups aligned to the attention
+ * block).  Per tile: P = exp(s - m) / l with the row's exact max m and sum
+ * l over all its kept keys, a = max of P over the tile's valid rows and
+ * keys, codes round_half_even(L P / a) (L = 127, or 7 with PA_ATTN_P4),
+ * and the tile contributes (codes V) * (a / L) * v_scale.  The kernel takes
+ * two passes over the kept tiles (Q K^T twice), so it is slower than the
+ * one-pass form above, whose per-tile scale is fixed at 1/L. */
+#define PA_ATTN_P_TILE 4u
 
 PA_API pa_status pa_block_sparse_attn(const void* q, const void* k, const void* v, pa_dtype dtype,
                                uint32_t flags, pa_shape shape, const int8_t* perms, const int32_t* idx,

@@ -134,8 +134,13 @@ def test_p4_flag_validation(lib):
     assert lib.pa_block_sparse_attn(FAKE, FAKE, FAKE, paro.PA_BF16, paro.PA_ATTN_P4, good, pp, FAKE,
                                     None, 1, None, None, None, FAKE, None, None) == paro.PA_ERR_INVALID_ARG
     assert b"P4" in lib.pa_last_error()
-    assert lib.pa_block_sparse_attn(FAKE, FAKE, FAKE, paro.PA_BF16, 4, good, pp, FAKE,
+    # PA_ATTN_P_TILE (4) needs int8 inputs too; bit 8 is unknown
+    assert lib.pa_block_sparse_attn(FAKE, FAKE, FAKE, paro.PA_BF16, paro.PA_ATTN_P_TILE, good, pp,
+                                    FAKE, None, 1, None, None, None, FAKE, None, None) == paro.PA_ERR_INVALID_ARG
+    assert b"P_TILE" in lib.pa_last_error()
+    assert lib.pa_block_sparse_attn(FAKE, FAKE, FAKE, paro.PA_BF16, 8, good, pp, FAKE,
                                     None, 1, None, None, None, FAKE, None, None) == paro.PA_ERR_INVALID_ARG
+    assert b"unknown flags" in lib.pa_last_error()
     assert lib.pa_quantize_int4(FAKE, paro.PA_I8, good, pp, FAKE, FAKE, None, None) == paro.PA_ERR_INVALID_ARG
 
 
