@@ -198,7 +198,9 @@ def percentiles(xs):
 def attn_kernel_name(pipe) -> str:
     if pipe.int8:
         return "attn_i8_kernel<tile>" if pipe.p_tile else "attn_i8_kernel"
-    return "attn_mma_kernel" if pipe.baseline else "attn_sm100_kernel"
+    # the tcgen05 kernel takes d = 128, block = 128; other shapes run mma.sync
+    tc = pipe.pr.d == 128 and pipe.pr.block == 128
+    return "attn_mma_kernel" if pipe.baseline or not tc else "attn_sm100_kernel"
 
 
 def step(pipe, qkv, ev=None):
