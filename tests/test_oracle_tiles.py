@@ -122,3 +122,26 @@ def test_candidate_names_and_counts():
     for block, shapes in ref.TILE_SHAPES.items():
         assert len(shapes) == 6 and all(a * b * c == block for a, b, c in shapes)
         assert len(set(shapes)) == 6
+
+
+def test_sics_picks_the_clustered_tile_blocking_closed_form():
+    """Rows equal up to scale inside each 2x8x8 tile (one random direction
+    per tile): only the mixed candidate 2x8x8 (id 8 at block 128) puts every
+    tile in one block, so each of its blocks has all 128 * 127 ordered pairs
+    at cosine 1 and it must win; q and k add their scores."""
+    F, H, W, d = 4, 16, 16, 16
+    rng = np.random.default_rng(9)
+    f, h, w = np.meshgrid(np.arange(F), np.arange(H), np.arange(W), indexing="ij")
+    tile = (f // 2, h // 8, w // 8)
+    xs = []
+    for _ in range(2):
+        dirs = rng.standard_normal((F // 2, H // 8, W // 8, d))
+        scale = rng.uniform(0.5, 2.0, size=(F * H * W, 1))
+        xs.append(dirs[tile].reshape(F * H * W, d) * scale)
+    scores = np.array([sel.sics_order(xs[0], (F, H, W), o, 128)
+                       + sel.sics_order(xs[1], (F, H, W), o, 128)
+                       for o in range(ref.N_ORDERS)])
+    nblocks = F * H * W // 128
+    assert abs(scores[8] - 2 * nblocks * 128 * 127) < 1e-9 * scores[8]
+    assert scores[8] > np.delete(scores, 8).max()
+    assert int(np.argmax(scores)) == 8
