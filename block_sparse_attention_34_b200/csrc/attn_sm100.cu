@@ -602,28 +602,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the group's P buffer is free once P V of its previous tile completed
       if (j >= 2 && !warp_wait(pv_done(j - 2), ring_par(j - 2), ctl)) return false;
       tc_fence_after();
-      // P = 2^(s*scale - m_j) as bf16 pairs into the group's P buffer; row
-      // sum in 8 chains
+      // P = 2^(s*scale - m_j) as bf16 pairs into the group's P buffer, two
+      // columns per paired f32x2 FMA and add; row sum in 4 paired chains
       const float neg_m = (m_j == -INFINITY ? 0.f : -m_j) + bias;
-      float rs[8];
+      const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(neg_m, neg_m);
+      float2 rs2[4];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) rs[u] = 0.f;
+      for (int u = 0; u < 4; ++u) rs2[u] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const int e = 32 * cc + 2 * c;
-          const float e0 = ex2(fmaf(__uint_as_float(sr[e]), scale_log2, neg_m));
-          const float e1 = ex2(fmaf(__uint_as_float(sr[e + 1]), scale_log2, neg_m));
-          rs[e & 7] += e0;
-          rs[(e + 1) & 7] += e1;
-          pk[c] = pack_bf16(e0, e1);
+          const float2 t =
+              ffma2(make_float2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), sc2, nm2);
+          const float2 ex = make_float2(ex2(t.x), ex2(t.y));
+          rs2[c & 3] = fadd2(rs2[c & 3], ex);
+          pk[c] = pack_bf16(ex.x, ex.y);
         }
         tmem_st16_async(lane_addr + p_col + 16 * cc, pk);
       }
       tmem_wait_st();
-      l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
+      l += ((rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y)) +
+           ((rs2[2].x + rs2[2].y) + (rs2[3].x + rs2[3].y));
       // O holds P V up to tile j-1 relative to m_prev: rescale it before
       // P V(j) once that MMA completed (rare: the reference moved)
       const bool need = m_prev != -INFINITY && m_j != m_prev;

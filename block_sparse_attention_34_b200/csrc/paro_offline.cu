@@ -200,11 +200,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (m_new != -INFINITY) {
           float acc = 0.f;
           if (valid >= 64) {
-            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+            // two columns per paired f32x2 FMA and add
+            const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-m_new, -m_new);
+            float2 a2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-            for (int c = 0; c < 64; ++c)
-              a4[c & 3] += ex2(fmaf(__uint_as_float(sr[c]), scale_log2, -m_new));
-            acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+            for (int c = 0; c < 64; c += 2) {
+              const float2 t = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
+                                     sc2, nm2);
+              a2[(c >> 1) & 1] = fadd2(a2[(c >> 1) & 1], make_float2(ex2(t.x), ex2(t.y)));
+            }
+            acc = (a2[0].x + a2[0].y) + (a2[1].x + a2[1].y);
           } else {
 #pragma unroll
             for (int c = 0; c < 64; ++c)
@@ -216,17 +221,25 @@ __global__ void __launch_bounds__(kThreads, 2)
       } else {
         float cnt = 0.f, sum = 0.f, mx = 0.f;
         if (row_ok && valid >= 64) {
-          float c4[4] = {0.f, 0.f, 0.f, 0.f}, s4[4] = {0.f, 0.f, 0.f, 0.f};
+          // two columns per paired f32x2 FMA, multiply and add
+          const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-m_row, -m_row);
+          const float2 il2 = make_float2(inv_l, inv_l);
+          float2 c2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+          float2 s2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
           float x4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const float pv = ex2(fmaf(__uint_as_float(sr[c]), scale_log2, -m_row)) * inv_l;
-            c4[c & 3] += pv < eps ? 1.f : 0.f;
-            s4[c & 3] += pv;
-            x4[c & 3] = fmaxf(x4[c & 3], pv);
+          for (int c = 0; c < 64; c += 2) {
+            const float2 t = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
+                                   sc2, nm2);
+            const float2 pv = fmul2(make_float2(ex2(t.x), ex2(t.y)), il2);
+            const int u = (c >> 1) & 1;
+            c2[u] = fadd2(c2[u], make_float2(pv.x < eps ? 1.f : 0.f, pv.y < eps ? 1.f : 0.f));
+            s2[u] = fadd2(s2[u], pv);
+            x4[2 * u] = fmaxf(x4[2 * u], pv.x);
+            x4[2 * u + 1] = fmaxf(x4[2 * u + 1], pv.y);
           }
-          cnt = (c4[0] + c4[1]) + (c4[2] + c4[3]);
-          sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+          cnt = (c2[0].x + c2[0].y) + (c2[1].x + c2[1].y);
+          sum = (s2[0].x + s2[0].y) + (s2[1].x + s2[1].y);
           mx = fmaxf(fmaxf(x4[0], x4[1]), fmaxf(x4[2], x4[3]));
         } else if (row_ok) {
 #pragma unroll

@@ -111,3 +111,77 @@ class Pipeline:
         self.select(q, k, v)
         self.attend(q, k, v)
         return self.out
+
+
+def chunk_ranges(B: int, heads: int, chunks: int):
+    """Split a [B, heads, ...] call into at most ``chunks`` pieces, each
+    contiguous in memory: head ranges of the one batch element when B = 1,
+    else ranges of whole batch elements.  Returns [(b0, b1, h0, h1)]."""
+    if B == 1:
+        n = max(1, min(chunks, heads))
+        cuts = [round(i * heads / n) for i in range(n + 1)]
+        return [(0, 1, cuts[i], cuts[i + 1]) for i in range(n) if cuts[i + 1] > cuts[i]]
+    n = max(1, min(chunks, B))
+    cuts = [round(i * B / n) for i in range(n + 1)]
+    return [(cuts[i], cuts[i + 1], 0, heads) for i in range(n) if cuts[i + 1] > cuts[i]]
+
+
+class StreamedPipeline:
+    """The same call on inputs in pinned host memory, with the copies
+    overlapped with the work: the layer is split into contiguous chunks of
+    heads (or batch elements), each with its own preallocated
+    :class:`Pipeline`; chunk c's host -> device copies run on a copy stream,
+    its selection and attention on a compute stream once they landed, and
+    its output's device -> host copy on a third stream once the attention
+    finished, so chunk c's work overlaps chunk c+1's upload and chunk c-1's
+    download.  Every step of the path is per head, so the result equals the
+    one-shot :class:`Pipeline`'s bit for bit."""
+
+    def __init__(self, B, heads, grid, d, block, perms, density, chunks=8, device="cuda",
+                 **kw):
+        dev = torch.device(device)
+        perms = list(perms)
+        self.ranges = chunk_ranges(B, heads, chunks)
+        self.pipes = [Pipeline(b1 - b0, h1 - h0, grid, d, block, perms[h0:h1], density,
+                               device=dev, **kw) for (b0, b1, h0, h1) in self.ranges]
+        p0 = self.pipes[0]
+        shape = (B, heads, p0.pr.N, d)
+        dtype = kw.get("dtype", torch.bfloat16)
+        self.dev_in = [[torch.empty((b1 - b0, h1 - h0) + shape[2:], dtype=dtype, device=dev)
+                        for _ in range(3)] for (b0, b1, h0, h1) in self.ranges]
+        self.streams = [torch.cuda.Stream(device=dev) for _ in range(3)]  # h2d, compute, d2h
+        self.k = p0.k
+
+    def run(self, host_q, host_k, host_v, host_out):
+        """host_q/k/v [B, heads, N, d] and host_out [B, heads, N, d] pinned
+        host tensors; returns host_out once its copies are enqueued (on the
+        caller's stream order: the caller's current stream waits for them)."""
+        cur = torch.cuda.current_stream()
+        h2d, comp, d2h = self.streams
+        for s in self.streams:
+            s.wait_stream(cur)  # nothing starts before the caller's prior work
+        for (b0, b1, h0, h1), pipe, dev in zip(self.ranges, self.pipes, self.dev_in):
+            with torch.cuda.stream(h2d):
+                for t, h in zip(dev, (host_q, host_k, host_v)):
+                    t.copy_(h[b0:b1, h0:h1], non_blocking=True)
+                landed = torch.cuda.Event()
+                landed.record(h2d)
+            with torch.cuda.stream(comp):
+                comp.wait_event(landed)
+                pipe.run(*dev)
+                done = torch.cuda.Event()
+                done.record(comp)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(done)
+                host_out[b0:b1, h0:h1].copy_(pipe.out, non_blocking=True)
+        for s in self.streams:
+            cur.wait_stream(s)
+        return host_out
+
+    def status(self) -> int:
+        """The first nonzero device status of the chunks (reads it back)."""
+        for pipe in self.pipes:
+            st = int(pipe.status.item())
+            if st != 0:
+                return st
+        return 0
