@@ -388,7 +388,8 @@ static pa_status attn_common(const void* q, const void* k, const void* v, pa_dty
   pa_status st = make_grid(shape, perms, true, &g);
   if (st != PA_OK) return st;
   PA_REQUIRE(dtype == PA_F32 || dtype == PA_BF16 || dtype == PA_I8, "dtype %d unknown", (int)dtype);
-  PA_REQUIRE(q && k && v && out && idx, "q, k, v, idx and out must be non-NULL");
+  PA_REQUIRE(q && k && v && out, "q, k, v and out must be non-NULL");
+  PA_REQUIRE(idx || k_max == 0, "idx must be non-NULL when k_max > 0");
   PA_REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out),
              "q, k, v and out must be 16-byte aligned");
   PA_REQUIRE(k_max >= 0 && k_max <= g.NB, "k_max=%d must be in [0, NB=%d]", k_max, g.NB);
@@ -453,8 +454,9 @@ pa_status pa_block_sparse_attn_compensated(const void* q, const void* k, const v
   if (st != PA_OK) return st;
   PA_REQUIRE(dtype == PA_F32 || dtype == PA_BF16,
              "dtype %d: pa_block_sparse_attn_compensated takes PA_F32 or PA_BF16", (int)dtype);
-  PA_REQUIRE(q && k && v && out && idx && k_pool && v_pool,
-             "q, k, v, idx, k_pool, v_pool and out must be non-NULL");
+  PA_REQUIRE(q && k && v && out && k_pool && v_pool,
+             "q, k, v, k_pool, v_pool and out must be non-NULL");
+  PA_REQUIRE(idx || k_max == 0, "idx must be non-NULL when k_max > 0");
   PA_REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out) &&
                  aligned16(k_pool) && aligned16(v_pool),
              "q, k, v, k_pool, v_pool and out must be 16-byte aligned");

@@ -296,7 +296,7 @@ PA_API pa_status pa_quantize_int4(const void* x, pa_dtype dtype, pa_shape shape,
  * idx [B,heads,NB,k] int32; each used entry in [0, NB), ascending, no
  * repeats (a malformed row is skipped with PA_ERR_DEVICE_CHECK on
  * dev_status; its rows of out are left unwritten).  A row whose count is
- * 0 produces zeros.
+ * 0 produces zeros; with k_max = 0 every row does, and idx may be NULL.
  *
  * dtype PA_BF16: q, k, v, out bf16, natural order; P rounded to bf16 for
  *   the P V product, fp32 accumulation.
@@ -372,7 +372,7 @@ PA_API pa_status pa_block_sparse_attn_mma(const void* q, const void* k, const vo
  *
  * Arguments, layouts, ownership and errors as pa_block_sparse_attn_mma
  * (dtype PA_F32 or PA_BF16, flags 0 or PA_ATTN_PERMUTED; k_max = 0 is
- * allowed and gives the compensation alone), plus:
+ * allowed, with idx NULL or not, and gives the compensation alone), plus:
  *   k_pool, v_pool  [B,heads,NB,d], 16-byte aligned, read only: the
  *                   means of the valid rows of each permuted block of k and
  *                   v (the pool output of pa_reorder or pa_block_score),

@@ -156,6 +156,29 @@ def test_offline_stage_validation(lib):
     assert lib.pa_paro_choose(FAKE, FAKE, good, float("inf"), FAKE, FAKE, None) == paro.PA_ERR_INVALID_ARG
 
 
+def test_empty_kept_lists_need_no_idx(lib):
+    """k_max = 0: idx is never read, so NULL passes the idx check; the call
+    here still fails validation, later, on a misaligned out (so no CUDA call
+    is made), and its message names the alignment, not idx.  k_max > 0 with
+    NULL idx is refused."""
+    good = paro.PaShape(1, 2, 4, 8, 8, 64, 64)
+    keep, pp = perms_of(0, 5)
+    bad_out = ctypes.c_void_p(4100)
+    st = lib.pa_block_sparse_attn(FAKE, FAKE, FAKE, paro.PA_BF16, 0, good, pp, None, None, 0,
+                                  None, None, None, bad_out, None, None)
+    assert st == paro.PA_ERR_INVALID_ARG and b"aligned" in lib.pa_last_error()
+    st = lib.pa_block_sparse_attn(FAKE, FAKE, FAKE, paro.PA_BF16, 0, good, pp, None, None, 1,
+                                  None, None, None, FAKE, None, None)
+    assert st == paro.PA_ERR_INVALID_ARG and b"idx" in lib.pa_last_error()
+    fn = lib.pa_block_sparse_attn_compensated
+    assert fn(FAKE, FAKE, FAKE, paro.PA_BF16, 0, good, pp, None, None, 0, FAKE, FAKE,
+              paro.PA_F32, bad_out, None, None) == paro.PA_ERR_INVALID_ARG
+    assert b"aligned" in lib.pa_last_error()
+    assert fn(FAKE, FAKE, FAKE, paro.PA_BF16, 0, good, pp, None, None, 2, FAKE, FAKE,
+              paro.PA_F32, FAKE, None, None) == paro.PA_ERR_INVALID_ARG
+    assert b"idx" in lib.pa_last_error()
+
+
 def test_compensated_attention_validation(lib):
     good = paro.PaShape(1, 2, 4, 8, 8, 64, 64)  # NB = 4
     keep, pp = perms_of(0, 5)
