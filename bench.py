@@ -234,17 +234,14 @@ def time_steps(pipe, qkv, steps, warmup, ws, device):
     return total_ms, attn_ms
 
 
-E2E_CHUNKS = 8
-
-
-def e2e_steps(w, perms, density, int8, kernel, device, host, host_out, steps):
+def e2e_steps(w, perms, density, int8, kernel, device, host, host_out, steps, chunks):
     """The same step through the public host-memory API
     (pipeline.StreamedPipeline): pinned host -> device copies of Q, K, V,
     the path, and the device -> host copy of O, all inside the timed region,
     with the copies of one chunk of heads overlapped with the work of the
     previous one.  One untimed call first (kernel attributes, allocator)."""
     sp = StreamedPipeline(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, perms, density,
-                          chunks=E2E_CHUNKS, device=device,
+                          chunks=chunks, device=device,
                           dtype=torch.float32 if w.dtype == "f32" else torch.bfloat16,
                           int8=int8, baseline=kernel == "mma")
     sp.run(*host, host_out)
@@ -414,7 +411,7 @@ def run_ours(a):
         host = [t.pin_memory() for t in (q, k, v)]
         host_out = torch.empty(pipe.out.shape, dtype=pipe.out.dtype).pin_memory()
         e_ms, n_chunks = e2e_steps(w, perms, dens, int8, a.kernel, device, host, host_out,
-                                   max(1, min(a.steps, 5)))
+                                   max(1, min(a.steps, 5)), a.e2e_chunks)
         e_ms = max_over_ranks(e_ms, ws, device)
         e2e = {"value": flops * ws / (e_ms / 1e3) / 1e12, "unit": "TFLOPS",
                "ms_per_step": e_ms,
@@ -800,6 +797,8 @@ def main(argv=None):
                     help="with --sweep: only the PASA compensation line")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-chunks", type=int, default=16,
+                    help="head chunks of the end-to-end (host memory) measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--ref-blocks", type=int, default=8)

@@ -599,30 +599,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(BMX0 + grp));  // release: the store above is visible to the waiter
       if (m_mine != -INFINITY) l *= ex2(m_mine - m_j);  // this group's sum, to m_j
       m_mine = m_j;
-      // the group's P buffer is free once P V of its previous tile completed
-      if (j >= 2 && !warp_wait(pv_done(j - 2), ring_par(j - 2), ctl)) return false;
-      tc_fence_after();
-      // P = 2^(s*scale - m_j) as bf16 pairs into the group's P buffer, two
-      // columns per paired f32x2 FMA and add; row sum in 4 paired chains
+      // P = 2^(s*scale - m_j) as bf16 pairs, two columns per paired f32x2
+      // FMA and add (row sum in 4 paired chains), all 128 columns into
+      // registers first: the group's P buffer is written only once P V of
+      // its previous tile completed, and that wait now overlaps the
+      // exponentials
       const float neg_m = (m_j == -INFINITY ? 0.f : -m_j) + bias;
       const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(neg_m, neg_m);
       float2 rs2[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) rs2[u] = make_float2(0.f, 0.f);
+      uint32_t pk[64];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int e = 32 * cc + 2 * c;
-          const float2 t =
-              ffma2(make_float2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), sc2, nm2);
-          const float2 ex = make_float2(ex2(t.x), ex2(t.y));
-          rs2[c & 3] = fadd2(rs2[c & 3], ex);
-          pk[c] = pack_bf16(ex.x, ex.y);
-        }
-        tmem_st16_async(lane_addr + p_col + 16 * cc, pk);
+      for (int c = 0; c < 64; ++c) {
+        const int e = 2 * c;
+        const float2 t =
+            ffma2(make_float2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), sc2, nm2);
+        const float2 ex = make_float2(ex2(t.x), ex2(t.y));
+        rs2[c & 3] = fadd2(rs2[c & 3], ex);
+        pk[c] = pack_bf16(ex.x, ex.y);
       }
+      if (j >= 2 && !warp_wait(pv_done(j - 2), ring_par(j - 2), ctl)) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc)
+        tmem_st16_async(lane_addr + p_col + 16 * cc,
+                        *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * cc]));
       tmem_wait_st();
       l += ((rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y)) +
            ((rs2[2].x + rs2[2].y) + (rs2[3].x + rs2[3].y));
