@@ -413,8 +413,21 @@ def run_ours(a):
         e_ms, n_chunks = e2e_steps(w, perms, dens, int8, a.kernel, device, host, host_out,
                                    max(1, min(a.steps, 5)), a.e2e_chunks)
         e_ms = max_over_ranks(e_ms, ws, device)
+        # the bound of this number: the host -> device copies of the step's
+        # inputs alone (the same pinned buffers, one stream)
+        for t, hsrc in zip(qkv, host):
+            t.copy_(hsrc, non_blocking=True)
+        torch.cuda.synchronize()
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record()
+        for t, hsrc in zip(qkv, host):
+            t.copy_(hsrc, non_blocking=True)
+        c1.record()
+        torch.cuda.synchronize()
+        h2d_ms = max_over_ranks(c0.elapsed_time(c1), ws, device)
         e2e = {"value": flops * ws / (e_ms / 1e3) / 1e12, "unit": "TFLOPS",
-               "ms_per_step": e_ms,
+               "ms_per_step": e_ms, "h2d_only_ms": h2d_ms,
+               "frac_of_h2d_bound": h2d_ms / e_ms,
                "api": f"pipeline.StreamedPipeline ({n_chunks} head chunks; copies on their own "
                       "streams, overlapped with the previous chunk's work)",
                "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in host)),

@@ -5,7 +5,8 @@
  *
  * The path, one attention call:
  *   1. per-head reorder of the flattened tokens to one of the six axis orders
- *      of [F, H, W]                  (PAROAttention, arXiv 2506.16054, Pith
+ *      of [F, H, W] (or one of SPADE's six 3D tile blockings)
+ *                                    (PAROAttention, arXiv 2506.16054, Pith
  *                                     verdict page, key_machinery);
  *   2. mean-pooled Q/K block summaries and block scores
  *                                    (SPADE, arXiv 2608.03335, Pith verdict
@@ -21,10 +22,13 @@
  *   5. inverse reorder of the output (fused into step 4's store).
  *
  * Around it: SPADE's selection variants (pa_sics_scores, pa_select_hybrid),
- * INT4 P V (pa_quantize_int4 with PA_ATTN_P4), PAROAttention's offline stage
+ * INT4 P V (pa_quantize_int4 with PA_ATTN_P4), the per-tile reading of the
+ * INT8/INT4 post-softmax map (PA_ATTN_P_TILE), PAROAttention's offline stage
  * (pa_map_row_stats, pa_map_block_stats, pa_paro_metric, pa_paro_choose) and
  * PASA's compensation of the unselected blocks
- * (pa_block_sparse_attn_compensated).
+ * (pa_block_sparse_attn_compensated, with pa_round_bf16 for bf16 block
+ * means); pa_clear_status resets the device status word, and
+ * pa_test_inject_v_stall is the host-set hook of the bounded-wait test.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
