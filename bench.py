@@ -141,10 +141,14 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            # the timed region starts once samples are flowing (up to 2 s)
+            t0 = time.monotonic()
+            while not self.lines and time.monotonic() - t0 < 2.0 and self.proc.poll() is None:
+                time.sleep(0.01)
         except (OSError, ValueError):
             self.proc = None
 
