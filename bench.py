@@ -498,6 +498,9 @@ def run_sweep(a):
     if a.pasa_only:
         run_sweep_pasa(device, peaks, peak_src, a.heads)
         return
+    if a.hbm_only:
+        run_sweep_hbm(device, peaks, peak_src, a.heads)
+        return
     names = a.sweep_workloads.split(",") if a.sweep_workloads else list(WORKLOADS)
     for name in ([] if a.selection_only else names):
         w = WORKLOADS[name]
@@ -553,8 +556,51 @@ def run_sweep(a):
         return
     run_sweep_selection(device, peaks, peak_src, a.heads)
     run_sweep_offline(device, peaks, peak_src, a.heads)
+    run_sweep_hbm(device, peaks, peak_src, a.heads)
     if not a.selection_only and not a.sweep_workloads:
         run_sweep_pasa(device, peaks, peak_src, a.heads)
+
+
+def run_sweep_hbm(device, peaks, peak_src, heads=None):
+    """The HBM-bound preparation kernels on the 720p layer against the
+    measured copy bandwidth: reorder with block means (pool_kernel: reads a
+    bf16 row, writes it permuted, plus the fp32 mean per block) and the
+    block-wise quantisation with block means (quant_kernel: reads a bf16
+    row, writes its int8 codes, plus a scale and a mean per block).
+    Algorithmic bytes per tensor: N rows read and written once, N_p
+    written (pad rows included), per-block outputs."""
+    w = WORKLOADS["720p_21x45x80"]
+    q, _, _, perms = make_inputs(w, heads=heads)
+    if heads is not None:
+        w = dataclasses.replace(w, heads=heads)
+    qd = q.to(device)
+    pr = paro.Problem(w.B, w.heads, (w.F, w.H, w.W), w.d, w.block, perms)
+    bh = w.B * w.heads
+    xp = torch.empty(pr.permuted, dtype=qd.dtype, device=device)
+    pool = torch.empty(pr.pooled, dtype=torch.float32, device=device)
+    x8 = torch.empty(pr.permuted, dtype=torch.int8, device=device)
+    sc = torch.empty(pr.per_block, dtype=torch.float32, device=device)
+    per_block = bh * pr.NB * (w.d * 4)  # fp32 block means
+    runs = {
+        "pool_kernel (reorder + block means)":
+            (lambda: paro.reorder(qd, pr, out=xp, pool=pool),
+             bh * (pr.N * w.d * 2 + pr.N_p * w.d * 2) + per_block),
+        "quant_kernel (8-bit codes + scales + block means)":
+            (lambda: paro.quantize_int8(qd, pr, x_q=x8, scales=sc, pool=pool),
+             bh * (pr.N * w.d * 2 + pr.N_p * w.d) + per_block + bh * pr.NB * 4),
+        "quant_kernel (4-bit codes + scales + block means)":
+            (lambda: paro.quantize_int8(qd, pr, x_q=x8, scales=sc, pool=pool, bits=4),
+             bh * (pr.N * w.d * 2 + pr.N_p * w.d) + per_block + bh * pr.NB * 4),
+    }
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
+    for name, (fn, nbytes) in runs.items():
+        ms = percentiles(timed_calls(fn))
+        gbs = nbytes / (ms["p50"] / 1e3) / 1e9
+        print(json.dumps({
+            "workload": w.name, "kernel": name, "heads": w.heads, "ms": ms, "bytes": nbytes,
+            "gbs_p50": gbs, "frac_of_hbm_p50": gbs / hbm, "peak_source": f"{peak_src} hbm_gbs",
+            "steps": 20, "warmup": 5,
+        }), flush=True)
 
 
 def timed_calls(fn, reps=20, warm=5):
@@ -810,6 +856,8 @@ def main(argv=None):
                     help="with --sweep: only the selection-variant lines")
     ap.add_argument("--sweep-workloads", default="",
                     help="with --sweep: comma-separated workload names (default: all)")
+    ap.add_argument("--hbm-only", action="store_true",
+                    help="with --sweep: only the HBM-bound preparation kernels")
     ap.add_argument("--pasa-only", action="store_true",
                     help="with --sweep: only the PASA compensation line")
     ap.add_argument("--no-dense", action="store_true")

@@ -260,52 +260,67 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const T* __restrict__ x
   const int p0 = i * BLOCK;
   const int valid = min(BLOCK, g.N - p0);
   const uint4* base = reinterpret_cast<const uint4*>(x + bh * (int64_t)g.N * g.d);
-  float v[RPT][E];
-  float amax = 0.f;
+  // the block's rows stay in registers as loaded (packed: half the
+  // registers for bf16, so more CTAs keep loads in flight), unpacked at
+  // each use
+  uint4 raw[RPT];
 #pragma unroll
   for (int u = 0; u < RPT; ++u) {
     const int r = rg + u * GROUPS;
-    if (r < valid) {
-      const int n = natural_index(g, order, p0 + r);
-      Chunk<T>::unpack(__ldg(base + (int64_t)n * VPR + c), v[u]);
-    } else {
+    raw[u] = r < valid ? __ldg(base + (int64_t)natural_index(g, order, p0 + r) * VPR + c)
+                       : make_uint4(0, 0, 0, 0);
+  }
+  float amax = 0.f;
+  float acc[E];
 #pragma unroll
-      for (int e = 0; e < E; ++e) v[u][e] = 0.f;
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+#pragma unroll
+  for (int u = 0; u < RPT; ++u) {
+    float f[E];
+    Chunk<T>::unpack(raw[u], f);
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      amax = fmaxf(amax, fabsf(f[e]));
+      acc[e] += f[e];
     }
-#pragma unroll
-    for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(v[u][e]));
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = amax;
   if (pool != nullptr) {
-    float acc[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = 0.f;
-#pragma unroll
-    for (int u = 0; u < RPT; ++u)
-#pragma unroll
-      for (int e = 0; e < E; ++e) acc[e] += v[u][e];
 #pragma unroll
     for (int e = 0; e < E; ++e) psum[rg][c * E + e] = acc[e];
   }
   __syncthreads();
+  // only the packed rows stay live across the reduction (the compiler may
+  // not keep the unpacked values from the first pass)
+#pragma unroll
+  for (int u = 0; u < RPT; ++u)
+    asm volatile("" : "+r"(raw[u].x), "+r"(raw[u].y), "+r"(raw[u].z), "+r"(raw[u].w));
   amax = 0.f;
 #pragma unroll
   for (int w = 0; w < kThreads / 32; ++w) amax = fmaxf(amax, red[w]);
   const float qf = (float)qmax;
   const float inv = amax > 0.f ? __fdiv_rn(qf, amax) : 0.f;
+  // code = rint_half_even(fl32(x * inv)): the product rounded to fp32 first
+  // (the reading), then added to 1.5 * 2^23, which rounds it to the nearest
+  // integer, ties to even (|x * inv| <= qmax < 2^22), held in the low bits
+  constexpr float kMagic = 12582912.0f;
+  constexpr int32_t kMagicBits = 0x4B400000;
   int8_t* outb = xq + (bh * (int64_t)g.Np + p0) * D;
 #pragma unroll
   for (int u = 0; u < RPT; ++u) {
     const int r = rg + u * GROUPS;
+    float f[E];
+    Chunk<T>::unpack(raw[u], f);
     uint32_t packed[E / 4];
 #pragma unroll
     for (int e4 = 0; e4 < E / 4; ++e4) {
       uint32_t wv = 0;
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
-        int qv = __float2int_rn(__fmul_rn(v[u][e4 * 4 + b], inv));
+        const float t = __fmul_rn(f[e4 * 4 + b], inv);
+        int qv = (int32_t)__float_as_uint(__fadd_rn(t, kMagic)) - kMagicBits;
         qv = max(-qmax, min(qmax, qv));
         wv |= (uint32_t)(qv & 0xFF) << (8 * b);
       }
