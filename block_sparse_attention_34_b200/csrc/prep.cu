@@ -99,6 +99,63 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(const T* __restrict__ x,
   }
 }
 
+// The same for sizes fixed at compile time (bf16, d = 128, block = 128, the
+// tcgen05 path's shape): each thread issues all its rows' loads before the
+// first store, so the CTA keeps its whole block in flight; the sums and the
+// outputs are the same, bit for bit (rows accumulated in the same order).
+template <typename T, int D, int BLOCK>
+__global__ void __launch_bounds__(kThreads) pool_kernel_fixed(const T* __restrict__ x,
+                                                              const __grid_constant__ Grid g,
+                                                              float* __restrict__ pool,
+                                                              T* __restrict__ xp) {
+  constexpr int E = Chunk<T>::n;
+  constexpr int VPR = D / E;
+  constexpr int GROUPS = kThreads / VPR;
+  constexpr int RPT = BLOCK / GROUPS;
+  __shared__ float red[GROUPS][D];
+  const int i = blockIdx.x;
+  const int64_t bh = blockIdx.y;
+  const int h = (int)(bh % g.heads);
+  const int order = g.perm[h];
+  const int c = threadIdx.x % VPR;
+  const int rg = threadIdx.x / VPR;
+  const int p0 = i * BLOCK;
+  const int valid = min(BLOCK, g.N - p0);
+  const uint4* base = reinterpret_cast<const uint4*>(x + bh * (int64_t)g.N * D);
+  uint4 u[RPT];
+#pragma unroll
+  for (int k = 0; k < RPT; ++k) {
+    const int r = rg + k * GROUPS;
+    u[k] = r < valid ? __ldg(base + (int64_t)natural_index(g, order, p0 + r) * VPR + c)
+                     : make_uint4(0, 0, 0, 0);
+  }
+  if (xp != nullptr) {
+    uint4* dst = reinterpret_cast<uint4*>(xp + (bh * (int64_t)g.Np + p0) * D);
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) dst[(int64_t)(rg + k * GROUPS) * VPR + c] = u[k];
+  }
+  if (pool == nullptr) return;  // uniform across the CTA
+  float acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+#pragma unroll
+  for (int k = 0; k < RPT; ++k) {
+    if (xp == nullptr && rg + k * GROUPS >= valid) break;  // as the generic loop's bound
+    float f[E];
+    Chunk<T>::unpack(u[k], f);
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] += f[e];
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) red[rg][c * E + e] = acc[e];
+  __syncthreads();
+  for (int col = threadIdx.x; col < D; col += kThreads) {
+    float sum = 0.f;
+    for (int r = 0; r < GROUPS; ++r) sum += red[r][col];
+    pool[(bh * g.NB + i) * D + col] = sum / (float)valid;
+  }
+}
+
 // --------------------------------------------------------------- scores ---
 // S[bh, i, j] = dot(qp[bh, i], kp[bh, j]) * inv_sqrt_d, fp32 SIMT tiles of
 // 64 x 64 (the whole matrix is < 0.1% of the attention FLOPs).
@@ -366,7 +423,10 @@ cudaError_t launch_reorder_pool(const void* x, void* xp, pa_dtype dt, const Grid
   const int groups = kThreads / (g.d / E);
   const size_t smem = (size_t)groups * g.d * sizeof(float);
   dim3 grid(g.NB, g.B * g.heads);
-  if (dt == PA_F32)
+  if (dt == PA_BF16 && g.d == 128 && g.block == 128)
+    pool_kernel_fixed<__nv_bfloat16, 128, 128><<<grid, kThreads, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), g, pool, static_cast<__nv_bfloat16*>(xp));
+  else if (dt == PA_F32)
     pool_kernel<float><<<grid, kThreads, smem, s>>>(static_cast<const float*>(x), g, pool,
                                                     static_cast<float*>(xp));
   else
