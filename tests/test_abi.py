@@ -353,3 +353,36 @@ def test_stall_hook_arguments_are_checked(lib):
     assert lib.pa_test_inject_v_stall(-1, 0, 1, 1_000_000) == paro.PA_ERR_INVALID_ARG
     assert lib.pa_test_inject_v_stall(0, 0, 1, 2_000_000_000) == paro.PA_ERR_INVALID_ARG
     assert lib.pa_test_inject_v_stall(-1, -1, -1, 0) == paro.PA_OK  # off
+
+
+def test_binding_chooses_the_p_reading_flags(monkeypatch):
+    """The flags the binding hands pa_block_sparse_attn for the INT8 and
+    INT4 paths: INT4 PV takes the per-tile reading (PA_ATTN_P_TILE) by
+    default, INT8 the one-pass form unless p_tile is asked for (a recording
+    stand-in for the library; CPU tensors, nothing dereferenced)."""
+    import torch
+
+    calls = []
+
+    class Recorder:
+        def pa_k_for_density(self, nb, density):
+            return ref.k_for_density(nb, density)
+
+        def pa_block_sparse_attn(self, *args):
+            calls.append(int(args[4]))  # flags
+            return paro.PA_OK
+
+        def __getattr__(self, name):
+            return lambda *args: paro.PA_OK
+
+    monkeypatch.setattr(paro, "_need_cuda", lambda *ts: None)
+    monkeypatch.setattr(paro, "_stream", lambda: None)
+    monkeypatch.setattr(paro, "load", lambda: Recorder())
+    q = torch.zeros((1, 2, 4 * 8 * 16, 128), dtype=torch.bfloat16)
+    for kw, want in [({"int8": True}, 0),
+                     ({"int8": True, "p_tile": True}, paro.PA_ATTN_P_TILE),
+                     ({"int8": True, "int4_pv": True}, paro.PA_ATTN_P4 | paro.PA_ATTN_P_TILE),
+                     ({"int8": True, "int4_pv": True, "p_tile": False}, paro.PA_ATTN_P4)]:
+        calls.clear()
+        paro.attention(q, q, q, (4, 8, 16), [0, 5], 128, 0.5, **kw)
+        assert calls == [want], (kw, calls)
