@@ -17,9 +17,11 @@
 //              memory lane quarter), one row per thread, all 128 keys of
 //              the tile.  A thread copies its row of S (128 fp32) from the
 //              group's S buffer into registers and releases the buffer, so
-//              QK^T two tiles ahead can start at once; it then writes its
-//              128 probabilities as bf16 pairs into the group's P buffer
-//              (the P V MMA's A operand).  Both groups accumulate into one
+//              QK^T two tiles ahead can start at once; it then computes
+//              its 128 probabilities as bf16 pairs in registers (scale,
+//              subtract and row sums as paired f32x2 instructions) and
+//              writes them into the group's P buffer (the P V MMA's A
+//              operand) once P V of the group's previous tile completed.  Both groups accumulate into one
 //              O, so every row has one reference max m_j, passed along the
 //              tile order through shared memory: m_j = m_{j-1} unless tile
 //              j's max exceeds it by more than 2^8 (then m_j is that max and
@@ -49,12 +51,14 @@
 // and section 3.3: the key blocks outside a query block's kept set enter
 // through a grouped first-order term), ceil(NB/128) pooled tiles follow the
 // kept tiles of every row: row c of pooled tile p is block b = 128p + c's
-// mean key and mean value (fp32 block means, rounded to bf16 by the loader
-// warps into the same swizzled stage layout), and the softmax adds log2 of
-// the block's valid key count to its score and gives kept blocks and
-// columns past NB the score -inf.  So block b adds n_b e^{q.kbar_b/sqrt(d)}
-// to the normaliser and that times vbar_b to the numerator, in the same
-// online softmax.
+// mean key and mean value (bf16 block means loaded with TMA like the K and
+// V tiles, or fp32 ones rounded to bf16 by the loader warps into the same
+// swizzled stage layout).  The softmax masks kept blocks and columns past
+// NB (per-tile use words from a bitset of the kept list), adds log2 of a
+// full block's key count, 7, to the exponent of every used column, and
+// gives the ragged last block its own count on its score.  So block b adds
+// n_b e^{q.kbar_b/sqrt(d)} to the normaliser and that times vbar_b to the
+// numerator, in the same online softmax.
 //
 // A K stage is refilled once its QK^T completes, a V stage once its P V
 // completes; each MMA group signals its completion with one commit.  Every mbarrier wait is bounded (about one second of
